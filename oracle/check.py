@@ -1,0 +1,61 @@
+"""Comparison rules between a computed layer output and the oracle's (test
+infrastructure only).
+
+Float outputs: per token row, the largest absolute difference divided by the
+row's largest reference magnitude (floor 1e-6), maximised over rows. This is
+the reading taken of "max relative error" for rows that may contain zeros.
+Bound: 2e-2 for bf16 storage, 1e-4 for the fp32 path.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+TOL_BF16 = 2e-2
+TOL_F32 = 1e-4
+TOL_GATE = 1e-5
+
+
+def row_rel_err(y, y_ref, floor=1e-6):
+    y = np.asarray(y, np.float64)
+    y_ref = np.asarray(y_ref, np.float64)
+    if y.shape != y_ref.shape:
+        raise ValueError(f"shape {y.shape} != {y_ref.shape}")
+    if y.size == 0:
+        return 0.0
+    num = np.abs(y - y_ref).max(axis=1)
+    den = np.maximum(np.abs(y_ref).max(axis=1), floor)
+    r = num / den
+    if np.isnan(r).any():
+        return float("inf")
+    return float(r.max())
+
+
+def tol_for(dtype: str) -> float:
+    return TOL_BF16 if dtype == "bf16" else TOL_F32
+
+
+def outputs_match(y, y_ref, dtype: str) -> bool:
+    return row_rel_err(y, y_ref) <= tol_for(dtype)
+
+
+def permutation_consistent(dest_row, perm_src, offsets, idx, n_kept=None):
+    """The combine source-index map is the inverse of the dispatch map on kept
+    slots, and each expert segment lists its tokens in ascending order."""
+    dest_row = np.asarray(dest_row)
+    perm_src = np.asarray(perm_src)
+    offsets = np.asarray(offsets)
+    idx = np.asarray(idx)
+    n = int(offsets[-1]) if n_kept is None else n_kept
+    tt, jj = np.nonzero(dest_row >= 0)
+    if len(tt) != n:
+        return False
+    if not np.array_equal(perm_src[dest_row[tt, jj]], tt):
+        return False
+    e = idx[tt, jj]
+    if not ((dest_row[tt, jj] >= offsets[e]) & (dest_row[tt, jj] < offsets[e + 1])).all():
+        return False
+    for a in range(len(offsets) - 1):
+        seg = perm_src[offsets[a]:offsets[a + 1]]
+        if seg.size > 1 and not (np.diff(seg) > 0).all():
+            return False
+    return True

@@ -1,0 +1,341 @@
+"""Pins of the CPU oracle to facts fixed outside it (CPU only).
+
+Each test checks the oracle against something it does not compute itself: the
+numbers the dispatch page prints for its two worked routing maps, brute force
+over all expert subsets, closed forms of identity-tagged tokens with
+scale-by-constant experts, and torch library routines on special cases that
+reduce to them (dense SwiGLU when E=k=1, a dense softmax mixture when k=E).
+The last group plants known mistakes in a copy of the combine step and checks
+that the comparison rules catch them.
+"""
+import itertools
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from oracle import check as C
+from oracle import cases
+import workloads as W
+
+RNG = np.random.default_rng(1234)
+
+
+# ---------------------------------------------------------------- worked maps
+def _load_maps(golden_dir):
+    with open(os.path.join(golden_dir, "dispatch_worked_maps.json")) as f:
+        return json.load(f)
+
+
+@pytest.mark.parametrize("name", ["map1", "map2"])
+def test_worked_routing_maps(golden_dir, name):
+    g = _load_maps(golden_dir)
+    toks = g["tokens"]
+    m = g["maps"][name]
+    idx = np.array([[m["expert_of_token"][t]] for t in toks], np.int32)
+    meta = O.dispatch_meta(idx, E=4, cap=-1)
+    assert meta["routed"].tolist() == m["counts_printed"]
+    assert meta["kept"].tolist() == m["counts_printed"]
+    assert meta["offsets"].tolist() == [0] + np.cumsum(m["counts_printed"]).tolist()
+    grouped = [[toks[t] for t in meta["perm_src"][meta["offsets"][e]:meta["offsets"][e + 1]]]
+               for e in range(4)]
+    assert grouped == m["expected_grouping_by_expert"]
+    remote = O.remote_assignments(idx[:, 0], tokens_per_rank=2, experts_per_rank=1)
+    assert remote == m["remote_vectors_printed"]
+    assert remote * g["row_bytes"] == m["remote_bytes_printed"]
+    assert C.permutation_consistent(meta["dest_row"], meta["perm_src"], meta["offsets"], idx)
+
+
+# ---------------------------------------------------------------- selection
+def _brute_topk(row, k):
+    """The k-subset whose every member beats every non-member under
+    (higher score, then lower index); slots ordered the same way."""
+    E = len(row)
+
+    def beats(a, b):
+        return row[a] > row[b] or (row[a] == row[b] and a < b)
+
+    winners = [S for S in itertools.combinations(range(E), k)
+               if all(beats(a, b) for a in S for b in range(E) if b not in S)]
+    assert len(winners) == 1
+    return sorted(winners[0], key=lambda e: (-row[e], e))
+
+
+def _tie_rows(T, E):
+    s = RNG.integers(-3, 4, size=(T, E)).astype(np.float32)   # many exact ties
+    s[0] = 1.0                                                 # all tied
+    s[1] = -np.inf                                             # all -inf
+    s[2, : E // 2] = -np.inf
+    return s
+
+
+@pytest.mark.parametrize("E", [1, 2, 3, 4, 6])
+def test_topk_against_brute_force(E):
+    s = _tie_rows(16, E)
+    for k in sorted({1, min(2, E), E}):
+        idx = O.topk_select(s, k)
+        for t in range(s.shape[0]):
+            assert idx[t].tolist() == _brute_topk(s[t].tolist(), k)
+
+
+def test_topk_against_library_sort():
+    s = RNG.standard_normal((300, 64)).astype(np.float32)
+    s[:, 5] = s[:, 9]                                          # planted ties
+    for k in (1, 6, 64):
+        idx = O.topk_select(s, k)
+        order = np.lexsort((np.broadcast_to(np.arange(64), s.shape), -s), axis=1)[:, :k]
+        assert np.array_equal(idx, order)
+
+
+def test_topk_matches_torch_topk_without_ties():
+    s = RNG.standard_normal((200, 16)).astype(np.float32)
+    idx = O.topk_select(s, 4)
+    ref = torch.topk(torch.from_numpy(s), 4, dim=1).indices.numpy()
+    assert np.array_equal(idx, ref)
+
+
+def test_nan_logits_count_as_minus_inf():
+    s = np.array([[0.5, np.nan, 0.2, np.nan]], np.float64)
+    s32, nan_row = O.decision_logits(s)
+    assert nan_row.tolist() == [True]
+    assert O.topk_select(s32, 3).tolist() == [[0, 2, 1]]
+
+
+# ---------------------------------------------------------------- gates
+def test_gates_are_softmax_over_picks():
+    s = RNG.standard_normal((100, 8)) * 3
+    idx = O.topk_select(s.astype(np.float32), 3)
+    g = O.gates(s, idx)
+    picked = torch.from_numpy(np.take_along_axis(s, idx.astype(np.int64), 1))
+    ref = torch.softmax(picked, dim=1).numpy()                    # library softmax
+    assert np.allclose(g, ref, rtol=1e-12, atol=1e-15)
+    assert np.allclose(g.sum(1), 1.0)
+    # equal to the full softmax renormalised (torch, different route)
+    p = torch.softmax(torch.from_numpy(s), dim=1).numpy()
+    pk = np.take_along_axis(p, idx.astype(np.int64), 1)
+    assert np.allclose(g, pk / pk.sum(1, keepdims=True), rtol=1e-12)
+
+
+def test_gates_degenerate_rows():
+    s = np.array([[-np.inf, -np.inf, -np.inf], [0.0, -np.inf, -np.inf]])
+    idx = O.topk_select(s.astype(np.float32), 2)
+    assert idx.tolist() == [[0, 1], [0, 1]]
+    g = O.gates(s, idx)
+    assert g.tolist() == [[0.0, 0.0], [1.0, 0.0]]
+
+
+def test_router_margin_closed_form():
+    s = np.array([[3.0, 1.0, 2.5, 0.0], [1.0, 1.0, 1.0, 0.5]])
+    assert O.router_margin(s, 1).tolist() == [0.5, 0.0]
+    assert O.router_margin(s, 3).tolist() == [1.0, 0.5]
+    assert O.min_adjacent_gap(s, 2).tolist() == [0.5, 0.0]
+
+
+def test_router_logits_closed_form():
+    h = np.array([[1.0, 2.0], [0.0, -1.0]])
+    w = np.array([[1.0, 0.0], [0.5, 0.5], [0.0, 0.0]])
+    b = np.array([0.0, 1.0, -np.inf])
+    s = O.router_logits(h, w, b)
+    assert s.tolist() == [[1.0, 2.5, -np.inf], [0.0, 0.5, -np.inf]]
+
+
+# ---------------------------------------------------------------- dispatch / capacity
+def _random_idx(T, E, k, seed):
+    r = np.random.default_rng(seed)
+    rows = [r.permutation(E)[:k] for _ in range(T)]
+    return np.stack(rows).astype(np.int32) if rows else np.zeros((0, k), np.int32)
+
+
+@pytest.mark.parametrize("T,E,k,cap", [(50, 5, 2, -1), (200, 8, 3, 40), (64, 4, 4, 10), (1, 3, 1, -1),
+                                       (0, 3, 1, -1), (30, 6, 2, 0)])
+def test_dispatch_invariants_and_capacity(T, E, k, cap):
+    idx = _random_idx(T, E, k, T + E)
+    meta = O.dispatch_meta(idx.reshape(T, k), E, cap)
+    routed = np.bincount(idx.ravel(), minlength=E)
+    assert meta["routed"].tolist() == routed.tolist()
+    assert meta["routed"].sum() == T * k
+    kept = routed if cap < 0 else np.minimum(routed, cap)
+    assert meta["kept"].tolist() == kept.tolist()
+    assert meta["offsets"][-1] == T * k - (0 if cap < 0 else np.maximum(routed - cap, 0).sum())
+    assert C.permutation_consistent(meta["dest_row"], meta["perm_src"], meta["offsets"], idx.reshape(T, k))
+    # the kept set of each expert is exactly its `cap` lowest token indices
+    for e in range(E):
+        users = sorted(t for t in range(T) if e in idx[t])
+        want = users if cap < 0 else users[:cap]
+        got = meta["perm_src"][meta["offsets"][e]:meta["offsets"][e + 1]].tolist()
+        assert got == want
+
+
+def test_invalid_routes_are_dropped_and_flagged():
+    idx = np.array([[0, 0], [1, 5], [-1, 2], [2, 1]], np.int32)
+    meta = O.dispatch_meta(idx, E=3, cap=-1)
+    assert meta["bad_route"]
+    assert (meta["dest_row"][0] >= 0).tolist() == [True, False]
+    assert (meta["dest_row"][1] >= 0).tolist() == [True, False]
+    assert (meta["dest_row"][2] >= 0).tolist() == [False, True]
+    assert meta["routed"].tolist() == [1, 2, 2]
+
+
+def test_capacity_formula_values():
+    assert O.capacity(16384, 6, 64) == 1920
+    assert O.capacity(64, 2, 4) == 40
+    assert O.capacity(8, 1, 4) == 2
+    assert W.capacity_factor_cap(16384, 6, 64) == 1920
+
+
+# ---------------------------------------------------------------- closed forms of the layer
+def test_identity_tagged_scale_experts_closed_form():
+    inp = cases.parity_inputs("tiny_f32_tagged")
+    wl = inp.wl
+    h = cases.as64(inp.h)
+    out = O.layer_forward(h, cases.as64(inp.w_router), None, wl.k, "scale")
+    idx, g, y = out["idx"], out["gate"], out["y"]
+    for t in range(wl.T):
+        c = t % wl.d
+        expect = (t + 1) * sum(g[t, j] * (idx[t, j] + 1) for j in range(wl.k))
+        row = y[t].copy()
+        assert row[c] == pytest.approx(expect, rel=1e-13)
+        row[c] = 0.0
+        assert not row.any()
+
+
+def test_identity_experts_return_input():
+    inp = cases.parity_inputs("tiny_f32")
+    wl = inp.wl
+    h = cases.as64(inp.h)
+    out = O.layer_forward(h, cases.as64(inp.w_router), None, wl.k, "identity")
+    assert np.allclose(out["y"], h, rtol=1e-14, atol=1e-14)
+
+
+def test_identity_experts_with_drops_scale_by_kept_gates():
+    h = RNG.standard_normal((40, 8))
+    w = RNG.standard_normal((4, 8))
+    out = O.layer_forward(h, w, None, 2, "identity", cap=10)
+    kept_gate = np.where(out["dest_row"] >= 0, out["gate"], 0.0).sum(1)
+    assert np.allclose(out["y"], h * kept_gate[:, None], rtol=1e-14, atol=1e-14)
+    assert (kept_gate < 1).any()                                # something was dropped
+
+
+def test_single_expert_is_dense_swiglu():
+    T, d, F = 20, 16, 24
+    h = RNG.standard_normal((T, d))
+    wg, wu, wd = RNG.standard_normal((1, F, d)), RNG.standard_normal((1, F, d)), RNG.standard_normal((1, d, F))
+    out = O.layer_forward(h, RNG.standard_normal((1, d)), None, 1, "swiglu",
+                          weights=lambda e: (wg[e], wu[e], wd[e]))
+    ht = torch.from_numpy(h)
+    ref = (torch.nn.functional.silu(ht @ torch.from_numpy(wg[0]).T) * (ht @ torch.from_numpy(wu[0]).T)) \
+        @ torch.from_numpy(wd[0]).T
+    assert np.allclose(out["y"], ref.numpy(), rtol=1e-12, atol=1e-12)
+    assert (out["gate"] == 1.0).all()
+
+
+def test_all_experts_is_dense_softmax_mixture():
+    T, d, F, E = 12, 8, 10, 4
+    h = RNG.standard_normal((T, d))
+    wr = RNG.standard_normal((E, d))
+    b = RNG.standard_normal(E)
+    wg, wu, wd = RNG.standard_normal((E, F, d)), RNG.standard_normal((E, F, d)), RNG.standard_normal((E, d, F))
+    out = O.layer_forward(h, wr, b, E, "swiglu", weights=lambda e: (wg[e], wu[e], wd[e]))
+    ht = torch.from_numpy(h)
+    p = torch.softmax(ht @ torch.from_numpy(wr).T + torch.from_numpy(b), dim=1)
+    ref = torch.zeros(T, d, dtype=torch.float64)
+    for e in range(E):
+        fe = (torch.nn.functional.silu(ht @ torch.from_numpy(wg[e]).T) * (ht @ torch.from_numpy(wu[e]).T)) \
+            @ torch.from_numpy(wd[e]).T
+        ref += p[:, e:e + 1] * fe
+    assert np.allclose(out["y"], ref.numpy(), rtol=1e-12, atol=1e-12)
+    assert (out["routed"] == T).all()
+
+
+def test_silu_against_library():
+    z = np.linspace(-30, 30, 1001)
+    assert np.allclose(O.silu(z), torch.nn.functional.silu(torch.from_numpy(z)).numpy(), rtol=1e-14, atol=1e-300)
+
+
+# ---------------------------------------------------------------- planted mistakes
+def _permuted_pipeline(h, idx, gate, meta, kind, wrong_index=False, swap_gates=False):
+    """CPU emulation of the grouped path: gather rows by expert, apply experts
+    per segment, scatter back. wrong_index plants the bug of scattering with the
+    pre-permutation index; swap_gates pairs each output with the other slot's
+    gate."""
+    x_perm = h[meta["perm_src"]]
+    y_perm = np.zeros_like(x_perm)
+    off = meta["offsets"]
+    for e in range(len(off) - 1):
+        y_perm[off[e]:off[e + 1]] = O.expert_apply(kind, e, x_perm[off[e]:off[e + 1]])
+    y = np.zeros_like(h)
+    T, k = idx.shape
+    for t in range(T):
+        for j in range(k):
+            r = meta["dest_row"][t, j]
+            if r < 0:
+                continue
+            src = y_perm[r] if not wrong_index else y_perm[min(t * k + j, len(y_perm) - 1)]
+            gj = gate[t, (j + 1) % k] if swap_gates else gate[t, j]
+            y[t] += gj * src
+    return y
+
+
+@pytest.mark.parametrize("kind", ["scale", "identity"])
+def test_checker_catches_planted_mistakes(kind):
+    inp = cases.parity_inputs("tiny_f32_tagged")
+    h = cases.as64(inp.h)
+    out = O.layer_forward(h, cases.as64(inp.w_router), None, inp.wl.k, kind)
+    meta = {k_: out[k_] for k_ in ("perm_src", "offsets", "dest_row")}
+    good = _permuted_pipeline(h, out["idx"], out["gate"], meta, kind)
+    assert C.row_rel_err(good, out["y"]) < 1e-12
+    bad_index = _permuted_pipeline(h, out["idx"], out["gate"], meta, kind, wrong_index=True)
+    assert not C.outputs_match(bad_index, out["y"], "f32")
+    if kind == "scale":   # identity experts sum to h whatever gate goes with which slot
+        bad_gate = _permuted_pipeline(h, out["idx"], out["gate"], meta, kind, swap_gates=True)
+        assert not C.outputs_match(bad_gate, out["y"], "f32")
+
+
+def test_permutation_check_catches_swapped_rows():
+    idx = _random_idx(40, 5, 2, 7)
+    meta = O.dispatch_meta(idx, 5)
+    assert C.permutation_consistent(meta["dest_row"], meta["perm_src"], meta["offsets"], idx)
+    dr = meta["dest_row"].copy()
+    a, b = np.argwhere(dr >= 0)[[0, 7]]
+    dr[tuple(a)], dr[tuple(b)] = dr[tuple(b)], dr[tuple(a)]
+    assert not C.permutation_consistent(dr, meta["perm_src"], meta["offsets"], idx)
+
+
+# ---------------------------------------------------------------- generator + margin pass
+def test_generator_is_deterministic_and_streams_differ():
+    wl = W.get("mixtral_scaled").with_(T=64)
+    a, b = W.draw_h(wl, 0), W.draw_h(wl, 0)
+    assert torch.equal(a, b)
+    assert not torch.equal(a, W.draw_h(wl, 1))
+    g0 = W.draw_w_gate(wl.with_(F=128, d=128, E=3), 0)
+    g1 = W.draw_w_gate(wl.with_(F=128, d=128, E=3), 0, experts=[1])
+    assert torch.equal(g0[1], g1[0])
+
+
+def test_margin_pass_reaches_min_gap():
+    inp = cases.parity_inputs("mixtral_scaled", weights=False)
+    s = O.router_logits(cases.as64(inp.h), cases.as64(inp.w_router), cases.as64(inp.bias))
+    assert O.min_adjacent_gap(s, inp.wl.k).min() >= cases.MIN_GAP
+
+
+def test_many_small_hot_bias_gives_half_the_assignments():
+    wl = W.get("many_small")
+    inp = cases.parity_inputs(wl, weights=False)
+    out = O.route(cases.as64(inp.h), cases.as64(inp.w_router), cases.as64(inp.bias), wl.k)
+    share = (out[0] < W.HOT_EXPERTS).mean()
+    assert abs(share - 0.5) <= 0.01
+    assert not (out[0] >= W.EMPTY_FROM).any()
+
+
+def test_skewed_bias_gives_hot_experts_and_empties():
+    wl = W.get("skewed")
+    inp = cases.parity_inputs(wl, weights=False)
+    idx = O.route(cases.as64(inp.h), cases.as64(inp.w_router), cases.as64(inp.bias), wl.k)[0]
+    counts = np.bincount(idx.ravel(), minlength=wl.E)
+    assert counts[list(W.SKEWED_EMPTY)].sum() == 0
+    assert counts.max() >= 5 * counts.mean()
+    assert O.dispatch_meta(idx, wl.E, O.capacity(wl.T, wl.k, wl.E))["kept"].max() == 1920
