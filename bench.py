@@ -1,0 +1,423 @@
+"""Benchmark of the MoE layer forward on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+One step is one whole layer forward (route, permute, grouped SwiGLU FFN,
+unpermute/combine) over one batch of T synthetic tokens, through the C ABI
+entry point moe_layer_forward. Under torchrun each rank runs its own batch on
+its own GPU (token-sharded replicas: weak scaling, no collective on the data
+path); `value` is the tokens of all ranks divided by the slowest rank's
+device time. Rank 0 prints one JSON line.
+
+--impl reference times the CPU oracle (fp64, numpy) on the host cores on a
+bounded token sample of the same workload; under torchrun only rank 0 runs it.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import re
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "MoE layer tokens/s; dispatch+combine HBM GB/s; grouped-GEMM TFLOPS (1 B200)"
+UNIT = "tokens/s"
+DEFAULT_WORKLOAD = "mixtral_8x7b"
+# tokens of the bounded CPU sample per workload (about 10-30 s of oracle work)
+CPU_SAMPLE = {"mixtral_8x7b": 512, "mixtral_scaled": 2048, "skewed": 1024, "many_small": 1024,
+              "tiny_f32": 64}
+PEAKS_PATH = os.path.join(ROOT, "MEASURED_PEAKS.json")
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+GEMM_PROFILE = os.path.join(ROOT, "profiles", "grouped_gemm_mixtral_8x7b.md")
+GEMM_SOURCES = [os.path.join(ROOT, "combine_router_gemm_softmax_b200", "csrc", f)
+                for f in ("grouped_ffn.cu", "moe_common.cuh")]
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--seed", type=int, default=0)
+    return ap.parse_args()
+
+
+def peaks():
+    if os.path.exists(PEAKS_PATH):
+        with open(PEAKS_PATH) as f:
+            p = json.load(f)
+        return p, "measured"
+    return FALLBACK_PEAKS, "fallback"
+
+
+def gemm_source_sha():
+    h = hashlib.sha256()
+    for p in GEMM_SOURCES:
+        with open(p, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic():
+    """DRAM bytes per grouped-GEMM launch pair from the committed ncu summary, if
+    it was taken on the current kernel source; else None."""
+    if not os.path.exists(GEMM_PROFILE):
+        return None
+    txt = open(GEMM_PROFILE).read()
+    m_sha = re.search(r"kernel_source_sha:\s*([0-9a-f]+)", txt)
+    m_b = re.search(r"traffic_bytes_per_step:\s*([0-9.eE+]+)", txt)
+    if not (m_sha and m_b) or m_sha.group(1) != gemm_source_sha():
+        return None
+    return float(m_b.group(1))
+
+
+# ---------------------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id):
+        self.gpu_id = gpu_id
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu_id), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+            time.sleep(0.3)
+        except OSError:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            time.sleep(0.2)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.lines:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx = float(parts[1])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[4:8]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------- CPU oracle
+def oracle_tokens_per_s(wl, n_tokens, seed=0):
+    """Oracle (as it stands) on the first n_tokens of the workload as their own
+    batch: route, dispatch metadata, experts and combine. Returns (tokens/s,
+    seconds, threads)."""
+    import oracle as O
+    from oracle import cases
+    import workloads as W
+    from threadpoolctl import threadpool_info
+
+    sub = wl.with_(T=min(n_tokens, wl.T))
+    inp = W.draw(sub, seed)
+    t0 = time.perf_counter()
+    O.layer_forward(cases.as64(inp.h), cases.as64(inp.w_router), cases.as64(inp.bias), sub.k, sub.expert_kind,
+                    cases.weights_fn(inp) if sub.expert_kind == "swiglu" else None, sub.capacity)
+    dt = time.perf_counter() - t0
+    threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    return sub.T / dt, dt, threads
+
+
+def run_reference(args, wl, rank):
+    if rank != 0:
+        return
+    n = CPU_SAMPLE.get(wl.name, 256)
+    for _ in range(args.warmup):
+        oracle_tokens_per_s(wl, n, args.seed)
+    times = []
+    threads = 1
+    for _ in range(args.steps):
+        _, dt, threads = oracle_tokens_per_s(wl, n, args.seed)
+        times.append(dt)
+    total = sum(times)
+    value = n * args.steps / total
+    sample = f"first {min(n, wl.T)} tokens of {wl.name} as their own batch, {args.steps} steps"
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic (seeded)", "config": config_dict(wl, args.gpus),
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def config_dict(wl, n):
+    return {"workload": wl.name, "T": wl.T, "d": wl.d, "E": wl.E, "k": wl.k, "d_ff": wl.F, "dtype": wl.dtype,
+            "expert_kind": wl.expert_kind, "capacity": wl.capacity, "global_batch": wl.T * n,
+            "parallelism": f"token-sharded replicas x{n}",
+            "l2": "not flushed: inputs larger than L2 (126 MB)"}
+
+
+# ---------------------------------------------------------------------------- GPU arm
+def main():
+    args = parse()
+    import torch
+
+    import workloads as W
+
+    wl = W.get(args.workload)
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, wl, rank)
+        return
+
+    import datetime
+
+    import torch.distributed as dist
+
+    import combine_router_gemm_softmax_b200 as M
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    # inputs: each rank draws its own batch (seed + rank), weights are the same
+    M.lib()
+    inp = W.draw(wl, args.seed)
+    h_host = W.draw_h(wl, args.seed + rank).pin_memory() if rank else inp.h.pin_memory()
+    cfg = M.config(wl.T, wl.d, wl.E, wl.k, wl.F, wl.dtype, wl.expert_kind, wl.capacity)
+    h = h_host.to(dev)
+    wr = inp.w_router.to(dev)
+    bias = None if inp.bias is None else inp.bias.to(dev)
+    w13 = wd = None
+    if wl.expert_kind == "swiglu":
+        wg, wu = inp.w_gate.to(dev), inp.w_up.to(dev)
+        w13 = M.moe_pack_weights(cfg, wg, wu)
+        del wg, wu
+        wd = inp.w_down.to(dev)
+    del inp
+    y = torch.empty((wl.T, wl.d), dtype=wl.torch_dtype, device=dev)
+    counts = torch.empty(wl.E, dtype=torch.int32, device=dev)
+    routed = torch.empty(wl.E, dtype=torch.int32, device=dev)
+    ws = M.workspace(cfg, M.MOE_OP_LAYER, dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        M.moe_layer_forward(cfg, h, wr, bias, w13, wd, y=y, routed_counts=routed, counts=counts, ws=ws,
+                            status=status, stream=stream)
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize()
+
+    # ------------------------------------------------ timed region (device events)
+    gpu_uuid = torch.cuda.get_device_properties(dev).uuid
+    sampler = ClockSampler(f"GPU-{gpu_uuid}")
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with sampler:
+        barrier()
+        torch.cuda.synchronize()
+        start.record(stream)
+        for _ in range(args.steps):
+            step()
+        end.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+    ms = start.elapsed_time(end)
+    ms_max = ms
+    if world > 1:
+        t = torch.tensor([ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_max = float(t.item())
+    value = wl.T * world * args.steps / (ms_max / 1e3)
+    launches_per_step = launches(cfg)
+    st = int(status.item())
+
+    # ------------------------------------------------ end to end: host buffers, copies inside the timed region
+    y_host = torch.empty((wl.T, wl.d), dtype=wl.torch_dtype, pin_memory=True)
+    for _ in range(2):
+        h.copy_(h_host, non_blocking=True)
+        step()
+        y_host.copy_(y, non_blocking=True)
+    torch.cuda.synchronize()
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        h.copy_(h_host, non_blocking=True)
+        step()
+        y_host.copy_(y, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    e2e_value = wl.T * world * args.steps / (e2e_ms / 1e3)
+    row_bytes = wl.d * wl.elem_bytes
+
+    # ------------------------------------------------ per stage (same stream, CUDA events)
+    stages = stage_times(M, cfg, wl, h, wr, bias, w13, wd, dev, stream, reps=max(3, min(args.steps, 10)))
+    barrier()
+
+    if rank == 0:
+        pk, pk_kind = peaks()
+        counts_np = counts.cpu().numpy()
+        A_kept = int(counts_np.sum())
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": max(args.warmup, 3), "ms_per_step": ms_max / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": wl.dtype,
+            "data": "synthetic: seeded N(0,1) tokens, N(0,1/fan_in) random-init weights",
+            "config": config_dict(wl, world),
+            "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": wl.T * row_bytes,
+                    "d2h_bytes_per_step": wl.T * row_bytes, "ms_per_step": e2e_ms / args.steps,
+                    "path": "pinned host h -> device, moe_layer_forward, device y -> pinned host"},
+            "gpu_launches": launches_per_step * args.steps,
+            "clocks": sampler.summary(),
+            "status_word": st,
+        }
+        line["stages"] = stage_report(stages, wl, A_kept, pk, pk_kind)
+        line["roofline"] = roofline(stages, wl, A_kept, pk, pk_kind)
+        line["routing"] = {"routed_counts_max": int(routed.max().item()),
+                           "routed_counts_mean": float(routed.float().mean().item()),
+                           "empty_experts": int((routed == 0).sum().item()), "kept": A_kept,
+                           "dropped": wl.T * wl.k - A_kept}
+        if not args.no_cpu_baseline and world == 1:
+            n = CPU_SAMPLE.get(wl.name, 256)
+            v, dt, threads = oracle_tokens_per_s(wl, n, args.seed)
+            line["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": threads, "kind": "oracle",
+                                    "sample": f"first {min(n, wl.T)} tokens of {wl.name} as their own batch, "
+                                              f"{dt:.1f} s"}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+def launches(cfg):
+    """Kernels one moe_layer_forward launches (router, count, scan, rank, copy,
+    expert stage, combine)."""
+    ffn = {0: 2, 1: 0, 2: 1}[cfg.expert_kind]
+    return 5 + ffn + 1
+
+
+def stage_times(M, cfg, wl, h, wr, bias, w13, wd, dev, stream, reps):
+    import torch
+
+    A = wl.T * wl.k
+    idx = torch.empty((wl.T, wl.k), dtype=torch.int32, device=dev)
+    gate = torch.empty((wl.T, wl.k), dtype=torch.float32, device=dev)
+    out = dict(routed_counts=torch.empty(wl.E, dtype=torch.int32, device=dev),
+               counts=torch.empty(wl.E, dtype=torch.int32, device=dev),
+               offsets=torch.empty(wl.E + 1, dtype=torch.int32, device=dev),
+               dest_row=torch.empty((wl.T, wl.k), dtype=torch.int32, device=dev),
+               perm_src=torch.empty(A, dtype=torch.int32, device=dev),
+               x_perm=torch.empty((A, wl.d), dtype=wl.torch_dtype, device=dev))
+    y_perm = torch.empty((A, wl.d), dtype=wl.torch_dtype, device=dev)
+    y = torch.empty((wl.T, wl.d), dtype=wl.torch_dtype, device=dev)
+    ws_p = M.workspace(cfg, M.MOE_OP_PERMUTE, dev)
+    ws_f = M.workspace(cfg, M.MOE_OP_GROUPED_FFN, dev)
+    calls = {
+        "route": lambda: M.moe_route(cfg, h, wr, bias, topk_idx=idx, topk_gate=gate, stream=stream),
+        "permute": lambda: M.moe_permute(cfg, h, idx, out=out, ws=ws_p, stream=stream),
+        "grouped_ffn": lambda: M.moe_grouped_ffn(cfg, out["x_perm"], out["offsets"], w13, wd, y_perm=y_perm,
+                                                 ws=ws_f, stream=stream),
+        "combine": lambda: M.moe_unpermute_combine(cfg, y_perm, out["dest_row"], gate, y=y, stream=stream),
+    }
+    res = {}
+    for name, fn in calls.items():
+        fn()
+        torch.cuda.synchronize()
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+        for a, b in evs:
+            a.record(stream)
+            fn()
+            b.record(stream)
+        torch.cuda.synchronize()
+        res[name] = statistics.median([a.elapsed_time(b) for a, b in evs])
+    return res
+
+
+def stage_report(st, wl, A_kept, pk, pk_kind):
+    s = wl.elem_bytes
+    T, d, E, k, F = wl.T, wl.d, wl.E, wl.k, wl.F
+    hbm = pk["hbm_gbs"]
+    tf = pk["bf16_tflops_sustained"]
+    router_b = T * d * s + E * d * s + T * k * 8
+    permute_b = T * d * s + A_kept * d * s
+    combine_b = A_kept * d * s + T * d * s + T * k * 8
+    flops = 6.0 * A_kept * d * F if wl.expert_kind == "swiglu" else 0.0
+    out = {
+        "route": {"us": 1e3 * st["route"], "GB/s": router_b / st["route"] / 1e6},
+        "permute": {"us": 1e3 * st["permute"], "GB/s": permute_b / st["permute"] / 1e6},
+        "grouped_ffn": {"us": 1e3 * st["grouped_ffn"]},
+        "combine": {"us": 1e3 * st["combine"], "GB/s": combine_b / st["combine"] / 1e6},
+    }
+    for key in ("route", "permute", "combine"):
+        out[key]["frac_hbm"] = out[key]["GB/s"] / hbm
+    if flops:
+        out["grouped_ffn"]["TFLOP/s"] = flops / st["grouped_ffn"] / 1e9
+        out["grouped_ffn"]["frac_bf16"] = out["grouped_ffn"]["TFLOP/s"] / tf
+    dc = (permute_b + combine_b) / ((st["permute"] + st["combine"]) / 1e3) / 1e9
+    out["dispatch_combine"] = {"GB/s": dc, "frac_hbm": dc / hbm}
+    out["peaks"] = {"hbm_gbs": hbm, "bf16_tflops_sustained": tf, "source": f"{pk_kind} (MEASURED_PEAKS.json)"
+                    if pk_kind == "measured" else "fallback"}
+    return out
+
+
+def roofline(st, wl, A_kept, pk, pk_kind):
+    if wl.expert_kind == "swiglu":
+        flops = 6.0 * A_kept * wl.d * wl.F
+        ach = flops / (st["grouped_ffn"] / 1e3) / 1e12
+        peak = pk["bf16_tflops_sustained"]
+        return {"bound": "tensor", "kernel": "grouped_gemm (SwiGLU GEMM1 + GEMM2, one call)", "achieved": ach,
+                "peak": peak, "unit": "TFLOP/s", "frac": ach / peak, "traffic": profiled_traffic(),
+                "peak_source": f"bf16_tflops_sustained, {pk_kind}"}
+    s = wl.elem_bytes
+    b = wl.T * wl.d * s + A_kept * wl.d * s
+    ach = b / (st["permute"] / 1e3) / 1e9
+    return {"bound": "hbm", "kernel": "permute", "achieved": ach, "peak": pk["hbm_gbs"], "unit": "GB/s",
+            "frac": ach / pk["hbm_gbs"], "traffic": None, "peak_source": f"hbm_gbs, {pk_kind}"}
+
+
+if __name__ == "__main__":
+    main()

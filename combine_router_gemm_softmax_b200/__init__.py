@@ -1,0 +1,20 @@
+"""B200 (sm_100a) token-choice Mixture-of-Experts layer forward.
+
+The computation lives in libmoe_b200.so (hand-written CUDA for sm_100a, C
+ABI in include/moe.h). This package only builds it and marshals torch
+tensors into its entry points:
+
+    moe_route              router scores, softmax, top-k, gates
+    moe_permute            per-expert counts/offsets, drops, dispatch permutation
+    moe_pack_weights       gate/up interleave for the grouped FFN
+    moe_grouped_ffn        grouped SwiGLU expert GEMMs over ragged groups
+    moe_unpermute_combine  return outputs to their tokens, gate-weighted
+    moe_layer_forward      all of the above on one stream
+"""
+from ._lib import (  # noqa: F401
+    EXPORTED, LIB_PATH, MOE_DTYPE_BF16, MOE_DTYPE_F32, MOE_ERR_CUDA, MOE_ERR_INVALID_ARG, MOE_ERR_NO_DEVICE,
+    MOE_ERR_UNSUPPORTED, MOE_ERR_WORKSPACE, MOE_EXPERT_IDENTITY, MOE_EXPERT_SCALE, MOE_EXPERT_SWIGLU, MOE_MAX_E,
+    MOE_MAX_K, MOE_OK, MOE_OP_GROUPED_FFN, MOE_OP_LAYER, MOE_OP_PERMUTE, MOE_OP_ROUTE, MOE_PACK_BLOCK,
+    MOE_STATUS_BAD_ROUTE, MOE_STATUS_NAN_LOGIT, MOE_STATUS_TIMEOUT, MoeConfig, MoeError, config, lib,
+    moe_grouped_ffn, moe_layer_forward, moe_pack_weights, moe_permute, moe_route, moe_unpermute_combine,
+    moe_workspace_size, workspace)

@@ -1,0 +1,250 @@
+"""ctypes binding of libmoe_b200.so (argument marshalling only).
+
+Every function here checks shapes, dtypes and devices of torch tensors, passes
+their device pointers and the current CUDA stream to the C ABI of the same
+name, and turns a non-zero return code into MoeError. All computation happens
+in the library's CUDA kernels; there is no other implementation to fall back
+to, so a missing library is an error.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmoe_b200.so")
+
+MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_WORKSPACE, MOE_ERR_CUDA, MOE_ERR_NO_DEVICE = range(6)
+MOE_STATUS_NAN_LOGIT, MOE_STATUS_BAD_ROUTE, MOE_STATUS_TIMEOUT = 1, 2, 4
+MOE_DTYPE_BF16, MOE_DTYPE_F32 = 0, 1
+MOE_EXPERT_SWIGLU, MOE_EXPERT_IDENTITY, MOE_EXPERT_SCALE = 0, 1, 2
+MOE_OP_ROUTE, MOE_OP_PERMUTE, MOE_OP_GROUPED_FFN, MOE_OP_LAYER = 0, 1, 2, 3
+MOE_MAX_E, MOE_MAX_K, MOE_PACK_BLOCK = 256, 8, 128
+
+EXPORTED = ("moe_workspace_size", "moe_status_string", "moe_version", "moe_pack_weights", "moe_route",
+            "moe_permute", "moe_grouped_ffn", "moe_unpermute_combine", "moe_layer_forward")
+
+
+class MoeError(RuntimeError):
+    def __init__(self, fn: str, code: int, text: str):
+        super().__init__(f"{fn} failed: {text} (code {code})")
+        self.code = code
+
+
+class MoeConfig(ctypes.Structure):
+    _fields_ = [("T", ctypes.c_int32), ("d", ctypes.c_int32), ("E", ctypes.c_int32), ("k", ctypes.c_int32),
+                ("d_ff", ctypes.c_int32), ("dtype", ctypes.c_int32), ("expert_kind", ctypes.c_int32),
+                ("capacity", ctypes.c_int32)]
+
+    def __repr__(self):
+        return "MoeConfig(" + ", ".join(f"{n}={getattr(self, n)}" for n, _ in self._fields_) + ")"
+
+    @property
+    def torch_dtype(self):
+        return torch.bfloat16 if self.dtype == MOE_DTYPE_BF16 else torch.float32
+
+
+_lib = None
+_lock = threading.Lock()
+
+P = ctypes.c_void_p
+I32 = ctypes.c_int32
+SZ = ctypes.c_size_t
+CFG = ctypes.POINTER(MoeConfig)
+
+_SIGS = {
+    "moe_workspace_size": (SZ, [CFG, I32]),
+    "moe_status_string": (ctypes.c_char_p, [I32]),
+    "moe_version": (I32, []),
+    "moe_pack_weights": (I32, [CFG, P, P, P, P]),
+    "moe_route": (I32, [CFG, P, P, P, P, P, P, P, SZ, P, P]),
+    "moe_permute": (I32, [CFG, P, P, P, P, P, P, P, P, P, SZ, P, P]),
+    "moe_grouped_ffn": (I32, [CFG, P, P, P, P, P, P, SZ, P, P]),
+    "moe_unpermute_combine": (I32, [CFG, P, P, P, P, P, P]),
+    "moe_layer_forward": (I32, [CFG, P, P, P, P, P, P, P, P, P, P, P, SZ, P, P]),
+}
+
+
+def lib() -> ctypes.CDLL:
+    """Load the CUDA library (raises if it has not been built)."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(LIB_PATH):
+                raise RuntimeError(f"{LIB_PATH} is missing; build it with "
+                                   "`python -m combine_router_gemm_softmax_b200.build`")
+            L = ctypes.CDLL(LIB_PATH)
+            for name, (res, args) in _SIGS.items():
+                f = getattr(L, name)
+                f.restype = res
+                f.argtypes = args
+            _lib = L
+    return _lib
+
+
+def config(T, d, E, k, d_ff, dtype="bf16", expert_kind="swiglu", capacity=-1) -> MoeConfig:
+    dt = {"bf16": MOE_DTYPE_BF16, "f32": MOE_DTYPE_F32, torch.bfloat16: MOE_DTYPE_BF16,
+          torch.float32: MOE_DTYPE_F32}[dtype]
+    kind = {"swiglu": MOE_EXPERT_SWIGLU, "identity": MOE_EXPERT_IDENTITY, "scale": MOE_EXPERT_SCALE}[expert_kind]
+    return MoeConfig(T, d, E, k, d_ff, dt, kind, capacity)
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if not isinstance(t, torch.Tensor):
+        raise TypeError("expected a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError("tensor must be on a CUDA device")
+    if not t.is_contiguous():
+        raise ValueError("tensor must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _check(t, shape, dtype, name):
+    if t is None:
+        return
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name}: shape {tuple(t.shape)} != {tuple(shape)}")
+    if t.dtype != dtype:
+        raise ValueError(f"{name}: dtype {t.dtype} != {dtype}")
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _rc(fn, code):
+    if code != MOE_OK:
+        raise MoeError(fn, code, lib().moe_status_string(code).decode())
+
+
+def _dev(ref):
+    return ref.device
+
+
+def moe_workspace_size(cfg: MoeConfig, op: int) -> int:
+    return int(lib().moe_workspace_size(ctypes.byref(cfg), op))
+
+
+def workspace(cfg: MoeConfig, op: int, device) -> torch.Tensor:
+    n = moe_workspace_size(cfg, op)
+    return torch.empty(max(n, 256), dtype=torch.uint8, device=device)
+
+
+def moe_pack_weights(cfg, w_gate, w_up, w13_packed=None, stream=None):
+    dt = cfg.torch_dtype
+    _check(w_gate, (cfg.E, cfg.d_ff, cfg.d), dt, "w_gate")
+    _check(w_up, (cfg.E, cfg.d_ff, cfg.d), dt, "w_up")
+    if w13_packed is None:
+        w13_packed = torch.empty((cfg.E, 2 * cfg.d_ff, cfg.d), dtype=dt, device=_dev(w_gate))
+    _check(w13_packed, (cfg.E, 2 * cfg.d_ff, cfg.d), dt, "w13_packed")
+    _rc("moe_pack_weights", lib().moe_pack_weights(ctypes.byref(cfg), _ptr(w_gate), _ptr(w_up), _ptr(w13_packed),
+                                                   _stream(stream)))
+    return w13_packed
+
+
+def moe_route(cfg, h, w_router, bias=None, logits_out=None, topk_idx=None, topk_gate=None, status=None,
+              stream=None):
+    dt = cfg.torch_dtype
+    dev = _dev(h)
+    _check(h, (cfg.T, cfg.d), dt, "h")
+    _check(w_router, (cfg.E, cfg.d), dt, "w_router")
+    _check(bias, (cfg.E,), torch.float32, "bias")
+    _check(logits_out, (cfg.T, cfg.E), torch.float32, "logits_out")
+    if topk_idx is None:
+        topk_idx = torch.empty((cfg.T, cfg.k), dtype=torch.int32, device=dev)
+    if topk_gate is None:
+        topk_gate = torch.empty((cfg.T, cfg.k), dtype=torch.float32, device=dev)
+    _check(topk_idx, (cfg.T, cfg.k), torch.int32, "topk_idx")
+    _check(topk_gate, (cfg.T, cfg.k), torch.float32, "topk_gate")
+    _rc("moe_route", lib().moe_route(ctypes.byref(cfg), _ptr(h), _ptr(w_router), _ptr(bias), _ptr(logits_out),
+                                     _ptr(topk_idx), _ptr(topk_gate), None, 0, _ptr(status), _stream(stream)))
+    return topk_idx, topk_gate
+
+
+def moe_permute(cfg, h, topk_idx, out=None, ws=None, status=None, stream=None):
+    """Returns dict routed_counts, counts, offsets, dest_row, perm_src, x_perm."""
+    dt = cfg.torch_dtype
+    dev = _dev(h)
+    A = cfg.T * cfg.k
+    _check(h, (cfg.T, cfg.d), dt, "h")
+    _check(topk_idx, (cfg.T, cfg.k), torch.int32, "topk_idx")
+    if out is None:
+        out = dict(routed_counts=torch.empty(cfg.E, dtype=torch.int32, device=dev),
+                   counts=torch.empty(cfg.E, dtype=torch.int32, device=dev),
+                   offsets=torch.empty(cfg.E + 1, dtype=torch.int32, device=dev),
+                   dest_row=torch.empty((cfg.T, cfg.k), dtype=torch.int32, device=dev),
+                   perm_src=torch.empty(max(A, 1), dtype=torch.int32, device=dev),
+                   x_perm=torch.empty((max(A, 1), cfg.d), dtype=dt, device=dev))
+    if ws is None:
+        ws = workspace(cfg, MOE_OP_PERMUTE, dev)
+    _rc("moe_permute", lib().moe_permute(
+        ctypes.byref(cfg), _ptr(h), _ptr(topk_idx), _ptr(out["routed_counts"]), _ptr(out["counts"]),
+        _ptr(out["offsets"]), _ptr(out["dest_row"]), _ptr(out["perm_src"]), _ptr(out["x_perm"]), _ptr(ws),
+        ws.numel(), _ptr(status), _stream(stream)))
+    return out
+
+
+def moe_grouped_ffn(cfg, x_perm, offsets, w13_packed=None, w_down=None, y_perm=None, ws=None, status=None,
+                    stream=None):
+    dt = cfg.torch_dtype
+    dev = _dev(x_perm)
+    rows = x_perm.shape[0]
+    if rows < max(cfg.T * cfg.k, 1):
+        raise ValueError("x_perm needs T*k rows")
+    _check(offsets, (cfg.E + 1,), torch.int32, "offsets")
+    if cfg.expert_kind == MOE_EXPERT_SWIGLU:
+        _check(w13_packed, (cfg.E, 2 * cfg.d_ff, cfg.d), dt, "w13_packed")
+        _check(w_down, (cfg.E, cfg.d, cfg.d_ff), dt, "w_down")
+    if y_perm is None:
+        y_perm = torch.empty((rows, cfg.d), dtype=dt, device=dev)
+    if ws is None:
+        ws = workspace(cfg, MOE_OP_GROUPED_FFN, dev)
+    _rc("moe_grouped_ffn", lib().moe_grouped_ffn(
+        ctypes.byref(cfg), _ptr(x_perm), _ptr(offsets), _ptr(w13_packed), _ptr(w_down), _ptr(y_perm), _ptr(ws),
+        ws.numel(), _ptr(status), _stream(stream)))
+    return y_perm
+
+
+def moe_unpermute_combine(cfg, y_perm, dest_row, topk_gate, y=None, status=None, stream=None):
+    dt = cfg.torch_dtype
+    _check(dest_row, (cfg.T, cfg.k), torch.int32, "dest_row")
+    _check(topk_gate, (cfg.T, cfg.k), torch.float32, "topk_gate")
+    if y is None:
+        y = torch.empty((cfg.T, cfg.d), dtype=dt, device=_dev(y_perm))
+    _check(y, (cfg.T, cfg.d), dt, "y")
+    _rc("moe_unpermute_combine", lib().moe_unpermute_combine(
+        ctypes.byref(cfg), _ptr(y_perm), _ptr(dest_row), _ptr(topk_gate), _ptr(y), _ptr(status), _stream(stream)))
+    return y
+
+
+def moe_layer_forward(cfg, h, w_router, bias=None, w13_packed=None, w_down=None, y=None, topk_idx=None,
+                      topk_gate=None, routed_counts=None, counts=None, ws=None, status=None, stream=None):
+    dt = cfg.torch_dtype
+    dev = _dev(h)
+    _check(h, (cfg.T, cfg.d), dt, "h")
+    _check(w_router, (cfg.E, cfg.d), dt, "w_router")
+    _check(bias, (cfg.E,), torch.float32, "bias")
+    if cfg.expert_kind == MOE_EXPERT_SWIGLU:
+        _check(w13_packed, (cfg.E, 2 * cfg.d_ff, cfg.d), dt, "w13_packed")
+        _check(w_down, (cfg.E, cfg.d, cfg.d_ff), dt, "w_down")
+    _check(topk_idx, (cfg.T, cfg.k), torch.int32, "topk_idx")
+    _check(topk_gate, (cfg.T, cfg.k), torch.float32, "topk_gate")
+    _check(routed_counts, (cfg.E,), torch.int32, "routed_counts")
+    _check(counts, (cfg.E,), torch.int32, "counts")
+    if y is None:
+        y = torch.empty((cfg.T, cfg.d), dtype=dt, device=dev)
+    _check(y, (cfg.T, cfg.d), dt, "y")
+    if ws is None:
+        ws = workspace(cfg, MOE_OP_LAYER, dev)
+    _rc("moe_layer_forward", lib().moe_layer_forward(
+        ctypes.byref(cfg), _ptr(h), _ptr(w_router), _ptr(bias), _ptr(w13_packed), _ptr(w_down), _ptr(y),
+        _ptr(topk_idx), _ptr(topk_gate), _ptr(routed_counts), _ptr(counts), _ptr(ws), ws.numel(), _ptr(status),
+        _stream(stream)))
+    return y

@@ -1,0 +1,348 @@
+// C ABI of the MoE layer: argument checks, workspace carving, TMA descriptor
+// encoding and stage launches. The stage order and the meaning of every
+// argument are documented in include/moe.h.
+#include <mutex>
+
+#include "moe_common.cuh"
+#include "moe_internal.h"
+
+namespace moe {
+
+int device_sm_count() {
+  static int cached[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) dev = 0;
+  if (dev >= 0 && dev < 64 && cached[dev] > 0) return cached[dev];
+  int n = 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 1;
+  if (dev >= 0 && dev < 64) cached[dev] = n;
+  return n;
+}
+
+namespace {
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// Row-major bf16 matrix [rows, cols], box of box_rows x 64 columns, 128-byte swizzle.
+int make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (enc == nullptr) return MOE_ERR_NO_DEVICE;
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {cols * 2};
+  const cuuint32_t box[2] = {64, box_rows};
+  const cuuint32_t es[2] = {1, 1};
+  const CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? MOE_OK : MOE_ERR_CUDA;
+}
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+int elem_bytes(const moe_config& c) { return c.dtype == MOE_DTYPE_BF16 ? 2 : 4; }
+
+int check_cfg(const moe_config* c) {
+  if (c == nullptr) return MOE_ERR_INVALID_ARG;
+  if (c->T < 0 || c->d <= 0 || c->E <= 0 || c->k <= 0 || c->capacity < -1) return MOE_ERR_INVALID_ARG;
+  if (c->dtype != MOE_DTYPE_BF16 && c->dtype != MOE_DTYPE_F32) return MOE_ERR_INVALID_ARG;
+  if (c->expert_kind < MOE_EXPERT_SWIGLU || c->expert_kind > MOE_EXPERT_SCALE) return MOE_ERR_INVALID_ARG;
+  if (c->expert_kind == MOE_EXPERT_SWIGLU && c->d_ff <= 0) return MOE_ERR_INVALID_ARG;
+  if (c->E > MOE_MAX_E || c->k > MOE_MAX_K || c->k > c->E) return MOE_ERR_UNSUPPORTED;
+  if (static_cast<long long>(c->T) * c->k >= (1LL << 31)) return MOE_ERR_UNSUPPORTED;
+  if (c->dtype == MOE_DTYPE_BF16) {
+    if (c->d % 128 != 0) return MOE_ERR_UNSUPPORTED;
+    if (c->expert_kind == MOE_EXPERT_SWIGLU && c->d_ff % 128 != 0) return MOE_ERR_UNSUPPORTED;
+  } else if (c->d % 4 != 0) {
+    return MOE_ERR_UNSUPPORTED;
+  }
+  return MOE_OK;
+}
+
+// Carves 256-byte aligned pieces off the workspace; with a null base it only
+// measures, so sizes and layout come from the same code.
+struct Carver {
+  uint8_t* base;
+  size_t off = 0;
+  explicit Carver(void* b) : base(static_cast<uint8_t*>(b)) {}
+  template <typename T>
+  T* take(size_t bytes) {
+    T* p = base ? reinterpret_cast<T*>(base + off) : nullptr;
+    off += (bytes + 255) & ~static_cast<size_t>(255);
+    return p;
+  }
+};
+
+struct PermuteScratch {
+  int32_t* chunk_counts;
+  int32_t* chunk_base;
+};
+
+PermuteScratch carve_permute(const moe_config& c, Carver& w) {
+  const size_t nc = (static_cast<size_t>(c.T) + kChunkTokens - 1) / kChunkTokens;
+  PermuteScratch p;
+  p.chunk_counts = w.take<int32_t>(nc * c.E * 4);
+  p.chunk_base = w.take<int32_t>(nc * c.E * 4);
+  return p;
+}
+
+void* carve_ffn(const moe_config& c, Carver& w) {
+  if (c.expert_kind != MOE_EXPERT_SWIGLU) return nullptr;
+  return w.take<void>(static_cast<size_t>(c.T) * c.k * c.d_ff * elem_bytes(c));
+}
+
+struct LayerBufs {
+  int32_t *idx, *routed, *kept, *offsets, *dest_row, *perm_src;
+  float* gate;
+  void *x_perm, *y_perm, *h_mid;
+  PermuteScratch perm;
+};
+
+LayerBufs carve_layer(const moe_config& c, Carver& w) {
+  const size_t A = static_cast<size_t>(c.T) * c.k;
+  const size_t row = static_cast<size_t>(c.d) * elem_bytes(c);
+  LayerBufs b;
+  b.idx = w.take<int32_t>(A * 4);
+  b.gate = w.take<float>(A * 4);
+  b.routed = w.take<int32_t>(c.E * 4);
+  b.kept = w.take<int32_t>(c.E * 4);
+  b.offsets = w.take<int32_t>((c.E + 1) * 4);
+  b.dest_row = w.take<int32_t>(A * 4);
+  b.perm_src = w.take<int32_t>(A * 4);
+  b.x_perm = w.take<void>(A * row);
+  b.y_perm = c.expert_kind == MOE_EXPERT_IDENTITY ? nullptr : w.take<void>(A * row);
+  b.perm = carve_permute(c, w);
+  b.h_mid = carve_ffn(c, w);
+  return b;
+}
+
+size_t ws_size(const moe_config& c, int op) {
+  Carver w(nullptr);
+  switch (op) {
+    case MOE_OP_ROUTE:
+      return 0;
+    case MOE_OP_PERMUTE:
+      carve_permute(c, w);
+      return w.off;
+    case MOE_OP_GROUPED_FFN:
+      carve_ffn(c, w);
+      return w.off;
+    case MOE_OP_LAYER:
+      carve_layer(c, w);
+      return w.off;
+    default:
+      return 0;
+  }
+}
+
+int cuda_rc(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+
+int route_impl(const moe_config& c, const void* h, const void* w_router, const float* bias, float* logits,
+               int32_t* idx, float* gate, int32_t* status, cudaStream_t s) {
+  if (c.T == 0) return MOE_OK;
+  if (c.dtype == MOE_DTYPE_F32)
+    return cuda_rc(launch_router_f32(static_cast<const float*>(h), static_cast<const float*>(w_router), c.T, c.d, c.E,
+                                     c.k, bias, logits, idx, gate, status, s));
+  const int npad = ((c.E + 15) / 16) * 16;
+  CUtensorMap tm_h, tm_w;
+  int rc = make_map(&tm_h, h, c.T, c.d, kTileM);
+  if (rc == MOE_OK) rc = make_map(&tm_w, w_router, c.E, c.d, npad);
+  if (rc != MOE_OK) return rc;
+  return cuda_rc(launch_router_tc(tm_h, tm_w, c.T, c.d, c.E, c.k, npad, bias, logits, idx, gate, status, s));
+}
+
+int permute_impl(const moe_config& c, const void* h, const int32_t* idx, int32_t* routed, int32_t* kept,
+                 int32_t* offsets, int32_t* dest_row, int32_t* perm_src, void* x_perm, const PermuteScratch& p,
+                 int32_t* status, cudaStream_t s) {
+  return cuda_rc(launch_permute(h, static_cast<size_t>(c.d) * elem_bytes(c), idx, c.T, c.k, c.E, c.capacity,
+                                p.chunk_counts, p.chunk_base, routed, kept, offsets, dest_row, perm_src, x_perm,
+                                status, s));
+}
+
+int ffn_impl(const moe_config& c, const void* x_perm, const int32_t* offsets, const void* w13, const void* w_down,
+             void* y_perm, void* h_mid, int32_t* status, cudaStream_t s) {
+  const int rows_max = c.T * c.k;
+  if (rows_max == 0) return MOE_OK;
+  if (c.expert_kind != MOE_EXPERT_SWIGLU)
+    return cuda_rc(launch_scale_rows(c.dtype, c.expert_kind, x_perm, offsets, y_perm, rows_max, c.d, c.E, s));
+  if (c.dtype == MOE_DTYPE_F32)
+    return cuda_rc(launch_ffn_f32(static_cast<const float*>(x_perm), offsets, static_cast<const float*>(w13),
+                                  static_cast<const float*>(w_down), static_cast<float*>(h_mid),
+                                  static_cast<float*>(y_perm), rows_max, c.d, c.d_ff, c.E, s));
+  const int F = c.d_ff, d = c.d, E = c.E;
+  CUtensorMap a1, b1, a2, b2;
+  int rc = make_map(&a1, x_perm, rows_max, d, kTileM);
+  if (rc == MOE_OK) rc = make_map(&b1, w13, static_cast<uint64_t>(E) * 2 * F, d, kGemmTileN);
+  if (rc == MOE_OK) rc = make_map(&a2, h_mid, rows_max, F, kTileM);
+  if (rc == MOE_OK) rc = make_map(&b2, w_down, static_cast<uint64_t>(E) * d, F, kGemmTileN);
+  if (rc != MOE_OK) return rc;
+  cudaError_t e = launch_grouped_gemm_tc(a1, b1, true, offsets, E, d, 2 * F, F / 128, F, F, h_mid, status, s);
+  if (e != cudaSuccess) return MOE_ERR_CUDA;
+  e = launch_grouped_gemm_tc(a2, b2, false, offsets, E, F, d, (d + kGemmTileN - 1) / kGemmTileN, d, d, y_perm,
+                             status, s);
+  return cuda_rc(e);
+}
+
+}  // namespace
+}  // namespace moe
+
+using namespace moe;
+
+extern "C" {
+
+int32_t moe_version(void) { return (1 << 16) | 0; }
+
+const char* moe_status_string(int32_t code) {
+  switch (code) {
+    case MOE_OK:
+      return "ok";
+    case MOE_ERR_INVALID_ARG:
+      return "invalid argument";
+    case MOE_ERR_UNSUPPORTED:
+      return "unsupported configuration or misaligned pointer";
+    case MOE_ERR_WORKSPACE:
+      return "workspace too small or misaligned";
+    case MOE_ERR_CUDA:
+      return "CUDA launch or runtime call failed";
+    case MOE_ERR_NO_DEVICE:
+      return "no usable sm_100 device or driver entry point";
+    default:
+      return "unknown status";
+  }
+}
+
+size_t moe_workspace_size(const moe_config* cfg, int32_t op) {
+  if (check_cfg(cfg) != MOE_OK) return 0;
+  return ws_size(*cfg, op);
+}
+
+int32_t moe_pack_weights(const moe_config* cfg, const void* w_gate, const void* w_up, void* w13_packed,
+                         moe_stream_t stream) {
+  int rc = check_cfg(cfg);
+  if (rc != MOE_OK) return rc;
+  if (cfg->expert_kind != MOE_EXPERT_SWIGLU) return MOE_ERR_INVALID_ARG;
+  if (!w_gate || !w_up || !w13_packed) return MOE_ERR_INVALID_ARG;
+  if (!aligned(w_gate, 16) || !aligned(w_up, 16) || !aligned(w13_packed, 16)) return MOE_ERR_UNSUPPORTED;
+  return cuda_rc(launch_pack_w13(w_gate, w_up, w13_packed, cfg->E, cfg->d_ff,
+                                 static_cast<size_t>(cfg->d) * elem_bytes(*cfg), static_cast<cudaStream_t>(stream)));
+}
+
+int32_t moe_route(const moe_config* cfg, const void* h, const void* w_router, const float* bias, float* logits_out,
+                  int32_t* topk_idx, float* topk_gate, void* workspace, size_t ws_bytes, int32_t* status_dev,
+                  moe_stream_t stream) {
+  (void)workspace;
+  (void)ws_bytes;
+  int rc = check_cfg(cfg);
+  if (rc != MOE_OK) return rc;
+  const bool tok = cfg->T > 0;  // token-sized arrays may be NULL when T == 0
+  if (!w_router || (tok && (!h || !topk_idx || !topk_gate))) return MOE_ERR_INVALID_ARG;
+  if (!aligned(h, 16) || !aligned(w_router, 16) || !aligned(topk_idx, 4) || !aligned(topk_gate, 4) ||
+      !aligned(bias, 4) || !aligned(logits_out, 4) || !aligned(status_dev, 4))
+    return MOE_ERR_UNSUPPORTED;
+  return route_impl(*cfg, h, w_router, bias, logits_out, topk_idx, topk_gate, status_dev,
+                    static_cast<cudaStream_t>(stream));
+}
+
+int32_t moe_permute(const moe_config* cfg, const void* h, const int32_t* topk_idx, int32_t* routed_counts,
+                    int32_t* counts, int32_t* offsets, int32_t* dest_row, int32_t* perm_src, void* x_perm,
+                    void* workspace, size_t ws_bytes, int32_t* status_dev, moe_stream_t stream) {
+  int rc = check_cfg(cfg);
+  if (rc != MOE_OK) return rc;
+  const bool tok = cfg->T > 0;  // token-sized arrays may be NULL when T == 0
+  if (!routed_counts || !counts || !offsets || (tok && (!h || !topk_idx || !dest_row || !perm_src || !x_perm)))
+    return MOE_ERR_INVALID_ARG;
+  if (!aligned(h, 16) || !aligned(x_perm, 16) || !aligned(topk_idx, 4) || !aligned(routed_counts, 4) ||
+      !aligned(counts, 4) || !aligned(offsets, 4) || !aligned(dest_row, 4) || !aligned(perm_src, 4) ||
+      !aligned(status_dev, 4))
+    return MOE_ERR_UNSUPPORTED;
+  const size_t need = ws_size(*cfg, MOE_OP_PERMUTE);
+  if (ws_bytes < need || (need > 0 && (!workspace || !aligned(workspace, 16)))) return MOE_ERR_WORKSPACE;
+  Carver w(workspace);
+  const PermuteScratch p = carve_permute(*cfg, w);
+  return permute_impl(*cfg, h, topk_idx, routed_counts, counts, offsets, dest_row, perm_src, x_perm, p, status_dev,
+                      static_cast<cudaStream_t>(stream));
+}
+
+int32_t moe_grouped_ffn(const moe_config* cfg, const void* x_perm, const int32_t* offsets, const void* w13_packed,
+                        const void* w_down, void* y_perm, void* workspace, size_t ws_bytes, int32_t* status_dev,
+                        moe_stream_t stream) {
+  int rc = check_cfg(cfg);
+  if (rc != MOE_OK) return rc;
+  const bool swiglu = cfg->expert_kind == MOE_EXPERT_SWIGLU;
+  const bool tok = cfg->T > 0;  // token-sized arrays may be NULL when T == 0
+  if (!offsets || (tok && (!x_perm || !y_perm)) || (swiglu && (!w13_packed || !w_down))) return MOE_ERR_INVALID_ARG;
+  if (!aligned(x_perm, 16) || !aligned(y_perm, 16) || !aligned(offsets, 4) || !aligned(status_dev, 4) ||
+      (swiglu && (!aligned(w13_packed, 16) || !aligned(w_down, 16))))
+    return MOE_ERR_UNSUPPORTED;
+  const size_t need = ws_size(*cfg, MOE_OP_GROUPED_FFN);
+  if (ws_bytes < need || (need > 0 && (!workspace || !aligned(workspace, 16)))) return MOE_ERR_WORKSPACE;
+  Carver w(workspace);
+  void* h_mid = carve_ffn(*cfg, w);
+  return ffn_impl(*cfg, x_perm, offsets, w13_packed, w_down, y_perm, h_mid, status_dev,
+                  static_cast<cudaStream_t>(stream));
+}
+
+int32_t moe_unpermute_combine(const moe_config* cfg, const void* y_perm, const int32_t* dest_row,
+                              const float* topk_gate, void* y, int32_t* status_dev, moe_stream_t stream) {
+  (void)status_dev;
+  int rc = check_cfg(cfg);
+  if (rc != MOE_OK) return rc;
+  if (cfg->T > 0 && (!y_perm || !dest_row || !topk_gate || !y)) return MOE_ERR_INVALID_ARG;
+  if (!aligned(y_perm, 16) || !aligned(y, 16) || !aligned(dest_row, 4) || !aligned(topk_gate, 4))
+    return MOE_ERR_UNSUPPORTED;
+  return cuda_rc(
+      launch_combine(cfg->dtype, y_perm, dest_row, topk_gate, y, cfg->T, cfg->k, cfg->d, static_cast<cudaStream_t>(stream)));
+}
+
+int32_t moe_layer_forward(const moe_config* cfg, const void* h, const void* w_router, const float* bias,
+                          const void* w13_packed, const void* w_down, void* y, int32_t* topk_idx, float* topk_gate,
+                          int32_t* routed_counts, int32_t* counts, void* workspace, size_t ws_bytes,
+                          int32_t* status_dev, moe_stream_t stream) {
+  int rc = check_cfg(cfg);
+  if (rc != MOE_OK) return rc;
+  const moe_config& c = *cfg;
+  const bool swiglu = c.expert_kind == MOE_EXPERT_SWIGLU;
+  if (!w_router || (c.T > 0 && (!h || !y)) || (swiglu && (!w13_packed || !w_down))) return MOE_ERR_INVALID_ARG;
+  if (!aligned(h, 16) || !aligned(w_router, 16) || !aligned(y, 16) || !aligned(bias, 4) || !aligned(topk_idx, 4) ||
+      !aligned(topk_gate, 4) || !aligned(routed_counts, 4) || !aligned(counts, 4) || !aligned(status_dev, 4) ||
+      (swiglu && (!aligned(w13_packed, 16) || !aligned(w_down, 16))))
+    return MOE_ERR_UNSUPPORTED;
+  const size_t need = ws_size(c, MOE_OP_LAYER);
+  if (ws_bytes < need || (need > 0 && (!workspace || !aligned(workspace, 16)))) return MOE_ERR_WORKSPACE;
+  Carver w(workspace);
+  LayerBufs b = carve_layer(c, w);
+  if (topk_idx) b.idx = topk_idx;
+  if (topk_gate) b.gate = topk_gate;
+  if (routed_counts) b.routed = routed_counts;
+  if (counts) b.kept = counts;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  rc = route_impl(c, h, w_router, bias, nullptr, b.idx, b.gate, status_dev, s);
+  if (rc != MOE_OK) return rc;
+  rc = permute_impl(c, h, b.idx, b.routed, b.kept, b.offsets, b.dest_row, b.perm_src, b.x_perm, b.perm, status_dev,
+                    s);
+  if (rc != MOE_OK) return rc;
+  const void* y_src = b.x_perm;
+  if (c.expert_kind != MOE_EXPERT_IDENTITY) {
+    rc = ffn_impl(c, b.x_perm, b.offsets, w13_packed, w_down, b.y_perm, b.h_mid, status_dev, s);
+    if (rc != MOE_OK) return rc;
+    y_src = b.y_perm;
+  }
+  return cuda_rc(launch_combine(c.dtype, y_src, b.dest_row, b.gate, y, c.T, c.k, c.d, s));
+}
+
+}  // extern "C"

@@ -1,0 +1,342 @@
+// Dispatch and return: per-expert counts and offsets from the routing map,
+// the stable permutation that groups token rows by expert (with the optional
+// capacity drop), and the weighted unpermute/combine.
+// ("MoE Token Dispatch: Why an All-Reduce Result Does Not Describe the
+// Exchange", "Follow one documented dispatch and return path"; capacity
+// resolved in token order as in "How Does Mixture-of-Experts Routing Affect
+// LLM Repeatability?"; archcrux "moe-unpermute-wrong-token" for the return.)
+//
+// Everything stays on the device: four kernels, no host synchronisation.
+//   count : per 128-token chunk, a histogram over experts (shared atomics;
+//           only the totals are used, so their order does not matter)
+//   scan  : one CTA; per expert an exclusive scan over chunks (the stable
+//           base rank of each chunk), then kept counts and offsets
+//   rank  : per chunk, every slot's rank among earlier tokens of the same
+//           expert, from per-warp bitmasks (popc), giving dest_row/perm_src
+//   copy  : one warp per token reads its row once (16-byte vectors) and writes
+//           it to each kept destination row
+// Nothing decides an order with atomics, so the permutation is deterministic.
+#include "moe_common.cuh"
+#include "moe_internal.h"
+
+namespace moe {
+
+namespace {
+
+// Raw expert indices of token t and a bitmask of its valid slots: in range
+// and not repeating an earlier slot of the same token.
+MOE_DEV uint32_t load_route(const int32_t* __restrict__ idx, int t, int k, int E, int (&ev)[kMaxK]) {
+  uint32_t valid = 0;
+#pragma unroll
+  for (int j = 0; j < kMaxK; ++j) {
+    ev[j] = -1;
+    if (j < k) {
+      const int v = idx[static_cast<size_t>(t) * k + j];
+      bool ok = v >= 0 && v < E;
+#pragma unroll
+      for (int jj = 0; jj < j; ++jj) ok = ok && (ev[jj] != v);
+      ev[j] = v;
+      if (ok) valid |= 1u << j;
+    }
+  }
+  return valid;
+}
+
+__global__ void __launch_bounds__(kChunkTokens) count_kernel(const int32_t* __restrict__ idx, int T, int k, int E,
+                                                             int n_chunks, int32_t* __restrict__ chunk_counts) {
+  __shared__ int hist[kMaxE];
+  for (int e = threadIdx.x; e < E; e += blockDim.x) hist[e] = 0;
+  __syncthreads();
+  const int t = blockIdx.x * kChunkTokens + threadIdx.x;
+  if (t < T) {
+    int ev[kMaxK];
+    const uint32_t valid = load_route(idx, t, k, E, ev);
+#pragma unroll
+    for (int j = 0; j < kMaxK; ++j)
+      if (valid & (1u << j)) atomicAdd(&hist[ev[j]], 1);
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x)
+    chunk_counts[static_cast<size_t>(e) * n_chunks + blockIdx.x] = hist[e];
+}
+
+constexpr int kScanPerLane = 8;
+
+__global__ void __launch_bounds__(1024) scan_kernel(const int32_t* __restrict__ chunk_counts,
+                                                    int32_t* __restrict__ chunk_base, int n_chunks, int E, int cap,
+                                                    int32_t* __restrict__ routed, int32_t* __restrict__ kept,
+                                                    int32_t* __restrict__ offsets) {
+  __shared__ int s_kept[kMaxE];
+  __shared__ int s_warp[8];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // one warp per expert column: exclusive scan over chunks
+  for (int e = warp; e < E; e += 32) {
+    const int32_t* col = chunk_counts + static_cast<size_t>(e) * n_chunks;
+    int32_t* base = chunk_base + static_cast<size_t>(e) * n_chunks;
+    int carry = 0;
+    for (int c0 = 0; c0 < n_chunks; c0 += 32 * kScanPerLane) {
+      int vals[kScanPerLane];
+      int sum = 0;
+#pragma unroll
+      for (int v = 0; v < kScanPerLane; ++v) {
+        const int c = c0 + lane * kScanPerLane + v;
+        vals[v] = c < n_chunks ? col[c] : 0;
+        sum += vals[v];
+      }
+      int inc = sum;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const int n = __shfl_up_sync(0xffffffffu, inc, off);
+        if (lane >= off) inc += n;
+      }
+      int run = carry + inc - sum;
+#pragma unroll
+      for (int v = 0; v < kScanPerLane; ++v) {
+        const int c = c0 + lane * kScanPerLane + v;
+        if (c < n_chunks) base[c] = run;
+        run += vals[v];
+      }
+      carry += __shfl_sync(0xffffffffu, inc, 31);
+    }
+    if (lane == 0) {
+      const int kk = cap < 0 ? carry : min(carry, cap);
+      routed[e] = carry;
+      kept[e] = kk;
+      s_kept[e] = kk;
+    }
+  }
+  __syncthreads();
+  // offsets = exclusive scan of kept counts over experts (threads 0..255)
+  if (threadIdx.x < kMaxE) {
+    const int e = threadIdx.x;
+    const int v = e < E ? s_kept[e] : 0;
+    int inc = v;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int n = __shfl_up_sync(0xffffffffu, inc, off);
+      if (lane >= off) inc += n;
+    }
+    if (lane == 31) s_warp[warp] = inc;
+    __syncwarp();
+    asm volatile("bar.sync 1, 256;" ::: "memory");
+    int before = 0;
+    for (int w = 0; w < warp; ++w) before += s_warp[w];
+    if (e < E) offsets[e] = before + inc - v;
+    if (e == E - 1) offsets[E] = before + inc;
+  }
+}
+
+__global__ void __launch_bounds__(kChunkTokens) rank_kernel(const int32_t* __restrict__ idx, int T, int k, int E,
+                                                            int cap, int n_chunks,
+                                                            const int32_t* __restrict__ chunk_base,
+                                                            const int32_t* __restrict__ offsets,
+                                                            int32_t* __restrict__ dest_row,
+                                                            int32_t* __restrict__ perm_src, int32_t* status) {
+  constexpr int kWarps = kChunkTokens / 32;
+  __shared__ uint32_t mask[kWarps][kMaxE];
+  __shared__ int wbase[kWarps][kMaxE];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int i = threadIdx.x; i < kWarps * kMaxE; i += blockDim.x) (&mask[0][0])[i] = 0u;
+  __syncthreads();
+  const int t = blockIdx.x * kChunkTokens + threadIdx.x;
+  int ev[kMaxK];
+  uint32_t valid = 0;
+  if (t < T) {
+    valid = load_route(idx, t, k, E, ev);
+#pragma unroll
+    for (int j = 0; j < kMaxK; ++j)
+      if (valid & (1u << j)) atomicOr(&mask[warp][ev[j]], 1u << lane);
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    int run = 0;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) {
+      wbase[w][e] = run;
+      run += __popc(mask[w][e]);
+    }
+  }
+  __syncthreads();
+  if (t < T) {
+    const uint32_t lt = lanemask_lt();
+#pragma unroll
+    for (int j = 0; j < kMaxK; ++j) {
+      if (j >= k) break;
+      int dest = -1;
+      if (valid & (1u << j)) {
+        const int e = ev[j];
+        const int r = chunk_base[static_cast<size_t>(e) * n_chunks + blockIdx.x] + wbase[warp][e] +
+                      __popc(mask[warp][e] & lt);
+        if (cap < 0 || r < cap) {
+          dest = offsets[e] + r;
+          perm_src[dest] = t;
+        }
+      }
+      dest_row[static_cast<size_t>(t) * k + j] = dest;
+    }
+    if (valid != ((1u << k) - 1u)) report_status(status, MOE_STATUS_BAD_ROUTE);
+  }
+}
+
+constexpr int kCopyUnroll = 8;
+
+// One warp per token: read the row once, write it to each kept destination.
+__global__ void __launch_bounds__(256) permute_copy_kernel(const uint4* __restrict__ h,
+                                                           const int32_t* __restrict__ dest_row,
+                                                           uint4* __restrict__ x_perm, int T, int k, int vpr) {
+  const int lane = threadIdx.x & 31;
+  const int nw = gridDim.x * (blockDim.x >> 5);
+  for (int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); t < T; t += nw) {
+    const int my_dest = lane < k ? dest_row[static_cast<size_t>(t) * k + lane] : -1;
+    const uint4* src = h + static_cast<size_t>(t) * vpr;
+    for (int v0 = 0; v0 < vpr; v0 += 32 * kCopyUnroll) {
+      uint4 buf[kCopyUnroll];
+#pragma unroll
+      for (int u = 0; u < kCopyUnroll; ++u) {
+        const int v = v0 + u * 32 + lane;
+        if (v < vpr) buf[u] = __ldg(src + v);
+      }
+#pragma unroll
+      for (int j = 0; j < kMaxK; ++j) {
+        if (j >= k) break;
+        const int dest = __shfl_sync(0xffffffffu, my_dest, j);
+        if (dest < 0) continue;
+        uint4* dst = x_perm + static_cast<size_t>(dest) * vpr;
+#pragma unroll
+        for (int u = 0; u < kCopyUnroll; ++u) {
+          const int v = v0 + u * 32 + lane;
+          if (v < vpr) dst[v] = buf[u];
+        }
+      }
+    }
+  }
+}
+
+// 16-byte vector <-> fp32 lanes for the two storage types.
+template <int DT>
+struct Vec;
+
+template <>
+struct Vec<MOE_DTYPE_BF16> {
+  static constexpr int N = 8;
+  MOE_DEV static void load(const uint4& q, float (&f)[8]) {
+    const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&q);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float2 x = __bfloat1622float2(p[i]);
+      f[2 * i] = x.x;
+      f[2 * i + 1] = x.y;
+    }
+  }
+  MOE_DEV static uint4 store(const float (&f)[8]) {
+    uint4 q;
+    q.x = pack_bf16x2(f[0], f[1]);
+    q.y = pack_bf16x2(f[2], f[3]);
+    q.z = pack_bf16x2(f[4], f[5]);
+    q.w = pack_bf16x2(f[6], f[7]);
+    return q;
+  }
+};
+
+template <>
+struct Vec<MOE_DTYPE_F32> {
+  static constexpr int N = 4;
+  MOE_DEV static void load(const uint4& q, float (&f)[4]) {
+    f[0] = __uint_as_float(q.x);
+    f[1] = __uint_as_float(q.y);
+    f[2] = __uint_as_float(q.z);
+    f[3] = __uint_as_float(q.w);
+  }
+  MOE_DEV static uint4 store(const float (&f)[4]) {
+    return make_uint4(__float_as_uint(f[0]), __float_as_uint(f[1]), __float_as_uint(f[2]), __float_as_uint(f[3]));
+  }
+};
+
+constexpr int kCombineUnroll = 2;
+
+// One warp per token: y[t] = sum_j gate[t,j] * y_perm[dest_row[t,j]] in fp32,
+// slots in order 0..k-1, dropped slots skipped.
+template <int DT>
+__global__ void __launch_bounds__(256) combine_kernel(const uint4* __restrict__ y_perm,
+                                                      const int32_t* __restrict__ dest_row,
+                                                      const float* __restrict__ gate, uint4* __restrict__ y, int T,
+                                                      int k, int vpr) {
+  using V = Vec<DT>;
+  const int lane = threadIdx.x & 31;
+  const int nw = gridDim.x * (blockDim.x >> 5);
+  for (int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); t < T; t += nw) {
+    const int my_dest = lane < k ? dest_row[static_cast<size_t>(t) * k + lane] : -1;
+    const float my_gate = lane < k ? gate[static_cast<size_t>(t) * k + lane] : 0.f;
+    for (int v0 = 0; v0 < vpr; v0 += 32 * kCombineUnroll) {
+      float acc[kCombineUnroll][V::N];
+#pragma unroll
+      for (int u = 0; u < kCombineUnroll; ++u)
+#pragma unroll
+        for (int i = 0; i < V::N; ++i) acc[u][i] = 0.f;
+#pragma unroll
+      for (int j = 0; j < kMaxK; ++j) {
+        if (j >= k) break;
+        const int dest = __shfl_sync(0xffffffffu, my_dest, j);
+        const float g = __shfl_sync(0xffffffffu, my_gate, j);
+        if (dest < 0) continue;
+        const uint4* src = y_perm + static_cast<size_t>(dest) * vpr;
+#pragma unroll
+        for (int u = 0; u < kCombineUnroll; ++u) {
+          const int v = v0 + u * 32 + lane;
+          if (v < vpr) {
+            float f[V::N];
+            V::load(__ldg(src + v), f);
+#pragma unroll
+            for (int i = 0; i < V::N; ++i) acc[u][i] = fmaf(g, f[i], acc[u][i]);
+          }
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < kCombineUnroll; ++u) {
+        const int v = v0 + u * 32 + lane;
+        if (v < vpr) y[static_cast<size_t>(t) * vpr + v] = V::store(acc[u]);
+      }
+    }
+  }
+}
+
+int warp_grid(int T) {
+  const int want = (T + 7) / 8;
+  const int cap = device_sm_count() * 8;
+  return want < cap ? (want > 0 ? want : 1) : cap;
+}
+
+}  // namespace
+
+cudaError_t launch_permute(const void* h, size_t row_bytes, const int32_t* idx, int T, int k, int E, int cap,
+                           int32_t* chunk_counts, int32_t* chunk_base, int32_t* routed, int32_t* kept,
+                           int32_t* offsets, int32_t* dest_row, int32_t* perm_src, void* x_perm,
+                           int32_t* status, cudaStream_t s) {
+  const int n_chunks = (T + kChunkTokens - 1) / kChunkTokens;
+  if (n_chunks > 0) count_kernel<<<n_chunks, kChunkTokens, 0, s>>>(idx, T, k, E, n_chunks, chunk_counts);
+  scan_kernel<<<1, 1024, 0, s>>>(chunk_counts, chunk_base, n_chunks, E, cap, routed, kept, offsets);
+  if (n_chunks > 0) {
+    rank_kernel<<<n_chunks, kChunkTokens, 0, s>>>(idx, T, k, E, cap, n_chunks, chunk_base, offsets, dest_row,
+                                                  perm_src, status);
+    const int vpr = static_cast<int>(row_bytes / 16);
+    permute_copy_kernel<<<warp_grid(T), 256, 0, s>>>(static_cast<const uint4*>(h), dest_row,
+                                                     static_cast<uint4*>(x_perm), T, k, vpr);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_combine(int dtype, const void* y_perm, const int32_t* dest_row, const float* gate, void* y,
+                           int T, int k, int d, cudaStream_t s) {
+  if (T == 0) return cudaSuccess;
+  const int elem = dtype == MOE_DTYPE_BF16 ? 2 : 4;
+  const int vpr = d * elem / 16;
+  if (dtype == MOE_DTYPE_BF16)
+    combine_kernel<MOE_DTYPE_BF16><<<warp_grid(T), 256, 0, s>>>(
+        static_cast<const uint4*>(y_perm), dest_row, gate, static_cast<uint4*>(y), T, k, vpr);
+  else
+    combine_kernel<MOE_DTYPE_F32><<<warp_grid(T), 256, 0, s>>>(static_cast<const uint4*>(y_perm), dest_row, gate,
+                                                               static_cast<uint4*>(y), T, k, vpr);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

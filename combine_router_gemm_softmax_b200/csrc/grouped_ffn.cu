@@ -1,0 +1,486 @@
+// Grouped expert FFN over variable-length groups ("Dropless MoE Is a Runtime
+// Problem as Much as a Model Design": one computation over a collection of
+// expert shapes instead of one GEMM per expert or padding to a capacity).
+//
+// bf16 path, two launches of one persistent tcgen05 kernel:
+//   GEMM1  [rows_e x d] x [2F x d]^T per expert, SwiGLU in the epilogue:
+//          h_mid = silu(x W_gate^T) * (x W_up^T), rounded to bf16
+//   GEMM2  [rows_e x F] x [d x F]^T per expert -> y_perm (bf16)
+// Tiles are 128 rows x 256 columns x 64-deep K slices. The tile list is built
+// on the device from the expert offsets (no host synchronisation): every CTA
+// reads offsets, counts ceil(rows_e / 128) row tiles per expert, and walks the
+// (row tile, column tile) grid in bands of 16 row tiles so that a wave of CTAs
+// shares A and B tiles in L2. grid = number of SMs; CTA c takes tiles c,
+// c + grid, ...
+//
+// Inside a CTA (192 threads): warp 0 issues TMA loads into a 4-stage ring of
+// shared-memory buffers, warp 1 allocates TMEM and one of its threads issues
+// tcgen05.mma into one of two 256-column fp32 accumulators, warps 2..5 drain
+// the other accumulator (tcgen05.ld, 32x32b: one thread per output row) and
+// store it, so the epilogue of tile i overlaps the main loop of tile i+1.
+// Rows past the end of an expert's group are computed on whatever the buffer
+// holds there and never stored.
+#include "moe_common.cuh"
+#include "moe_internal.h"
+
+namespace moe {
+
+namespace {
+
+constexpr int kBM = kTileM;       // 128
+constexpr int kBN = kGemmTileN;   // 256
+constexpr int kBK = 64;
+constexpr int kStages = 4;
+constexpr int kGroupM = 16;
+constexpr int kGemmThreads = 192;
+constexpr uint32_t kABytes = kBM * kBK * 2;
+constexpr uint32_t kBBytes = kBN * kBK * 2;
+constexpr uint32_t kStageBytes = kABytes + kBBytes;
+constexpr uint32_t kTmemCols = 2 * kBN;
+
+constexpr size_t gemm_smem_bytes() {
+  return 1024 + kStages * static_cast<size_t>(kStageBytes) + (2 * kStages + 5) * 8 + 16 + 2 * (kMaxE + 1) * 4;
+}
+
+struct GemmArgs {
+  const int32_t* offsets;
+  int E;
+  int K;             // reduction length, a multiple of 64
+  int n_per_expert;  // rows of B per expert (2F for GEMM1, d for GEMM2)
+  int n_tiles;       // column tiles per expert
+  int out_cols;      // columns of D
+  int ldd;           // row stride of D in elements
+  __nv_bfloat16* D;
+  int32_t* status;
+};
+
+// tile -> (expert, row tile within the expert, column tile)
+MOE_DEV void decode_tile(long long tile, int m_total, int n_tiles, const int* prefix, int E, int& e, int& m,
+                         int& n) {
+  const long long band_size = static_cast<long long>(kGroupM) * n_tiles;
+  const int band = static_cast<int>(tile / band_size);
+  const int within = static_cast<int>(tile - band * band_size);
+  const int m0 = band * kGroupM;
+  const int rows = min(kGroupM, m_total - m0);
+  n = within / rows;
+  const int gm = m0 + within % rows;
+  int lo = 0, hi = E;  // prefix[lo] <= gm < prefix[hi]
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (prefix[mid] <= gm)
+      lo = mid;
+    else
+      hi = mid;
+  }
+  e = lo;
+  m = gm - prefix[lo];
+}
+
+template <bool kSwiGLU>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    grouped_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
+                        const GemmArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align_1024(smem_raw);
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + kStages * kABytes;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kStages * kStageBytes);
+  uint64_t* empty = full + kStages;
+  uint64_t* tfull = empty + kStages;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* drain = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  int* consumed_slot = reinterpret_cast<int*>(tmem_slot + 2);
+  int* s_off = reinterpret_cast<int*>(tmem_slot + 4);  // [E+1]
+  int* prefix = s_off + (kMaxE + 1);                   // [E+1]
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int E = a.E;
+  const int nkb = a.K / kBK;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&tfull[i], 1);
+      mbar_init(&tempty[i], 4);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    *consumed_slot = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(&tm_a);
+    tma_prefetch_desc(&tm_b);
+  }
+  for (int e = threadIdx.x; e <= E; e += blockDim.x) s_off[e] = a.offsets[e];
+  __syncthreads();
+  if (warp == 0) {
+    // row tiles per expert, exclusive prefix over experts (8 experts per lane)
+    int loc[8];
+    int sum = 0;
+#pragma unroll
+    for (int v = 0; v < 8; ++v) {
+      const int e = lane * 8 + v;
+      loc[v] = e < E ? (s_off[e + 1] - s_off[e] + kBM - 1) / kBM : 0;
+      sum += loc[v];
+    }
+    int inc = sum;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int nb = __shfl_up_sync(0xffffffffu, inc, off);
+      if (lane >= off) inc += nb;
+    }
+    int run = inc - sum;
+#pragma unroll
+    for (int v = 0; v < 8; ++v) {
+      const int e = lane * 8 + v;
+      if (e < E) prefix[e] = run;
+      run += loc[v];
+    }
+    if (lane == 31) prefix[E] = inc;
+  } else if (warp == 1) {
+    tmem_alloc(tmem_slot, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const int m_total = prefix[E];
+  const long long total = static_cast<long long>(m_total) * a.n_tiles;
+
+  int issued = 0;
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---------------------------------------------------------------- TMA producer
+      int stage = 0;
+      uint32_t phase = 0;
+      bool stop = false;
+      for (long long tile = blockIdx.x; tile < total && !stop; tile += gridDim.x) {
+        int e, m, n;
+        decode_tile(tile, m_total, a.n_tiles, prefix, E, e, m, n);
+        const int a_row = s_off[e] + m * kBM;
+        const int b_row = e * a.n_per_expert + n * kBN;
+        for (int kb = 0; kb < nkb; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag)) {
+            *abort_flag = 1;
+            stop = true;
+            break;
+          }
+          mbar_expect_tx(&full[stage], kStageBytes);
+          tma_load_2d(sA + stage * kABytes, &tm_a, &full[stage], kb * kBK, a_row);
+          tma_load_2d(sB + stage * kBBytes, &tm_b, &full[stage], kb * kBK, b_row);
+          ++issued;
+          if (++stage == kStages) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ---------------------------------------------------------------- MMA issuer
+      const uint32_t idesc = idesc_bf16_f32(kBM, kBN);
+      int stage = 0;
+      uint32_t phase = 0;
+      int consumed = 0, local = 0;
+      bool stop = false;
+      for (long long tile = blockIdx.x; tile < total && !stop; tile += gridDim.x, ++local) {
+        const int acc = local & 1;
+        const uint32_t acc_phase = (local >> 1) & 1;
+        if (!mbar_wait(&tempty[acc], acc_phase ^ 1, abort_flag)) {
+          *abort_flag = 1;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem + acc * kBN;
+        for (int kb = 0; kb < nkb; ++kb) {
+          if (!mbar_wait(&full[stage], phase, abort_flag)) {
+            *abort_flag = 1;
+            stop = true;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sa = smem_addr(sA + stage * kABytes);
+          const uint32_t sb = smem_addr(sB + stage * kBBytes);
+#pragma unroll
+          for (int kk = 0; kk < kBK / 16; ++kk)
+            umma_bf16(d_tmem, sw128_kmajor_desc(sa + kk * 32), sw128_kmajor_desc(sb + kk * 32), idesc,
+                      (kb | kk) != 0);
+          umma_commit(&empty[stage]);
+          ++consumed;
+          if (++stage == kStages) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+        if (!stop) umma_commit(&tfull[acc]);
+      }
+      *consumed_slot = consumed;
+      umma_commit(drain);
+      mbar_wait(drain, 0, nullptr);
+    }
+  } else {
+    // ---------------------------------------------------------------- epilogue
+    const int q = warp & 3;  // TMEM lane quadrant this warp may read
+    const int row = q * 32 + lane;
+    int local = 0;
+    for (long long tile = blockIdx.x; tile < total; tile += gridDim.x, ++local) {
+      int e, m, n;
+      decode_tile(tile, m_total, a.n_tiles, prefix, E, e, m, n);
+      const int acc = local & 1;
+      const uint32_t acc_phase = (local >> 1) & 1;
+      if (!mbar_wait(&tfull[acc], acc_phase, abort_flag)) {
+        *abort_flag = 1;
+        break;
+      }
+      tc_fence_after();
+      const int rows_valid = min(kBM, s_off[e + 1] - s_off[e] - m * kBM);
+      const bool valid = row < rows_valid;
+      const size_t grow = static_cast<size_t>(s_off[e] + m * kBM + row);
+      const uint32_t tbase = tmem + acc * kBN + (static_cast<uint32_t>(q * 32) << 16);
+      if constexpr (kSwiGLU) {
+        // columns [0,128) of the tile are gate, [128,256) the matching up
+        __nv_bfloat16* out = a.D + grow * a.ldd + n * (kBN / 2);
+#pragma unroll 1
+        for (int c = 0; c < kBN / 2; c += 32) {
+          uint32_t g[32], u[32];
+          tmem_ld32(tbase + c, g);
+          tmem_ld32(tbase + kBN / 2 + c, u);
+          tmem_ld_wait();
+          if (valid) {
+            uint32_t p[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              const float h0 = silu_f(__uint_as_float(g[2 * i])) * __uint_as_float(u[2 * i]);
+              const float h1 = silu_f(__uint_as_float(g[2 * i + 1])) * __uint_as_float(u[2 * i + 1]);
+              p[i] = pack_bf16x2(h0, h1);
+            }
+            uint4* dst = reinterpret_cast<uint4*>(out + c);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) dst[i] = make_uint4(p[4 * i], p[4 * i + 1], p[4 * i + 2], p[4 * i + 3]);
+          }
+        }
+      } else {
+        __nv_bfloat16* out = a.D + grow * a.ldd + n * kBN;
+#pragma unroll 1
+        for (int c = 0; c < kBN; c += 32) {
+          if (n * kBN + c >= a.out_cols) break;
+          uint32_t v[32];
+          tmem_ld32(tbase + c, v);
+          tmem_ld_wait();
+          if (valid) {
+            uint32_t p[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) p[i] = pack_bf16x2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
+            uint4* dst = reinterpret_cast<uint4*>(out + c);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) dst[i] = make_uint4(p[4 * i], p[4 * i + 1], p[4 * i + 2], p[4 * i + 3]);
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tempty[acc]);
+    }
+  }
+  __syncwarp();
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (*abort_flag) {
+    if (threadIdx.x == 0) report_status(a.status, MOE_STATUS_TIMEOUT);
+    if (warp == 0 && lane == 0) {
+      // loads issued but never consumed must land before the CTA leaves
+      for (int i = *consumed_slot; i < issued; ++i) mbar_wait(&full[i % kStages], (i / kStages) & 1, nullptr);
+    }
+  }
+  __syncthreads();
+  if (warp == 1) tmem_dealloc(tmem, kTmemCols);
+}
+
+// ------------------------------------------------------------------ helpers for the other paths
+MOE_DEV int expert_of_row(const int32_t* __restrict__ off, int E, int r) {
+  int lo = 0, hi = E;  // off[lo] <= r < off[hi]
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (off[mid] <= r)
+      lo = mid;
+    else
+      hi = mid;
+  }
+  return lo;
+}
+
+// Packed row of gate row f (is_up = 0) or up row f (is_up = 1) inside one expert.
+MOE_DEV int packed_row(int f, int F, int is_up) {
+  const int b = f / MOE_PACK_BLOCK;
+  const int w = f - b * MOE_PACK_BLOCK;
+  const int pb = min(MOE_PACK_BLOCK, F - b * MOE_PACK_BLOCK);
+  return 2 * b * MOE_PACK_BLOCK + (is_up ? pb : 0) + w;
+}
+
+// fp32 path, first projection: h_mid[r,f] = silu(x_r . Wg_f) * (x_r . Wu_f)
+__global__ void ffn1_f32_kernel(const float* __restrict__ x, const int32_t* __restrict__ off,
+                                const float* __restrict__ w13, float* __restrict__ h_mid, int rows_max, int d,
+                                int F, int E) {
+  const int n = off[E];
+  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x;
+       i < static_cast<long long>(rows_max) * F; i += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const int r = static_cast<int>(i / F), f = static_cast<int>(i % F);
+    if (r >= n) continue;
+    const int e = expert_of_row(off, E, r);
+    const float* xr = x + static_cast<size_t>(r) * d;
+    const float* wg = w13 + (static_cast<size_t>(e) * 2 * F + packed_row(f, F, 0)) * d;
+    const float* wu = w13 + (static_cast<size_t>(e) * 2 * F + packed_row(f, F, 1)) * d;
+    float ag = 0.f, au = 0.f;
+    for (int c = 0; c < d; ++c) {
+      ag = fmaf(xr[c], wg[c], ag);
+      au = fmaf(xr[c], wu[c], au);
+    }
+    h_mid[static_cast<size_t>(r) * F + f] = silu_f(ag) * au;
+  }
+}
+
+// fp32 path, second projection: y[r,c] = h_mid_r . Wd_c
+__global__ void ffn2_f32_kernel(const float* __restrict__ h_mid, const int32_t* __restrict__ off,
+                                const float* __restrict__ wd, float* __restrict__ y, int rows_max, int d, int F,
+                                int E) {
+  const int n = off[E];
+  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x;
+       i < static_cast<long long>(rows_max) * d; i += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const int r = static_cast<int>(i / d), c = static_cast<int>(i % d);
+    if (r >= n) continue;
+    const int e = expert_of_row(off, E, r);
+    const float* hr = h_mid + static_cast<size_t>(r) * F;
+    const float* wc = wd + (static_cast<size_t>(e) * d + c) * F;
+    float acc = 0.f;
+    for (int f = 0; f < F; ++f) acc = fmaf(hr[f], wc[f], acc);
+    y[static_cast<size_t>(r) * d + c] = acc;
+  }
+}
+
+// Identity (bit copy) and scale-by-(e+1) test experts, one warp per row.
+template <int DT>
+__global__ void __launch_bounds__(256) scale_rows_kernel(const uint4* __restrict__ x, const int32_t* __restrict__ off,
+                                                         uint4* __restrict__ y, int rows_max, int vpr, int E,
+                                                         int scale) {
+  const int lane = threadIdx.x & 31;
+  const int n = min(off[E], rows_max);
+  const int nw = gridDim.x * (blockDim.x >> 5);
+  for (int r = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); r < n; r += nw) {
+    const float s = scale ? static_cast<float>(expert_of_row(off, E, r) + 1) : 1.f;
+    for (int v = lane; v < vpr; v += 32) {
+      uint4 q = __ldg(x + static_cast<size_t>(r) * vpr + v);
+      if (scale) {
+        if (DT == MOE_DTYPE_BF16) {
+          __nv_bfloat162* p = reinterpret_cast<__nv_bfloat162*>(&q);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const float2 f = __bfloat1622float2(p[i]);
+            p[i] = __floats2bfloat162_rn(f.x * s, f.y * s);
+          }
+        } else {
+          q.x = __float_as_uint(__uint_as_float(q.x) * s);
+          q.y = __float_as_uint(__uint_as_float(q.y) * s);
+          q.z = __float_as_uint(__uint_as_float(q.z) * s);
+          q.w = __float_as_uint(__uint_as_float(q.w) * s);
+        }
+      }
+      y[static_cast<size_t>(r) * vpr + v] = q;
+    }
+  }
+}
+
+// Packed gate/up layout, one warp per packed row.
+__global__ void __launch_bounds__(256) pack_w13_kernel(const uint4* __restrict__ wg, const uint4* __restrict__ wu,
+                                                       uint4* __restrict__ w13, int E, int F, int vpr) {
+  const int lane = threadIdx.x & 31;
+  const long long rows = static_cast<long long>(E) * 2 * F;
+  const long long nw = static_cast<long long>(gridDim.x) * (blockDim.x >> 5);
+  for (long long p = blockIdx.x * static_cast<long long>(blockDim.x >> 5) + (threadIdx.x >> 5); p < rows; p += nw) {
+    const int e = static_cast<int>(p / (2 * F));
+    const int w = static_cast<int>(p - static_cast<long long>(e) * 2 * F);
+    const int b = w / (2 * MOE_PACK_BLOCK);
+    const int in_blk = w - b * 2 * MOE_PACK_BLOCK;
+    const int pb = min(MOE_PACK_BLOCK, F - b * MOE_PACK_BLOCK);
+    const bool up = in_blk >= pb;
+    const int f = b * MOE_PACK_BLOCK + (up ? in_blk - pb : in_blk);
+    const uint4* src = (up ? wu : wg) + (static_cast<size_t>(e) * F + f) * vpr;
+    uint4* dst = w13 + static_cast<size_t>(p) * vpr;
+    for (int v = lane; v < vpr; v += 32) dst[v] = __ldg(src + v);
+  }
+}
+
+int blocks_for(long long work, int per_block) {
+  long long b = (work + per_block - 1) / per_block;
+  const long long cap = static_cast<long long>(device_sm_count()) * 16;
+  if (b > cap) b = cap;
+  return b < 1 ? 1 : static_cast<int>(b);
+}
+
+}  // namespace
+
+cudaError_t launch_grouped_gemm_tc(const CUtensorMap& tm_a, const CUtensorMap& tm_b, bool swiglu,
+                                   const int32_t* offsets, int E, int K, int n_per_expert, int n_tiles,
+                                   int out_cols, int ldd, void* D, int32_t* status, cudaStream_t s) {
+  GemmArgs a{offsets, E, K, n_per_expert, n_tiles, out_cols, ldd, static_cast<__nv_bfloat16*>(D), status};
+  const size_t smem = gemm_smem_bytes();
+  const int grid = device_sm_count();
+  cudaError_t err;
+  if (swiglu) {
+    err = cudaFuncSetAttribute(grouped_gemm_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(smem));
+    if (err != cudaSuccess) return err;
+    grouped_gemm_kernel<true><<<grid, kGemmThreads, smem, s>>>(tm_a, tm_b, a);
+  } else {
+    err = cudaFuncSetAttribute(grouped_gemm_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(smem));
+    if (err != cudaSuccess) return err;
+    grouped_gemm_kernel<false><<<grid, kGemmThreads, smem, s>>>(tm_a, tm_b, a);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_ffn_f32(const float* x_perm, const int32_t* offsets, const float* w13, const float* wd,
+                           float* h_mid, float* y_perm, int rows_max, int d, int F, int E, cudaStream_t s) {
+  if (rows_max == 0) return cudaSuccess;
+  ffn1_f32_kernel<<<blocks_for(static_cast<long long>(rows_max) * F, 256), 256, 0, s>>>(x_perm, offsets, w13, h_mid,
+                                                                                        rows_max, d, F, E);
+  ffn2_f32_kernel<<<blocks_for(static_cast<long long>(rows_max) * d, 256), 256, 0, s>>>(h_mid, offsets, wd, y_perm,
+                                                                                        rows_max, d, F, E);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_scale_rows(int dtype, int kind, const void* x_perm, const int32_t* offsets, void* y_perm,
+                              int rows_max, int d, int E, cudaStream_t s) {
+  if (rows_max == 0) return cudaSuccess;
+  const int elem = dtype == MOE_DTYPE_BF16 ? 2 : 4;
+  const int vpr = d * elem / 16;
+  const int scale = kind == MOE_EXPERT_SCALE;
+  const int grid = blocks_for(rows_max, 8);
+  if (dtype == MOE_DTYPE_BF16)
+    scale_rows_kernel<MOE_DTYPE_BF16><<<grid, 256, 0, s>>>(static_cast<const uint4*>(x_perm), offsets,
+                                                           static_cast<uint4*>(y_perm), rows_max, vpr, E, scale);
+  else
+    scale_rows_kernel<MOE_DTYPE_F32><<<grid, 256, 0, s>>>(static_cast<const uint4*>(x_perm), offsets,
+                                                          static_cast<uint4*>(y_perm), rows_max, vpr, E, scale);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_pack_w13(const void* w_gate, const void* w_up, void* w13, int E, int F, size_t row_bytes,
+                            cudaStream_t s) {
+  const long long rows = static_cast<long long>(E) * 2 * F;
+  if (rows == 0) return cudaSuccess;
+  pack_w13_kernel<<<blocks_for(rows, 8), 256, 0, s>>>(static_cast<const uint4*>(w_gate),
+                                                      static_cast<const uint4*>(w_up), static_cast<uint4*>(w13), E, F,
+                                                      static_cast<int>(row_bytes / 16));
+  return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -1,0 +1,47 @@
+// Internal launch interface between the C ABI layer and the kernels.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/moe.h"
+
+namespace moe {
+
+// Tokens per dispatch chunk (one CTA of the count and rank kernels).
+constexpr int kChunkTokens = 128;
+// Rows per tile of the tensor-core kernels.
+constexpr int kTileM = 128;
+// Columns per output tile of the grouped expert GEMM.
+constexpr int kGemmTileN = 256;
+
+int device_sm_count();
+
+// router.cu
+cudaError_t launch_router_tc(const CUtensorMap& tm_h, const CUtensorMap& tm_w, int T, int d, int E, int k,
+                             int npad, const float* bias, float* logits, int32_t* idx, float* gate,
+                             int32_t* status, cudaStream_t s);
+cudaError_t launch_router_f32(const float* h, const float* w, int T, int d, int E, int k, const float* bias,
+                              float* logits, int32_t* idx, float* gate, int32_t* status, cudaStream_t s);
+
+// dispatch.cu
+cudaError_t launch_permute(const void* h, size_t row_bytes, const int32_t* idx, int T, int k, int E, int cap,
+                           int32_t* chunk_counts, int32_t* chunk_base, int32_t* routed, int32_t* kept,
+                           int32_t* offsets, int32_t* dest_row, int32_t* perm_src, void* x_perm,
+                           int32_t* status, cudaStream_t s);
+cudaError_t launch_combine(int dtype, const void* y_perm, const int32_t* dest_row, const float* gate, void* y,
+                           int T, int k, int d, cudaStream_t s);
+
+// grouped_ffn.cu
+cudaError_t launch_grouped_gemm_tc(const CUtensorMap& tm_a, const CUtensorMap& tm_b, bool swiglu,
+                                   const int32_t* offsets, int E, int K, int n_per_expert, int n_tiles,
+                                   int out_cols, int ldd, void* D, int32_t* status, cudaStream_t s);
+cudaError_t launch_ffn_f32(const float* x_perm, const int32_t* offsets, const float* w13, const float* wd,
+                           float* h_mid, float* y_perm, int rows_max, int d, int F, int E, cudaStream_t s);
+cudaError_t launch_scale_rows(int dtype, int kind, const void* x_perm, const int32_t* offsets, void* y_perm,
+                              int rows_max, int d, int E, cudaStream_t s);
+cudaError_t launch_pack_w13(const void* w_gate, const void* w_up, void* w13, int E, int F, size_t row_bytes,
+                            cudaStream_t s);
+
+}  // namespace moe

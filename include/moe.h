@@ -1,0 +1,194 @@
+/*
+ * moe.h -- C ABI of the B200 (sm_100a) token-choice Mixture-of-Experts layer.
+ *
+ * One forward pass of the layer is
+ *
+ *     s_t = h_t W_r^T (+ b)                 router scores
+ *     E_t = TopK(s_t, k)                     expert choice
+ *     g_t = softmax(s_t) renormalised over E_t
+ *     y_t = sum_{e in E_t} g_{t,e} f_e(h_t)  combine
+ *
+ * ("How Does Mixture-of-Experts Routing Affect LLM Repeatability?", the
+ * simplified token-choice layer), carried out as the stages of "MoE Token
+ * Dispatch: Why an All-Reduce Result Does Not Describe the Exchange", section
+ * "Follow one documented dispatch and return path": per-expert counts from the
+ * routing map, a permutation that groups token rows by expert, the experts,
+ * and the return of every output to its original token position. On one GPU
+ * the dispatch and the return are on-device permutations.
+ *
+ * Conventions for every entry point:
+ *  - Tensor arguments are DEVICE pointers owned by the caller. The library
+ *    never allocates, frees or keeps device memory; scratch comes from the
+ *    caller's `workspace` (size from moe_workspace_size). Pointers must be
+ *    16-byte aligned.
+ *  - Row-major throughout. Weights are "out x in" (the reduction index is the
+ *    contiguous one), i.e. W_r [E, d], W_gate/W_up [E, F, d], W_down [E, d, F].
+ *  - `dtype` (MOE_DTYPE_*) is the storage type of h, the expert weights, the
+ *    permuted rows and y. The router weight has the same type; the router bias
+ *    is always fp32. Logits and gates are fp32, indices int32. Arithmetic
+ *    accumulates in fp32 on both paths.
+ *  - Every call only enqueues work on `stream` (a cudaStream_t; NULL is the
+ *    legacy default stream) and never synchronises. Counts and offsets stay on
+ *    the device.
+ *  - Return value: MOE_OK or a host-side error (MOE_ERR_*), detected before
+ *    anything is enqueued, except MOE_ERR_CUDA, which reports a failed launch.
+ *  - Data errors found on the device never trap: they are OR-ed into
+ *    *status_dev (MOE_STATUS_* bits) when status_dev is not NULL. The caller
+ *    zeroes it and reads it when convenient.
+ *
+ * Limits: 1 <= E <= 256, 1 <= k <= min(E, 8), T >= 0, T*k < 2^31.
+ * bf16 path: d and F multiples of 128. fp32 path: d a multiple of 4.
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* host-side return codes */
+#define MOE_OK              0
+#define MOE_ERR_INVALID_ARG 1  /* NULL where a pointer is required, bad sizes */
+#define MOE_ERR_UNSUPPORTED 2  /* outside the limits above, misaligned pointer */
+#define MOE_ERR_WORKSPACE   3  /* workspace too small or misaligned */
+#define MOE_ERR_CUDA        4  /* a kernel launch or CUDA runtime call failed */
+#define MOE_ERR_NO_DEVICE   5  /* no usable sm_100 device / driver entry point */
+
+/* asynchronous status bits, OR-ed into *status_dev */
+#define MOE_STATUS_NAN_LOGIT 1  /* a router logit was NaN (treated as -inf) */
+#define MOE_STATUS_BAD_ROUTE 2  /* an index out of [0,E) or repeated within a token (slot dropped) */
+#define MOE_STATUS_TIMEOUT   4  /* a bounded on-chip wait gave up (output invalid) */
+
+#define MOE_DTYPE_BF16 0
+#define MOE_DTYPE_F32  1
+
+#define MOE_EXPERT_SWIGLU   0  /* f_e(x) = W_down,e (silu(W_gate,e x) * (W_up,e x)) */
+#define MOE_EXPERT_IDENTITY 1  /* f_e(x) = x       (test expert) */
+#define MOE_EXPERT_SCALE    2  /* f_e(x) = (e+1) x (test expert) */
+
+#define MOE_OP_ROUTE       0
+#define MOE_OP_PERMUTE     1
+#define MOE_OP_GROUPED_FFN 2
+#define MOE_OP_LAYER       3
+
+#define MOE_MAX_E 256
+#define MOE_MAX_K 8
+#define MOE_PACK_BLOCK 128
+
+typedef struct moe_config {
+  int32_t T;            /* tokens */
+  int32_t d;            /* hidden size */
+  int32_t E;            /* experts */
+  int32_t k;            /* experts per token */
+  int32_t d_ff;         /* expert FFN width F */
+  int32_t dtype;        /* MOE_DTYPE_* */
+  int32_t expert_kind;  /* MOE_EXPERT_* */
+  int32_t capacity;     /* -1: dropless; >= 0: per-expert cap in assignments */
+} moe_config;
+
+typedef void* moe_stream_t; /* cudaStream_t */
+
+/* Bytes of workspace the given operation needs (MOE_OP_*). 0 on invalid cfg. */
+MOE_API size_t moe_workspace_size(const moe_config* cfg, int32_t op);
+
+/* Text for a MOE_OK / MOE_ERR_* code. Never NULL. */
+MOE_API const char* moe_status_string(int32_t code);
+
+/* ABI version, (major << 16) | minor. */
+MOE_API int32_t moe_version(void);
+
+/* moe_pack_weights -- lay out the gate and up projections for the grouped FFN.
+ * w_gate, w_up: [E, F, d]. w13_packed: [E, 2F, d], written. For each expert,
+ * rows are interleaved in blocks of MOE_PACK_BLOCK (128) rows: block b holds
+ * gate rows [128b, 128b+n) followed by up rows [128b, 128b+n), n = min(128,
+ * F-128b). This lets one output tile of the first expert GEMM see matching
+ * gate and up columns, so the SwiGLU product is formed in its epilogue.
+ * W_down is used as given, [E, d, F]. Runs once per set of weights. */
+MOE_API int32_t moe_pack_weights(const moe_config* cfg, const void* w_gate, const void* w_up,
+                         void* w13_packed, moe_stream_t stream);
+
+/* moe_route -- router scores, softmax and top-k.
+ * ("How Does Mixture-of-Experts Routing Affect LLM Repeatability?": s_t =
+ * h_t W_r, E_t = TopK(s_t, k), gate g_{t,e}; deterministic tie handling.)
+ * h [T, d], w_router [E, d] (dtype), bias [E] fp32 or NULL.
+ * logits_out [T, E] fp32 or NULL: s_t with the bias added.
+ * topk_idx [T, k] int32: slot j holds the expert with the (j+1)-th highest
+ *   score; equal scores go to the lower expert index; NaN counts as -inf.
+ * topk_gate [T, k] fp32: softmax over all E experts renormalised over the k
+ *   picks (= softmax over the k picked scores). A token whose scores are all
+ *   -inf gets experts 0..k-1 with gate 0.
+ * Scores are accumulated in fp32 (bf16 products on tensor cores for bf16). */
+MOE_API int32_t moe_route(const moe_config* cfg, const void* h, const void* w_router, const float* bias,
+                  float* logits_out, int32_t* topk_idx, float* topk_gate,
+                  void* workspace, size_t ws_bytes, int32_t* status_dev, moe_stream_t stream);
+
+/* moe_permute -- per-expert counts, offsets, drop decisions and the dispatch
+ * permutation ("MoE Token Dispatch ...", "Follow one documented dispatch and
+ * return path"; capacity resolved in token order as in "How Does
+ * Mixture-of-Experts Routing Affect LLM Repeatability?").
+ * topk_idx [T, k] int32 may come from moe_route or be supplied by the caller
+ * (route replay). Slots with an index outside [0,E) or repeating an earlier
+ * slot's expert are dropped and flag MOE_STATUS_BAD_ROUTE.
+ * rank(t,j) = number of tokens t' < t that picked the same expert. The slot is
+ * kept iff capacity < 0 or rank < capacity.
+ * Outputs (all written):
+ *   routed_counts [E]  assignments per expert before drops
+ *   counts [E]         kept assignments per expert
+ *   offsets [E+1]      exclusive prefix sum of counts; offsets[E] = kept total
+ *   dest_row [T, k]    row of x_perm holding slot (t,j), -1 if dropped
+ *   perm_src [T*k]     token of each x_perm row (first offsets[E] entries valid)
+ *   x_perm [T*k, d]    x_perm[dest_row[t,j]] = h[t], bitwise; rows of expert e
+ *                      are [offsets[e], offsets[e+1]) in ascending token order;
+ *                      rows past offsets[E] are left untouched. */
+MOE_API int32_t moe_permute(const moe_config* cfg, const void* h, const int32_t* topk_idx,
+                    int32_t* routed_counts, int32_t* counts, int32_t* offsets,
+                    int32_t* dest_row, int32_t* perm_src, void* x_perm,
+                    void* workspace, size_t ws_bytes, int32_t* status_dev, moe_stream_t stream);
+
+/* moe_grouped_ffn -- all experts over their variable-length row groups in one
+ * grouped computation ("Dropless MoE Is a Runtime Problem as Much as a Model
+ * Design": one implementation over a collection of expert shapes, no padding).
+ * x_perm [T*k, d] and offsets [E+1] as written by moe_permute; the group sizes
+ * are read on the device (no host synchronisation).
+ * w13_packed [E, 2F, d] from moe_pack_weights, w_down [E, d, F] (SwiGLU only;
+ * may be NULL for the identity and scale experts).
+ * y_perm [T*k, d]: y_perm[r] = f_e(x_perm[r]) for r in [offsets[e], offsets[e+1]).
+ * bf16 path: silu(gate) * up is rounded to bf16 before the down projection. */
+MOE_API int32_t moe_grouped_ffn(const moe_config* cfg, const void* x_perm, const int32_t* offsets,
+                        const void* w13_packed, const void* w_down, void* y_perm,
+                        void* workspace, size_t ws_bytes, int32_t* status_dev, moe_stream_t stream);
+
+/* moe_unpermute_combine -- return every expert output to its token and
+ * weight it (archcrux "moe-unpermute-wrong-token": outputs restored to their
+ * original positions; top-k weights tied to the same token).
+ * y[t] = sum_{j=0..k-1, dest_row[t,j] >= 0} topk_gate[t,j] * y_perm[dest_row[t,j]],
+ * accumulated in fp32 in slot order, stored in dtype. Dropped slots add
+ * nothing and the kept gates are not renormalised. */
+MOE_API int32_t moe_unpermute_combine(const moe_config* cfg, const void* y_perm, const int32_t* dest_row,
+                              const float* topk_gate, void* y, int32_t* status_dev,
+                              moe_stream_t stream);
+
+/* moe_layer_forward -- the whole layer on one stream: route, permute, grouped
+ * FFN, unpermute/combine. Intermediates live in the workspace
+ * (moe_workspace_size(cfg, MOE_OP_LAYER)). Optional outputs (NULL to skip):
+ * topk_idx [T,k], topk_gate [T,k], routed_counts [E], counts [E]. */
+MOE_API int32_t moe_layer_forward(const moe_config* cfg, const void* h, const void* w_router,
+                          const float* bias, const void* w13_packed, const void* w_down, void* y,
+                          int32_t* topk_idx, float* topk_gate, int32_t* routed_counts,
+                          int32_t* counts, void* workspace, size_t ws_bytes,
+                          int32_t* status_dev, moe_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_B200_H */

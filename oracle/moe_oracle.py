@@ -131,6 +131,8 @@ def min_adjacent_gap(s, k):
     both the picked set and the slot order are away from a boundary)."""
     srt = -np.sort(-np.asarray(s, F64), axis=1)
     top = srt[:, :min(k + 1, srt.shape[1])]
+    if top.shape[1] < 2:
+        return np.full(top.shape[0], np.inf)
     with np.errstate(invalid="ignore"):
         gaps = top[:, :-1] - top[:, 1:]
     gaps = np.where(np.isnan(gaps), np.inf, gaps)   # -inf - -inf: both out of reach

@@ -1,0 +1,111 @@
+"""The C ABI library loads and exports what include/moe.h declares (CPU only).
+
+No compute call is made here: the argument checks below all fail before the
+library touches CUDA.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+import combine_router_gemm_softmax_b200 as M
+from combine_router_gemm_softmax_b200 import _lib
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "moe.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    from combine_router_gemm_softmax_b200 import build
+    build.build()
+    return M.lib()
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(moe_[a-z_]+)\s*\(", src)))
+
+
+def test_header_declares_the_entry_points():
+    names = declared_functions()
+    for n in ("moe_route", "moe_permute", "moe_grouped_ffn", "moe_unpermute_combine", "moe_layer_forward",
+              "moe_workspace_size", "moe_pack_weights"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(L):
+    for n in declared_functions():
+        assert hasattr(L, n), n
+    assert set(declared_functions()) <= set(_lib.EXPORTED)
+
+
+def test_header_constants_match_binding():
+    src = open(HEADER).read()
+    consts = dict(re.findall(r"#define\s+(MOE_[A-Z0-9_]+)\s+(-?\d+)", src))
+    for name, val in consts.items():
+        assert getattr(_lib, name) == int(val), name
+
+
+def test_version_and_status_strings(L):
+    assert L.moe_version() >> 16 == 1
+    assert L.moe_status_string(0) == b"ok"
+    assert b"workspace" in L.moe_status_string(3)
+    assert L.moe_status_string(99) == b"unknown status"
+
+
+def test_workspace_sizes(L):
+    cfg = M.config(4096, 1024, 8, 2, 3584)
+    assert M.moe_workspace_size(cfg, M.MOE_OP_ROUTE) == 0
+    nc = 4096 // 128
+    assert M.moe_workspace_size(cfg, M.MOE_OP_PERMUTE) == 2 * ((nc * 8 * 4 + 255) // 256 * 256)
+    assert M.moe_workspace_size(cfg, M.MOE_OP_GROUPED_FFN) == 4096 * 2 * 3584 * 2
+    layer = M.moe_workspace_size(cfg, M.MOE_OP_LAYER)
+    assert layer > 2 * 4096 * 2 * 1024 * 2 + 4096 * 2 * 3584 * 2
+    ident = M.config(4096, 1024, 8, 2, 3584, expert_kind="identity")
+    assert M.moe_workspace_size(ident, M.MOE_OP_GROUPED_FFN) == 0
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(E=300), M.MOE_ERR_UNSUPPORTED),
+    (dict(k=9, E=16), M.MOE_ERR_UNSUPPORTED),
+    (dict(k=5, E=4), M.MOE_ERR_UNSUPPORTED),
+    (dict(d=96), M.MOE_ERR_UNSUPPORTED),
+    (dict(d_ff=200), M.MOE_ERR_UNSUPPORTED),
+    (dict(T=-1), M.MOE_ERR_INVALID_ARG),
+    (dict(capacity=-2), M.MOE_ERR_INVALID_ARG),
+])
+def test_config_rejected_before_any_cuda_call(L, kw, code):
+    base = dict(T=64, d=128, E=8, k=2, d_ff=256)
+    base.update(kw)
+    cfg = M.config(**base)
+    assert M.moe_workspace_size(cfg, M.MOE_OP_LAYER) == 0
+    rc = L.moe_route(ctypes.byref(cfg), None, None, None, None, None, None, None, 0, None, None)
+    assert rc == code
+
+
+def test_null_pointers_rejected(L):
+    cfg = M.config(64, 128, 8, 2, 256)
+    assert L.moe_route(ctypes.byref(cfg), None, None, None, None, None, None, None, 0, None, None) \
+        == M.MOE_ERR_INVALID_ARG
+    assert L.moe_unpermute_combine(ctypes.byref(cfg), None, None, None, None, None, None) == M.MOE_ERR_INVALID_ARG
+    assert L.moe_layer_forward(ctypes.byref(cfg), None, None, None, None, None, None, None, None, None, None, None,
+                               0, None, None) == M.MOE_ERR_INVALID_ARG
+    assert L.moe_pack_weights(None, None, None, None, None) == M.MOE_ERR_INVALID_ARG
+
+
+def test_misaligned_pointer_rejected(L):
+    cfg = M.config(64, 128, 8, 2, 256)
+    p = ctypes.c_void_p(0x1000)
+    odd = ctypes.c_void_p(0x1008)
+    rc = L.moe_route(ctypes.byref(cfg), odd, p, None, None, p, p, None, 0, None, None)
+    assert rc == M.MOE_ERR_UNSUPPORTED
+
+
+def test_small_workspace_rejected(L):
+    cfg = M.config(4096, 1024, 8, 2, 3584)
+    p = ctypes.c_void_p(0x1000)
+    rc = L.moe_permute(ctypes.byref(cfg), p, p, p, p, p, p, p, p, p, 16, None, None)
+    assert rc == M.MOE_ERR_WORKSPACE

@@ -1,0 +1,338 @@
+"""Parity of the CUDA path with the CPU oracle, called through the C ABI.
+
+Bars: routing indices, counts, offsets, drop decisions, dest_row/perm_src and
+the permuted rows are bit-exact; gates within 1e-5 relative; layer outputs
+within the per-row relative bound (2e-2 for bf16 storage, 1e-4 for fp32).
+"""
+import numpy as np
+import pytest
+import torch
+
+import combine_router_gemm_softmax_b200 as M
+import oracle as O
+import workloads as W
+from oracle import cases
+from oracle import check as C
+
+from gpu_cases import DEV, DeviceCase, cfg_for, np64, np_, oracle_y, parity_case, workload
+
+pytestmark = pytest.mark.gpu
+
+LAYER_CASES = ["tiny_f32", "tiny_f32_tagged", "small_ragged", "small_skewed", "small_skewed_capacity",
+               "small_many", "mixtral_scaled", "skewed", "skewed_capacity", "many_small", "many_small_identity",
+               "mixtral_8x7b"]
+FULL_ORACLE = {"tiny_f32", "tiny_f32_tagged", "small_ragged", "small_skewed", "small_skewed_capacity",
+               "small_many", "many_small_identity"}
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _device():
+    assert torch.cuda.is_available(), "these tests need a CUDA device"
+    torch.cuda.set_device(0)
+    M.lib()
+
+
+_dev_cache = {}
+
+
+def dev_case(name):
+    if name not in _dev_cache:
+        _dev_cache.clear()
+        torch.cuda.empty_cache()
+        inp, _ = parity_case(name)
+        _dev_cache[name] = DeviceCase(inp)
+    return _dev_cache[name]
+
+
+def gate_close(g, ref):
+    return np.allclose(g, ref, rtol=C.TOL_GATE, atol=1e-7)
+
+
+# ------------------------------------------------------------------ router
+@pytest.mark.parametrize("name", ["tiny_f32", "small_ragged", "small_many", "mixtral_scaled", "skewed",
+                                  "many_small", "mixtral_8x7b"])
+def test_route_matches_oracle(name):
+    dc = dev_case(name)
+    _, ref = parity_case(name)
+    wl = dc.wl
+    logits = torch.empty((wl.T, wl.E), dtype=torch.float32, device=DEV)
+    dc.status.zero_()
+    idx, gate = M.moe_route(dc.cfg, dc.h, dc.w_router, dc.bias, logits_out=logits, status=dc.status)
+    torch.cuda.synchronize()
+    assert np.array_equal(np_(idx), ref["idx"])
+    assert gate_close(np64(gate), ref["gate"])
+    s = ref["logits"]
+    fin = np.isfinite(s)
+    got = np64(logits)
+    assert np.array_equal(np.isfinite(got), fin)
+    assert np.allclose(got[fin], s[fin], rtol=1e-4, atol=1e-4)
+    assert int(dc.status.item()) == 0
+
+
+def _int_valued(T, d, E, seed, lo=-2, hi=3):
+    r = np.random.default_rng(seed)
+    return (r.integers(lo, hi, size=(T, d)).astype(np.float32), r.integers(lo, hi, size=(E, d)).astype(np.float32))
+
+
+@pytest.mark.parametrize("dtype,T,d,E,k", [("bf16", 300, 128, 8, 2), ("bf16", 129, 256, 64, 6),
+                                           ("bf16", 200, 128, 128, 8), ("f32", 77, 32, 6, 3)])
+def test_route_exact_ties_go_to_lowest_index(dtype, T, d, E, k):
+    """Small integers make every score exact in fp32 and fp64, so planted ties
+    are real ties on both sides."""
+    h, w = _int_valued(T, d, E, seed=T + E)
+    w[E // 2] = w[0]                      # expert E/2 always ties expert 0
+    w[E - 1] = w[1]
+    tdt = torch.bfloat16 if dtype == "bf16" else torch.float32
+    cfg = M.config(T, d, E, k, 128, dtype)
+    ht, wt = torch.from_numpy(h).to(tdt), torch.from_numpy(w).to(tdt)
+    idx, gate = M.moe_route(cfg, ht.to(DEV), wt.to(DEV))
+    ref_idx, ref_gate, _, _ = O.route(h.astype(np.float64), w.astype(np.float64), None, k)
+    assert np.array_equal(np_(idx), ref_idx)
+    assert gate_close(np64(gate), ref_gate)
+
+
+def test_route_nan_and_all_minus_inf():
+    T, d, E, k = 130, 128, 16, 4
+    h, w = _int_valued(T, d, E, seed=5)
+    h[3, 7] = np.nan                      # NaN scores for every expert of token 3
+    bias = np.zeros(E, np.float32)
+    bias[E - 3:] = -np.inf
+    hb = torch.from_numpy(h).to(torch.bfloat16)
+    cfg = M.config(T, d, E, k, 128)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    idx, gate = M.moe_route(cfg, hb.to(DEV), torch.from_numpy(w).to(torch.bfloat16).to(DEV),
+                            torch.from_numpy(bias).to(DEV), status=status)
+    ref_idx, ref_gate, _, nan_row = O.route(hb.double().numpy(), w.astype(np.float64), bias.astype(np.float64), k)
+    assert nan_row[3]
+    assert np.array_equal(np_(idx), ref_idx)
+    assert np_(idx)[3].tolist() == [0, 1, 2, 3]
+    assert np.all(np64(gate)[3] == 0)
+    assert gate_close(np64(gate), ref_gate)
+    assert int(status.item()) & M.MOE_STATUS_NAN_LOGIT
+    # all experts at -inf: picks 0..k-1, gate 0
+    cfg2 = M.config(4, d, E, k, 128)
+    idx2, gate2 = M.moe_route(cfg2, hb[:4].to(DEV), torch.from_numpy(w).to(torch.bfloat16).to(DEV),
+                              torch.full((E,), -float("inf"), device=DEV))
+    assert np_(idx2).tolist() == [[0, 1, 2, 3]] * 4
+    assert np.all(np64(gate2) == 0)
+
+
+def test_route_batch_invariance():
+    """A token's scores do not depend on which other tokens share the batch."""
+    dc = dev_case("small_ragged")
+    wl = dc.wl
+    full = torch.empty((wl.T, wl.E), dtype=torch.float32, device=DEV)
+    M.moe_route(dc.cfg, dc.h, dc.w_router, dc.bias, logits_out=full)
+    for lo, hi in ((0, 1), (5, 300), (517, 1000)):
+        sub = cfg_for(wl.with_(T=hi - lo))
+        part = torch.empty((hi - lo, wl.E), dtype=torch.float32, device=DEV)
+        M.moe_route(sub, dc.h[lo:hi].contiguous(), dc.w_router, dc.bias, logits_out=part)
+        assert torch.equal(part, full[lo:hi])
+    perm = torch.randperm(wl.T, generator=torch.Generator().manual_seed(0)).to(DEV)
+    shuffled = torch.empty_like(full)
+    M.moe_route(dc.cfg, dc.h[perm].contiguous(), dc.w_router, dc.bias, logits_out=shuffled)
+    assert torch.equal(shuffled, full[perm])
+
+
+# ------------------------------------------------------------------ permute
+def _permute_check(T, d, E, k, idx, cap=-1, dtype="bf16", seed=0):
+    tdt = torch.bfloat16 if dtype == "bf16" else torch.float32
+    h = torch.from_numpy(np.random.default_rng(seed).standard_normal((T, d)).astype(np.float32)).to(tdt)
+    cfg = M.config(T, d, E, k, 128, dtype, capacity=cap)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    out = M.moe_permute(cfg, h.to(DEV), torch.from_numpy(np.asarray(idx, np.int32)).to(DEV), status=status)
+    torch.cuda.synchronize()
+    ref = O.dispatch_meta(np.asarray(idx), E, cap)
+    n = int(ref["offsets"][-1])
+    assert np_(out["routed_counts"]).tolist() == ref["routed"].tolist()
+    assert np_(out["counts"]).tolist() == ref["kept"].tolist()
+    assert np_(out["offsets"]).tolist() == ref["offsets"].tolist()
+    assert np.array_equal(np_(out["dest_row"]), ref["dest_row"])
+    assert np.array_equal(np_(out["perm_src"])[:n], ref["perm_src"])
+    xp = out["x_perm"][:n].cpu()
+    want = h[torch.from_numpy(ref["perm_src"])]
+    bits = torch.int16 if dtype == "bf16" else torch.int32
+    assert torch.equal(xp.view(bits), want.view(bits))
+    bad = bool(int(status.item()) & M.MOE_STATUS_BAD_ROUTE)
+    assert bad == ref["bad_route"]
+    return out, ref
+
+
+@pytest.mark.parametrize("which", ["map1", "map2"])
+def test_permute_worked_maps(golden_dir, which):
+    """The two four-rank routing maps printed on the dispatch page, 2 KiB rows."""
+    import json
+    import os
+    g = json.load(open(os.path.join(golden_dir, "dispatch_worked_maps.json")))
+    m = g["maps"][which]
+    idx = [[m["expert_of_token"][t]] for t in g["tokens"]]
+    out, _ = _permute_check(8, g["row_bytes"] // 2, 4, 1, idx)
+    assert np_(out["counts"]).tolist() == m["counts_printed"]
+    toks = g["tokens"]
+    off = np_(out["offsets"])
+    ps = np_(out["perm_src"])
+    assert [[toks[t] for t in ps[off[e]:off[e + 1]]] for e in range(4)] == m["expected_grouping_by_expert"]
+
+
+def _routes(kind, T, E, k, seed=0):
+    r = np.random.default_rng(seed)
+    if kind == "random":
+        return np.stack([r.permutation(E)[:k] for _ in range(T)])
+    if kind == "all_to_one":                        # every token's first pick is expert 0
+        rows = [np.concatenate([[0], r.permutation(np.arange(1, E))[:k - 1]]) for _ in range(T)]
+        return np.stack(rows)
+    if kind == "empty_experts":                     # only even experts are used
+        return np.stack([r.permutation(np.arange(0, E, 2))[:k] for _ in range(T)])
+    if kind == "bad":
+        idx = np.stack([r.permutation(E)[:k] for _ in range(T)])
+        idx[3, 1] = E + 5
+        idx[10, 0] = -1
+        idx[20, 1] = idx[20, 0]
+        return idx
+    raise ValueError(kind)
+
+
+@pytest.mark.parametrize("kind,T,E,k,cap", [
+    ("random", 1000, 8, 2, -1), ("random", 4097, 64, 6, -1), ("all_to_one", 700, 16, 3, -1),
+    ("empty_experts", 513, 32, 4, -1), ("all_to_one", 700, 16, 3, 100), ("random", 999, 40, 4, 50),
+    ("bad", 300, 8, 2, -1), ("random", 1, 8, 2, -1), ("random", 128, 256, 8, -1), ("random", 300, 4, 4, 0)])
+def test_permute_injected_routes(kind, T, E, k, cap):
+    _permute_check(T, 256, E, k, _routes(kind, T, E, k), cap)
+
+
+def test_permute_fp32_rows():
+    _permute_check(100, 36, 5, 2, _routes("random", 100, 5, 2), dtype="f32")
+
+
+def test_permute_zero_tokens():
+    cfg = M.config(0, 128, 8, 2, 128)
+    out = M.moe_permute(cfg, torch.empty((0, 128), dtype=torch.bfloat16, device=DEV),
+                        torch.empty((0, 2), dtype=torch.int32, device=DEV))
+    torch.cuda.synchronize()
+    assert np_(out["offsets"]).tolist() == [0] * 9
+    assert np_(out["routed_counts"]).tolist() == [0] * 8
+
+
+# ------------------------------------------------------------------ grouped FFN (fed by the oracle's dispatch)
+@pytest.mark.parametrize("name", ["tiny_f32", "small_ragged", "small_skewed", "small_many", "mixtral_scaled"])
+def test_grouped_ffn_matches_oracle(name):
+    dc = dev_case(name)
+    inp, ref = parity_case(name)
+    wl = dc.wl
+    A = wl.T * wl.k
+    x_perm = torch.zeros((A, wl.d), dtype=wl.torch_dtype)
+    n = int(ref["offsets"][-1])
+    x_perm[:n] = inp.h[ref["perm_src"]]
+    offsets = torch.from_numpy(ref["offsets"].astype(np.int32))
+    y_perm = M.moe_grouped_ffn(dc.cfg, x_perm.to(DEV), offsets.to(DEV), dc.w13, dc.w_down, status=dc.status)
+    torch.cuda.synchronize()
+    got = np64(y_perm[:n])
+    rows = np.linspace(0, n - 1, min(n, 1536)).astype(np.int64)
+    want = np.zeros((len(rows), wl.d))
+    xs = cases.as64(x_perm)
+    wf = cases.weights_fn(inp)
+    for e in range(wl.E):
+        sel = np.nonzero((rows >= ref["offsets"][e]) & (rows < ref["offsets"][e + 1]))[0]
+        if sel.size:
+            want[sel] = O.swiglu_expert(xs[rows[sel]], *wf(e))
+    assert C.row_rel_err(got[rows], want) <= C.tol_for(wl.dtype)
+
+
+@pytest.mark.parametrize("kind", ["identity", "scale"])
+def test_combine_matches_oracle(kind):
+    """Combine alone, fed y_perm = f_e(x_perm) for the identity and scale
+    experts built on the CPU from the oracle's dispatch."""
+    name = "small_skewed_capacity"
+    inp, ref = parity_case(name)
+    wl = inp.wl.with_(expert_kind=kind)
+    A = wl.T * wl.k
+    n = int(ref["offsets"][-1])
+    h64 = cases.as64(inp.h)
+    y_perm = np.zeros((A, wl.d))
+    for e in range(wl.E):
+        a, b = ref["offsets"][e], ref["offsets"][e + 1]
+        y_perm[a:b] = O.expert_apply(kind, e, h64[ref["perm_src"][a:b]])
+    cfg = cfg_for(wl)
+    y = M.moe_unpermute_combine(cfg, torch.from_numpy(y_perm).to(torch.bfloat16).to(DEV),
+                                torch.from_numpy(ref["dest_row"].astype(np.int32)).to(DEV),
+                                torch.from_numpy(ref["gate"].astype(np.float32)).to(DEV))
+    want = O.combine(h64, ref["idx"], ref["gate"], ref["dest_row"], kind)
+    assert C.row_rel_err(np64(y), want) <= C.TOL_BF16
+    assert n < A                                   # this case drops assignments
+
+
+# ------------------------------------------------------------------ whole layer
+@pytest.mark.parametrize("name", LAYER_CASES)
+def test_layer_matches_oracle(name):
+    dc = dev_case(name)
+    inp, ref = parity_case(name)
+    wl = dc.wl
+    dc.status.zero_()
+    out = dc.layer()
+    torch.cuda.synchronize()
+    assert np.array_equal(np_(out["topk_idx"]), ref["idx"])
+    assert gate_close(np64(out["topk_gate"]), ref["gate"])
+    assert np_(out["routed_counts"]).tolist() == ref["routed"].tolist()
+    assert np_(out["counts"]).tolist() == ref["kept"].tolist()
+    assert int(dc.status.item()) == 0
+    if name in FULL_ORACLE:
+        tokens = None
+    else:
+        tokens = cases.sample_tokens(ref["idx"], ref["dest_row"], 1024)
+    want = oracle_y(name, tokens)
+    got = np64(out["y"]) if tokens is None else np64(out["y"][torch.from_numpy(tokens).to(DEV)])
+    err = C.row_rel_err(got, want)
+    assert err <= C.tol_for(wl.dtype), err
+
+
+def test_layer_identity_tagged_closed_form():
+    """Identity-tagged tokens with scale experts: every output row is zero
+    except position t mod d, which holds (t+1) * sum_j g_j (e_j + 1)."""
+    dc = dev_case("tiny_f32_tagged")
+    out = dc.layer()
+    y = np64(out["y"])
+    idx, g = np_(out["topk_idx"]), np64(out["topk_gate"])
+    for t in range(dc.wl.T):
+        c = t % dc.wl.d
+        row = y[t].copy()
+        assert row[c] == pytest.approx((t + 1) * float((g[t] * (idx[t] + 1)).sum()), rel=1e-5)
+        row[c] = 0
+        assert not row.any()
+
+
+def test_layer_is_deterministic():
+    dc = dev_case("small_skewed_capacity")
+    a = dc.layer()["y"].clone()
+    b = dc.layer()["y"]
+    assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+
+
+@pytest.mark.parametrize("T,E,k,cap", [(0, 8, 2, -1), (1, 8, 2, -1), (129, 1, 1, -1), (200, 8, 8, -1),
+                                       (300, 8, 2, 0)])
+def test_layer_edge_cases(T, E, k, cap):
+    wl = W.Workload("edge", T=T, d=128, E=E, k=k, F=128, bias="none", capacity=cap)
+    inp = W.draw(wl, 3)
+    if T:
+        inp = cases.enforce_margin(inp, 3)
+    dc = DeviceCase(inp)
+    out = dc.layer()
+    torch.cuda.synchronize()
+    if T == 0:
+        assert out["y"].numel() == 0
+        return
+    ref = O.layer_forward(cases.as64(inp.h), cases.as64(inp.w_router), None, k, "swiglu", cases.weights_fn(inp),
+                          cap)
+    assert np.array_equal(np_(out["topk_idx"]), ref["idx"])
+    assert C.row_rel_err(np64(out["y"]), ref["y"]) <= C.TOL_BF16
+    if cap == 0:
+        assert not out["y"].any()
+
+
+def test_workspace_guard_bytes_untouched():
+    """Bytes past the workspace the library asked for stay untouched."""
+    dc = dev_case("small_ragged")
+    need = M.moe_workspace_size(dc.cfg, M.MOE_OP_LAYER)
+    ws = torch.full((need + 4096,), 0x5A, dtype=torch.uint8, device=DEV)
+    dc.layer(ws=ws[:need])
+    torch.cuda.synchronize()
+    assert bool((ws[need:] == 0x5A).all())

@@ -176,7 +176,7 @@ def draw_bias(wl: Workload, seed: int = 0, hot_bias: float | None = None) -> tor
         return None
     if wl.bias == "zipf_3_empty":
         b = np.array([2.0 * math.log(1.0 / (e + 1)) for e in range(E)], np.float64)
-        b[list(SKEWED_EMPTY)] = -np.inf
+        b[[e for e in SKEWED_EMPTY if e < E]] = -np.inf
         return torch.from_numpy(b.astype(np.float32))
     if wl.bias == "gauss_0.5":
         z = normal(seed, (STREAM_BIAS,), (E,))
