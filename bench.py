@@ -32,7 +32,7 @@ METRIC = "MoE layer tokens/s; dispatch+combine HBM GB/s; grouped-GEMM TFLOPS (1 
 UNIT = "tokens/s"
 DEFAULT_WORKLOAD = "mixtral_8x7b"
 # tokens of the bounded CPU sample per workload (about 10-30 s of oracle work)
-CPU_SAMPLE = {"mixtral_8x7b": 512, "mixtral_scaled": 2048, "skewed": 1024, "many_small": 1024,
+CPU_SAMPLE = {"mixtral_8x7b": 8192, "mixtral_scaled": 4096, "skewed": 4096, "many_small": 4096,
               "tiny_f32": 64}
 PEAKS_PATH = os.path.join(ROOT, "MEASURED_PEAKS.json")
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}

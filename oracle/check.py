@@ -14,6 +14,11 @@ TOL_BF16 = 2e-2
 TOL_F32 = 1e-4
 TOL_GATE = 1e-5
 
+# Router scores: the kernel accumulates bf16 (or fp32) products in fp32, the
+# oracle in fp64; scores must agree within LOGIT_ATOL + LOGIT_RTOL * |s|.
+LOGIT_ATOL = 1e-4
+LOGIT_RTOL = 1e-4
+
 
 def row_rel_err(y, y_ref, floor=1e-6):
     y = np.asarray(y, np.float64)
@@ -59,3 +64,29 @@ def permutation_consistent(dest_row, perm_src, offsets, idx, n_kept=None):
         if seg.size > 1 and not (np.diff(seg) > 0).all():
             return False
     return True
+
+
+def logits_match(s, s_ref):
+    """Finite pattern identical, finite values within the score tolerance."""
+    s = np.asarray(s, np.float64)
+    s_ref = np.asarray(s_ref, np.float64)
+    fin = np.isfinite(s_ref)
+    if not np.array_equal(np.isfinite(s), fin):
+        return False
+    return bool(np.all(np.abs(s[fin] - s_ref[fin]) <= LOGIT_ATOL + LOGIT_RTOL * np.abs(s_ref[fin])))
+
+
+def gate_bound(gate_ref, s_picked_ref):
+    """Allowed |g - g_ref| per slot when the scores themselves may differ by
+    the score tolerance. A gate renormalised over the picks is
+    g_j = exp(s_j) / sum_i exp(s_i), so dg_j/ds_i = g_j (delta_ij - g_i) and
+    |dg_j| <= g_j * 2 * max_i |ds_i|; TOL_GATE covers fp32 exp and division."""
+    g = np.asarray(gate_ref, np.float64)
+    sp = np.asarray(s_picked_ref, np.float64)
+    ds = np.where(np.isfinite(sp), LOGIT_ATOL + LOGIT_RTOL * np.abs(sp), 0.0).max(axis=1, keepdims=True)
+    return g * (2.0 * ds + TOL_GATE) + 1e-7
+
+
+def gates_match(gate, gate_ref, logits_ref, idx_ref):
+    sp = np.take_along_axis(np.asarray(logits_ref, np.float64), np.asarray(idx_ref, np.int64), axis=1)
+    return bool(np.all(np.abs(np.asarray(gate, np.float64) - gate_ref) <= gate_bound(gate_ref, sp)))

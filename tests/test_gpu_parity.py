@@ -44,8 +44,8 @@ def dev_case(name):
     return _dev_cache[name]
 
 
-def gate_close(g, ref):
-    return np.allclose(g, ref, rtol=C.TOL_GATE, atol=1e-7)
+def gate_close(g, ref, logits_ref, idx_ref):
+    return C.gates_match(g, ref, logits_ref, idx_ref)
 
 
 # ------------------------------------------------------------------ router
@@ -60,12 +60,8 @@ def test_route_matches_oracle(name):
     idx, gate = M.moe_route(dc.cfg, dc.h, dc.w_router, dc.bias, logits_out=logits, status=dc.status)
     torch.cuda.synchronize()
     assert np.array_equal(np_(idx), ref["idx"])
-    assert gate_close(np64(gate), ref["gate"])
-    s = ref["logits"]
-    fin = np.isfinite(s)
-    got = np64(logits)
-    assert np.array_equal(np.isfinite(got), fin)
-    assert np.allclose(got[fin], s[fin], rtol=1e-4, atol=1e-4)
+    assert C.logits_match(np64(logits), ref["logits"])
+    assert gate_close(np64(gate), ref["gate"], ref["logits"], ref["idx"])
     assert int(dc.status.item()) == 0
 
 
@@ -86,9 +82,9 @@ def test_route_exact_ties_go_to_lowest_index(dtype, T, d, E, k):
     cfg = M.config(T, d, E, k, 128, dtype)
     ht, wt = torch.from_numpy(h).to(tdt), torch.from_numpy(w).to(tdt)
     idx, gate = M.moe_route(cfg, ht.to(DEV), wt.to(DEV))
-    ref_idx, ref_gate, _, _ = O.route(h.astype(np.float64), w.astype(np.float64), None, k)
+    ref_idx, ref_gate, ref_s, _ = O.route(h.astype(np.float64), w.astype(np.float64), None, k)
     assert np.array_equal(np_(idx), ref_idx)
-    assert gate_close(np64(gate), ref_gate)
+    assert gate_close(np64(gate), ref_gate, ref_s, ref_idx)
 
 
 def test_route_nan_and_all_minus_inf():
@@ -102,12 +98,13 @@ def test_route_nan_and_all_minus_inf():
     status = torch.zeros(1, dtype=torch.int32, device=DEV)
     idx, gate = M.moe_route(cfg, hb.to(DEV), torch.from_numpy(w).to(torch.bfloat16).to(DEV),
                             torch.from_numpy(bias).to(DEV), status=status)
-    ref_idx, ref_gate, _, nan_row = O.route(hb.double().numpy(), w.astype(np.float64), bias.astype(np.float64), k)
+    ref_idx, ref_gate, ref_s, nan_row = O.route(hb.double().numpy(), w.astype(np.float64), bias.astype(np.float64),
+                                                k)
     assert nan_row[3]
     assert np.array_equal(np_(idx), ref_idx)
     assert np_(idx)[3].tolist() == [0, 1, 2, 3]
     assert np.all(np64(gate)[3] == 0)
-    assert gate_close(np64(gate), ref_gate)
+    assert gate_close(np64(gate), ref_gate, ref_s, ref_idx)
     assert int(status.item()) & M.MOE_STATUS_NAN_LOGIT
     # all experts at -inf: picks 0..k-1, gate 0
     cfg2 = M.config(4, d, E, k, 128)
@@ -271,7 +268,7 @@ def test_layer_matches_oracle(name):
     out = dc.layer()
     torch.cuda.synchronize()
     assert np.array_equal(np_(out["topk_idx"]), ref["idx"])
-    assert gate_close(np64(out["topk_gate"]), ref["gate"])
+    assert gate_close(np64(out["topk_gate"]), ref["gate"], ref["logits"], ref["idx"])
     assert np_(out["routed_counts"]).tolist() == ref["routed"].tolist()
     assert np_(out["counts"]).tolist() == ref["kept"].tolist()
     assert int(dc.status.item()) == 0
