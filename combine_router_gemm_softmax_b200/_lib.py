@@ -25,7 +25,8 @@ MOE_OP_ROUTE, MOE_OP_PERMUTE, MOE_OP_GROUPED_FFN, MOE_OP_LAYER = 0, 1, 2, 3
 MOE_MAX_E, MOE_MAX_K, MOE_PACK_BLOCK = 256, 8, 128
 
 EXPORTED = ("moe_workspace_size", "moe_status_string", "moe_version", "moe_pack_weights", "moe_route",
-            "moe_permute", "moe_grouped_ffn", "moe_unpermute_combine", "moe_layer_forward")
+            "moe_permute", "moe_grouped_ffn", "moe_unpermute_combine", "moe_layer_forward",
+            "moe_permute_static_scratch")
 
 
 class MoeError(RuntimeError):
@@ -65,6 +66,7 @@ _SIGS = {
     "moe_grouped_ffn": (I32, [CFG, P, P, P, P, P, P, SZ, P, P]),
     "moe_unpermute_combine": (I32, [CFG, P, P, P, P, P, P]),
     "moe_layer_forward": (I32, [CFG, P, P, P, P, P, P, P, P, P, P, P, SZ, P, P]),
+    "moe_permute_static_scratch": (I32, [CFG, P, P, P, P, P, P, P, P, P, P]),
 }
 
 
@@ -248,3 +250,27 @@ def moe_layer_forward(cfg, h, w_router, bias=None, w13_packed=None, w_down=None,
         _ptr(topk_idx), _ptr(topk_gate), _ptr(routed_counts), _ptr(counts), _ptr(ws), ws.numel(), _ptr(status),
         _stream(stream)))
     return y
+
+
+def moe_permute_static_scratch(cfg, h, topk_idx, out=None, status=None, stream=None):
+    """moe_permute without a workspace argument, for callers that cannot
+    allocate device memory; the library keeps the scratch in a fixed 1 MiB
+    device array shared by all calls (calls that overlap on the GPU race).
+    Returns the same dict as moe_permute."""
+    dt = cfg.torch_dtype
+    dev = _dev(h)
+    A = cfg.T * cfg.k
+    _check(h, (cfg.T, cfg.d), dt, "h")
+    _check(topk_idx, (cfg.T, cfg.k), torch.int32, "topk_idx")
+    if out is None:
+        out = dict(routed_counts=torch.empty(cfg.E, dtype=torch.int32, device=dev),
+                   counts=torch.empty(cfg.E, dtype=torch.int32, device=dev),
+                   offsets=torch.empty(cfg.E + 1, dtype=torch.int32, device=dev),
+                   dest_row=torch.empty((cfg.T, cfg.k), dtype=torch.int32, device=dev),
+                   perm_src=torch.empty(max(A, 1), dtype=torch.int32, device=dev),
+                   x_perm=torch.empty((max(A, 1), cfg.d), dtype=dt, device=dev))
+    _rc("moe_permute_static_scratch", lib().moe_permute_static_scratch(
+        ctypes.byref(cfg), _ptr(h), _ptr(topk_idx), _ptr(out["routed_counts"]), _ptr(out["counts"]),
+        _ptr(out["offsets"]), _ptr(out["dest_row"]), _ptr(out["perm_src"]), _ptr(out["x_perm"]), _ptr(status),
+        _stream(stream)))
+    return out

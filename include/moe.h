@@ -187,6 +187,27 @@ MOE_API int32_t moe_layer_forward(const moe_config* cfg, const void* h, const vo
                           int32_t* counts, void* workspace, size_t ws_bytes,
                           int32_t* status_dev, moe_stream_t stream);
 
+/* moe_permute_static_scratch -- moe_permute for callers that cannot allocate.
+ * The paper has no counterpart for this entry point. It is for code that has
+ * no way to pass a workspace: a host framework or memory pool that owns all
+ * device memory and forbids allocations outside it, or a latency-critical
+ * path that must not allocate. Inputs, outputs and results are exactly those
+ * of moe_permute; the permute scratch lives instead in a fixed 1 MiB array in
+ * the library's device image, which every GPU that loads the library holds
+ * until the process exits.
+ * Limit: 2 * roundup256(4 * E * ceil(T/128)) bytes must fit in 1 MiB
+ * (E * ceil(T/128) <= 131072, e.g. T <= 65536 at E = 256); larger problems
+ * return MOE_ERR_WORKSPACE and enqueue nothing.
+ * All calls share the array: calls that may overlap on the GPU (streams with
+ * no ordering between them) race and give wrong results. Nothing in the array
+ * needs to start at zero. The first call on a device looks up the array's
+ * address on that device; make it before any stream capture. No cudaMalloc,
+ * cudaFree or other allocating call is made. */
+MOE_API int32_t moe_permute_static_scratch(const moe_config* cfg, const void* h, const int32_t* topk_idx,
+                                           int32_t* routed_counts, int32_t* counts, int32_t* offsets,
+                                           int32_t* dest_row, int32_t* perm_src, void* x_perm,
+                                           int32_t* status_dev, moe_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif
