@@ -189,6 +189,21 @@ def run_reference(args, wl, rank):
     print(json.dumps(line), flush=True)
 
 
+def combine_ranks(ms_local, tokens_per_rank, steps, world, device=None):
+    """Whole-job throughput of token-sharded replicas: every rank processed
+    tokens_per_rank tokens per step; the job took as long as its slowest rank.
+    Returns (max device ms over ranks, tokens/s of all ranks)."""
+    import torch
+    import torch.distributed as dist
+
+    ms = float(ms_local)
+    if world > 1:
+        t = torch.tensor([ms], dtype=torch.float64, device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    return ms, tokens_per_rank * world * steps / (ms / 1e3)
+
+
 def config_dict(wl, n, flush=None):
     c = {"workload": wl.name, "T": wl.T, "d": wl.d, "E": wl.E, "k": wl.k, "d_ff": wl.F, "dtype": wl.dtype,
          "expert_kind": wl.expert_kind, "capacity": wl.capacity, "global_batch": wl.T * n,
@@ -288,12 +303,7 @@ def main():
         torch.cuda.synchronize()
         barrier()
     ms = sum(a.elapsed_time(b) for a, b in evs)
-    ms_max = ms
-    if world > 1:
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_max = float(t.item())
-    value = wl.T * world * args.steps / (ms_max / 1e3)
+    ms_max, value = combine_ranks(ms, wl.T, args.steps, world, dev)
     launches_per_step = launches(cfg)
     st = int(status.item())
 
@@ -313,12 +323,7 @@ def main():
         y_host.copy_(y, non_blocking=True)
     e1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1)
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
-    e2e_value = wl.T * world * args.steps / (e2e_ms / 1e3)
+    e2e_ms, e2e_value = combine_ranks(e0.elapsed_time(e1), wl.T, args.steps, world, dev)
     row_bytes = wl.d * wl.elem_bytes
 
     # ------------------------------------------------ per stage (same stream, CUDA events)

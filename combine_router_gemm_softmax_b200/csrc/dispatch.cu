@@ -13,8 +13,8 @@
 //           base rank of each chunk), then kept counts and offsets
 //   rank  : per chunk, every slot's rank among earlier tokens of the same
 //           expert, from per-warp bitmasks (popc), giving dest_row/perm_src
-//   copy  : one warp per token reads its row once (16-byte vectors) and writes
-//           it to each kept destination row
+//   copy  : TMA bulk copies: each token row is bulk-loaded into shared memory
+//           once and bulk-stored to each kept destination row
 // Nothing decides an order with atomics, so the permutation is deterministic.
 #include "moe_common.cuh"
 #include "moe_internal.h"
@@ -178,38 +178,77 @@ __global__ void __launch_bounds__(kChunkTokens) rank_kernel(const int32_t* __res
   }
 }
 
-constexpr int kCopyUnroll = 8;
+constexpr int kCopyBuffers = 8;     // shared-memory row buffers per CTA
+constexpr int kCopyLead = 4;        // row loads kept in flight ahead of the stores
+constexpr int kCopyPiece = 8192;    // bytes per bulk transfer
+// Tokens per CTA: small blocks give many CTAs per SM and the most row loads in
+// flight (measured on B200 for 4-8 KiB rows and k = 2..8).
+constexpr int kCopyTokensPerCta = 4;
 
-// One warp per token: read the row once, write it to each kept destination.
-__global__ void __launch_bounds__(256) permute_copy_kernel(const uint4* __restrict__ h,
-                                                           const int32_t* __restrict__ dest_row,
-                                                           uint4* __restrict__ x_perm, int T, int k, int vpr) {
-  const int lane = threadIdx.x & 31;
-  const int nw = gridDim.x * (blockDim.x >> 5);
-  for (int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); t < T; t += nw) {
-    const int my_dest = lane < k ? dest_row[static_cast<size_t>(t) * k + lane] : -1;
-    const uint4* src = h + static_cast<size_t>(t) * vpr;
-    for (int v0 = 0; v0 < vpr; v0 += 32 * kCopyUnroll) {
-      uint4 buf[kCopyUnroll];
-#pragma unroll
-      for (int u = 0; u < kCopyUnroll; ++u) {
-        const int v = v0 + u * 32 + lane;
-        if (v < vpr) buf[u] = __ldg(src + v);
-      }
-#pragma unroll
-      for (int j = 0; j < kMaxK; ++j) {
-        if (j >= k) break;
-        const int dest = __shfl_sync(0xffffffffu, my_dest, j);
-        if (dest < 0) continue;
-        uint4* dst = x_perm + static_cast<size_t>(dest) * vpr;
-#pragma unroll
-        for (int u = 0; u < kCopyUnroll; ++u) {
-          const int v = v0 + u * 32 + lane;
-          if (v < vpr) dst[v] = buf[u];
-        }
-      }
+// Row copy with the TMA engine. Each CTA owns a contiguous block of tokens and
+// stages their dest_row entries in shared memory; one thread then runs a
+// pipeline: bulk-load a row (or a piece of it) into one of 8 buffers, and when
+// it lands, bulk-store it to every kept destination row. Each row is read from
+// HBM once; a few instructions move a whole row.
+__global__ void __launch_bounds__(32) permute_copy_bulk_kernel(const uint8_t* __restrict__ h,
+                                                               const int32_t* __restrict__ dest_row,
+                                                               uint8_t* __restrict__ x_perm, int T, int k, int rb,
+                                                               int tokens_per_cta, int32_t* status) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((128u - (smem_addr(smem_raw) & 127u)) & 127u);
+  const int piece = rb < kCopyPiece ? rb : kCopyPiece;
+  const int n_pieces = (rb + piece - 1) / piece;
+  uint8_t* buf = smem;                                                    // kCopyBuffers x piece
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kCopyBuffers * piece);
+  int* dests = reinterpret_cast<int*>(bars + kCopyBuffers);               // tokens_per_cta x k
+  const int lane = threadIdx.x;
+  const int t0 = blockIdx.x * tokens_per_cta;
+  const int nt = min(tokens_per_cta, T - t0);
+  if (nt <= 0) return;
+  for (int i = lane; i < nt * k; i += 32) dests[i] = dest_row[static_cast<size_t>(t0) * k + i];
+  if (lane == 0) {
+    for (int b = 0; b < kCopyBuffers; ++b) mbar_init(&bars[b], 1);
+    fence_mbar_init();
+  }
+  __syncwarp();
+  if (lane != 0) return;
+
+  const int n = nt * n_pieces;
+  int issued = 0;
+  auto issue = [&](int m) {
+    const int b = m % kCopyBuffers;
+    const int off = (m % n_pieces) * piece;
+    const uint32_t bytes = static_cast<uint32_t>(min(piece, rb - off));
+    mbar_expect_tx(&bars[b], bytes);
+    bulk_load(buf + b * piece, h + static_cast<size_t>(t0 + m / n_pieces) * rb + off, bytes, &bars[b]);
+    ++issued;
+  };
+  for (int m = 0; m < kCopyLead && m < n; ++m) issue(m);
+  int m = 0;
+  for (; m < n; ++m) {
+    const int b = m % kCopyBuffers;
+    if (!mbar_wait(&bars[b], (m / kCopyBuffers) & 1, nullptr)) {
+      report_status(status, MOE_STATUS_TIMEOUT);
+      break;
+    }
+    const int tl = m / n_pieces;
+    const int off = (m % n_pieces) * piece;
+    const uint32_t bytes = static_cast<uint32_t>(min(piece, rb - off));
+    for (int j = 0; j < k; ++j) {
+      const int dest = dests[tl * k + j];
+      if (dest >= 0) bulk_store(x_perm + static_cast<size_t>(dest) * rb + off, buf + b * piece, bytes);
+    }
+    bulk_commit();
+    if (m + kCopyLead < n) {
+      // buffer (m + lead) % 8 was last used by unit m + lead - 8, whose stores
+      // were committed 8 - lead groups ago
+      bulk_wait_read<kCopyBuffers - kCopyLead>();
+      issue(m + kCopyLead);
     }
   }
+  for (int r = m + 1; r < issued; ++r)  // only after a timeout: let issued loads land
+    mbar_wait(&bars[r % kCopyBuffers], (r / kCopyBuffers) & 1, nullptr);
+  bulk_wait_all();
 }
 
 // 16-byte vector <-> fp32 lanes for the two storage types.
@@ -252,52 +291,80 @@ struct Vec<MOE_DTYPE_F32> {
   }
 };
 
-constexpr int kCombineUnroll = 2;
-
 // One warp per token: y[t] = sum_j gate[t,j] * y_perm[dest_row[t,j]] in fp32,
-// slots in order 0..k-1, dropped slots skipped.
-template <int DT>
+// slots in order 0..k-1, dropped slots skipped. All k rows of U segments are
+// loaded before any of them is used, so k*U 16-byte loads per lane are in
+// flight (k*U = 8 for k <= 8).
+template <int DT, int K>
 __global__ void __launch_bounds__(256) combine_kernel(const uint4* __restrict__ y_perm,
                                                       const int32_t* __restrict__ dest_row,
                                                       const float* __restrict__ gate, uint4* __restrict__ y, int T,
-                                                      int k, int vpr) {
+                                                      int vpr) {
   using V = Vec<DT>;
+  constexpr int U = K >= 8 ? 1 : 8 / K;
   const int lane = threadIdx.x & 31;
   const int nw = gridDim.x * (blockDim.x >> 5);
   for (int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); t < T; t += nw) {
-    const int my_dest = lane < k ? dest_row[static_cast<size_t>(t) * k + lane] : -1;
-    const float my_gate = lane < k ? gate[static_cast<size_t>(t) * k + lane] : 0.f;
-    for (int v0 = 0; v0 < vpr; v0 += 32 * kCombineUnroll) {
-      float acc[kCombineUnroll][V::N];
+    const int my_dest = lane < K ? dest_row[static_cast<size_t>(t) * K + lane] : -1;
+    const float my_gate = lane < K ? gate[static_cast<size_t>(t) * K + lane] : 0.f;
+    int dst[K];
+    float g[K];
 #pragma unroll
-      for (int u = 0; u < kCombineUnroll; ++u)
+    for (int j = 0; j < K; ++j) {
+      dst[j] = __shfl_sync(0xffffffffu, my_dest, j);
+      g[j] = __shfl_sync(0xffffffffu, my_gate, j);
+    }
+    for (int v0 = 0; v0 < vpr; v0 += 32 * U) {
+      uint4 q[K][U];
 #pragma unroll
-        for (int i = 0; i < V::N; ++i) acc[u][i] = 0.f;
+      for (int j = 0; j < K; ++j)
 #pragma unroll
-      for (int j = 0; j < kMaxK; ++j) {
-        if (j >= k) break;
-        const int dest = __shfl_sync(0xffffffffu, my_dest, j);
-        const float g = __shfl_sync(0xffffffffu, my_gate, j);
-        if (dest < 0) continue;
-        const uint4* src = y_perm + static_cast<size_t>(dest) * vpr;
-#pragma unroll
-        for (int u = 0; u < kCombineUnroll; ++u) {
+        for (int u = 0; u < U; ++u) {
           const int v = v0 + u * 32 + lane;
-          if (v < vpr) {
-            float f[V::N];
-            V::load(__ldg(src + v), f);
-#pragma unroll
-            for (int i = 0; i < V::N; ++i) acc[u][i] = fmaf(g, f[i], acc[u][i]);
-          }
+          q[j][u] = (dst[j] >= 0 && v < vpr) ? __ldg(y_perm + static_cast<size_t>(dst[j]) * vpr + v)
+                                             : make_uint4(0, 0, 0, 0);
         }
-      }
 #pragma unroll
-      for (int u = 0; u < kCombineUnroll; ++u) {
+      for (int u = 0; u < U; ++u) {
+        float acc[V::N];
+#pragma unroll
+        for (int i = 0; i < V::N; ++i) acc[i] = 0.f;
+#pragma unroll
+        for (int j = 0; j < K; ++j) {
+          if (dst[j] < 0) continue;
+          float f[V::N];
+          V::load(q[j][u], f);
+#pragma unroll
+          for (int i = 0; i < V::N; ++i) acc[i] = fmaf(g[j], f[i], acc[i]);
+        }
         const int v = v0 + u * 32 + lane;
-        if (v < vpr) y[static_cast<size_t>(t) * vpr + v] = V::store(acc[u]);
+        if (v < vpr) y[static_cast<size_t>(t) * vpr + v] = V::store(acc);
       }
     }
   }
+}
+
+template <int DT>
+cudaError_t launch_combine_k(const uint4* y_perm, const int32_t* dest_row, const float* gate, uint4* y, int T, int k,
+                             int vpr, int grid, cudaStream_t s) {
+  switch (k) {
+#define MOE_COMBINE_K(KK) \
+  case KK:                \
+    combine_kernel<DT, KK><<<grid, 256, 0, s>>>(y_perm, dest_row, gate, y, T, vpr); \
+    break;
+    MOE_COMBINE_K(1)
+    MOE_COMBINE_K(2)
+    MOE_COMBINE_K(3)
+    MOE_COMBINE_K(4)
+    MOE_COMBINE_K(5)
+    MOE_COMBINE_K(6)
+    MOE_COMBINE_K(7)
+    MOE_COMBINE_K(8)
+#undef MOE_COMBINE_K
+    default:
+      return cudaErrorInvalidValue;
+  }
+  return cudaGetLastError();
 }
 
 int warp_grid(int T) {
@@ -318,9 +385,15 @@ cudaError_t launch_permute(const void* h, size_t row_bytes, const int32_t* idx, 
   if (n_chunks > 0) {
     rank_kernel<<<n_chunks, kChunkTokens, 0, s>>>(idx, T, k, E, cap, n_chunks, chunk_base, offsets, dest_row,
                                                   perm_src, status);
-    const int vpr = static_cast<int>(row_bytes / 16);
-    permute_copy_kernel<<<warp_grid(T), 256, 0, s>>>(static_cast<const uint4*>(h), dest_row,
-                                                     static_cast<uint4*>(x_perm), T, k, vpr);
+    const int tpc = kCopyTokensPerCta;
+    const int piece = static_cast<int>(row_bytes < kCopyPiece ? row_bytes : kCopyPiece);
+    const size_t smem = 128 + static_cast<size_t>(kCopyBuffers) * piece + kCopyBuffers * 8 + tpc * k * 4;
+    cudaError_t err = cudaFuncSetAttribute(permute_copy_bulk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           static_cast<int>(smem));
+    if (err != cudaSuccess) return err;
+    permute_copy_bulk_kernel<<<(T + tpc - 1) / tpc, 32, smem, s>>>(static_cast<const uint8_t*>(h), dest_row,
+                                                                   static_cast<uint8_t*>(x_perm), T, k,
+                                                                   static_cast<int>(row_bytes), tpc, status);
   }
   return cudaGetLastError();
 }
@@ -331,12 +404,10 @@ cudaError_t launch_combine(int dtype, const void* y_perm, const int32_t* dest_ro
   const int elem = dtype == MOE_DTYPE_BF16 ? 2 : 4;
   const int vpr = d * elem / 16;
   if (dtype == MOE_DTYPE_BF16)
-    combine_kernel<MOE_DTYPE_BF16><<<warp_grid(T), 256, 0, s>>>(
-        static_cast<const uint4*>(y_perm), dest_row, gate, static_cast<uint4*>(y), T, k, vpr);
-  else
-    combine_kernel<MOE_DTYPE_F32><<<warp_grid(T), 256, 0, s>>>(static_cast<const uint4*>(y_perm), dest_row, gate,
-                                                               static_cast<uint4*>(y), T, k, vpr);
-  return cudaGetLastError();
+    return launch_combine_k<MOE_DTYPE_BF16>(static_cast<const uint4*>(y_perm), dest_row, gate,
+                                            static_cast<uint4*>(y), T, k, vpr, warp_grid(T), s);
+  return launch_combine_k<MOE_DTYPE_F32>(static_cast<const uint4*>(y_perm), dest_row, gate, static_cast<uint4*>(y),
+                                         T, k, vpr, warp_grid(T), s);
 }
 
 }  // namespace moe

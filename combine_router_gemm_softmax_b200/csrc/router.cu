@@ -24,6 +24,10 @@ constexpr int kRouterBK = 64;
 constexpr uint32_t kRouterABytes = kTileM * kRouterBK * 2;
 
 // Running top-k of one token, sorted by (score descending, expert ascending).
+// Empty slots hold NaN, which compares false against everything, so they are
+// never ranked ahead of a candidate. An insertion counts the held entries
+// that stay ahead of the candidate (independent compares) and shifts the
+// tail down by one: no loop-carried chain through the k slots.
 struct TopList {
   float v[kMaxK];
   int i[kMaxK];
@@ -31,31 +35,37 @@ struct TopList {
   MOE_DEV void init() {
 #pragma unroll
     for (int j = 0; j < kMaxK; ++j) {
-      v[j] = -INFINITY;
+      v[j] = __int_as_float(0x7fffffff);
       i[j] = -1;
     }
   }
 
-  // Walk the held entries in order, carrying the candidate; whenever the
-  // carried entry ranks ahead of the held one (held slot empty, higher score,
-  // or equal score and lower index) the two swap. The list stays sorted and a
-  // candidate that does not beat the last entry falls off the end. Written
-  // without an early exit so the list stays in registers.
-  MOE_DEV void push(float x, int e, int k) {
-    float cv = x;
-    int ci = e;
+  MOE_DEV void insert_at(int p, float x, int e) {
 #pragma unroll
-    for (int j = 0; j < kMaxK; ++j) {
-      if (j < k) {
-        const bool ahead = (i[j] < 0) || (cv > v[j]) || (cv == v[j] && ci < i[j]);
-        const float tv = ahead ? v[j] : cv;
-        const int ti = ahead ? i[j] : ci;
-        v[j] = ahead ? cv : v[j];
-        i[j] = ahead ? ci : i[j];
-        cv = tv;
-        ci = ti;
-      }
+    for (int j = kMaxK - 1; j >= 0; --j) {
+      const float pv = j > 0 ? v[j - 1] : x;
+      const int pi = j > 0 ? i[j - 1] : e;
+      const bool move = j > p, put = j == p;
+      v[j] = move ? pv : (put ? x : v[j]);
+      i[j] = move ? pi : (put ? e : i[j]);
     }
+  }
+
+  // Candidates of one list arrive in ascending expert index, so a held entry
+  // with an equal score stays ahead (lower index wins).
+  MOE_DEV void push_ascending(float x, int e, int k) {
+    int p = 0;
+#pragma unroll
+    for (int j = 0; j < kMaxK; ++j) p += (j < k && v[j] >= x) ? 1 : 0;
+    insert_at(p, x, e);
+  }
+
+  // Candidate in any index order (merging another list); e < 0 is an empty slot.
+  MOE_DEV void push_any(float x, int e, int k) {
+    int p = 0;
+#pragma unroll
+    for (int j = 0; j < kMaxK; ++j) p += (j < k && (v[j] > x || (v[j] == x && i[j] < e))) ? 1 : 0;
+    insert_at(e < 0 ? k : p, x, e);
   }
 
   // Writes slot indices and gates: softmax over the picked scores.
@@ -87,7 +97,7 @@ struct RouterArgs {
   int32_t* status;
 };
 
-__global__ void __launch_bounds__(128) router_tc_kernel(const __grid_constant__ CUtensorMap tm_h,
+__global__ void __launch_bounds__(256) router_tc_kernel(const __grid_constant__ CUtensorMap tm_h,
                                                         const __grid_constant__ CUtensorMap tm_w,
                                                         const RouterArgs a) {
   extern __shared__ uint8_t smem_raw[];
@@ -118,7 +128,8 @@ __global__ void __launch_bounds__(128) router_tc_kernel(const __grid_constant__ 
     tma_prefetch_desc(&tm_h);
     tma_prefetch_desc(&tm_w);
   }
-  for (int e = threadIdx.x; e < a.E; e += blockDim.x) sbias[e] = a.bias ? a.bias[e] : 0.f;
+  for (int e = threadIdx.x; e < a.npad; e += blockDim.x)
+    sbias[e] = e >= a.E ? -INFINITY : (a.bias ? a.bias[e] : 0.f);
   if (warp == 0) {
     tmem_alloc(tmem_slot, a.tmem_cols);
     tmem_relinquish();
@@ -171,36 +182,54 @@ __global__ void __launch_bounds__(128) router_tc_kernel(const __grid_constant__ 
 
   bool ok = mbar_wait(done, 0, nullptr);
   tc_fence_after();
-  if (*abort_flag) ok = false;
+  ok = __syncthreads_and(ok && !*abort_flag);  // the same decision in every thread
 
   if (ok) {
-    const int row = warp * 32 + lane;
+    // 8 warps: warp w reads TMEM lane quadrant (w & 3), i.e. token rows
+    // 32*(w&3) .. +31, and every other 16-column chunk starting at 16*(w>>2).
+    // The two partial lists of a row are merged through shared memory.
+    const int q = warp & 3, half = warp >> 2;
+    const int row = q * 32 + lane;
     const int t = tile * kTileM + row;
     TopList top;
     top.init();
     bool nan = false;
-    const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);
-    for (int c0 = 0; c0 < a.npad; c0 += 16) {
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>(q * 32) << 16);
+    float* lrow = (a.logits != nullptr && t < a.T) ? a.logits + static_cast<size_t>(t) * a.E : nullptr;
+    for (int c0 = half * 16; c0 < a.npad; c0 += 32) {
       uint32_t r[16];
       tmem_ld16(lane_base + c0, r);
       tmem_ld_wait();
 #pragma unroll
       for (int j = 0; j < 16; ++j) {
-        const int e = c0 + j;
-        if (e < a.E) {
-          float x = __uint_as_float(r[j]) + sbias[e];
-          if (a.logits != nullptr && t < a.T) a.logits[static_cast<size_t>(t) * a.E + e] = x;
-          if (x != x) {
-            nan = true;
-            x = -INFINITY;
-          }
-          top.push(x, e, a.k);
-        }
+        float x = __uint_as_float(r[j]) + sbias[c0 + j];  // padded experts carry -inf
+        if (lrow != nullptr && c0 + j < a.E) lrow[c0 + j] = x;
+        nan |= x != x;
+        x = x != x ? -INFINITY : x;
+        top.push_ascending(x, c0 + j, a.k);
       }
     }
-    if (t < a.T) {
-      top.write(a.idx + static_cast<size_t>(t) * a.k, a.gate + static_cast<size_t>(t) * a.k, a.k);
-      if (nan) report_status(a.status, MOE_STATUS_NAN_LOGIT);
+    float* xv = reinterpret_cast<float*>(smem);  // stage buffers are free once the MMAs are done
+    int* xi = reinterpret_cast<int*>(smem + kTileM * kMaxK * 4);
+    int* xn = reinterpret_cast<int*>(smem + 2 * kTileM * kMaxK * 4);
+    if (half == 1) {
+#pragma unroll
+      for (int j = 0; j < kMaxK; ++j) {
+        xv[row * kMaxK + j] = top.v[j];
+        xi[row * kMaxK + j] = top.i[j];
+      }
+      xn[row] = nan;
+    }
+    __syncthreads();
+    if (half == 0) {
+#pragma unroll
+      for (int j = 0; j < kMaxK; ++j)
+        if (j < a.k) top.push_any(xv[row * kMaxK + j], xi[row * kMaxK + j], a.k);
+      nan |= xn[row] != 0;
+      if (t < a.T) {
+        top.write(a.idx + static_cast<size_t>(t) * a.k, a.gate + static_cast<size_t>(t) * a.k, a.k);
+        if (nan) report_status(a.status, MOE_STATUS_NAN_LOGIT);
+      }
     }
   } else if (threadIdx.x == 0) {
     report_status(a.status, MOE_STATUS_TIMEOUT);
@@ -244,7 +273,7 @@ __global__ void __launch_bounds__(256) router_f32_kernel(const float* __restrict
           nan = true;
           x = -INFINITY;
         }
-        top.push(x, e, a.k);
+        top.push_ascending(x, e, a.k);
       }
       top.write(a.idx + static_cast<size_t>(t) * a.k, a.gate + static_cast<size_t>(t) * a.k, a.k);
       if (nan) report_status(a.status, MOE_STATUS_NAN_LOGIT);
@@ -272,7 +301,7 @@ cudaError_t launch_router_tc(const CUtensorMap& tm_h, const CUtensorMap& tm_w, i
                                          static_cast<int>(smem));
   if (err != cudaSuccess) return err;
   const int grid = (T + kTileM - 1) / kTileM;
-  router_tc_kernel<<<grid, 128, smem, s>>>(tm_h, tm_w, a);
+  router_tc_kernel<<<grid, 256, smem, s>>>(tm_h, tm_w, a);
   return cudaGetLastError();
 }
 

@@ -333,3 +333,32 @@ def test_workspace_guard_bytes_untouched():
     dc.layer(ws=ws[:need])
     torch.cuda.synchronize()
     assert bool((ws[need:] == 0x5A).all())
+
+
+def test_layer_replays_from_a_cuda_graph():
+    """The whole layer is stream-ordered with no host synchronisation, so it
+    captures into a CUDA graph; replays match eager runs bit for bit, also
+    after new tokens are copied into the captured input buffer."""
+    dc = dev_case("small_skewed_capacity")
+    wl = dc.wl
+    h_static = dc.h.clone()
+    y_static = torch.empty((wl.T, wl.d), dtype=wl.torch_dtype, device=DEV)
+    ws = M.workspace(dc.cfg, M.MOE_OP_LAYER, DEV)
+
+    def run(h, y):
+        return M.moe_layer_forward(dc.cfg, h, dc.w_router, dc.bias, dc.w13, dc.w_down, y=y, ws=ws)
+
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        run(h_static, y_static)
+    torch.cuda.current_stream().wait_stream(side)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        run(h_static, y_static)
+    for h_new in (dc.h, dc.h.flip(0).contiguous()):
+        h_static.copy_(h_new)
+        graph.replay()
+        eager = run(h_new.clone(), torch.empty_like(y_static))
+        torch.cuda.synchronize()
+        assert torch.equal(y_static.view(torch.int16), eager.view(torch.int16))

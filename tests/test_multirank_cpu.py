@@ -1,0 +1,59 @@
+"""The multi-GPU bench path on CPU: two gloo ranks, token-sharded replicas.
+
+Each rank times its own batch; the job's device time is the slowest rank's,
+and throughput counts the tokens of every rank (weak scaling, no collective on
+the data path, only the max-reduce of the timings)."""
+import os
+import socket
+
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _worker(rank, world, port, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    import bench
+    ms_local = [12.0, 15.5][rank]
+    ms, value = bench.combine_ranks(ms_local, tokens_per_rank=1000, steps=4, world=world, device="cpu")
+    q.put((rank, ms, value))
+    dist.barrier()
+    dist.destroy_process_group()
+
+
+def test_two_gloo_ranks_take_the_slowest_rank_and_all_tokens():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = sorted(q.get(timeout=120) for _ in procs)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    for rank, ms, value in res:
+        assert ms == 15.5
+        assert value == pytest.approx(1000 * 2 * 4 / 15.5e-3)
+
+
+def test_single_rank_needs_no_process_group():
+    import bench
+    ms, value = bench.combine_ranks(10.0, 500, 3, 1)
+    assert ms == 10.0 and value == pytest.approx(500 * 3 / 10e-3)
+
+
+def test_launch_count_per_step():
+    import bench
+    import combine_router_gemm_softmax_b200 as M
+    assert bench.launches(M.config(64, 128, 8, 2, 128)) == 8
+    assert bench.launches(M.config(64, 128, 8, 2, 128, expert_kind="identity")) == 6
+    assert bench.launches(M.config(64, 128, 8, 2, 128, expert_kind="scale")) == 7
