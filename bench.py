@@ -54,6 +54,7 @@ def parse():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--gemm-tiles", choices=["auto", "single", "pair"], default="auto")
     return ap.parse_args()
 
 
@@ -248,7 +249,7 @@ def main():
     M.lib()
     inp = W.draw(wl, args.seed)
     h_host = W.draw_h(wl, args.seed + rank).pin_memory() if rank else inp.h.pin_memory()
-    cfg = M.config(wl.T, wl.d, wl.E, wl.k, wl.F, wl.dtype, wl.expert_kind, wl.capacity)
+    cfg = M.config(wl.T, wl.d, wl.E, wl.k, wl.F, wl.dtype, wl.expert_kind, wl.capacity, args.gemm_tiles)
     h = h_host.to(dev)
     wr = inp.w_router.to(dev)
     bias = None if inp.bias is None else inp.bias.to(dev)
@@ -339,7 +340,7 @@ def main():
             "warmup": max(args.warmup, 3), "ms_per_step": ms_max / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": wl.dtype,
             "data": "synthetic: seeded N(0,1) tokens, N(0,1/fan_in) random-init weights",
-            "config": config_dict(wl, world, flush),
+            "config": {**config_dict(wl, world, flush), "gemm_tiles": args.gemm_tiles},
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": wl.T * row_bytes,
                     "d2h_bytes_per_step": wl.T * row_bytes, "ms_per_step": e2e_ms / args.steps,
                     "path": "pinned host h -> device, moe_layer_forward, device y -> pinned host"},

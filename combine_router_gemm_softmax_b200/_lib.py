@@ -22,6 +22,7 @@ MOE_STATUS_NAN_LOGIT, MOE_STATUS_BAD_ROUTE, MOE_STATUS_TIMEOUT = 1, 2, 4
 MOE_DTYPE_BF16, MOE_DTYPE_F32 = 0, 1
 MOE_EXPERT_SWIGLU, MOE_EXPERT_IDENTITY, MOE_EXPERT_SCALE = 0, 1, 2
 MOE_OP_ROUTE, MOE_OP_PERMUTE, MOE_OP_GROUPED_FFN, MOE_OP_LAYER = 0, 1, 2, 3
+MOE_GEMM_TILES_AUTO, MOE_GEMM_TILES_SINGLE, MOE_GEMM_TILES_PAIR = 0, 1, 2
 MOE_MAX_E, MOE_MAX_K, MOE_PACK_BLOCK = 256, 8, 128
 
 EXPORTED = ("moe_workspace_size", "moe_status_string", "moe_version", "moe_pack_weights", "moe_route",
@@ -38,7 +39,7 @@ class MoeError(RuntimeError):
 class MoeConfig(ctypes.Structure):
     _fields_ = [("T", ctypes.c_int32), ("d", ctypes.c_int32), ("E", ctypes.c_int32), ("k", ctypes.c_int32),
                 ("d_ff", ctypes.c_int32), ("dtype", ctypes.c_int32), ("expert_kind", ctypes.c_int32),
-                ("capacity", ctypes.c_int32)]
+                ("capacity", ctypes.c_int32), ("gemm_tiles", ctypes.c_int32)]
 
     def __repr__(self):
         return "MoeConfig(" + ", ".join(f"{n}={getattr(self, n)}" for n, _ in self._fields_) + ")"
@@ -87,11 +88,12 @@ def lib() -> ctypes.CDLL:
     return _lib
 
 
-def config(T, d, E, k, d_ff, dtype="bf16", expert_kind="swiglu", capacity=-1) -> MoeConfig:
+def config(T, d, E, k, d_ff, dtype="bf16", expert_kind="swiglu", capacity=-1, gemm_tiles="auto") -> MoeConfig:
     dt = {"bf16": MOE_DTYPE_BF16, "f32": MOE_DTYPE_F32, torch.bfloat16: MOE_DTYPE_BF16,
           torch.float32: MOE_DTYPE_F32}[dtype]
     kind = {"swiglu": MOE_EXPERT_SWIGLU, "identity": MOE_EXPERT_IDENTITY, "scale": MOE_EXPERT_SCALE}[expert_kind]
-    return MoeConfig(T, d, E, k, d_ff, dt, kind, capacity)
+    tiles = {"auto": MOE_GEMM_TILES_AUTO, "single": MOE_GEMM_TILES_SINGLE, "pair": MOE_GEMM_TILES_PAIR}[gemm_tiles]
+    return MoeConfig(T, d, E, k, d_ff, dt, kind, capacity, tiles)
 
 
 def _ptr(t):

@@ -4,6 +4,7 @@
 #include <mutex>
 
 #include "moe_common.cuh"
+
 #include "moe_internal.h"
 
 namespace moe {
@@ -62,6 +63,7 @@ int check_cfg(const moe_config* c) {
   if (c->T < 0 || c->d <= 0 || c->E <= 0 || c->k <= 0 || c->capacity < -1) return MOE_ERR_INVALID_ARG;
   if (c->dtype != MOE_DTYPE_BF16 && c->dtype != MOE_DTYPE_F32) return MOE_ERR_INVALID_ARG;
   if (c->expert_kind < MOE_EXPERT_SWIGLU || c->expert_kind > MOE_EXPERT_SCALE) return MOE_ERR_INVALID_ARG;
+  if (c->gemm_tiles < MOE_GEMM_TILES_AUTO || c->gemm_tiles > MOE_GEMM_TILES_PAIR) return MOE_ERR_INVALID_ARG;
   if (c->expert_kind == MOE_EXPERT_SWIGLU && c->d_ff <= 0) return MOE_ERR_INVALID_ARG;
   if (c->E > MOE_MAX_E || c->k > MOE_MAX_K || c->k > c->E) return MOE_ERR_UNSUPPORTED;
   if (static_cast<long long>(c->T) * c->k >= (1LL << 31)) return MOE_ERR_UNSUPPORTED;
@@ -185,16 +187,21 @@ int ffn_impl(const moe_config& c, const void* x_perm, const int32_t* offsets, co
                                   static_cast<const float*>(w_down), static_cast<float*>(h_mid),
                                   static_cast<float*>(y_perm), rows_max, c.d, c.d_ff, c.E, s));
   const int F = c.d_ff, d = c.d, E = c.E;
+  // Tile shape: single-CTA 128x256 tiles unless the caller asks for CTA pairs
+  // (256x256, each CTA of the pair stages half of the B tile).
+  const bool pair = c.gemm_tiles == MOE_GEMM_TILES_PAIR;
   CUtensorMap a1, b1, a2, b2;
   int rc = make_map(&a1, x_perm, rows_max, d, kTileM);
-  if (rc == MOE_OK) rc = make_map(&b1, w13, static_cast<uint64_t>(E) * 2 * F, d, kGemmTileN);
+  if (rc == MOE_OK) rc = make_map(&b1, w13, static_cast<uint64_t>(E) * 2 * F, d, pair ? 128 : kGemmTileN);
   if (rc == MOE_OK) rc = make_map(&a2, h_mid, rows_max, F, kTileM);
-  if (rc == MOE_OK) rc = make_map(&b2, w_down, static_cast<uint64_t>(E) * d, F, kGemmTileN);
+  if (rc == MOE_OK) rc = make_map(&b2, w_down, static_cast<uint64_t>(E) * d, F, pair ? 128 : kGemmTileN);
   if (rc != MOE_OK) return rc;
-  cudaError_t e = launch_grouped_gemm_tc(a1, b1, true, offsets, E, d, 2 * F, F / 128, F, F, h_mid, status, s);
+  cudaError_t e = (pair ? launch_grouped_gemm_pair : launch_grouped_gemm_tc)(a1, b1, true, offsets, E, d, 2 * F,
+                                                                              F / 128, F, F, h_mid, status, s);
   if (e != cudaSuccess) return MOE_ERR_CUDA;
-  e = launch_grouped_gemm_tc(a2, b2, false, offsets, E, F, d, (d + kGemmTileN - 1) / kGemmTileN, d, d, y_perm,
-                             status, s);
+  e = (pair ? launch_grouped_gemm_pair : launch_grouped_gemm_tc)(a2, b2, false, offsets, E, F, d,
+                                                                  (d + kGemmTileN - 1) / kGemmTileN, d, d, y_perm,
+                                                                  status, s);
   return cuda_rc(e);
 }
 

@@ -304,6 +304,264 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   if (warp == 1) tmem_dealloc(tmem, kTmemCols);
 }
 
+// ------------------------------------------------------------------ CTA-pair variant
+// Same computation on 256 x 256 tiles shared by a pair of CTAs (a cluster of
+// two SMs). Each CTA loads its own 128 rows of A and 128 rows of B per K
+// slice into its own shared memory; the pair's leader issues one
+// tcgen05.mma.cta_group::2 per 16-deep step, reading both CTAs' operands, and
+// each CTA's TMEM receives its own 128 output rows x 256 columns. Per output
+// element this halves the B bytes every SM stages and the tile bytes the L2
+// serves, compared with the single-CTA 128 x 256 tile.
+//   barriers: full[s] lives in the leader and counts both CTAs' bytes; each
+//   CTA's empty[s] and tfull[a] are signalled by the leader's commit to both
+//   CTAs; tempty[a] lives in the leader and takes one arrival per epilogue
+//   warp of both CTAs (8).
+constexpr int kPairStages = 6;
+constexpr int kPairBM = 256;
+constexpr uint32_t kPairHalfBytes = 128 * kBK * 2;                 // one CTA's A or B slice
+constexpr uint32_t kPairPad = 16384;                               // keeps any operand over-read in bounds
+
+constexpr size_t pair_smem_bytes() {
+  return 1024 + 2 * kPairStages * static_cast<size_t>(kPairHalfBytes) + kPairPad + (2 * kPairStages + 5) * 8 + 16 +
+         2 * (kMaxE + 1) * 4;
+}
+
+template <bool kSwiGLU>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
+                             const GemmArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align_1024(smem_raw);
+  uint8_t* sB = smem;                                           // kPairStages x 16 KB
+  uint8_t* sA = smem + kPairStages * kPairHalfBytes;             // kPairStages x 16 KB
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + 2 * kPairStages * kPairHalfBytes + kPairPad);
+  uint64_t* empty = full + kPairStages;
+  uint64_t* tfull = empty + kPairStages;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* drain = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  int* consumed_slot = reinterpret_cast<int*>(tmem_slot + 2);
+  int* s_off = reinterpret_cast<int*>(tmem_slot + 4);
+  int* prefix = s_off + (kMaxE + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+  const int E = a.E;
+  const int nkb = a.K / kBK;
+  const uint32_t peer_abort = mapa_shared(smem_addr(const_cast<int*>(abort_flag)), rank ^ 1u);
+  auto raise_abort = [&]() {
+    *abort_flag = 1;
+    st_shared_cluster_u32(peer_abort, 1u);
+  };
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kPairStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&tfull[i], 1);
+      mbar_init(&tempty[i], 8);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    *consumed_slot = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(&tm_a);
+    tma_prefetch_desc(&tm_b);
+  }
+  for (int e = threadIdx.x; e <= E; e += blockDim.x) s_off[e] = a.offsets[e];
+  __syncthreads();
+  if (warp == 0) {
+    int loc[8];
+    int sum = 0;
+#pragma unroll
+    for (int v = 0; v < 8; ++v) {
+      const int e = lane * 8 + v;
+      loc[v] = e < E ? (s_off[e + 1] - s_off[e] + kPairBM - 1) / kPairBM : 0;
+      sum += loc[v];
+    }
+    int inc = sum;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int nb = __shfl_up_sync(0xffffffffu, inc, off);
+      if (lane >= off) inc += nb;
+    }
+    int run = inc - sum;
+#pragma unroll
+    for (int v = 0; v < 8; ++v) {
+      const int e = lane * 8 + v;
+      if (e < E) prefix[e] = run;
+      run += loc[v];
+    }
+    if (lane == 31) prefix[E] = inc;
+  } else if (warp == 1) {
+    tmem_alloc_pair(tmem_slot, kTmemCols);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  cluster_sync();  // both CTAs' barriers initialised before any cross-CTA signal
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const int m_total = prefix[E];
+  const long long total = static_cast<long long>(m_total) * a.n_tiles;
+  const int pair_id = blockIdx.x >> 1, n_pairs = gridDim.x >> 1;
+
+  int issued = 0;
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---------------------------------------------------------------- TMA producer (both CTAs)
+      const uint32_t full_leader = mapa_shared(smem_addr(&full[0]), 0);
+      int stage = 0;
+      uint32_t phase = 0;
+      bool stop = false;
+      for (long long tile = pair_id; tile < total && !stop; tile += n_pairs) {
+        int e, m, n;
+        decode_tile(tile, m_total, a.n_tiles, prefix, E, e, m, n);
+        const int a_row = s_off[e] + m * kPairBM + static_cast<int>(rank) * 128;
+        const int b_row = e * a.n_per_expert + n * kBN + static_cast<int>(rank) * 128;
+        for (int kb = 0; kb < nkb; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag)) {
+            raise_abort();
+            stop = true;
+            break;
+          }
+          if (leader) mbar_expect_tx(&full[stage], 4 * kPairHalfBytes);
+          tma_load_2d_pair(sA + stage * kPairHalfBytes, &tm_a, full_leader + stage * 8, kb * kBK, a_row);
+          tma_load_2d_pair(sB + stage * kPairHalfBytes, &tm_b, full_leader + stage * 8, kb * kBK, b_row);
+          ++issued;
+          if (++stage == kPairStages) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && leader) {
+      // ---------------------------------------------------------------- MMA issuer (leader only)
+      const uint32_t idesc = idesc_bf16_f32(kPairBM, kBN);
+      int stage = 0;
+      uint32_t phase = 0;
+      int consumed = 0, local = 0;
+      bool stop = false;
+      for (long long tile = pair_id; tile < total && !stop; tile += n_pairs, ++local) {
+        const int acc = local & 1;
+        const uint32_t acc_phase = (local >> 1) & 1;
+        if (!mbar_wait(&tempty[acc], acc_phase ^ 1, abort_flag)) {
+          raise_abort();
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem + acc * kBN;
+        for (int kb = 0; kb < nkb; ++kb) {
+          if (!mbar_wait(&full[stage], phase, abort_flag)) {
+            raise_abort();
+            stop = true;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sa = smem_addr(sA + stage * kPairHalfBytes);
+          const uint32_t sb = smem_addr(sB + stage * kPairHalfBytes);
+#pragma unroll
+          for (int kk = 0; kk < kBK / 16; ++kk)
+            umma_bf16_pair(d_tmem, sw128_kmajor_desc(sa + kk * 32), sw128_kmajor_desc(sb + kk * 32), idesc,
+                           (kb | kk) != 0);
+          umma_commit_pair_all(&empty[stage], 0x3);
+          ++consumed;
+          if (++stage == kPairStages) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+        if (!stop) umma_commit_pair_all(&tfull[acc], 0x3);
+      }
+      *consumed_slot = consumed;
+      umma_commit_pair(drain);
+      mbar_wait(drain, 0, nullptr);
+    }
+  } else {
+    // ---------------------------------------------------------------- epilogue (both CTAs)
+    const uint32_t tempty_leader = mapa_shared(smem_addr(&tempty[0]), 0);
+    const int q = warp & 3;
+    const int row = q * 32 + lane;
+    int local = 0;
+    for (long long tile = pair_id; tile < total; tile += n_pairs, ++local) {
+      int e, m, n;
+      decode_tile(tile, m_total, a.n_tiles, prefix, E, e, m, n);
+      const int acc = local & 1;
+      const uint32_t acc_phase = (local >> 1) & 1;
+      if (!mbar_wait(&tfull[acc], acc_phase, abort_flag)) {
+        raise_abort();
+        break;
+      }
+      tc_fence_after();
+      const int row0 = m * kPairBM + static_cast<int>(rank) * 128;  // first row of this CTA within the group
+      const int rows_valid = min(128, s_off[e + 1] - s_off[e] - row0);
+      const bool valid = row < rows_valid;
+      const size_t grow = static_cast<size_t>(s_off[e] + row0 + row);
+      const uint32_t tbase = tmem + acc * kBN + (static_cast<uint32_t>(q * 32) << 16);
+      if constexpr (kSwiGLU) {
+        __nv_bfloat16* out = a.D + grow * a.ldd + n * (kBN / 2);
+#pragma unroll 1
+        for (int c = 0; c < kBN / 2; c += 32) {
+          uint32_t g[32], u[32];
+          tmem_ld32(tbase + c, g);
+          tmem_ld32(tbase + kBN / 2 + c, u);
+          tmem_ld_wait();
+          if (valid) {
+            uint32_t p[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              const float h0 = silu_f(__uint_as_float(g[2 * i])) * __uint_as_float(u[2 * i]);
+              const float h1 = silu_f(__uint_as_float(g[2 * i + 1])) * __uint_as_float(u[2 * i + 1]);
+              p[i] = pack_bf16x2(h0, h1);
+            }
+            uint4* dst = reinterpret_cast<uint4*>(out + c);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) dst[i] = make_uint4(p[4 * i], p[4 * i + 1], p[4 * i + 2], p[4 * i + 3]);
+          }
+        }
+      } else {
+        __nv_bfloat16* out = a.D + grow * a.ldd + n * kBN;
+#pragma unroll 1
+        for (int c = 0; c < kBN; c += 32) {
+          if (n * kBN + c >= a.out_cols) break;
+          uint32_t v[32];
+          tmem_ld32(tbase + c, v);
+          tmem_ld_wait();
+          if (valid) {
+            uint32_t p[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) p[i] = pack_bf16x2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
+            uint4* dst = reinterpret_cast<uint4*>(out + c);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) dst[i] = make_uint4(p[4 * i], p[4 * i + 1], p[4 * i + 2], p[4 * i + 3]);
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(tempty_leader + acc * 8);
+    }
+  }
+  __syncwarp();
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (*abort_flag) {
+    if (threadIdx.x == 0) report_status(a.status, MOE_STATUS_TIMEOUT);
+    if (warp == 0 && lane == 0 && leader) {
+      for (int i = *consumed_slot; i < issued; ++i) mbar_wait(&full[i % kPairStages], (i / kPairStages) & 1, nullptr);
+    }
+  }
+  cluster_sync();  // neither CTA leaves while the pair's MMAs or signals may still touch it
+  if (warp == 1) tmem_dealloc_pair(tmem, kTmemCols);
+}
+
 // ------------------------------------------------------------------ helpers for the other paths
 MOE_DEV int expert_of_row(const int32_t* __restrict__ off, int E, int r) {
   int lo = 0, hi = E;  // off[lo] <= r < off[hi]
@@ -444,6 +702,40 @@ cudaError_t launch_grouped_gemm_tc(const CUtensorMap& tm_a, const CUtensorMap& t
     if (err != cudaSuccess) return err;
     grouped_gemm_kernel<false><<<grid, kGemmThreads, smem, s>>>(tm_a, tm_b, a);
   }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_grouped_gemm_pair(const CUtensorMap& tm_a, const CUtensorMap& tm_b, bool swiglu,
+                                     const int32_t* offsets, int E, int K, int n_per_expert, int n_tiles, int out_cols,
+                                     int ldd, void* D, int32_t* status, cudaStream_t s) {
+  GemmArgs a{offsets, E, K, n_per_expert, n_tiles, out_cols, ldd, static_cast<__nv_bfloat16*>(D), status};
+  const size_t smem = pair_smem_bytes();
+  const int grid = (device_sm_count() / 2) * 2;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid, 1, 1);
+  cfg.blockDim = dim3(kGemmThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t err;
+  if (swiglu) {
+    err = cudaFuncSetAttribute(grouped_gemm_pair_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(smem));
+    if (err != cudaSuccess) return err;
+    err = cudaLaunchKernelEx(&cfg, grouped_gemm_pair_kernel<true>, tm_a, tm_b, a);
+  } else {
+    err = cudaFuncSetAttribute(grouped_gemm_pair_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(smem));
+    if (err != cudaSuccess) return err;
+    err = cudaLaunchKernelEx(&cfg, grouped_gemm_pair_kernel<false>, tm_a, tm_b, a);
+  }
+  if (err != cudaSuccess) return err;
   return cudaGetLastError();
 }
 

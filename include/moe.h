@@ -75,6 +75,15 @@ extern "C" {
 #define MOE_EXPERT_IDENTITY 1  /* f_e(x) = x       (test expert) */
 #define MOE_EXPERT_SCALE    2  /* f_e(x) = (e+1) x (test expert) */
 
+/* Grouped-GEMM tiles (bf16 path). SINGLE: 128x256 tiles, one SM each. PAIR:
+ * 256x256 tiles shared by two SMs of a cluster (tcgen05 cta_group::2), which
+ * halves the operand bytes each SM stages but moves operands between the
+ * two SMs; under the 1 kW power cap it measured about 5% slower per layer on
+ * B200, so AUTO picks SINGLE. */
+#define MOE_GEMM_TILES_AUTO   0
+#define MOE_GEMM_TILES_SINGLE 1
+#define MOE_GEMM_TILES_PAIR   2
+
 #define MOE_OP_ROUTE       0
 #define MOE_OP_PERMUTE     1
 #define MOE_OP_GROUPED_FFN 2
@@ -93,6 +102,7 @@ typedef struct moe_config {
   int32_t dtype;        /* MOE_DTYPE_* */
   int32_t expert_kind;  /* MOE_EXPERT_* */
   int32_t capacity;     /* -1: dropless; >= 0: per-expert cap in assignments */
+  int32_t gemm_tiles;   /* MOE_GEMM_TILES_*: tile shape of the bf16 grouped GEMMs */
 } moe_config;
 
 typedef void* moe_stream_t; /* cudaStream_t */

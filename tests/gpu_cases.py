@@ -28,6 +28,15 @@ SMALL = {
         capacity=W.capacity_factor_cap(777, 4, 40)),
     "small_many": W.get("many_small").with_(
         name="small_many", T=640, d=256, E=128, k=8, F=256),
+    # CTA-pair GEMM tiles: 256-row tiles with a ragged last tile per expert
+    # (one CTA of the pair may have no valid rows), and d = 384 gives a
+    # half-empty second column tile in the down projection
+    "small_pair": W.get("mixtral_scaled").with_(
+        name="small_pair", T=2100, d=384, E=4, k=2, F=384, bias="gauss_0.5", gemm_tiles="pair"),
+    "small_pair_wide": W.get("mixtral_scaled").with_(
+        name="small_pair_wide", T=2100, d=2048, E=4, k=2, F=640, bias="gauss_0.5", gemm_tiles="pair"),
+    "small_skewed_pair": W.get("skewed").with_(
+        name="small_skewed_pair", T=777, d=256, E=40, k=4, F=384, gemm_tiles="pair"),
 }
 
 
@@ -36,7 +45,7 @@ def workload(name):
 
 
 def cfg_for(wl) -> M.MoeConfig:
-    return M.config(wl.T, wl.d, wl.E, wl.k, wl.F, wl.dtype, wl.expert_kind, wl.capacity)
+    return M.config(wl.T, wl.d, wl.E, wl.k, wl.F, wl.dtype, wl.expert_kind, wl.capacity, wl.gemm_tiles)
 
 
 @functools.lru_cache(maxsize=3)

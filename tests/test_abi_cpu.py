@@ -86,6 +86,15 @@ def test_config_rejected_before_any_cuda_call(L, kw, code):
     assert rc == code
 
 
+def test_gemm_tiles_value_checked(L):
+    cfg = M.config(64, 128, 8, 2, 256)
+    cfg.gemm_tiles = 7
+    assert L.moe_route(ctypes.byref(cfg), None, None, None, None, None, None, None, 0, None, None) \
+        == M.MOE_ERR_INVALID_ARG
+    for tiles in ("auto", "single", "pair"):
+        assert M.moe_workspace_size(M.config(64, 128, 8, 2, 256, gemm_tiles=tiles), M.MOE_OP_LAYER) > 0
+
+
 def test_null_pointers_rejected(L):
     cfg = M.config(64, 128, 8, 2, 256)
     assert L.moe_route(ctypes.byref(cfg), None, None, None, None, None, None, None, 0, None, None) \

@@ -19,10 +19,10 @@ from gpu_cases import DEV, DeviceCase, cfg_for, np64, np_, oracle_y, parity_case
 pytestmark = pytest.mark.gpu
 
 LAYER_CASES = ["tiny_f32", "tiny_f32_tagged", "small_ragged", "small_skewed", "small_skewed_capacity",
-               "small_many", "mixtral_scaled", "skewed", "skewed_capacity", "many_small", "many_small_identity",
+               "small_many", "small_pair", "small_pair_wide", "small_skewed_pair", "mixtral_scaled", "skewed", "skewed_capacity", "many_small", "many_small_identity",
                "mixtral_8x7b"]
 FULL_ORACLE = {"tiny_f32", "tiny_f32_tagged", "small_ragged", "small_skewed", "small_skewed_capacity",
-               "small_many", "many_small_identity"}
+               "small_many", "small_pair", "small_pair_wide", "small_skewed_pair", "many_small_identity"}
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -211,7 +211,8 @@ def test_permute_zero_tokens():
 
 
 # ------------------------------------------------------------------ grouped FFN (fed by the oracle's dispatch)
-@pytest.mark.parametrize("name", ["tiny_f32", "small_ragged", "small_skewed", "small_many", "mixtral_scaled"])
+@pytest.mark.parametrize("name", ["tiny_f32", "small_ragged", "small_skewed", "small_many", "small_pair",
+                                  "small_pair_wide", "mixtral_scaled"])
 def test_grouped_ffn_matches_oracle(name):
     dc = dev_case(name)
     inp, ref = parity_case(name)

@@ -51,6 +51,7 @@ class Workload:
     capacity: -1 for dropless, else the per-expert cap in assignments.
     expert_kind: "swiglu" | "identity" | "scale"
     tagged: identity-tagged tokens h_t = (t+1) * onehot(t mod d).
+    gemm_tiles: "auto" | "single" | "pair" (tile shape of the grouped GEMMs).
     """
 
     name: str
@@ -64,6 +65,7 @@ class Workload:
     capacity: int = -1
     expert_kind: str = "swiglu"
     tagged: bool = False
+    gemm_tiles: str = "auto"
     note: str = ""
 
     @property
