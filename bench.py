@@ -309,22 +309,12 @@ def main():
     st = int(status.item())
 
     # ------------------------------------------------ end to end: host buffers, copies inside the timed region
-    y_host = torch.empty((wl.T, wl.d), dtype=wl.torch_dtype, pin_memory=True)
-    for _ in range(2):
-        h.copy_(h_host, non_blocking=True)
-        step()
-        y_host.copy_(y, non_blocking=True)
-    torch.cuda.synchronize()
-    barrier()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(args.steps):
-        h.copy_(h_host, non_blocking=True)
-        step()
-        y_host.copy_(y, non_blocking=True)
-    e1.record(stream)
-    torch.cuda.synchronize()
-    e2e_ms, e2e_value = combine_ranks(e0.elapsed_time(e1), wl.T, args.steps, world, dev)
+    # Every step copies its tokens from pinned host memory to the device, runs
+    # the layer and copies its result back. Two device slots and separate copy
+    # streams let step i+1's upload and step i-1's download overlap step i's
+    # compute, as a serving loop would run it.
+    e2e_ms = run_e2e(M, cfg, wl, h_host, h, y, wr, bias, w13, wd, ws, stream, dev, args.steps, barrier)
+    e2e_ms, e2e_value = combine_ranks(e2e_ms, wl.T, args.steps, world, dev)
     row_bytes = wl.d * wl.elem_bytes
 
     # ------------------------------------------------ per stage (same stream, CUDA events)
@@ -343,7 +333,9 @@ def main():
             "config": {**config_dict(wl, world, flush), "gemm_tiles": args.gemm_tiles},
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": wl.T * row_bytes,
                     "d2h_bytes_per_step": wl.T * row_bytes, "ms_per_step": e2e_ms / args.steps,
-                    "path": "pinned host h -> device, moe_layer_forward, device y -> pinned host"},
+                    "path": "pinned host h -> device, moe_layer_forward, device y -> pinned host; "
+                            "two device slots, upload and download on their own streams overlap the "
+                            "neighbouring steps' compute"},
             "gpu_launches": launches_per_step * args.steps,
             "clocks": sampler.summary(),
             "status_word": st,
@@ -363,6 +355,50 @@ def main():
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.destroy_process_group()
+
+
+def run_e2e(M, cfg, wl, h_host, h0, y0, wr, bias, w13, wd, ws, stream, dev, steps, barrier):
+    """Device time of `steps` host-to-host layer steps (upload, layer, download),
+    double-buffered over two device slots. Returns milliseconds."""
+    import torch
+
+    s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    h_dev = [h0, torch.empty_like(h0)]
+    y_dev = [y0, torch.empty_like(y0)]
+    y_host = [torch.empty(y0.shape, dtype=y0.dtype, pin_memory=True) for _ in range(2)]
+    ev = {k: [torch.cuda.Event() for _ in range(2)] for k in ("in", "comp", "out")}
+
+    def run(n):
+        for i in range(n):
+            sl = i % 2
+            if i >= 2:
+                s_in.wait_event(ev["comp"][sl])          # slot's previous step has read its tokens
+            with torch.cuda.stream(s_in):
+                h_dev[sl].copy_(h_host, non_blocking=True)
+            ev["in"][sl].record(s_in)
+            stream.wait_event(ev["in"][sl])
+            if i >= 2:
+                stream.wait_event(ev["out"][sl])         # slot's previous result has been downloaded
+            M.moe_layer_forward(cfg, h_dev[sl], wr, bias, w13, wd, y=y_dev[sl], ws=ws, stream=stream)
+            ev["comp"][sl].record(stream)
+            s_out.wait_event(ev["comp"][sl])
+            with torch.cuda.stream(s_out):
+                y_host[sl].copy_(y_dev[sl], non_blocking=True)
+            ev["out"][sl].record(s_out)
+        for sl in range(min(n, 2)):
+            stream.wait_event(ev["out"][sl])
+
+    run(2)
+    torch.cuda.synchronize()
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    s_in.wait_event(e0)
+    s_out.wait_event(e0)
+    run(steps)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1)
 
 
 def launches(cfg):
