@@ -402,10 +402,15 @@ def run_e2e(M, cfg, wl, h_host, h0, y0, wr, bias, w13, wd, ws, stream, dev, step
 
 
 def launches(cfg):
-    """Kernels one moe_layer_forward launches (router, count, scan, rank, copy,
-    expert stage, combine)."""
+    """Kernels one moe_layer_forward launches: router (which also counts the
+    experts per 128-token tile on the bf16 path; the fp32 path adds a count
+    kernel), a separate scan only for large E * ceil(T/128), rank, row copy,
+    the expert stage and the combine."""
+    n_chunks = (cfg.T + 127) // 128
+    count = 0 if cfg.dtype == 0 else 1
+    scan = 0 if cfg.E * n_chunks <= 8192 else 1
     ffn = {0: 2, 1: 0, 2: 1}[cfg.expert_kind]
-    return 5 + ffn + 1
+    return 1 + count + scan + 1 + 1 + ffn + 1
 
 
 def stage_times(M, cfg, wl, h, wr, bias, w13, wd, dev, stream, reps):

@@ -154,8 +154,10 @@ size_t ws_size(const moe_config& c, int op) {
 
 int cuda_rc(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
 
+// chunk_counts (may be NULL, bf16 path only): the router also writes the
+// expert histogram of every 128-token tile, which the dispatch needs.
 int route_impl(const moe_config& c, const void* h, const void* w_router, const float* bias, float* logits,
-               int32_t* idx, float* gate, int32_t* status, cudaStream_t s) {
+               int32_t* idx, float* gate, int32_t* chunk_counts, int32_t* status, cudaStream_t s) {
   if (c.T == 0) return MOE_OK;
   if (c.dtype == MOE_DTYPE_F32)
     return cuda_rc(launch_router_f32(static_cast<const float*>(h), static_cast<const float*>(w_router), c.T, c.d, c.E,
@@ -165,15 +167,16 @@ int route_impl(const moe_config& c, const void* h, const void* w_router, const f
   int rc = make_map(&tm_h, h, c.T, c.d, kTileM);
   if (rc == MOE_OK) rc = make_map(&tm_w, w_router, c.E, c.d, npad);
   if (rc != MOE_OK) return rc;
-  return cuda_rc(launch_router_tc(tm_h, tm_w, c.T, c.d, c.E, c.k, npad, bias, logits, idx, gate, status, s));
+  return cuda_rc(
+      launch_router_tc(tm_h, tm_w, c.T, c.d, c.E, c.k, npad, bias, logits, idx, gate, chunk_counts, status, s));
 }
 
 int permute_impl(const moe_config& c, const void* h, const int32_t* idx, int32_t* routed, int32_t* kept,
                  int32_t* offsets, int32_t* dest_row, int32_t* perm_src, void* x_perm, const PermuteScratch& p,
-                 int32_t* status, cudaStream_t s) {
+                 bool counts_ready, int32_t* status, cudaStream_t s) {
   return cuda_rc(launch_permute(h, static_cast<size_t>(c.d) * elem_bytes(c), idx, c.T, c.k, c.E, c.capacity,
                                 p.chunk_counts, p.chunk_base, routed, kept, offsets, dest_row, perm_src, x_perm,
-                                status, s));
+                                counts_ready, status, s));
 }
 
 int ffn_impl(const moe_config& c, const void* x_perm, const int32_t* offsets, const void* w13, const void* w_down,
@@ -261,7 +264,7 @@ int32_t moe_route(const moe_config* cfg, const void* h, const void* w_router, co
   if (!aligned(h, 16) || !aligned(w_router, 16) || !aligned(topk_idx, 4) || !aligned(topk_gate, 4) ||
       !aligned(bias, 4) || !aligned(logits_out, 4) || !aligned(status_dev, 4))
     return MOE_ERR_UNSUPPORTED;
-  return route_impl(*cfg, h, w_router, bias, logits_out, topk_idx, topk_gate, status_dev,
+  return route_impl(*cfg, h, w_router, bias, logits_out, topk_idx, topk_gate, nullptr, status_dev,
                     static_cast<cudaStream_t>(stream));
 }
 
@@ -281,8 +284,8 @@ int32_t moe_permute(const moe_config* cfg, const void* h, const int32_t* topk_id
   if (ws_bytes < need || (need > 0 && (!workspace || !aligned(workspace, 16)))) return MOE_ERR_WORKSPACE;
   Carver w(workspace);
   const PermuteScratch p = carve_permute(*cfg, w);
-  return permute_impl(*cfg, h, topk_idx, routed_counts, counts, offsets, dest_row, perm_src, x_perm, p, status_dev,
-                      static_cast<cudaStream_t>(stream));
+  return permute_impl(*cfg, h, topk_idx, routed_counts, counts, offsets, dest_row, perm_src, x_perm, p, false,
+                      status_dev, static_cast<cudaStream_t>(stream));
 }
 
 int32_t moe_grouped_ffn(const moe_config* cfg, const void* x_perm, const int32_t* offsets, const void* w13_packed,
@@ -338,10 +341,13 @@ int32_t moe_layer_forward(const moe_config* cfg, const void* h, const void* w_ro
   if (routed_counts) b.routed = routed_counts;
   if (counts) b.kept = counts;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  rc = route_impl(c, h, w_router, bias, nullptr, b.idx, b.gate, status_dev, s);
+  // the bf16 router also writes the per-tile expert histogram the dispatch needs
+  const bool router_counts = c.dtype == MOE_DTYPE_BF16;
+  rc = route_impl(c, h, w_router, bias, nullptr, b.idx, b.gate, router_counts ? b.perm.chunk_counts : nullptr,
+                  status_dev, s);
   if (rc != MOE_OK) return rc;
-  rc = permute_impl(c, h, b.idx, b.routed, b.kept, b.offsets, b.dest_row, b.perm_src, b.x_perm, b.perm, status_dev,
-                    s);
+  rc = permute_impl(c, h, b.idx, b.routed, b.kept, b.offsets, b.dest_row, b.perm_src, b.x_perm, b.perm,
+                    router_counts, status_dev, s);
   if (rc != MOE_OK) return rc;
   const void* y_src = b.x_perm;
   if (c.expert_kind != MOE_EXPERT_IDENTITY) {

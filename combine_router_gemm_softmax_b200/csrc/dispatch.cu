@@ -6,11 +6,13 @@
 // resolved in token order as in "How Does Mixture-of-Experts Routing Affect
 // LLM Repeatability?"; archcrux "moe-unpermute-wrong-token" for the return.)
 //
-// Everything stays on the device: four kernels, no host synchronisation.
+// Everything stays on the device, no host synchronisation:
 //   count : per 128-token chunk, a histogram over experts (shared atomics;
-//           only the totals are used, so their order does not matter)
-//   scan  : one CTA; per expert an exclusive scan over chunks (the stable
-//           base rank of each chunk), then kept counts and offsets
+//           only the totals are used, so their order does not matter). In
+//           the whole-layer path the router's epilogue writes these counts.
+//   scan  : per expert an exclusive scan over chunks (the stable base rank of
+//           each chunk), then kept counts and offsets. Done inside every rank
+//           CTA when the counts matrix is small, else by one separate CTA.
 //   rank  : per chunk, every slot's rank among earlier tokens of the same
 //           expert, from per-warp bitmasks (popc), giving dest_row/perm_src
 //   copy  : TMA bulk copies: each token row is bulk-loaded into shared memory
@@ -57,7 +59,7 @@ __global__ void __launch_bounds__(kChunkTokens) count_kernel(const int32_t* __re
   }
   __syncthreads();
   for (int e = threadIdx.x; e < E; e += blockDim.x)
-    chunk_counts[static_cast<size_t>(e) * n_chunks + blockIdx.x] = hist[e];
+    chunk_counts[static_cast<size_t>(blockIdx.x) * E + e] = hist[e];
 }
 
 constexpr int kScanPerLane = 8;
@@ -69,10 +71,8 @@ __global__ void __launch_bounds__(1024) scan_kernel(const int32_t* __restrict__ 
   __shared__ int s_kept[kMaxE];
   __shared__ int s_warp[8];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  // one warp per expert column: exclusive scan over chunks
+  // one warp per expert column: exclusive scan over chunks (tables are [chunk][E])
   for (int e = warp; e < E; e += 32) {
-    const int32_t* col = chunk_counts + static_cast<size_t>(e) * n_chunks;
-    int32_t* base = chunk_base + static_cast<size_t>(e) * n_chunks;
     int carry = 0;
     for (int c0 = 0; c0 < n_chunks; c0 += 32 * kScanPerLane) {
       int vals[kScanPerLane];
@@ -80,7 +80,7 @@ __global__ void __launch_bounds__(1024) scan_kernel(const int32_t* __restrict__ 
 #pragma unroll
       for (int v = 0; v < kScanPerLane; ++v) {
         const int c = c0 + lane * kScanPerLane + v;
-        vals[v] = c < n_chunks ? col[c] : 0;
+        vals[v] = c < n_chunks ? chunk_counts[static_cast<size_t>(c) * E + e] : 0;
         sum += vals[v];
       }
       int inc = sum;
@@ -93,7 +93,7 @@ __global__ void __launch_bounds__(1024) scan_kernel(const int32_t* __restrict__ 
 #pragma unroll
       for (int v = 0; v < kScanPerLane; ++v) {
         const int c = c0 + lane * kScanPerLane + v;
-        if (c < n_chunks) base[c] = run;
+        if (c < n_chunks) chunk_base[static_cast<size_t>(c) * E + e] = run;
         run += vals[v];
       }
       carry += __shfl_sync(0xffffffffu, inc, 31);
@@ -126,19 +126,107 @@ __global__ void __launch_bounds__(1024) scan_kernel(const int32_t* __restrict__ 
   }
 }
 
-__global__ void __launch_bounds__(kChunkTokens) rank_kernel(const int32_t* __restrict__ idx, int T, int k, int E,
-                                                            int cap, int n_chunks,
-                                                            const int32_t* __restrict__ chunk_base,
-                                                            const int32_t* __restrict__ offsets,
-                                                            int32_t* __restrict__ dest_row,
-                                                            int32_t* __restrict__ perm_src, int32_t* status) {
+// Chunk-counts matrices up to this many entries are scanned inside every rank
+// CTA (each CTA needs its chunk's base rank for every expert and the offsets);
+// larger ones go through scan_kernel first.
+constexpr int kFusedScanMax = 8192;
+
+MOE_DEV int warp_sum(int v) {
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+  return v;
+}
+
+// Ranks of one 128-token chunk: rank(t,j) = tokens before t (in earlier
+// chunks, then in earlier warps of this chunk, then in lower lanes) that
+// picked the same expert. With kFusedScan the chunk bases and offsets are
+// computed here from the per-chunk counts, and CTA 0 writes the counts and
+// offsets; otherwise they come from scan_kernel.
+template <bool kFusedScan>
+__global__ void __launch_bounds__(kChunkTokens) rank_kernel(
+    const int32_t* __restrict__ idx, int T, int k, int E, int cap, int n_chunks,
+    const int32_t* __restrict__ chunk_table,  // counts [n_chunks][E] (fused) or bases [n_chunks][E]
+    const int32_t* __restrict__ offsets_in, int32_t* __restrict__ routed_out, int32_t* __restrict__ kept_out,
+    int32_t* __restrict__ offsets_out, int32_t* __restrict__ dest_row, int32_t* __restrict__ perm_src,
+    int32_t* status) {
   constexpr int kWarps = kChunkTokens / 32;
   __shared__ uint32_t mask[kWarps][kMaxE];
   __shared__ int wbase[kWarps][kMaxE];
+  __shared__ int s_base[kMaxE];
+  __shared__ int s_kept[kMaxE];
+  __shared__ int s_off[kMaxE + 1];
+  __shared__ int s_warp[kWarps];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int chunk = blockIdx.x;
   for (int i = threadIdx.x; i < kWarps * kMaxE; i += blockDim.x) (&mask[0][0])[i] = 0u;
+
+  if constexpr (kFusedScan) {
+    // per expert: tokens of earlier chunks (this chunk's base rank) and the
+    // total. Each expert's chunks are split over 128/E threads so that every
+    // thread has a few independent, coalesced loads in flight.
+    __shared__ int p_before[kChunkTokens], p_tot[kChunkTokens];
+    for (int e_base = 0; e_base < E; e_base += kChunkTokens) {
+      const int ne = min(E - e_base, kChunkTokens);
+      const int groups = kChunkTokens / ne;
+      int before = 0, tot = 0;
+      if (threadIdx.x < groups * ne) {
+        const int e = e_base + threadIdx.x % ne, g = threadIdx.x / ne;
+#pragma unroll 8
+        for (int c = g; c < n_chunks; c += groups) {
+          const int v = chunk_table[static_cast<size_t>(c) * E + e];
+          tot += v;
+          before += c < chunk ? v : 0;
+        }
+      }
+      p_before[threadIdx.x] = before;
+      p_tot[threadIdx.x] = tot;
+      __syncthreads();
+      if (threadIdx.x < ne) {
+        int b = 0, tt = 0;
+        for (int g = 0; g < groups; ++g) {
+          b += p_before[g * ne + threadIdx.x];
+          tt += p_tot[g * ne + threadIdx.x];
+        }
+        const int e = e_base + threadIdx.x;
+        s_base[e] = b;
+        s_kept[e] = cap < 0 ? tt : min(tt, cap);
+        if (chunk == 0) {
+          routed_out[e] = tt;
+          kept_out[e] = s_kept[e];
+        }
+      }
+      __syncthreads();
+    }
+    __syncthreads();
+    // offsets: exclusive scan of kept counts, two experts per thread
+    const int e0 = 2 * threadIdx.x;
+    const int v0 = e0 < E ? s_kept[e0] : 0, v1 = e0 + 1 < E ? s_kept[e0 + 1] : 0;
+    int inc = v0 + v1;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int nb = __shfl_up_sync(0xffffffffu, inc, off);
+      if (lane >= off) inc += nb;
+    }
+    if (lane == 31) s_warp[warp] = inc;
+    __syncthreads();
+    int before = 0;
+    for (int w = 0; w < warp; ++w) before += s_warp[w];
+    const int excl = before + inc - v0 - v1;
+    if (e0 < E) s_off[e0] = excl;
+    if (e0 + 1 < E) s_off[e0 + 1] = excl + v0;
+    if (threadIdx.x == blockDim.x - 1) s_off[E] = before + inc;
+    __syncthreads();
+    if (chunk == 0)
+      for (int e = threadIdx.x; e <= E; e += blockDim.x) offsets_out[e] = s_off[e];
+  } else {
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+      s_base[e] = chunk_table[static_cast<size_t>(chunk) * E + e];
+      s_off[e] = offsets_in[e];
+    }
+  }
   __syncthreads();
-  const int t = blockIdx.x * kChunkTokens + threadIdx.x;
+
+  const int t = chunk * kChunkTokens + threadIdx.x;
   int ev[kMaxK];
   uint32_t valid = 0;
   if (t < T) {
@@ -165,10 +253,9 @@ __global__ void __launch_bounds__(kChunkTokens) rank_kernel(const int32_t* __res
       int dest = -1;
       if (valid & (1u << j)) {
         const int e = ev[j];
-        const int r = chunk_base[static_cast<size_t>(e) * n_chunks + blockIdx.x] + wbase[warp][e] +
-                      __popc(mask[warp][e] & lt);
+        const int r = s_base[e] + wbase[warp][e] + __popc(mask[warp][e] & lt);
         if (cap < 0 || r < cap) {
-          dest = offsets[e] + r;
+          dest = s_off[e] + r;
           perm_src[dest] = t;
         }
       }
@@ -378,13 +465,21 @@ int warp_grid(int T) {
 cudaError_t launch_permute(const void* h, size_t row_bytes, const int32_t* idx, int T, int k, int E, int cap,
                            int32_t* chunk_counts, int32_t* chunk_base, int32_t* routed, int32_t* kept,
                            int32_t* offsets, int32_t* dest_row, int32_t* perm_src, void* x_perm,
-                           int32_t* status, cudaStream_t s) {
+                           bool counts_ready, int32_t* status, cudaStream_t s) {
   const int n_chunks = (T + kChunkTokens - 1) / kChunkTokens;
-  if (n_chunks > 0) count_kernel<<<n_chunks, kChunkTokens, 0, s>>>(idx, T, k, E, n_chunks, chunk_counts);
-  scan_kernel<<<1, 1024, 0, s>>>(chunk_counts, chunk_base, n_chunks, E, cap, routed, kept, offsets);
+  if (n_chunks > 0 && !counts_ready)
+    count_kernel<<<n_chunks, kChunkTokens, 0, s>>>(idx, T, k, E, n_chunks, chunk_counts);
+  const bool fused = n_chunks > 0 && static_cast<long long>(E) * n_chunks <= kFusedScanMax;
+  if (fused) {
+    rank_kernel<true><<<n_chunks, kChunkTokens, 0, s>>>(idx, T, k, E, cap, n_chunks, chunk_counts, nullptr, routed,
+                                                        kept, offsets, dest_row, perm_src, status);
+  } else {
+    scan_kernel<<<1, 1024, 0, s>>>(chunk_counts, chunk_base, n_chunks, E, cap, routed, kept, offsets);
+    if (n_chunks > 0)
+      rank_kernel<false><<<n_chunks, kChunkTokens, 0, s>>>(idx, T, k, E, cap, n_chunks, chunk_base, offsets,
+                                                           nullptr, nullptr, nullptr, dest_row, perm_src, status);
+  }
   if (n_chunks > 0) {
-    rank_kernel<<<n_chunks, kChunkTokens, 0, s>>>(idx, T, k, E, cap, n_chunks, chunk_base, offsets, dest_row,
-                                                  perm_src, status);
     const int tpc = kCopyTokensPerCta;
     const int piece = static_cast<int>(row_bytes < kCopyPiece ? row_bytes : kCopyPiece);
     const size_t smem = 128 + static_cast<size_t>(kCopyBuffers) * piece + kCopyBuffers * 8 + tpc * k * 4;

@@ -19,9 +19,10 @@ constexpr int kGemmTileN = 256;
 int device_sm_count();
 
 // router.cu
+// chunk_counts (may be NULL): per-128-token-tile expert histogram [ceil(T/128)][E].
 cudaError_t launch_router_tc(const CUtensorMap& tm_h, const CUtensorMap& tm_w, int T, int d, int E, int k,
                              int npad, const float* bias, float* logits, int32_t* idx, float* gate,
-                             int32_t* status, cudaStream_t s);
+                             int32_t* chunk_counts, int32_t* status, cudaStream_t s);
 cudaError_t launch_router_f32(const float* h, const float* w, int T, int d, int E, int k, const float* bias,
                               float* logits, int32_t* idx, float* gate, int32_t* status, cudaStream_t s);
 
@@ -29,7 +30,7 @@ cudaError_t launch_router_f32(const float* h, const float* w, int T, int d, int 
 cudaError_t launch_permute(const void* h, size_t row_bytes, const int32_t* idx, int T, int k, int E, int cap,
                            int32_t* chunk_counts, int32_t* chunk_base, int32_t* routed, int32_t* kept,
                            int32_t* offsets, int32_t* dest_row, int32_t* perm_src, void* x_perm,
-                           int32_t* status, cudaStream_t s);
+                           bool counts_ready, int32_t* status, cudaStream_t s);
 cudaError_t launch_combine(int dtype, const void* y_perm, const int32_t* dest_row, const float* gate, void* y,
                            int T, int k, int d, cudaStream_t s);
 

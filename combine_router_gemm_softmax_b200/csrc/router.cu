@@ -94,10 +94,12 @@ struct RouterArgs {
   float* logits;
   int32_t* idx;
   float* gate;
+  int32_t* chunk_counts;  // [n_tiles][E] expert histogram per 128-token tile, or NULL
+  int n_tiles;
   int32_t* status;
 };
 
-__global__ void __launch_bounds__(256) router_tc_kernel(const __grid_constant__ CUtensorMap tm_h,
+__global__ void __launch_bounds__(256, 2) router_tc_kernel(const __grid_constant__ CUtensorMap tm_h,
                                                         const __grid_constant__ CUtensorMap tm_w,
                                                         const RouterArgs a) {
   extern __shared__ uint8_t smem_raw[];
@@ -128,8 +130,10 @@ __global__ void __launch_bounds__(256) router_tc_kernel(const __grid_constant__ 
     tma_prefetch_desc(&tm_h);
     tma_prefetch_desc(&tm_w);
   }
+  __shared__ int s_hist[kMaxE];
   for (int e = threadIdx.x; e < a.npad; e += blockDim.x)
     sbias[e] = e >= a.E ? -INFINITY : (a.bias ? a.bias[e] : 0.f);
+  for (int e = threadIdx.x; e < a.E; e += blockDim.x) s_hist[e] = 0;
   if (warp == 0) {
     tmem_alloc(tmem_slot, a.tmem_cols);
     tmem_relinquish();
@@ -229,7 +233,17 @@ __global__ void __launch_bounds__(256) router_tc_kernel(const __grid_constant__ 
       if (t < a.T) {
         top.write(a.idx + static_cast<size_t>(t) * a.k, a.gate + static_cast<size_t>(t) * a.k, a.k);
         if (nan) report_status(a.status, MOE_STATUS_NAN_LOGIT);
+        if (a.chunk_counts != nullptr) {
+#pragma unroll
+          for (int j = 0; j < kMaxK; ++j)
+            if (j < a.k) atomicAdd(&s_hist[top.i[j]], 1);
+        }
       }
+    }
+    if (a.chunk_counts != nullptr) {
+      __syncthreads();
+      for (int e = threadIdx.x; e < a.E; e += blockDim.x)
+        a.chunk_counts[static_cast<size_t>(tile) * a.E + e] = s_hist[e];
     }
   } else if (threadIdx.x == 0) {
     report_status(a.status, MOE_STATUS_TIMEOUT);
@@ -292,15 +306,17 @@ uint32_t pow2_at_least(uint32_t x, uint32_t lo) {
 
 cudaError_t launch_router_tc(const CUtensorMap& tm_h, const CUtensorMap& tm_w, int T, int d, int E, int k,
                              int npad, const float* bias, float* logits, int32_t* idx, float* gate,
-                             int32_t* status, cudaStream_t s) {
+                             int32_t* chunk_counts, int32_t* status, cudaStream_t s) {
   if (T == 0) return cudaSuccess;
-  RouterArgs a{T, d, E, k, npad, static_cast<int>(pow2_at_least(npad, 32)), bias, logits, idx, gate, status};
+  const int grid = (T + kTileM - 1) / kTileM;
+  RouterArgs a{T,    d,      E,   k,    npad,         static_cast<int>(pow2_at_least(npad, 32)),
+               bias, logits, idx, gate, chunk_counts, grid,
+               status};
   const size_t stage_bytes = kRouterABytes + static_cast<size_t>(npad) * kRouterBK * 2;
   const size_t smem = 1024 + kRouterStages * stage_bytes + (2 * kRouterStages + 1) * 8 + 16 + kMaxE * 4;
   cudaError_t err = cudaFuncSetAttribute(router_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
   if (err != cudaSuccess) return err;
-  const int grid = (T + kTileM - 1) / kTileM;
   router_tc_kernel<<<grid, 256, smem, s>>>(tm_h, tm_w, a);
   return cudaGetLastError();
 }
@@ -308,7 +324,7 @@ cudaError_t launch_router_tc(const CUtensorMap& tm_h, const CUtensorMap& tm_w, i
 cudaError_t launch_router_f32(const float* h, const float* w, int T, int d, int E, int k, const float* bias,
                               float* logits, int32_t* idx, float* gate, int32_t* status, cudaStream_t s) {
   if (T == 0) return cudaSuccess;
-  RouterArgs a{T, d, E, k, E, 0, bias, logits, idx, gate, status};
+  RouterArgs a{T, d, E, k, E, 0, bias, logits, idx, gate, nullptr, 0, status};
   const int grid = (T + 7) / 8 < 4096 ? (T + 7) / 8 : 4096;
   router_f32_kernel<<<grid, 256, 8 * E * sizeof(float), s>>>(h, w, a);
   return cudaGetLastError();

@@ -192,7 +192,9 @@ def _routes(kind, T, E, k, seed=0):
 @pytest.mark.parametrize("kind,T,E,k,cap", [
     ("random", 1000, 8, 2, -1), ("random", 4097, 64, 6, -1), ("all_to_one", 700, 16, 3, -1),
     ("empty_experts", 513, 32, 4, -1), ("all_to_one", 700, 16, 3, 100), ("random", 999, 40, 4, 50),
-    ("bad", 300, 8, 2, -1), ("random", 1, 8, 2, -1), ("random", 128, 256, 8, -1), ("random", 300, 4, 4, 0)])
+    ("bad", 300, 8, 2, -1), ("random", 1, 8, 2, -1), ("random", 128, 256, 8, -1), ("random", 300, 4, 4, 0),
+    # E * ceil(T/128) > 8192: chunk bases come from the separate scan kernel
+    ("random", 8320, 256, 2, -1), ("all_to_one", 8320, 256, 3, 70)])
 def test_permute_injected_routes(kind, T, E, k, cap):
     _permute_check(T, 256, E, k, _routes(kind, T, E, k), cap)
 
