@@ -162,7 +162,7 @@ int route_impl(const moe_config& c, const void* h, const void* w_router, const f
   if (c.dtype == MOE_DTYPE_F32)
     return cuda_rc(launch_router_f32(static_cast<const float*>(h), static_cast<const float*>(w_router), c.T, c.d, c.E,
                                      c.k, bias, logits, idx, gate, status, s));
-  const int npad = ((c.E + 15) / 16) * 16;
+  const int npad = router_npad(c.E);
   CUtensorMap tm_h, tm_w;
   int rc = make_map(&tm_h, h, c.T, c.d, kTileM);
   if (rc == MOE_OK) rc = make_map(&tm_w, w_router, c.E, c.d, npad);

@@ -19,6 +19,12 @@ constexpr int kGemmTileN = 256;
 int device_sm_count();
 
 // router.cu
+// Padded expert count of the router's score tile: a multiple of 16, or of 32
+// from 49 experts on, where a CTA pair splits the reduction over d and each
+// CTA ranks half of the experts.
+constexpr int kRouterSplitMin = 64;
+inline int router_npad(int E) { return E > 48 ? (E + 31) / 32 * 32 : (E + 15) / 16 * 16; }
+inline bool router_splits_experts(int npad) { return npad >= kRouterSplitMin; }
 // chunk_counts (may be NULL): per-128-token-tile expert histogram [ceil(T/128)][E].
 cudaError_t launch_router_tc(const CUtensorMap& tm_h, const CUtensorMap& tm_w, int T, int d, int E, int k,
                              int npad, const float* bias, float* logits, int32_t* idx, float* gate,

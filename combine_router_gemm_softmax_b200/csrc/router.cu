@@ -3,13 +3,23 @@
 // LLM Repeatability?", the simplified token-choice layer and its note on
 // stable score ordering and deterministic tie handling).
 //
-// bf16 path: one CTA per 128 tokens. The score tile (128 tokens x E padded to
-// a multiple of 16) is a tcgen05 GEMM: TMA brings 128x64 slices of h and the
-// whole router weight slice into shared memory through a 4-stage mbarrier
-// pipeline, one thread issues the MMAs, the fp32 accumulator lives in TMEM.
-// The epilogue reads TMEM with the 32x32b shape, so each thread owns one
-// token's full score row and does bias, NaN handling, top-k and gates in
-// registers. The kernel streams h once: it is bound by HBM reads of h.
+// bf16 path: one CTA per 128 tokens computes the score tile (128 tokens x E
+// padded) as a tcgen05 GEMM: TMA brings 128x64 slices of h and the matching
+// slice of W_r into shared memory through an mbarrier ring, one thread issues
+// the MMAs, the fp32 accumulator lives in TMEM. The epilogue reads TMEM with
+// the 32x32b shape, so each thread owns one token row: bias, NaN handling,
+// top-k and gates happen in registers (8 warps: two per TMEM lane quadrant,
+// each taking every other 16-column chunk, their lists merged through shared
+// memory). The kernel streams h once and is bound by HBM reads of h.
+//
+// From 49 experts on, a pair of CTAs (a cluster of two) shares each tile and
+// splits the reduction: CTA r multiplies the r-th half of d for all experts,
+// so each CTA streams half of the tile's h and W_r. Each CTA then hands the
+// partner the partial scores of the experts the partner owns (through
+// distributed shared memory), adds the partner's half to its own experts'
+// scores, ranks its half of the experts, and rank 1 hands its top-k lists to
+// rank 0, which merges them and writes the result.
+#include <limits.h>
 #include <math.h>
 
 #include "moe_common.cuh"
@@ -19,77 +29,93 @@ namespace moe {
 
 namespace {
 
-constexpr int kRouterStages = 4;
+constexpr int kRouterMaxStages = 8;
 constexpr int kRouterBK = 64;
 constexpr uint32_t kRouterABytes = kTileM * kRouterBK * 2;
 
-// Running top-k of one token, sorted by (score descending, expert ascending).
-// Empty slots hold NaN, which compares false against everything, so they are
-// never ranked ahead of a candidate. An insertion counts the held entries
-// that stay ahead of the candidate (independent compares) and shifts the
-// tail down by one: no loop-carried chain through the k slots.
+// Top-K of one token under the order (score descending, expert ascending):
+// an unsorted set of K entries plus its worst entry (lowest score, ties to
+// the highest expert index). A candidate that does not beat the worst entry
+// costs one comparison; one that does replaces it, and the new worst entry is
+// found again. sort() puts the set in slot order at the end. Empty slots hold
+// (-inf, INT_MAX), which any real candidate beats.
+template <int K>
 struct TopList {
-  float v[kMaxK];
-  int i[kMaxK];
+  float v[K];
+  int i[K];
+  float wv;
+  int wi;
 
   MOE_DEV void init() {
 #pragma unroll
-    for (int j = 0; j < kMaxK; ++j) {
-      v[j] = __int_as_float(0x7fffffff);
-      i[j] = -1;
+    for (int j = 0; j < K; ++j) {
+      v[j] = -INFINITY;
+      i[j] = INT_MAX;
     }
+    wv = -INFINITY;
+    wi = INT_MAX;
   }
 
-  MOE_DEV void insert_at(int p, float x, int e) {
+  MOE_DEV void push(float x, int e) {
+    if (!(x > wv || (x == wv && e < wi))) return;
+    bool done = false;
 #pragma unroll
-    for (int j = kMaxK - 1; j >= 0; --j) {
-      const float pv = j > 0 ? v[j - 1] : x;
-      const int pi = j > 0 ? i[j - 1] : e;
-      const bool move = j > p, put = j == p;
-      v[j] = move ? pv : (put ? x : v[j]);
-      i[j] = move ? pi : (put ? e : i[j]);
+    for (int j = 0; j < K; ++j) {
+      const bool here = !done && v[j] == wv && i[j] == wi;
+      v[j] = here ? x : v[j];
+      i[j] = here ? e : i[j];
+      done = done || here;
     }
-  }
-
-  // Candidates of one list arrive in ascending expert index, so a held entry
-  // with an equal score stays ahead (lower index wins).
-  MOE_DEV void push_ascending(float x, int e, int k) {
-    int p = 0;
+    float nv = v[0];
+    int ni = i[0];
 #pragma unroll
-    for (int j = 0; j < kMaxK; ++j) p += (j < k && v[j] >= x) ? 1 : 0;
-    insert_at(p, x, e);
+    for (int j = 1; j < K; ++j) {
+      const bool worse = v[j] < nv || (v[j] == nv && i[j] > ni);
+      nv = worse ? v[j] : nv;
+      ni = worse ? i[j] : ni;
+    }
+    wv = nv;
+    wi = ni;
   }
 
-  // Candidate in any index order (merging another list); e < 0 is an empty slot.
-  MOE_DEV void push_any(float x, int e, int k) {
-    int p = 0;
+  MOE_DEV void sort() {
 #pragma unroll
-    for (int j = 0; j < kMaxK; ++j) p += (j < k && (v[j] > x || (v[j] == x && i[j] < e))) ? 1 : 0;
-    insert_at(e < 0 ? k : p, x, e);
+    for (int x = 1; x < K; ++x)
+#pragma unroll
+      for (int y = x; y > 0; --y) {
+        const bool sw = v[y] > v[y - 1] || (v[y] == v[y - 1] && i[y] < i[y - 1]);
+        const float tv = v[y];
+        const int ti = i[y];
+        v[y] = sw ? v[y - 1] : v[y];
+        i[y] = sw ? i[y - 1] : i[y];
+        v[y - 1] = sw ? tv : v[y - 1];
+        i[y - 1] = sw ? ti : i[y - 1];
+      }
   }
 
-  // Writes slot indices and gates: softmax over the picked scores.
-  MOE_DEV void write(int32_t* idx, float* gate, int k) const {
+  // Slot indices and gates (softmax over the picked scores); call after sort().
+  MOE_DEV void write(int32_t* idx, float* gate) const {
     const float m = v[0];
-    float w[kMaxK];
+    float w[K];
     float sum = 0.f;
 #pragma unroll
-    for (int j = 0; j < kMaxK; ++j) {
-      w[j] = 0.f;
-      if (j < k && m > -INFINITY) w[j] = expf(v[j] - m);
+    for (int j = 0; j < K; ++j) {
+      w[j] = m > -INFINITY ? expf(v[j] - m) : 0.f;
       sum += w[j];
     }
 #pragma unroll
-    for (int j = 0; j < kMaxK; ++j)
-      if (j < k) {
-        idx[j] = i[j];
-        gate[j] = sum > 0.f ? w[j] / sum : 0.f;
-      }
+    for (int j = 0; j < K; ++j) {
+      idx[j] = i[j];
+      gate[j] = sum > 0.f ? w[j] / sum : 0.f;
+    }
   }
 };
 
 struct RouterArgs {
-  int T, d, E, k, npad, tmem_cols;
+  int T, d, E, npad, tmem_cols;
+  int ncols;   // experts this CTA ranks: npad, or npad/2 when a CTA pair splits the reduction
+  int stages;  // depth of the TMA ring (<= kRouterMaxStages)
+  int split;   // 1: CTA pairs split the reduction over d (clusters of two)
   const float* bias;
   float* logits;
   int32_t* idx;
@@ -99,27 +125,37 @@ struct RouterArgs {
   int32_t* status;
 };
 
-__global__ void __launch_bounds__(256, 2) router_tc_kernel(const __grid_constant__ CUtensorMap tm_h,
-                                                        const __grid_constant__ CUtensorMap tm_w,
-                                                        const RouterArgs a) {
+template <int K>
+__global__ void __launch_bounds__(256, 1) router_tc_kernel(const __grid_constant__ CUtensorMap tm_h,
+                                                           const __grid_constant__ CUtensorMap tm_w,
+                                                           const RouterArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align_1024(smem_raw);
   const uint32_t b_bytes = static_cast<uint32_t>(a.npad) * kRouterBK * 2;
   const uint32_t stage_bytes = kRouterABytes + b_bytes;  // a multiple of 2048
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kRouterStages * stage_bytes);
-  uint64_t* empty = full + kRouterStages;
-  uint64_t* done = empty + kRouterStages;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + a.stages * stage_bytes);
+  uint64_t* empty = full + kRouterMaxStages;
+  uint64_t* done = empty + kRouterMaxStages;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   int* consumed_slot = reinterpret_cast<int*>(tmem_slot + 2);
-  float* sbias = reinterpret_cast<float*>(tmem_slot + 4);
+  float* sbias = reinterpret_cast<float*>(tmem_slot + 4);         // [kMaxE]
+  float* pair_v = sbias + kMaxE;                                    // [128][K] lists handed over by rank 1
+  int* pair_i = reinterpret_cast<int*>(pair_v + kTileM * K);        // [128][K]
+  int* pair_nan = pair_i + kTileM * K;                              // [128]
+  float* recv = reinterpret_cast<float*>(                           // [128][ncols] partner's partial scores,
+      (reinterpret_cast<uintptr_t>(pair_nan + kTileM) + 15) & ~static_cast<uintptr_t>(15));  // 16-byte aligned
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int nkb = a.d / kRouterBK;
-  const int tile = blockIdx.x;
+  const uint32_t rank = a.split ? cluster_ctarank() : 0u;
+  const int tile = a.split ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
+  const int col0 = static_cast<int>(rank) * a.ncols;  // first expert this CTA ranks
+  const int nkb_all = a.d / kRouterBK;
+  const int nkb = a.split ? nkb_all / 2 : nkb_all;     // k-blocks this CTA multiplies
+  const int kb0 = static_cast<int>(rank) * nkb;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kRouterStages; ++s) {
+    for (int s = 0; s < a.stages; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
@@ -131,8 +167,10 @@ __global__ void __launch_bounds__(256, 2) router_tc_kernel(const __grid_constant
     tma_prefetch_desc(&tm_w);
   }
   __shared__ int s_hist[kMaxE];
-  for (int e = threadIdx.x; e < a.npad; e += blockDim.x)
-    sbias[e] = e >= a.E ? -INFINITY : (a.bias ? a.bias[e] : 0.f);
+  for (int j = threadIdx.x; j < a.ncols; j += blockDim.x) {
+    const int e = col0 + j;
+    sbias[j] = e >= a.E ? -INFINITY : (a.bias ? a.bias[e] : 0.f);
+  }
   for (int e = threadIdx.x; e < a.E; e += blockDim.x) s_hist[e] = 0;
   if (warp == 0) {
     tmem_alloc(tmem_slot, a.tmem_cols);
@@ -147,25 +185,25 @@ __global__ void __launch_bounds__(256, 2) router_tc_kernel(const __grid_constant
   if (warp == 0 && lane == 0) {
     // TMA producer
     for (int kb = 0; kb < nkb; ++kb) {
-      const int s = kb % kRouterStages;
-      const uint32_t round = kb / kRouterStages;
+      const int s = kb % a.stages;
+      const uint32_t round = kb / a.stages;
       if (!mbar_wait(&empty[s], (round & 1) ^ 1, abort_flag)) {
         *abort_flag = 1;
         break;
       }
       uint8_t* st = smem + s * stage_bytes;
       mbar_expect_tx(&full[s], stage_bytes);
-      tma_load_2d(st, &tm_h, &full[s], kb * kRouterBK, tile * kTileM);
-      tma_load_2d(st + kRouterABytes, &tm_w, &full[s], kb * kRouterBK, 0);
+      tma_load_2d(st, &tm_h, &full[s], (kb0 + kb) * kRouterBK, tile * kTileM);
+      tma_load_2d(st + kRouterABytes, &tm_w, &full[s], (kb0 + kb) * kRouterBK, 0);
       ++issued;
     }
   } else if (warp == 1 && lane == 0) {
-    // MMA issuer
+    // MMA issuer: all npad expert columns over this CTA's k-blocks
     const uint32_t idesc = idesc_bf16_f32(kTileM, a.npad);
     int kb = 0;
     for (; kb < nkb; ++kb) {
-      const int s = kb % kRouterStages;
-      const uint32_t round = kb / kRouterStages;
+      const int s = kb % a.stages;
+      const uint32_t round = kb / a.stages;
       if (!mbar_wait(&full[s], round & 1, abort_flag)) {
         *abort_flag = 1;
         break;
@@ -188,55 +226,97 @@ __global__ void __launch_bounds__(256, 2) router_tc_kernel(const __grid_constant
   tc_fence_after();
   ok = __syncthreads_and(ok && !*abort_flag);  // the same decision in every thread
 
+  // Thread layout of the epilogue: warp w reads TMEM lane quadrant (w & 3),
+  // i.e. token rows 32*(w&3) .. +31; the two warps of a quadrant take every
+  // other 16-column chunk (starting at 16*(w>>2)).
+  const int q = warp & 3, half = warp >> 2;
+  const int row = q * 32 + lane;
+  const int t = tile * kTileM + row;
+  const uint32_t lane_base = tmem + (static_cast<uint32_t>(q * 32) << 16);
+
+  if (a.split) {
+    // hand the partner the partial scores of the experts it ranks
+    if (ok) {
+      const int pcol0 = static_cast<int>(rank ^ 1u) * a.ncols;
+      const uint32_t dst = mapa_shared(smem_addr(recv + row * a.ncols), rank ^ 1u);
+      for (int c0 = half * 16; c0 < a.ncols; c0 += 32) {
+        uint32_t r[16];
+        tmem_ld16(lane_base + pcol0 + c0, r);
+        tmem_ld_wait();
+#pragma unroll
+        for (int j = 0; j < 16; j += 4)
+          st_shared_cluster_v4(dst + 4 * (c0 + j), r[j], r[j + 1], r[j + 2], r[j + 3]);
+      }
+    }
+    cluster_sync();  // every thread of both CTAs, whatever happened above
+  }
+
+  TopList<K> top;
+  top.init();
+  bool nan = false;
   if (ok) {
-    // 8 warps: warp w reads TMEM lane quadrant (w & 3), i.e. token rows
-    // 32*(w&3) .. +31, and every other 16-column chunk starting at 16*(w>>2).
-    // The two partial lists of a row are merged through shared memory.
-    const int q = warp & 3, half = warp >> 2;
-    const int row = q * 32 + lane;
-    const int t = tile * kTileM + row;
-    TopList top;
-    top.init();
-    bool nan = false;
-    const uint32_t lane_base = tmem + (static_cast<uint32_t>(q * 32) << 16);
     float* lrow = (a.logits != nullptr && t < a.T) ? a.logits + static_cast<size_t>(t) * a.E : nullptr;
-    for (int c0 = half * 16; c0 < a.npad; c0 += 32) {
+    for (int c0 = half * 16; c0 < a.ncols; c0 += 32) {
       uint32_t r[16];
-      tmem_ld16(lane_base + c0, r);
+      tmem_ld16(lane_base + col0 + c0, r);
       tmem_ld_wait();
 #pragma unroll
       for (int j = 0; j < 16; ++j) {
-        float x = __uint_as_float(r[j]) + sbias[c0 + j];  // padded experts carry -inf
-        if (lrow != nullptr && c0 + j < a.E) lrow[c0 + j] = x;
+        const int e = col0 + c0 + j;
+        float x = __uint_as_float(r[j]);
+        if (a.split) x += recv[row * a.ncols + c0 + j];
+        x += sbias[c0 + j];  // padded experts carry -inf
+        if (lrow != nullptr && e < a.E) lrow[e] = x;
         nan |= x != x;
         x = x != x ? -INFINITY : x;
-        top.push_ascending(x, c0 + j, a.k);
+        top.push(x, e);
       }
     }
     float* xv = reinterpret_cast<float*>(smem);  // stage buffers are free once the MMAs are done
-    int* xi = reinterpret_cast<int*>(smem + kTileM * kMaxK * 4);
-    int* xn = reinterpret_cast<int*>(smem + 2 * kTileM * kMaxK * 4);
+    int* xi = reinterpret_cast<int*>(smem + kTileM * K * 4);
+    int* xn = reinterpret_cast<int*>(smem + 2 * kTileM * K * 4);
     if (half == 1) {
 #pragma unroll
-      for (int j = 0; j < kMaxK; ++j) {
-        xv[row * kMaxK + j] = top.v[j];
-        xi[row * kMaxK + j] = top.i[j];
+      for (int j = 0; j < K; ++j) {
+        xv[row * K + j] = top.v[j];
+        xi[row * K + j] = top.i[j];
       }
       xn[row] = nan;
     }
     __syncthreads();
     if (half == 0) {
 #pragma unroll
-      for (int j = 0; j < kMaxK; ++j)
-        if (j < a.k) top.push_any(xv[row * kMaxK + j], xi[row * kMaxK + j], a.k);
+      for (int j = 0; j < K; ++j) top.push(xv[row * K + j], xi[row * K + j]);
       nan |= xn[row] != 0;
+      if (a.split && rank == 1) {
+        const uint32_t dv = mapa_shared(smem_addr(pair_v + row * K), 0);
+        const uint32_t di = mapa_shared(smem_addr(pair_i + row * K), 0);
+#pragma unroll
+        for (int j = 0; j < K; ++j) {
+          st_shared_cluster_u32(dv + 4 * j, __float_as_uint(top.v[j]));
+          st_shared_cluster_u32(di + 4 * j, static_cast<uint32_t>(top.i[j]));
+        }
+        st_shared_cluster_u32(mapa_shared(smem_addr(pair_nan + row), 0), nan ? 1u : 0u);
+      }
+    }
+  } else if (threadIdx.x == 0) {
+    report_status(a.status, MOE_STATUS_TIMEOUT);
+  }
+  if (a.split) cluster_sync();  // every thread of both CTAs, whatever happened above
+  if (ok && rank == 0) {
+    if (half == 0) {
+      if (a.split) {
+#pragma unroll
+        for (int j = 0; j < K; ++j) top.push(pair_v[row * K + j], pair_i[row * K + j]);
+        nan |= pair_nan[row] != 0;
+      }
+      top.sort();
       if (t < a.T) {
-        top.write(a.idx + static_cast<size_t>(t) * a.k, a.gate + static_cast<size_t>(t) * a.k, a.k);
+        top.write(a.idx + static_cast<size_t>(t) * K, a.gate + static_cast<size_t>(t) * K);
         if (nan) report_status(a.status, MOE_STATUS_NAN_LOGIT);
         if (a.chunk_counts != nullptr) {
 #pragma unroll
-          for (int j = 0; j < kMaxK; ++j)
-            if (j < a.k) atomicAdd(&s_hist[top.i[j]], 1);
+          for (int j = 0; j < K; ++j) atomicAdd(&s_hist[top.i[j]], 1);
         }
       }
     }
@@ -245,8 +325,6 @@ __global__ void __launch_bounds__(256, 2) router_tc_kernel(const __grid_constant
       for (int e = threadIdx.x; e < a.E; e += blockDim.x)
         a.chunk_counts[static_cast<size_t>(tile) * a.E + e] = s_hist[e];
     }
-  } else if (threadIdx.x == 0) {
-    report_status(a.status, MOE_STATUS_TIMEOUT);
   }
 
   tc_fence_before();
@@ -254,13 +332,14 @@ __global__ void __launch_bounds__(256, 2) router_tc_kernel(const __grid_constant
   if (warp == 0 && lane == 0 && *abort_flag) {
     // loads issued but never consumed must land before the CTA leaves
     for (int kb = *consumed_slot; kb < issued; ++kb)
-      mbar_wait(&full[kb % kRouterStages], (kb / kRouterStages) & 1, nullptr);
+      mbar_wait(&full[kb % a.stages], (kb / a.stages) & 1, nullptr);
   }
   __syncthreads();
   if (warp == 0) tmem_dealloc(tmem, a.tmem_cols);
 }
 
 // fp32 path: one warp per token, lanes over experts, fp32 FMA in index order.
+template <int K>
 __global__ void __launch_bounds__(256) router_f32_kernel(const float* __restrict__ h, const float* __restrict__ w,
                                                          const RouterArgs a) {
   extern __shared__ float slog[];  // [8 warps][E]
@@ -278,7 +357,7 @@ __global__ void __launch_bounds__(256) router_f32_kernel(const float* __restrict
     }
     __syncwarp();
     if (lane == 0) {
-      TopList top;
+      TopList<K> top;
       top.init();
       bool nan = false;
       for (int e = 0; e < a.E; ++e) {
@@ -287,9 +366,10 @@ __global__ void __launch_bounds__(256) router_f32_kernel(const float* __restrict
           nan = true;
           x = -INFINITY;
         }
-        top.push_ascending(x, e, a.k);
+        top.push(x, e);
       }
-      top.write(a.idx + static_cast<size_t>(t) * a.k, a.gate + static_cast<size_t>(t) * a.k, a.k);
+      top.sort();
+      top.write(a.idx + static_cast<size_t>(t) * K, a.gate + static_cast<size_t>(t) * K);
       if (nan) report_status(a.status, MOE_STATUS_NAN_LOGIT);
     }
     __syncwarp();
@@ -302,31 +382,126 @@ uint32_t pow2_at_least(uint32_t x, uint32_t lo) {
   return p;
 }
 
+template <int K>
+cudaError_t launch_router_tc_k(const CUtensorMap& tm_h, const CUtensorMap& tm_w, RouterArgs a, int tiles,
+                               cudaStream_t s) {
+  const size_t stage_bytes = kRouterABytes + static_cast<size_t>(a.npad) * kRouterBK * 2;
+  const size_t fixed = 1024 + (2 * kRouterMaxStages + 1) * 8 + 16 + kMaxE * 4 + static_cast<size_t>(kTileM) * K * 8 +
+                       kTileM * 4 + 16 + (a.split ? static_cast<size_t>(kTileM) * a.ncols * 4 : 0);
+  const size_t budget = 227 * 1024 - 1024 /* static histogram */ - fixed;
+  int fit = static_cast<int>(budget / stage_bytes);
+  fit = fit > kRouterMaxStages ? kRouterMaxStages : fit;
+  // every CTA on its own SM: the deepest ring that fits; otherwise a ring
+  // small enough for two CTAs per SM (at most 4 stages)
+  const int ctas = (a.split ? 2 : 1) * tiles;
+  if (ctas <= device_sm_count()) {
+    a.stages = fit;
+  } else {
+    const size_t half_budget = 113 * 1024 - 1024 - fixed;
+    const int two = static_cast<int>(half_budget / stage_bytes);
+    a.stages = two >= 2 ? (two < 4 ? two : 4) : (fit < 4 ? fit : 4);
+  }
+  if (a.stages < 2) return cudaErrorInvalidConfiguration;
+  const size_t smem = fixed + a.stages * stage_bytes;
+  cudaError_t err = cudaFuncSetAttribute(router_tc_kernel<K>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+  if (err != cudaSuccess) return err;
+  if (!a.split) {
+    router_tc_kernel<K><<<tiles, 256, smem, s>>>(tm_h, tm_w, a);
+    return cudaGetLastError();
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * tiles, 1, 1);
+  cfg.blockDim = dim3(256, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  err = cudaLaunchKernelEx(&cfg, router_tc_kernel<K>, tm_h, tm_w, a);
+  if (err != cudaSuccess) return err;
+  return cudaGetLastError();
+}
+
 }  // namespace
 
 cudaError_t launch_router_tc(const CUtensorMap& tm_h, const CUtensorMap& tm_w, int T, int d, int E, int k,
                              int npad, const float* bias, float* logits, int32_t* idx, float* gate,
                              int32_t* chunk_counts, int32_t* status, cudaStream_t s) {
   if (T == 0) return cudaSuccess;
-  const int grid = (T + kTileM - 1) / kTileM;
-  RouterArgs a{T,    d,      E,   k,    npad,         static_cast<int>(pow2_at_least(npad, 32)),
-               bias, logits, idx, gate, chunk_counts, grid,
-               status};
-  const size_t stage_bytes = kRouterABytes + static_cast<size_t>(npad) * kRouterBK * 2;
-  const size_t smem = 1024 + kRouterStages * stage_bytes + (2 * kRouterStages + 1) * 8 + 16 + kMaxE * 4;
-  cudaError_t err = cudaFuncSetAttribute(router_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(smem));
-  if (err != cudaSuccess) return err;
-  router_tc_kernel<<<grid, 256, smem, s>>>(tm_h, tm_w, a);
-  return cudaGetLastError();
+  const int tiles = (T + kTileM - 1) / kTileM;
+  const int split = router_splits_experts(npad) ? 1 : 0;
+  RouterArgs a{};
+  a.T = T;
+  a.d = d;
+  a.E = E;
+  a.npad = npad;
+  a.tmem_cols = static_cast<int>(pow2_at_least(npad, 32));
+  a.ncols = split ? npad / 2 : npad;
+  a.stages = 4;
+  a.split = split;
+  a.bias = bias;
+  a.logits = logits;
+  a.idx = idx;
+  a.gate = gate;
+  a.chunk_counts = chunk_counts;
+  a.n_tiles = tiles;
+  a.status = status;
+  switch (k) {
+#define MOE_ROUTER_K(KK) \
+  case KK:               \
+    return launch_router_tc_k<KK>(tm_h, tm_w, a, tiles, s);
+    MOE_ROUTER_K(1)
+    MOE_ROUTER_K(2)
+    MOE_ROUTER_K(3)
+    MOE_ROUTER_K(4)
+    MOE_ROUTER_K(5)
+    MOE_ROUTER_K(6)
+    MOE_ROUTER_K(7)
+    MOE_ROUTER_K(8)
+#undef MOE_ROUTER_K
+    default:
+      return cudaErrorInvalidValue;
+  }
 }
 
 cudaError_t launch_router_f32(const float* h, const float* w, int T, int d, int E, int k, const float* bias,
                               float* logits, int32_t* idx, float* gate, int32_t* status, cudaStream_t s) {
   if (T == 0) return cudaSuccess;
-  RouterArgs a{T, d, E, k, E, 0, bias, logits, idx, gate, nullptr, 0, status};
+  RouterArgs a{};
+  a.T = T;
+  a.d = d;
+  a.E = E;
+  a.npad = E;
+  a.ncols = E;
+  a.bias = bias;
+  a.logits = logits;
+  a.idx = idx;
+  a.gate = gate;
+  a.status = status;
   const int grid = (T + 7) / 8 < 4096 ? (T + 7) / 8 : 4096;
-  router_f32_kernel<<<grid, 256, 8 * E * sizeof(float), s>>>(h, w, a);
+  const size_t smem = 8 * static_cast<size_t>(E) * sizeof(float);
+  switch (k) {
+#define MOE_ROUTER_F32_K(KK)                                \
+  case KK:                                                  \
+    router_f32_kernel<KK><<<grid, 256, smem, s>>>(h, w, a); \
+    break;
+    MOE_ROUTER_F32_K(1)
+    MOE_ROUTER_F32_K(2)
+    MOE_ROUTER_F32_K(3)
+    MOE_ROUTER_F32_K(4)
+    MOE_ROUTER_F32_K(5)
+    MOE_ROUTER_F32_K(6)
+    MOE_ROUTER_F32_K(7)
+    MOE_ROUTER_F32_K(8)
+#undef MOE_ROUTER_F32_K
+    default:
+      return cudaErrorInvalidValue;
+  }
   return cudaGetLastError();
 }
 

@@ -71,7 +71,8 @@ def _int_valued(T, d, E, seed, lo=-2, hi=3):
 
 
 @pytest.mark.parametrize("dtype,T,d,E,k", [("bf16", 300, 128, 8, 2), ("bf16", 129, 256, 64, 6),
-                                           ("bf16", 200, 128, 128, 8), ("f32", 77, 32, 6, 3)])
+                                           ("bf16", 200, 128, 128, 8), ("bf16", 150, 128, 100, 4),
+                                           ("bf16", 140, 128, 256, 8), ("f32", 77, 32, 6, 3)])
 def test_route_exact_ties_go_to_lowest_index(dtype, T, d, E, k):
     """Small integers make every score exact in fp32 and fp64, so planted ties
     are real ties on both sides."""
