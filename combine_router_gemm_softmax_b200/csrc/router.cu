@@ -140,11 +140,17 @@ __global__ void __launch_bounds__(256, 1) router_tc_kernel(const __grid_constant
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   int* consumed_slot = reinterpret_cast<int*>(tmem_slot + 2);
   float* sbias = reinterpret_cast<float*>(tmem_slot + 4);         // [kMaxE]
-  float* pair_v = sbias + kMaxE;                                    // [128][K] lists handed over by rank 1
-  int* pair_i = reinterpret_cast<int*>(pair_v + kTileM * K);        // [128][K]
+  // Per-token arrays are stored token-minor ([slot][128]) so a warp's 32
+  // tokens hit 32 different banks.
+  float* pair_v = sbias + kMaxE;                                    // [K][128] lists handed over by rank 1
+  int* pair_i = reinterpret_cast<int*>(pair_v + kTileM * K);        // [K][128]
   int* pair_nan = pair_i + kTileM * K;                              // [128]
-  float* recv = reinterpret_cast<float*>(                           // [128][ncols] partner's partial scores,
-      (reinterpret_cast<uintptr_t>(pair_nan + kTileM) + 15) & ~static_cast<uintptr_t>(15));  // 16-byte aligned
+  // [128][rs] partner's partial scores, 16-byte aligned; the row stride
+  // rs = ncols + 4 puts the 8 rows of a quarter warp's 16-byte accesses in
+  // distinct bank groups
+  float* recv = reinterpret_cast<float*>(
+      (reinterpret_cast<uintptr_t>(pair_nan + kTileM) + 15) & ~static_cast<uintptr_t>(15));
+  const int rs = a.ncols + 4;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = a.split ? cluster_ctarank() : 0u;
@@ -238,7 +244,7 @@ __global__ void __launch_bounds__(256, 1) router_tc_kernel(const __grid_constant
     // hand the partner the partial scores of the experts it ranks
     if (ok) {
       const int pcol0 = static_cast<int>(rank ^ 1u) * a.ncols;
-      const uint32_t dst = mapa_shared(smem_addr(recv + row * a.ncols), rank ^ 1u);
+      const uint32_t dst = mapa_shared(smem_addr(recv + row * rs), rank ^ 1u);
       for (int c0 = half * 16; c0 < a.ncols; c0 += 32) {
         uint32_t r[16];
         tmem_ld16(lane_base + pcol0 + c0, r);
@@ -259,12 +265,21 @@ __global__ void __launch_bounds__(256, 1) router_tc_kernel(const __grid_constant
     for (int c0 = half * 16; c0 < a.ncols; c0 += 32) {
       uint32_t r[16];
       tmem_ld16(lane_base + col0 + c0, r);
+      float part[16];  // the partner's partial scores, read while the TMEM load is in flight
+#pragma unroll
+      for (int j = 0; j < 16; j += 4) {
+        float4 p = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (a.split) p = *reinterpret_cast<const float4*>(recv + row * rs + c0 + j);
+        part[j] = p.x;
+        part[j + 1] = p.y;
+        part[j + 2] = p.z;
+        part[j + 3] = p.w;
+      }
       tmem_ld_wait();
 #pragma unroll
       for (int j = 0; j < 16; ++j) {
         const int e = col0 + c0 + j;
-        float x = __uint_as_float(r[j]);
-        if (a.split) x += recv[row * a.ncols + c0 + j];
+        float x = __uint_as_float(r[j]) + part[j];
         x += sbias[c0 + j];  // padded experts carry -inf
         if (lrow != nullptr && e < a.E) lrow[e] = x;
         nan |= x != x;
@@ -278,23 +293,23 @@ __global__ void __launch_bounds__(256, 1) router_tc_kernel(const __grid_constant
     if (half == 1) {
 #pragma unroll
       for (int j = 0; j < K; ++j) {
-        xv[row * K + j] = top.v[j];
-        xi[row * K + j] = top.i[j];
+        xv[j * kTileM + row] = top.v[j];
+        xi[j * kTileM + row] = top.i[j];
       }
       xn[row] = nan;
     }
     __syncthreads();
     if (half == 0) {
 #pragma unroll
-      for (int j = 0; j < K; ++j) top.push(xv[row * K + j], xi[row * K + j]);
+      for (int j = 0; j < K; ++j) top.push(xv[j * kTileM + row], xi[j * kTileM + row]);
       nan |= xn[row] != 0;
       if (a.split && rank == 1) {
-        const uint32_t dv = mapa_shared(smem_addr(pair_v + row * K), 0);
-        const uint32_t di = mapa_shared(smem_addr(pair_i + row * K), 0);
+        const uint32_t dv = mapa_shared(smem_addr(pair_v + row), 0);
+        const uint32_t di = mapa_shared(smem_addr(pair_i + row), 0);
 #pragma unroll
         for (int j = 0; j < K; ++j) {
-          st_shared_cluster_u32(dv + 4 * j, __float_as_uint(top.v[j]));
-          st_shared_cluster_u32(di + 4 * j, static_cast<uint32_t>(top.i[j]));
+          st_shared_cluster_u32(dv + 4 * j * kTileM, __float_as_uint(top.v[j]));
+          st_shared_cluster_u32(di + 4 * j * kTileM, static_cast<uint32_t>(top.i[j]));
         }
         st_shared_cluster_u32(mapa_shared(smem_addr(pair_nan + row), 0), nan ? 1u : 0u);
       }
@@ -307,7 +322,7 @@ __global__ void __launch_bounds__(256, 1) router_tc_kernel(const __grid_constant
     if (half == 0) {
       if (a.split) {
 #pragma unroll
-        for (int j = 0; j < K; ++j) top.push(pair_v[row * K + j], pair_i[row * K + j]);
+        for (int j = 0; j < K; ++j) top.push(pair_v[j * kTileM + row], pair_i[j * kTileM + row]);
         nan |= pair_nan[row] != 0;
       }
       top.sort();
@@ -387,7 +402,7 @@ cudaError_t launch_router_tc_k(const CUtensorMap& tm_h, const CUtensorMap& tm_w,
                                cudaStream_t s) {
   const size_t stage_bytes = kRouterABytes + static_cast<size_t>(a.npad) * kRouterBK * 2;
   const size_t fixed = 1024 + (2 * kRouterMaxStages + 1) * 8 + 16 + kMaxE * 4 + static_cast<size_t>(kTileM) * K * 8 +
-                       kTileM * 4 + 16 + (a.split ? static_cast<size_t>(kTileM) * a.ncols * 4 : 0);
+                       kTileM * 4 + 16 + (a.split ? static_cast<size_t>(kTileM) * (a.ncols + 4) * 4 : 0);
   const size_t budget = 227 * 1024 - 1024 /* static histogram */ - fixed;
   int fit = static_cast<int>(budget / stage_bytes);
   fit = fit > kRouterMaxStages ? kRouterMaxStages : fit;
