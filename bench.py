@@ -270,9 +270,9 @@ def main():
     status = torch.zeros(1, dtype=torch.int32, device=dev)
     stream = torch.cuda.current_stream(dev)
 
-    def step():
+    def step(stage_events=None):
         M.moe_layer_forward(cfg, h, wr, bias, w13, wd, y=y, routed_counts=routed, counts=counts, ws=ws,
-                            status=status, stream=stream)
+                            status=status, stream=stream, stage_events=stage_events)
 
     for _ in range(max(args.warmup, 3)):
         step()
@@ -288,8 +288,14 @@ def main():
     scrub = torch.empty(256 << 20, dtype=torch.uint8, device=dev) if flush else None
     gpu_uuid = torch.cuda.get_device_properties(dev).uuid
     sampler = ClockSampler(f"GPU-{gpu_uuid}")
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-           for _ in range(args.steps if flush else 1)]
+    # every timed step records 5 events on the launching stream: before the
+    # router and after the router, the dispatch, the expert stage and the
+    # combine, so each kernel stage is timed inside the steps themselves
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    for row in ev:
+        for e in row:
+            e.record(stream)
+    torch.cuda.synchronize()
     with sampler:
         barrier()
         torch.cuda.synchronize()
@@ -297,20 +303,18 @@ def main():
         # launches before the device reaches them, so the events bracket device
         # work only (host launch cost is part of the end-to-end figure below)
         torch.cuda._sleep(HOST_LEAD_CYCLES)
-        if flush:
-            for a, b in evs:
+        for i in range(args.steps):
+            if flush:
                 scrub.fill_(1)
-                a.record(stream)
-                step()
-                b.record(stream)
-        else:
-            evs[0][0].record(stream)
-            for _ in range(args.steps):
-                step()
-            evs[0][1].record(stream)
+            step(ev[i])
         torch.cuda.synchronize()
         barrier()
-    ms = sum(a.elapsed_time(b) for a, b in evs)
+    if flush:
+        ms = sum(row[0].elapsed_time(row[4]) for row in ev)   # each step alone, scrub excluded
+    else:
+        ms = ev[0][0].elapsed_time(ev[-1][4])                 # steps back to back
+    stages = {name: statistics.mean(row[i].elapsed_time(row[i + 1]) for row in ev)
+              for i, name in enumerate(("route", "permute", "grouped_ffn", "combine"))}
     ms_max, value = combine_ranks(ms, wl.T, args.steps, world, dev)
     launches_per_step = launches(cfg)
     st = int(status.item())
@@ -324,8 +328,6 @@ def main():
     e2e_ms, e2e_value = combine_ranks(e2e_ms, wl.T, args.steps, world, dev)
     row_bytes = wl.d * wl.elem_bytes
 
-    # ------------------------------------------------ per stage (same stream, CUDA events)
-    stages = stage_times(M, cfg, wl, h, wr, bias, w13, wd, dev, stream, scrub, reps=max(3, min(args.steps, 10)))
     barrier()
 
     if rank == 0:
@@ -418,49 +420,6 @@ def launches(cfg):
     scan = 0 if cfg.E * n_chunks <= 8192 else 1
     ffn = {0: 2, 1: 0, 2: 1}[cfg.expert_kind]
     return 1 + count + scan + 1 + 1 + ffn + 1
-
-
-def stage_times(M, cfg, wl, h, wr, bias, w13, wd, dev, stream, scrub, reps):
-    """Median device time of each stage called on its own through the C ABI.
-    Like the whole step, each call starts with a cold L2 when `scrub` is given,
-    and a spin kernel lets the host queue all calls ahead of the device."""
-    import torch
-
-    A = wl.T * wl.k
-    idx = torch.empty((wl.T, wl.k), dtype=torch.int32, device=dev)
-    gate = torch.empty((wl.T, wl.k), dtype=torch.float32, device=dev)
-    out = dict(routed_counts=torch.empty(wl.E, dtype=torch.int32, device=dev),
-               counts=torch.empty(wl.E, dtype=torch.int32, device=dev),
-               offsets=torch.empty(wl.E + 1, dtype=torch.int32, device=dev),
-               dest_row=torch.empty((wl.T, wl.k), dtype=torch.int32, device=dev),
-               perm_src=torch.empty(A, dtype=torch.int32, device=dev),
-               x_perm=torch.empty((A, wl.d), dtype=wl.torch_dtype, device=dev))
-    y_perm = torch.empty((A, wl.d), dtype=wl.torch_dtype, device=dev)
-    y = torch.empty((wl.T, wl.d), dtype=wl.torch_dtype, device=dev)
-    ws_p = M.workspace(cfg, M.MOE_OP_PERMUTE, dev)
-    ws_f = M.workspace(cfg, M.MOE_OP_GROUPED_FFN, dev)
-    calls = {
-        "route": lambda: M.moe_route(cfg, h, wr, bias, topk_idx=idx, topk_gate=gate, stream=stream),
-        "permute": lambda: M.moe_permute(cfg, h, idx, out=out, ws=ws_p, stream=stream),
-        "grouped_ffn": lambda: M.moe_grouped_ffn(cfg, out["x_perm"], out["offsets"], w13, wd, y_perm=y_perm,
-                                                 ws=ws_f, stream=stream),
-        "combine": lambda: M.moe_unpermute_combine(cfg, y_perm, out["dest_row"], gate, y=y, stream=stream),
-    }
-    res = {}
-    for name, fn in calls.items():
-        fn()
-        torch.cuda.synchronize()
-        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
-        torch.cuda._sleep(HOST_LEAD_CYCLES)
-        for a, b in evs:
-            if scrub is not None:
-                scrub.fill_(1)
-            a.record(stream)
-            fn()
-            b.record(stream)
-        torch.cuda.synchronize()
-        res[name] = statistics.median([a.elapsed_time(b) for a, b in evs])
-    return res
 
 
 def stage_report(st, wl, A_kept, pk, pk_kind):

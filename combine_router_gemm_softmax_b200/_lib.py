@@ -27,7 +27,7 @@ MOE_MAX_E, MOE_MAX_K, MOE_PACK_BLOCK = 256, 8, 128
 
 EXPORTED = ("moe_workspace_size", "moe_status_string", "moe_version", "moe_pack_weights", "moe_route",
             "moe_permute", "moe_grouped_ffn", "moe_unpermute_combine", "moe_layer_forward",
-            "moe_permute_static_scratch")
+            "moe_permute_static_scratch", "moe_layer_forward_timed")
 
 
 class MoeError(RuntimeError):
@@ -68,6 +68,7 @@ _SIGS = {
     "moe_unpermute_combine": (I32, [CFG, P, P, P, P, P, P]),
     "moe_layer_forward": (I32, [CFG, P, P, P, P, P, P, P, P, P, P, P, SZ, P, P]),
     "moe_permute_static_scratch": (I32, [CFG, P, P, P, P, P, P, P, P, P, P]),
+    "moe_layer_forward_timed": (I32, [CFG, P, P, P, P, P, P, P, P, P, P, P, SZ, P, P, P]),
 }
 
 
@@ -229,7 +230,11 @@ def moe_unpermute_combine(cfg, y_perm, dest_row, topk_gate, y=None, status=None,
 
 
 def moe_layer_forward(cfg, h, w_router, bias=None, w13_packed=None, w_down=None, y=None, topk_idx=None,
-                      topk_gate=None, routed_counts=None, counts=None, ws=None, status=None, stream=None):
+                      topk_gate=None, routed_counts=None, counts=None, ws=None, status=None, stream=None,
+                      stage_events=None):
+    """The whole layer; returns y. stage_events: None, or 5 torch.cuda.Event
+    (or None) recorded before the router and after the router, the dispatch,
+    the expert stage and the combine (moe_layer_forward_timed)."""
     dt = cfg.torch_dtype
     dev = _dev(h)
     _check(h, (cfg.T, cfg.d), dt, "h")
@@ -247,11 +252,25 @@ def moe_layer_forward(cfg, h, w_router, bias=None, w13_packed=None, w_down=None,
     _check(y, (cfg.T, cfg.d), dt, "y")
     if ws is None:
         ws = workspace(cfg, MOE_OP_LAYER, dev)
-    _rc("moe_layer_forward", lib().moe_layer_forward(
-        ctypes.byref(cfg), _ptr(h), _ptr(w_router), _ptr(bias), _ptr(w13_packed), _ptr(w_down), _ptr(y),
-        _ptr(topk_idx), _ptr(topk_gate), _ptr(routed_counts), _ptr(counts), _ptr(ws), ws.numel(), _ptr(status),
-        _stream(stream)))
+    args = (ctypes.byref(cfg), _ptr(h), _ptr(w_router), _ptr(bias), _ptr(w13_packed), _ptr(w_down), _ptr(y),
+            _ptr(topk_idx), _ptr(topk_gate), _ptr(routed_counts), _ptr(counts), _ptr(ws), ws.numel(), _ptr(status),
+            _stream(stream))
+    if stage_events is None:
+        _rc("moe_layer_forward", lib().moe_layer_forward(*args))
+        return y
+    if len(stage_events) != 5:
+        raise ValueError("stage_events needs 5 entries")
+    handles = (ctypes.c_void_p * 5)(*[None if e is None else _event_handle(e) for e in stage_events])
+    _rc("moe_layer_forward_timed", lib().moe_layer_forward_timed(*args, handles))
     return y
+
+
+def _event_handle(ev):
+    """Raw cudaEvent_t of a torch.cuda.Event; torch creates the event on its
+    first record, so an event that was never recorded is recorded once here."""
+    if not ev.cuda_event:
+        ev.record()
+    return ctypes.c_void_p(ev.cuda_event)
 
 
 def moe_permute_static_scratch(cfg, h, topk_idx, out=None, status=None, stream=None):

@@ -323,6 +323,15 @@ int32_t moe_layer_forward(const moe_config* cfg, const void* h, const void* w_ro
                           const void* w13_packed, const void* w_down, void* y, int32_t* topk_idx, float* topk_gate,
                           int32_t* routed_counts, int32_t* counts, void* workspace, size_t ws_bytes,
                           int32_t* status_dev, moe_stream_t stream) {
+  return moe_layer_forward_timed(cfg, h, w_router, bias, w13_packed, w_down, y, topk_idx, topk_gate, routed_counts,
+                                 counts, workspace, ws_bytes, status_dev, stream, nullptr);
+}
+
+int32_t moe_layer_forward_timed(const moe_config* cfg, const void* h, const void* w_router, const float* bias,
+                                const void* w13_packed, const void* w_down, void* y, int32_t* topk_idx,
+                                float* topk_gate, int32_t* routed_counts, int32_t* counts, void* workspace,
+                                size_t ws_bytes, int32_t* status_dev, moe_stream_t stream,
+                                void* const* stage_events) {
   int rc = check_cfg(cfg);
   if (rc != MOE_OK) return rc;
   const moe_config& c = *cfg;
@@ -341,21 +350,29 @@ int32_t moe_layer_forward(const moe_config* cfg, const void* h, const void* w_ro
   if (routed_counts) b.routed = routed_counts;
   if (counts) b.kept = counts;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  auto mark = [&](int i) {
+    if (stage_events == nullptr || stage_events[i] == nullptr) return MOE_OK;
+    return cuda_rc(cudaEventRecord(static_cast<cudaEvent_t>(stage_events[i]), s));
+  };
+  if ((rc = mark(0)) != MOE_OK) return rc;
   // the bf16 router also writes the per-tile expert histogram the dispatch needs
   const bool router_counts = c.dtype == MOE_DTYPE_BF16;
   rc = route_impl(c, h, w_router, bias, nullptr, b.idx, b.gate, router_counts ? b.perm.chunk_counts : nullptr,
                   status_dev, s);
-  if (rc != MOE_OK) return rc;
+  if (rc != MOE_OK || (rc = mark(1)) != MOE_OK) return rc;
   rc = permute_impl(c, h, b.idx, b.routed, b.kept, b.offsets, b.dest_row, b.perm_src, b.x_perm, b.perm,
                     router_counts, status_dev, s);
-  if (rc != MOE_OK) return rc;
+  if (rc != MOE_OK || (rc = mark(2)) != MOE_OK) return rc;
   const void* y_src = b.x_perm;
   if (c.expert_kind != MOE_EXPERT_IDENTITY) {
     rc = ffn_impl(c, b.x_perm, b.offsets, w13_packed, w_down, b.y_perm, b.h_mid, status_dev, s);
     if (rc != MOE_OK) return rc;
     y_src = b.y_perm;
   }
-  return cuda_rc(launch_combine(c.dtype, y_src, b.dest_row, b.gate, y, c.T, c.k, c.d, s));
+  if ((rc = mark(3)) != MOE_OK) return rc;
+  rc = cuda_rc(launch_combine(c.dtype, y_src, b.dest_row, b.gate, y, c.T, c.k, c.d, s));
+  if (rc != MOE_OK) return rc;
+  return mark(4);
 }
 
 }  // extern "C"

@@ -9,9 +9,11 @@
 // Tiles are 128 rows x 256 columns x 64-deep K slices. The tile list is built
 // on the device from the expert offsets (no host synchronisation): every CTA
 // reads offsets, counts ceil(rows_e / 128) row tiles per expert, and walks the
-// (row tile, column tile) grid in bands of 16 row tiles so that a wave of CTAs
-// shares A and B tiles in L2. grid = number of SMs; CTA c takes tiles c,
-// c + grid, ...
+// (row tile, column tile) grid in bands of row tiles so that a wave of CTAs
+// shares A and B tiles in L2. A band holds about 64 MB of A (8 to 32 row
+// tiles: 32 for the Mixtral-sized gate/up GEMM with K = 4096, 16 for its down
+// projection with K = 14336), so the band stays in L2 while the weights stream
+// through it once. grid = number of SMs; CTA c takes tiles c, c + grid, ...
 //
 // Inside a CTA (192 threads): warp 0 issues TMA loads into a 4-stage ring of
 // shared-memory buffers, warp 1 allocates TMEM and one of its threads issues
@@ -31,7 +33,6 @@ constexpr int kBM = kTileM;       // 128
 constexpr int kBN = kGemmTileN;   // 256
 constexpr int kBK = 64;
 constexpr int kStages = 4;
-constexpr int kGroupM = 16;
 constexpr int kGemmThreads = 192;
 constexpr uint32_t kABytes = kBM * kBK * 2;
 constexpr uint32_t kBBytes = kBN * kBK * 2;
@@ -52,16 +53,17 @@ struct GemmArgs {
   int ldd;           // row stride of D in elements
   __nv_bfloat16* D;
   int32_t* status;
+  int band;          // row tiles per band of the tile walk
 };
 
 // tile -> (expert, row tile within the expert, column tile)
-MOE_DEV void decode_tile(long long tile, int m_total, int n_tiles, const int* prefix, int E, int& e, int& m,
-                         int& n) {
-  const long long band_size = static_cast<long long>(kGroupM) * n_tiles;
+MOE_DEV void decode_tile(long long tile, int m_total, int n_tiles, int band_rows, const int* prefix, int E, int& e,
+                         int& m, int& n) {
+  const long long band_size = static_cast<long long>(band_rows) * n_tiles;
   const int band = static_cast<int>(tile / band_size);
   const int within = static_cast<int>(tile - band * band_size);
-  const int m0 = band * kGroupM;
-  const int rows = min(kGroupM, m_total - m0);
+  const int m0 = band * band_rows;
+  const int rows = min(band_rows, m_total - m0);
   n = within / rows;
   const int gm = m0 + within % rows;
   int lo = 0, hi = E;  // prefix[lo] <= gm < prefix[hi]
@@ -161,7 +163,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       bool stop = false;
       for (long long tile = blockIdx.x; tile < total && !stop; tile += gridDim.x) {
         int e, m, n;
-        decode_tile(tile, m_total, a.n_tiles, prefix, E, e, m, n);
+        decode_tile(tile, m_total, a.n_tiles, a.band, prefix, E, e, m, n);
         const int a_row = s_off[e] + m * kBM;
         const int b_row = e * a.n_per_expert + n * kBN;
         for (int kb = 0; kb < nkb; ++kb) {
@@ -231,7 +233,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     int local = 0;
     for (long long tile = blockIdx.x; tile < total; tile += gridDim.x, ++local) {
       int e, m, n;
-      decode_tile(tile, m_total, a.n_tiles, prefix, E, e, m, n);
+      decode_tile(tile, m_total, a.n_tiles, a.band, prefix, E, e, m, n);
       const int acc = local & 1;
       const uint32_t acc_phase = (local >> 1) & 1;
       if (!mbar_wait(&tfull[acc], acc_phase, abort_flag)) {
@@ -419,7 +421,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       bool stop = false;
       for (long long tile = pair_id; tile < total && !stop; tile += n_pairs) {
         int e, m, n;
-        decode_tile(tile, m_total, a.n_tiles, prefix, E, e, m, n);
+        decode_tile(tile, m_total, a.n_tiles, a.band, prefix, E, e, m, n);
         const int a_row = s_off[e] + m * kPairBM + static_cast<int>(rank) * 128;
         const int b_row = e * a.n_per_expert + n * kBN + static_cast<int>(rank) * 128;
         for (int kb = 0; kb < nkb; ++kb) {
@@ -490,7 +492,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     int local = 0;
     for (long long tile = pair_id; tile < total; tile += n_pairs, ++local) {
       int e, m, n;
-      decode_tile(tile, m_total, a.n_tiles, prefix, E, e, m, n);
+      decode_tile(tile, m_total, a.n_tiles, a.band, prefix, E, e, m, n);
       const int acc = local & 1;
       const uint32_t acc_phase = (local >> 1) & 1;
       if (!mbar_wait(&tfull[acc], acc_phase, abort_flag)) {
@@ -682,12 +684,22 @@ int blocks_for(long long work, int per_block) {
   return b < 1 ? 1 : static_cast<int>(b);
 }
 
+// Row tiles per band: the largest power of two in [lo, hi] whose A rows
+// (tile_rows x K bf16 each) stay within 64 MB, half of the L2.
+int band_rows(int tile_rows, int K, int lo, int hi) {
+  const long long tile_bytes = static_cast<long long>(tile_rows) * K * 2;
+  int b = hi;
+  while (b > lo && b * tile_bytes > (64ll << 20)) b >>= 1;
+  return b;
+}
+
 }  // namespace
 
 cudaError_t launch_grouped_gemm_tc(const CUtensorMap& tm_a, const CUtensorMap& tm_b, bool swiglu,
                                    const int32_t* offsets, int E, int K, int n_per_expert, int n_tiles,
                                    int out_cols, int ldd, void* D, int32_t* status, cudaStream_t s) {
-  GemmArgs a{offsets, E, K, n_per_expert, n_tiles, out_cols, ldd, static_cast<__nv_bfloat16*>(D), status};
+  GemmArgs a{offsets, E, K, n_per_expert, n_tiles, out_cols, ldd, static_cast<__nv_bfloat16*>(D), status,
+             band_rows(kBM, K, 8, 32)};
   const size_t smem = gemm_smem_bytes();
   const int grid = device_sm_count();
   cudaError_t err;
@@ -708,7 +720,8 @@ cudaError_t launch_grouped_gemm_tc(const CUtensorMap& tm_a, const CUtensorMap& t
 cudaError_t launch_grouped_gemm_pair(const CUtensorMap& tm_a, const CUtensorMap& tm_b, bool swiglu,
                                      const int32_t* offsets, int E, int K, int n_per_expert, int n_tiles, int out_cols,
                                      int ldd, void* D, int32_t* status, cudaStream_t s) {
-  GemmArgs a{offsets, E, K, n_per_expert, n_tiles, out_cols, ldd, static_cast<__nv_bfloat16*>(D), status};
+  GemmArgs a{offsets, E, K, n_per_expert, n_tiles, out_cols, ldd, static_cast<__nv_bfloat16*>(D), status,
+             band_rows(2 * kBM, K, 4, 16)};
   const size_t smem = pair_smem_bytes();
   const int grid = (device_sm_count() / 2) * 2;
   cudaLaunchConfig_t cfg = {};

@@ -238,6 +238,10 @@ MOE_DEV void st_shared_cluster_u32(uint32_t cluster_saddr, uint32_t v) {
   asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(cluster_saddr), "r"(v) : "memory");
 }
 
+MOE_DEV void st_shared_cluster_u64(uint32_t cluster_saddr, uint64_t v) {
+  asm volatile("st.shared::cluster.u64 [%0], %1;" ::"r"(cluster_saddr), "l"(v) : "memory");
+}
+
 // 16-byte store into another CTA's shared memory (address 16-byte aligned).
 MOE_DEV void st_shared_cluster_v4(uint32_t cluster_saddr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
   asm volatile("st.shared::cluster.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(cluster_saddr), "r"(a), "r"(b), "r"(c),

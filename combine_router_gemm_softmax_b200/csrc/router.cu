@@ -111,6 +111,68 @@ struct TopList {
   }
 };
 
+// Order-preserving 64-bit key of (score, expert) for the tensor-core path:
+// a larger key ranks first, i.e. a higher score, then the lower expert index.
+// The high word maps the fp32 score onto unsigned order (-0 ranks as +0, as
+// it compares in fp32); the low word is the complemented expert index. Key 0
+// is below every real key (-inf maps to 0x007fffff) and marks an empty slot.
+MOE_DEV uint64_t rank_key(float x, int e) {
+  uint32_t u = __float_as_uint(x);
+  u = u == 0x80000000u ? 0u : u;
+  u = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+  return (static_cast<uint64_t>(u) << 32) | static_cast<uint32_t>(~static_cast<uint32_t>(e));
+}
+MOE_DEV float key_score(uint64_t k) {
+  const uint32_t u = static_cast<uint32_t>(k >> 32);
+  return __uint_as_float((u & 0x80000000u) ? (u & 0x7fffffffu) : ~u);
+}
+MOE_DEV int key_expert(uint64_t k) { return static_cast<int>(~static_cast<uint32_t>(k)); }
+
+// Compare-exchange: the larger key to slot i, the smaller to slot l.
+MOE_DEV void cx(uint64_t& i, uint64_t& l) {
+  const uint64_t a = i, b = l;
+  const bool s = a < b;
+  i = s ? b : a;
+  l = s ? a : b;
+}
+
+// Bitonic sort of N keys (N a power of two) into descending order. All loops
+// unroll, so every index is a compile-time constant and the keys stay in
+// registers; each layer is N/2 independent compare-exchanges.
+template <int N>
+MOE_DEV void sort_desc(uint64_t* v) {
+#pragma unroll
+  for (int k = 2; k <= N; k <<= 1)
+#pragma unroll
+    for (int j = k >> 1; j > 0; j >>= 1)
+#pragma unroll
+      for (int i = 0; i < N; ++i) {
+        const int l = i ^ j;
+        if (l > i) {
+          if ((i & k) == 0)
+            cx(v[i], v[l]);
+          else
+            cx(v[l], v[i]);
+        }
+      }
+}
+
+// a, b sorted descending: a becomes the N largest keys of both, descending.
+// max(a[i], b[N-1-i]) is a bitonic sequence holding the N largest keys; a
+// half-cleaner network then sorts it.
+template <int N>
+MOE_DEV void merge_top(uint64_t* a, const uint64_t* b) {
+#pragma unroll
+  for (int i = 0; i < N; ++i) a[i] = a[i] > b[N - 1 - i] ? a[i] : b[N - 1 - i];
+#pragma unroll
+  for (int j = N >> 1; j > 0; j >>= 1)
+#pragma unroll
+    for (int i = 0; i < N; ++i) {
+      const int l = i ^ j;
+      if (l > i) cx(a[i], a[l]);
+    }
+}
+
 struct RouterArgs {
   int T, d, E, npad, tmem_cols;
   int ncols;   // experts this CTA ranks: npad, or npad/2 when a CTA pair splits the reduction
@@ -125,10 +187,18 @@ struct RouterArgs {
   int32_t* status;
 };
 
+// Candidate lists hold KP keys, K rounded up to a power of two (<= 8), so
+// they merge with bitonic networks; the first K entries are the result.
+template <int K>
+__host__ __device__ constexpr int list_len() {
+  return K <= 1 ? 1 : K <= 2 ? 2 : K <= 4 ? 4 : 8;
+}
+
 template <int K>
 __global__ void __launch_bounds__(256, 1) router_tc_kernel(const __grid_constant__ CUtensorMap tm_h,
                                                            const __grid_constant__ CUtensorMap tm_w,
                                                            const RouterArgs a) {
+  constexpr int KP = list_len<K>();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align_1024(smem_raw);
   const uint32_t b_bytes = static_cast<uint32_t>(a.npad) * kRouterBK * 2;
@@ -141,10 +211,9 @@ __global__ void __launch_bounds__(256, 1) router_tc_kernel(const __grid_constant
   int* consumed_slot = reinterpret_cast<int*>(tmem_slot + 2);
   float* sbias = reinterpret_cast<float*>(tmem_slot + 4);         // [kMaxE]
   // Per-token arrays are stored token-minor ([slot][128]) so a warp's 32
-  // tokens hit 32 different banks.
-  float* pair_v = sbias + kMaxE;                                    // [K][128] lists handed over by rank 1
-  int* pair_i = reinterpret_cast<int*>(pair_v + kTileM * K);        // [K][128]
-  int* pair_nan = pair_i + kTileM * K;                              // [128]
+  // tokens touch consecutive words.
+  uint64_t* pair_k = reinterpret_cast<uint64_t*>(sbias + kMaxE);   // [KP][128] keys handed over by rank 1
+  int* pair_nan = reinterpret_cast<int*>(pair_k + kTileM * KP);     // [128]
   // [128][rs] partner's partial scores, 16-byte aligned; the row stride
   // rs = ncols + 4 puts the 8 rows of a quarter warp's 16-byte accesses in
   // distinct bank groups
@@ -257,8 +326,11 @@ __global__ void __launch_bounds__(256, 1) router_tc_kernel(const __grid_constant
     cluster_sync();  // every thread of both CTAs, whatever happened above
   }
 
-  TopList<K> top;
-  top.init();
+  // Each 16-column chunk: bitonic-sort groups of KP keys, merge the groups
+  // down to the chunk's best KP, merge those into the running list.
+  uint64_t top[KP];
+#pragma unroll
+  for (int j = 0; j < KP; ++j) top[j] = 0;
   bool nan = false;
   if (ok) {
     float* lrow = (a.logits != nullptr && t < a.T) ? a.logits + static_cast<size_t>(t) * a.E : nullptr;
@@ -276,6 +348,7 @@ __global__ void __launch_bounds__(256, 1) router_tc_kernel(const __grid_constant
         part[j + 3] = p.w;
       }
       tmem_ld_wait();
+      uint64_t key[16];
 #pragma unroll
       for (int j = 0; j < 16; ++j) {
         const int e = col0 + c0 + j;
@@ -283,34 +356,34 @@ __global__ void __launch_bounds__(256, 1) router_tc_kernel(const __grid_constant
         x += sbias[c0 + j];  // padded experts carry -inf
         if (lrow != nullptr && e < a.E) lrow[e] = x;
         nan |= x != x;
-        x = x != x ? -INFINITY : x;
-        top.push(x, e);
+        key[j] = rank_key(x != x ? -INFINITY : x, e);
       }
+#pragma unroll
+      for (int g = 0; g < 16; g += KP) sort_desc<KP>(key + g);
+#pragma unroll
+      for (int w = KP; w < 16; w <<= 1)
+#pragma unroll
+        for (int g = 0; g + w < 16; g += 2 * w) merge_top<KP>(key + g, key + g + w);
+      merge_top<KP>(top, key);
     }
-    float* xv = reinterpret_cast<float*>(smem);  // stage buffers are free once the MMAs are done
-    int* xi = reinterpret_cast<int*>(smem + kTileM * K * 4);
-    int* xn = reinterpret_cast<int*>(smem + 2 * kTileM * K * 4);
+    uint64_t* xk = reinterpret_cast<uint64_t*>(smem);  // stage buffers are free once the MMAs are done
+    int* xn = reinterpret_cast<int*>(smem + kTileM * KP * 8);
     if (half == 1) {
 #pragma unroll
-      for (int j = 0; j < K; ++j) {
-        xv[j * kTileM + row] = top.v[j];
-        xi[j * kTileM + row] = top.i[j];
-      }
+      for (int j = 0; j < KP; ++j) xk[j * kTileM + row] = top[j];
       xn[row] = nan;
     }
     __syncthreads();
     if (half == 0) {
+      uint64_t other[KP];
 #pragma unroll
-      for (int j = 0; j < K; ++j) top.push(xv[j * kTileM + row], xi[j * kTileM + row]);
+      for (int j = 0; j < KP; ++j) other[j] = xk[j * kTileM + row];
+      merge_top<KP>(top, other);
       nan |= xn[row] != 0;
       if (a.split && rank == 1) {
-        const uint32_t dv = mapa_shared(smem_addr(pair_v + row), 0);
-        const uint32_t di = mapa_shared(smem_addr(pair_i + row), 0);
+        const uint32_t dk = mapa_shared(smem_addr(pair_k + row), 0);
 #pragma unroll
-        for (int j = 0; j < K; ++j) {
-          st_shared_cluster_u32(dv + 4 * j * kTileM, __float_as_uint(top.v[j]));
-          st_shared_cluster_u32(di + 4 * j * kTileM, static_cast<uint32_t>(top.i[j]));
-        }
+        for (int j = 0; j < KP; ++j) st_shared_cluster_u64(dk + 8 * j * kTileM, top[j]);
         st_shared_cluster_u32(mapa_shared(smem_addr(pair_nan + row), 0), nan ? 1u : 0u);
       }
     }
@@ -321,17 +394,33 @@ __global__ void __launch_bounds__(256, 1) router_tc_kernel(const __grid_constant
   if (ok && rank == 0) {
     if (half == 0) {
       if (a.split) {
+        uint64_t other[KP];
 #pragma unroll
-        for (int j = 0; j < K; ++j) top.push(pair_v[j * kTileM + row], pair_i[j * kTileM + row]);
+        for (int j = 0; j < KP; ++j) other[j] = pair_k[j * kTileM + row];
+        merge_top<KP>(top, other);
         nan |= pair_nan[row] != 0;
       }
-      top.sort();
       if (t < a.T) {
-        top.write(a.idx + static_cast<size_t>(t) * K, a.gate + static_cast<size_t>(t) * K);
+        // gates: softmax over the K picked scores (slot 0 holds the largest)
+        const float m = key_score(top[0]);
+        float w[K];
+        float sum = 0.f;
+#pragma unroll
+        for (int j = 0; j < K; ++j) {
+          w[j] = m > -INFINITY ? expf(key_score(top[j]) - m) : 0.f;
+          sum += w[j];
+        }
+        int32_t* it = a.idx + static_cast<size_t>(t) * K;
+        float* gt = a.gate + static_cast<size_t>(t) * K;
+#pragma unroll
+        for (int j = 0; j < K; ++j) {
+          it[j] = key_expert(top[j]);
+          gt[j] = sum > 0.f ? w[j] / sum : 0.f;
+        }
         if (nan) report_status(a.status, MOE_STATUS_NAN_LOGIT);
         if (a.chunk_counts != nullptr) {
 #pragma unroll
-          for (int j = 0; j < K; ++j) atomicAdd(&s_hist[top.i[j]], 1);
+          for (int j = 0; j < K; ++j) atomicAdd(&s_hist[key_expert(top[j])], 1);
         }
       }
     }
@@ -401,7 +490,7 @@ template <int K>
 cudaError_t launch_router_tc_k(const CUtensorMap& tm_h, const CUtensorMap& tm_w, RouterArgs a, int tiles,
                                cudaStream_t s) {
   const size_t stage_bytes = kRouterABytes + static_cast<size_t>(a.npad) * kRouterBK * 2;
-  const size_t fixed = 1024 + (2 * kRouterMaxStages + 1) * 8 + 16 + kMaxE * 4 + static_cast<size_t>(kTileM) * K * 8 +
+  const size_t fixed = 1024 + (2 * kRouterMaxStages + 1) * 8 + 16 + kMaxE * 4 + static_cast<size_t>(kTileM) * list_len<K>() * 8 +
                        kTileM * 4 + 16 + (a.split ? static_cast<size_t>(kTileM) * (a.ncols + 4) * 4 : 0);
   const size_t budget = 227 * 1024 - 1024 /* static histogram */ - fixed;
   int fit = static_cast<int>(budget / stage_bytes);

@@ -197,6 +197,23 @@ MOE_API int32_t moe_layer_forward(const moe_config* cfg, const void* h, const vo
                           int32_t* counts, void* workspace, size_t ws_bytes,
                           int32_t* status_dev, moe_stream_t stream);
 
+/* moe_layer_forward_timed -- moe_layer_forward that also records caller-owned
+ * CUDA events between its stages, so a caller can time each stage inside a
+ * real layer step (the stand-alone stage calls differ: moe_permute counts the
+ * routes itself, while in the layer the router does). The pages have no
+ * counterpart for this entry point; it is a measurement hook.
+ * stage_events: NULL (then this is moe_layer_forward), or an array of 5
+ * cudaEvent_t handles, each may be NULL. Recorded on `stream`:
+ *   [0] before the router, [1] after the router, [2] after the dispatch
+ *   (rank + row copy), [3] after the expert stage, [4] after the combine.
+ * The events stay owned by the caller and must be created on the current
+ * device; a failed record returns MOE_ERR_CUDA and enqueues no later stage. */
+MOE_API int32_t moe_layer_forward_timed(const moe_config* cfg, const void* h, const void* w_router,
+                                        const float* bias, const void* w13_packed, const void* w_down, void* y,
+                                        int32_t* topk_idx, float* topk_gate, int32_t* routed_counts,
+                                        int32_t* counts, void* workspace, size_t ws_bytes,
+                                        int32_t* status_dev, moe_stream_t stream, void* const* stage_events);
+
 /* moe_permute_static_scratch -- moe_permute for callers that cannot allocate.
  * The paper has no counterpart for this entry point. It is for code that has
  * no way to pass a workspace: a host framework or memory pool that owns all

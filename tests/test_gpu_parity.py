@@ -366,3 +366,27 @@ def test_layer_replays_from_a_cuda_graph():
         eager = run(h_new.clone(), torch.empty_like(y_static))
         torch.cuda.synchronize()
         assert torch.equal(y_static.view(torch.int16), eager.view(torch.int16))
+
+
+def test_layer_stage_events_time_the_same_layer():
+    """moe_layer_forward_timed gives the same output bit for bit and records
+    its 5 events in stage order on the launching stream."""
+    dc = dev_case("small_skewed")
+    wl = dc.wl
+    ws = M.workspace(dc.cfg, M.MOE_OP_LAYER, DEV)
+    y0 = M.moe_layer_forward(dc.cfg, dc.h, dc.w_router, dc.bias, dc.w13, dc.w_down, ws=ws)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(5)]
+    y1 = M.moe_layer_forward(dc.cfg, dc.h, dc.w_router, dc.bias, dc.w13, dc.w_down, ws=ws, stage_events=ev)
+    torch.cuda.synchronize()
+    assert torch.equal(y0.view(torch.int16), y1.view(torch.int16))
+    parts = [ev[i].elapsed_time(ev[i + 1]) for i in range(4)]
+    assert all(p >= 0 for p in parts)
+    assert parts[2] > 0  # the expert stage did work between its two events
+    assert abs(sum(parts) - ev[0].elapsed_time(ev[4])) < 1e-2
+    # NULL entries are skipped
+    y2 = M.moe_layer_forward(dc.cfg, dc.h, dc.w_router, dc.bias, dc.w13, dc.w_down, ws=ws,
+                             stage_events=[None, ev[1], None, None, ev[4]])
+    torch.cuda.synchronize()
+    assert torch.equal(y0.view(torch.int16), y2.view(torch.int16))
+    with pytest.raises(ValueError):
+        M.moe_layer_forward(dc.cfg, dc.h, dc.w_router, dc.bias, dc.w13, dc.w_down, ws=ws, stage_events=ev[:3])
