@@ -195,6 +195,34 @@ def dispatch_meta(idx, E, cap=-1):
                 perm_src=perm_src, rank=rank, bad_route=bool((~ok).any()))
 
 
+def dispatch_meta_padded(idx, E, cap):
+    """The padded capacity-based layout, the comparison arm of the evaluation
+    the dropless page proposes ("Dropless MoE Is a Runtime Problem as Much as
+    a Model Design": grouped GEMM avoids "padding all experts to a common
+    capacity"; its reproducible-evaluation paragraph compares padded
+    capacity-based against dropless). Every expert owns a buffer of exactly
+    cap rows: expert e's rows are [e*cap, (e+1)*cap). The kept assignments and
+    their ranks are those of the capacity mode (dispatch_meta with the same
+    cap); a kept assignment of rank r goes to row e*cap + r, and the rows past
+    an expert's kept count are padding (perm_src = -1, a zero row in x_perm).
+
+    Returns dispatch_meta's dict with offsets [E+1] = e*cap, dest_row [T,k] and
+    perm_src [E*cap] in this layout.
+    """
+    if cap < 0:
+        raise ValueError("the padded layout needs a capacity")
+    m = dispatch_meta(idx, E, cap)
+    idx = np.asarray(idx)
+    offsets = np.arange(E + 1, dtype=np.int64) * cap
+    dest_row = np.full(idx.shape, -1, np.int64)
+    keep = m["dest_row"] >= 0
+    tt, jj = np.nonzero(keep)
+    dest_row[tt, jj] = offsets[idx[tt, jj]] + m["rank"][tt, jj]
+    perm_src = np.full(E * cap, -1, np.int64)
+    perm_src[dest_row[tt, jj]] = tt
+    return dict(m, offsets=offsets, dest_row=dest_row, perm_src=perm_src)
+
+
 def silu(z):
     """silu(z) = z / (1 + exp(-z))."""
     with np.errstate(over="ignore"):

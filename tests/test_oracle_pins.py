@@ -170,6 +170,33 @@ def test_dispatch_invariants_and_capacity(T, E, k, cap):
         assert got == want
 
 
+@pytest.mark.parametrize("T,E,k,cap", [(200, 8, 3, 40), (64, 4, 4, 10), (30, 6, 2, 0), (9, 3, 1, 5)])
+def test_padded_layout_brute_force(T, E, k, cap):
+    """Padded capacity layout, from its definition by brute force: expert e
+    owns rows [e*cap, (e+1)*cap); the first min(routed_e, cap) hold the tokens
+    that picked e, in ascending order; the rest are padding (-1)."""
+    idx = _random_idx(T, E, k, 7 * T + E).reshape(T, k)
+    pm = O.dispatch_meta_padded(idx, E, cap)
+    assert pm["offsets"].tolist() == [e * cap for e in range(E + 1)]
+    assert len(pm["perm_src"]) == E * cap
+    for e in range(E):
+        users = [t for t in range(T) if e in idx[t]]
+        kept = users[:cap]
+        seg = pm["perm_src"][e * cap:(e + 1) * cap].tolist()
+        assert seg == kept + [-1] * (cap - len(kept))
+        for r, t in enumerate(kept):
+            j = list(idx[t]).index(e)
+            assert pm["dest_row"][t, j] == e * cap + r
+        for t in users[cap:]:
+            assert pm["dest_row"][t, list(idx[t]).index(e)] == -1
+    # the same assignments are kept as in the compact capacity layout
+    cm = O.dispatch_meta(idx, E, cap)
+    assert ((pm["dest_row"] >= 0) == (cm["dest_row"] >= 0)).all()
+    assert pm["kept"].tolist() == cm["kept"].tolist()
+    with pytest.raises(ValueError):
+        O.dispatch_meta_padded(idx, E, -1)
+
+
 def test_invalid_routes_are_dropped_and_flagged():
     idx = np.array([[0, 0], [1, 5], [-1, 2], [2, 1]], np.int32)
     meta = O.dispatch_meta(idx, E=3, cap=-1)
