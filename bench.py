@@ -210,7 +210,7 @@ def combine_ranks(ms_local, tokens_per_rank, steps, world, device=None):
 
 def config_dict(wl, n, flush=None):
     c = {"workload": wl.name, "T": wl.T, "d": wl.d, "E": wl.E, "k": wl.k, "d_ff": wl.F, "dtype": wl.dtype,
-         "expert_kind": wl.expert_kind, "capacity": wl.capacity, "global_batch": wl.T * n,
+         "expert_kind": wl.expert_kind, "capacity": wl.capacity, "layout": wl.layout, "global_batch": wl.T * n,
          "parallelism": f"token-sharded replicas x{n}"}
     if flush is not None:
         c["l2"] = ("flushed between steps (256 MB write), steps timed one by one" if flush
@@ -252,7 +252,7 @@ def main():
     M.lib()
     inp = W.draw(wl, args.seed)
     h_host = W.draw_h(wl, args.seed + rank).pin_memory() if rank else inp.h.pin_memory()
-    cfg = M.config(wl.T, wl.d, wl.E, wl.k, wl.F, wl.dtype, wl.expert_kind, wl.capacity, args.gemm_tiles)
+    cfg = M.config(wl.T, wl.d, wl.E, wl.k, wl.F, wl.dtype, wl.expert_kind, wl.capacity, args.gemm_tiles, wl.layout)
     h = h_host.to(dev)
     wr = inp.w_router.to(dev)
     bias = None if inp.bias is None else inp.bias.to(dev)
@@ -414,12 +414,13 @@ def launches(cfg):
     """Kernels one moe_layer_forward launches: router (which also counts the
     experts per 128-token tile on the bf16 path; the fp32 path adds a count
     kernel), a separate scan only for large E * ceil(T/128), rank, row copy,
-    the expert stage and the combine."""
+    the zero fill of the padded layout, the expert stage and the combine."""
     n_chunks = (cfg.T + 127) // 128
     count = 0 if cfg.dtype == 0 else 1
     scan = 0 if cfg.E * n_chunks <= 8192 else 1
+    pad = 1 if cfg.layout == 1 and cfg.capacity > 0 else 0
     ffn = {0: 2, 1: 0, 2: 1}[cfg.expert_kind]
-    return 1 + count + scan + 1 + 1 + ffn + 1
+    return 1 + count + scan + 1 + 1 + pad + ffn + 1
 
 
 def stage_report(st, wl, A_kept, pk, pk_kind):

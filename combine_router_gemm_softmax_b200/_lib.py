@@ -23,6 +23,7 @@ MOE_DTYPE_BF16, MOE_DTYPE_F32 = 0, 1
 MOE_EXPERT_SWIGLU, MOE_EXPERT_IDENTITY, MOE_EXPERT_SCALE = 0, 1, 2
 MOE_OP_ROUTE, MOE_OP_PERMUTE, MOE_OP_GROUPED_FFN, MOE_OP_LAYER = 0, 1, 2, 3
 MOE_GEMM_TILES_AUTO, MOE_GEMM_TILES_SINGLE, MOE_GEMM_TILES_PAIR = 0, 1, 2
+MOE_LAYOUT_COMPACT, MOE_LAYOUT_PADDED = 0, 1
 MOE_MAX_E, MOE_MAX_K, MOE_PACK_BLOCK = 256, 8, 128
 
 EXPORTED = ("moe_workspace_size", "moe_status_string", "moe_version", "moe_pack_weights", "moe_route",
@@ -39,7 +40,7 @@ class MoeError(RuntimeError):
 class MoeConfig(ctypes.Structure):
     _fields_ = [("T", ctypes.c_int32), ("d", ctypes.c_int32), ("E", ctypes.c_int32), ("k", ctypes.c_int32),
                 ("d_ff", ctypes.c_int32), ("dtype", ctypes.c_int32), ("expert_kind", ctypes.c_int32),
-                ("capacity", ctypes.c_int32), ("gemm_tiles", ctypes.c_int32)]
+                ("capacity", ctypes.c_int32), ("gemm_tiles", ctypes.c_int32), ("layout", ctypes.c_int32)]
 
     def __repr__(self):
         return "MoeConfig(" + ", ".join(f"{n}={getattr(self, n)}" for n, _ in self._fields_) + ")"
@@ -89,12 +90,19 @@ def lib() -> ctypes.CDLL:
     return _lib
 
 
-def config(T, d, E, k, d_ff, dtype="bf16", expert_kind="swiglu", capacity=-1, gemm_tiles="auto") -> MoeConfig:
+def config(T, d, E, k, d_ff, dtype="bf16", expert_kind="swiglu", capacity=-1, gemm_tiles="auto",
+           layout="compact") -> MoeConfig:
     dt = {"bf16": MOE_DTYPE_BF16, "f32": MOE_DTYPE_F32, torch.bfloat16: MOE_DTYPE_BF16,
           torch.float32: MOE_DTYPE_F32}[dtype]
     kind = {"swiglu": MOE_EXPERT_SWIGLU, "identity": MOE_EXPERT_IDENTITY, "scale": MOE_EXPERT_SCALE}[expert_kind]
     tiles = {"auto": MOE_GEMM_TILES_AUTO, "single": MOE_GEMM_TILES_SINGLE, "pair": MOE_GEMM_TILES_PAIR}[gemm_tiles]
-    return MoeConfig(T, d, E, k, d_ff, dt, kind, capacity, tiles)
+    lay = {"compact": MOE_LAYOUT_COMPACT, "padded": MOE_LAYOUT_PADDED}[layout]
+    return MoeConfig(T, d, E, k, d_ff, dt, kind, capacity, tiles, lay)
+
+
+def perm_rows(cfg) -> int:
+    """Rows P of x_perm, y_perm and perm_src: T*k, or E*capacity in the padded layout."""
+    return cfg.E * cfg.capacity if cfg.layout == MOE_LAYOUT_PADDED else cfg.T * cfg.k
 
 
 def _ptr(t):
@@ -177,7 +185,7 @@ def moe_permute(cfg, h, topk_idx, out=None, ws=None, status=None, stream=None):
     """Returns dict routed_counts, counts, offsets, dest_row, perm_src, x_perm."""
     dt = cfg.torch_dtype
     dev = _dev(h)
-    A = cfg.T * cfg.k
+    A = perm_rows(cfg)
     _check(h, (cfg.T, cfg.d), dt, "h")
     _check(topk_idx, (cfg.T, cfg.k), torch.int32, "topk_idx")
     if out is None:
@@ -201,8 +209,8 @@ def moe_grouped_ffn(cfg, x_perm, offsets, w13_packed=None, w_down=None, y_perm=N
     dt = cfg.torch_dtype
     dev = _dev(x_perm)
     rows = x_perm.shape[0]
-    if rows < max(cfg.T * cfg.k, 1):
-        raise ValueError("x_perm needs T*k rows")
+    if rows < max(perm_rows(cfg), 1):
+        raise ValueError("x_perm needs perm_rows(cfg) rows")
     _check(offsets, (cfg.E + 1,), torch.int32, "offsets")
     if cfg.expert_kind == MOE_EXPERT_SWIGLU:
         _check(w13_packed, (cfg.E, 2 * cfg.d_ff, cfg.d), dt, "w13_packed")
@@ -280,7 +288,7 @@ def moe_permute_static_scratch(cfg, h, topk_idx, out=None, status=None, stream=N
     Returns the same dict as moe_permute."""
     dt = cfg.torch_dtype
     dev = _dev(h)
-    A = cfg.T * cfg.k
+    A = perm_rows(cfg)
     _check(h, (cfg.T, cfg.d), dt, "h")
     _check(topk_idx, (cfg.T, cfg.k), torch.int32, "topk_idx")
     if out is None:

@@ -58,15 +58,25 @@ bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p
 
 int elem_bytes(const moe_config& c) { return c.dtype == MOE_DTYPE_BF16 ? 2 : 4; }
 
+// Rows of the permuted buffers: kept rows only (at most T*k), or capacity
+// rows per expert in the padded layout.
+size_t perm_rows(const moe_config& c) {
+  return c.layout == MOE_LAYOUT_PADDED ? static_cast<size_t>(c.E) * c.capacity : static_cast<size_t>(c.T) * c.k;
+}
+
 int check_cfg(const moe_config* c) {
   if (c == nullptr) return MOE_ERR_INVALID_ARG;
   if (c->T < 0 || c->d <= 0 || c->E <= 0 || c->k <= 0 || c->capacity < -1) return MOE_ERR_INVALID_ARG;
   if (c->dtype != MOE_DTYPE_BF16 && c->dtype != MOE_DTYPE_F32) return MOE_ERR_INVALID_ARG;
   if (c->expert_kind < MOE_EXPERT_SWIGLU || c->expert_kind > MOE_EXPERT_SCALE) return MOE_ERR_INVALID_ARG;
   if (c->gemm_tiles < MOE_GEMM_TILES_AUTO || c->gemm_tiles > MOE_GEMM_TILES_PAIR) return MOE_ERR_INVALID_ARG;
+  if (c->layout != MOE_LAYOUT_COMPACT && c->layout != MOE_LAYOUT_PADDED) return MOE_ERR_INVALID_ARG;
+  if (c->layout == MOE_LAYOUT_PADDED && c->capacity < 0) return MOE_ERR_INVALID_ARG;
   if (c->expert_kind == MOE_EXPERT_SWIGLU && c->d_ff <= 0) return MOE_ERR_INVALID_ARG;
   if (c->E > MOE_MAX_E || c->k > MOE_MAX_K || c->k > c->E) return MOE_ERR_UNSUPPORTED;
   if (static_cast<long long>(c->T) * c->k >= (1LL << 31)) return MOE_ERR_UNSUPPORTED;
+  if (c->layout == MOE_LAYOUT_PADDED && static_cast<long long>(c->E) * c->capacity >= (1LL << 31))
+    return MOE_ERR_UNSUPPORTED;
   if (c->dtype == MOE_DTYPE_BF16) {
     if (c->d % 128 != 0) return MOE_ERR_UNSUPPORTED;
     if (c->expert_kind == MOE_EXPERT_SWIGLU && c->d_ff % 128 != 0) return MOE_ERR_UNSUPPORTED;
@@ -105,7 +115,7 @@ PermuteScratch carve_permute(const moe_config& c, Carver& w) {
 
 void* carve_ffn(const moe_config& c, Carver& w) {
   if (c.expert_kind != MOE_EXPERT_SWIGLU) return nullptr;
-  return w.take<void>(static_cast<size_t>(c.T) * c.k * c.d_ff * elem_bytes(c));
+  return w.take<void>(perm_rows(c) * c.d_ff * elem_bytes(c));
 }
 
 struct LayerBufs {
@@ -117,6 +127,7 @@ struct LayerBufs {
 
 LayerBufs carve_layer(const moe_config& c, Carver& w) {
   const size_t A = static_cast<size_t>(c.T) * c.k;
+  const size_t P = perm_rows(c);
   const size_t row = static_cast<size_t>(c.d) * elem_bytes(c);
   LayerBufs b;
   b.idx = w.take<int32_t>(A * 4);
@@ -125,9 +136,9 @@ LayerBufs carve_layer(const moe_config& c, Carver& w) {
   b.kept = w.take<int32_t>(c.E * 4);
   b.offsets = w.take<int32_t>((c.E + 1) * 4);
   b.dest_row = w.take<int32_t>(A * 4);
-  b.perm_src = w.take<int32_t>(A * 4);
-  b.x_perm = w.take<void>(A * row);
-  b.y_perm = c.expert_kind == MOE_EXPERT_IDENTITY ? nullptr : w.take<void>(A * row);
+  b.perm_src = w.take<int32_t>(P * 4);
+  b.x_perm = w.take<void>(P * row);
+  b.y_perm = c.expert_kind == MOE_EXPERT_IDENTITY ? nullptr : w.take<void>(P * row);
   b.perm = carve_permute(c, w);
   b.h_mid = carve_ffn(c, w);
   return b;
@@ -171,17 +182,20 @@ int route_impl(const moe_config& c, const void* h, const void* w_router, const f
       launch_router_tc(tm_h, tm_w, c.T, c.d, c.E, c.k, npad, bias, logits, idx, gate, chunk_counts, status, s));
 }
 
+// pdl (here and in ffn_impl): the first kernel may launch as a programmatic
+// dependent of the previous kernel on the stream, which must belong to the
+// same library call.
 int permute_impl(const moe_config& c, const void* h, const int32_t* idx, int32_t* routed, int32_t* kept,
                  int32_t* offsets, int32_t* dest_row, int32_t* perm_src, void* x_perm, const PermuteScratch& p,
-                 bool counts_ready, int32_t* status, cudaStream_t s) {
+                 bool counts_ready, bool pdl, int32_t* status, cudaStream_t s) {
   return cuda_rc(launch_permute(h, static_cast<size_t>(c.d) * elem_bytes(c), idx, c.T, c.k, c.E, c.capacity,
-                                p.chunk_counts, p.chunk_base, routed, kept, offsets, dest_row, perm_src, x_perm,
-                                counts_ready, status, s));
+                                c.layout == MOE_LAYOUT_PADDED, p.chunk_counts, p.chunk_base, routed, kept, offsets,
+                                dest_row, perm_src, x_perm, counts_ready, pdl, status, s));
 }
 
 int ffn_impl(const moe_config& c, const void* x_perm, const int32_t* offsets, const void* w13, const void* w_down,
-             void* y_perm, void* h_mid, int32_t* status, cudaStream_t s) {
-  const int rows_max = c.T * c.k;
+             void* y_perm, void* h_mid, bool pdl, int32_t* status, cudaStream_t s) {
+  const int rows_max = static_cast<int>(perm_rows(c));
   if (rows_max == 0) return MOE_OK;
   if (c.expert_kind != MOE_EXPERT_SWIGLU)
     return cuda_rc(launch_scale_rows(c.dtype, c.expert_kind, x_perm, offsets, y_perm, rows_max, c.d, c.E, s));
@@ -200,11 +214,11 @@ int ffn_impl(const moe_config& c, const void* x_perm, const int32_t* offsets, co
   if (rc == MOE_OK) rc = make_map(&b2, w_down, static_cast<uint64_t>(E) * d, F, pair ? 128 : kGemmTileN);
   if (rc != MOE_OK) return rc;
   cudaError_t e = (pair ? launch_grouped_gemm_pair : launch_grouped_gemm_tc)(a1, b1, true, offsets, E, d, 2 * F,
-                                                                              F / 128, F, F, h_mid, status, s);
+                                                                              F / 128, F, F, h_mid, status, pdl, s);
   if (e != cudaSuccess) return MOE_ERR_CUDA;
   e = (pair ? launch_grouped_gemm_pair : launch_grouped_gemm_tc)(a2, b2, false, offsets, E, F, d,
                                                                   (d + kGemmTileN - 1) / kGemmTileN, d, d, y_perm,
-                                                                  status, s);
+                                                                  status, true, s);
   return cuda_rc(e);
 }
 
@@ -285,7 +299,7 @@ int32_t moe_permute(const moe_config* cfg, const void* h, const int32_t* topk_id
   Carver w(workspace);
   const PermuteScratch p = carve_permute(*cfg, w);
   return permute_impl(*cfg, h, topk_idx, routed_counts, counts, offsets, dest_row, perm_src, x_perm, p, false,
-                      status_dev, static_cast<cudaStream_t>(stream));
+                      false, status_dev, static_cast<cudaStream_t>(stream));
 }
 
 int32_t moe_grouped_ffn(const moe_config* cfg, const void* x_perm, const int32_t* offsets, const void* w13_packed,
@@ -303,7 +317,7 @@ int32_t moe_grouped_ffn(const moe_config* cfg, const void* x_perm, const int32_t
   if (ws_bytes < need || (need > 0 && (!workspace || !aligned(workspace, 16)))) return MOE_ERR_WORKSPACE;
   Carver w(workspace);
   void* h_mid = carve_ffn(*cfg, w);
-  return ffn_impl(*cfg, x_perm, offsets, w13_packed, w_down, y_perm, h_mid, status_dev,
+  return ffn_impl(*cfg, x_perm, offsets, w13_packed, w_down, y_perm, h_mid, false, status_dev,
                   static_cast<cudaStream_t>(stream));
 }
 
@@ -316,7 +330,8 @@ int32_t moe_unpermute_combine(const moe_config* cfg, const void* y_perm, const i
   if (!aligned(y_perm, 16) || !aligned(y, 16) || !aligned(dest_row, 4) || !aligned(topk_gate, 4))
     return MOE_ERR_UNSUPPORTED;
   return cuda_rc(
-      launch_combine(cfg->dtype, y_perm, dest_row, topk_gate, y, cfg->T, cfg->k, cfg->d, static_cast<cudaStream_t>(stream)));
+      launch_combine(cfg->dtype, y_perm, dest_row, topk_gate, y, cfg->T, cfg->k, cfg->d, false,
+                     static_cast<cudaStream_t>(stream)));
 }
 
 int32_t moe_layer_forward(const moe_config* cfg, const void* h, const void* w_router, const float* bias,
@@ -360,17 +375,20 @@ int32_t moe_layer_forward_timed(const moe_config* cfg, const void* h, const void
   rc = route_impl(c, h, w_router, bias, nullptr, b.idx, b.gate, router_counts ? b.perm.chunk_counts : nullptr,
                   status_dev, s);
   if (rc != MOE_OK || (rc = mark(1)) != MOE_OK) return rc;
+  // after the router, every kernel of the layer launches as a programmatic
+  // dependent of the one before it, so its launch and prologue overlap the
+  // previous kernel's tail
   rc = permute_impl(c, h, b.idx, b.routed, b.kept, b.offsets, b.dest_row, b.perm_src, b.x_perm, b.perm,
-                    router_counts, status_dev, s);
+                    router_counts, true, status_dev, s);
   if (rc != MOE_OK || (rc = mark(2)) != MOE_OK) return rc;
   const void* y_src = b.x_perm;
   if (c.expert_kind != MOE_EXPERT_IDENTITY) {
-    rc = ffn_impl(c, b.x_perm, b.offsets, w13_packed, w_down, b.y_perm, b.h_mid, status_dev, s);
+    rc = ffn_impl(c, b.x_perm, b.offsets, w13_packed, w_down, b.y_perm, b.h_mid, true, status_dev, s);
     if (rc != MOE_OK) return rc;
     y_src = b.y_perm;
   }
   if ((rc = mark(3)) != MOE_OK) return rc;
-  rc = cuda_rc(launch_combine(c.dtype, y_src, b.dest_row, b.gate, y, c.T, c.k, c.d, s));
+  rc = cuda_rc(launch_combine(c.dtype, y_src, b.dest_row, b.gate, y, c.T, c.k, c.d, true, s));
   if (rc != MOE_OK) return rc;
   return mark(4);
 }

@@ -46,6 +46,7 @@ MOE_DEV uint32_t load_route(const int32_t* __restrict__ idx, int t, int k, int E
 
 __global__ void __launch_bounds__(kChunkTokens) count_kernel(const int32_t* __restrict__ idx, int T, int k, int E,
                                                              int n_chunks, int32_t* __restrict__ chunk_counts) {
+  pdl_wait();
   __shared__ int hist[kMaxE];
   for (int e = threadIdx.x; e < E; e += blockDim.x) hist[e] = 0;
   __syncthreads();
@@ -66,8 +67,9 @@ constexpr int kScanPerLane = 8;
 
 __global__ void __launch_bounds__(1024) scan_kernel(const int32_t* __restrict__ chunk_counts,
                                                     int32_t* __restrict__ chunk_base, int n_chunks, int E, int cap,
-                                                    int32_t* __restrict__ routed, int32_t* __restrict__ kept,
-                                                    int32_t* __restrict__ offsets) {
+                                                    int padded, int32_t* __restrict__ routed,
+                                                    int32_t* __restrict__ kept, int32_t* __restrict__ offsets) {
+  pdl_wait();
   __shared__ int s_kept[kMaxE];
   __shared__ int s_warp[8];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -121,8 +123,8 @@ __global__ void __launch_bounds__(1024) scan_kernel(const int32_t* __restrict__ 
     asm volatile("bar.sync 1, 256;" ::: "memory");
     int before = 0;
     for (int w = 0; w < warp; ++w) before += s_warp[w];
-    if (e < E) offsets[e] = before + inc - v;
-    if (e == E - 1) offsets[E] = before + inc;
+    if (e < E) offsets[e] = padded ? e * cap : before + inc - v;
+    if (e == E - 1) offsets[E] = padded ? E * cap : before + inc;
   }
 }
 
@@ -144,7 +146,7 @@ MOE_DEV int warp_sum(int v) {
 // offsets; otherwise they come from scan_kernel.
 template <bool kFusedScan>
 __global__ void __launch_bounds__(kChunkTokens) rank_kernel(
-    const int32_t* __restrict__ idx, int T, int k, int E, int cap, int n_chunks,
+    const int32_t* __restrict__ idx, int T, int k, int E, int cap, int padded, int n_chunks,
     const int32_t* __restrict__ chunk_table,  // counts [n_chunks][E] (fused) or bases [n_chunks][E]
     const int32_t* __restrict__ offsets_in, int32_t* __restrict__ routed_out, int32_t* __restrict__ kept_out,
     int32_t* __restrict__ offsets_out, int32_t* __restrict__ dest_row, int32_t* __restrict__ perm_src,
@@ -156,6 +158,7 @@ __global__ void __launch_bounds__(kChunkTokens) rank_kernel(
   __shared__ int s_kept[kMaxE];
   __shared__ int s_off[kMaxE + 1];
   __shared__ int s_warp[kWarps];
+  pdl_wait();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int chunk = blockIdx.x;
   for (int i = threadIdx.x; i < kWarps * kMaxE; i += blockDim.x) (&mask[0][0])[i] = 0u;
@@ -212,9 +215,9 @@ __global__ void __launch_bounds__(kChunkTokens) rank_kernel(
     int before = 0;
     for (int w = 0; w < warp; ++w) before += s_warp[w];
     const int excl = before + inc - v0 - v1;
-    if (e0 < E) s_off[e0] = excl;
-    if (e0 + 1 < E) s_off[e0 + 1] = excl + v0;
-    if (threadIdx.x == blockDim.x - 1) s_off[E] = before + inc;
+    if (e0 < E) s_off[e0] = padded ? e0 * cap : excl;
+    if (e0 + 1 < E) s_off[e0 + 1] = padded ? (e0 + 1) * cap : excl + v0;
+    if (threadIdx.x == blockDim.x - 1) s_off[E] = padded ? E * cap : before + inc;
     __syncthreads();
     if (chunk == 0)
       for (int e = threadIdx.x; e <= E; e += blockDim.x) offsets_out[e] = s_off[e];
@@ -265,6 +268,26 @@ __global__ void __launch_bounds__(kChunkTokens) rank_kernel(
   }
 }
 
+// Padded layout: rows e*cap + i with i >= kept[e] are padding. One warp per
+// row writes zeros (16-byte stores) and marks perm_src -1; kept rows are
+// skipped (the row copy writes them).
+__global__ void __launch_bounds__(256) pad_rows_kernel(const int32_t* __restrict__ kept, int E, int cap,
+                                                       uint4* __restrict__ x_perm, int vpr,
+                                                       int32_t* __restrict__ perm_src) {
+  pdl_wait();
+  const int lane = threadIdx.x & 31;
+  const long long rows = static_cast<long long>(E) * cap;
+  const long long nw = static_cast<long long>(gridDim.x) * (blockDim.x >> 5);
+  for (long long r = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); r < rows; r += nw) {
+    const int e = static_cast<int>(r / cap);
+    const int i = static_cast<int>(r - static_cast<long long>(e) * cap);
+    if (i < kept[e]) continue;
+    uint4* row = x_perm + r * vpr;
+    for (int v = lane; v < vpr; v += 32) row[v] = make_uint4(0, 0, 0, 0);
+    if (lane == 0) perm_src[r] = -1;
+  }
+}
+
 constexpr int kCopyBuffers = 8;     // shared-memory row buffers per CTA
 constexpr int kCopyLead = 4;        // row loads kept in flight ahead of the stores
 constexpr int kCopyPiece = 8192;    // bytes per bulk transfer
@@ -281,6 +304,7 @@ __global__ void __launch_bounds__(32) permute_copy_bulk_kernel(const uint8_t* __
                                                                const int32_t* __restrict__ dest_row,
                                                                uint8_t* __restrict__ x_perm, int T, int k, int rb,
                                                                int tokens_per_cta, int32_t* status) {
+  pdl_wait();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((128u - (smem_addr(smem_raw) & 127u)) & 127u);
   const int piece = rb < kCopyPiece ? rb : kCopyPiece;
@@ -389,6 +413,7 @@ __global__ void __launch_bounds__(256) combine_kernel(const uint4* __restrict__ 
                                                       int vpr) {
   using V = Vec<DT>;
   constexpr int U = K >= 8 ? 1 : 8 / K;
+  pdl_wait();
   const int lane = threadIdx.x & 31;
   const int nw = gridDim.x * (blockDim.x >> 5);
   for (int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); t < T; t += nw) {
@@ -433,11 +458,13 @@ __global__ void __launch_bounds__(256) combine_kernel(const uint4* __restrict__ 
 
 template <int DT>
 cudaError_t launch_combine_k(const uint4* y_perm, const int32_t* dest_row, const float* gate, uint4* y, int T, int k,
-                             int vpr, int grid, cudaStream_t s) {
+                             int vpr, int grid, bool pdl, cudaStream_t s) {
+  cudaError_t err = cudaSuccess;
   switch (k) {
-#define MOE_COMBINE_K(KK) \
-  case KK:                \
-    combine_kernel<DT, KK><<<grid, 256, 0, s>>>(y_perm, dest_row, gate, y, T, vpr); \
+#define MOE_COMBINE_K(KK)                                                                                       \
+  case KK:                                                                                                     \
+    err = launch_kernel(combine_kernel<DT, KK>, dim3(grid), dim3(256), 0, s, pdl, 1, y_perm, dest_row, gate, y, T, \
+                        vpr);                                                                                  \
     break;
     MOE_COMBINE_K(1)
     MOE_COMBINE_K(2)
@@ -451,7 +478,7 @@ cudaError_t launch_combine_k(const uint4* y_perm, const int32_t* dest_row, const
     default:
       return cudaErrorInvalidValue;
   }
-  return cudaGetLastError();
+  return err != cudaSuccess ? err : cudaGetLastError();
 }
 
 int warp_grid(int T) {
@@ -463,46 +490,71 @@ int warp_grid(int T) {
 }  // namespace
 
 cudaError_t launch_permute(const void* h, size_t row_bytes, const int32_t* idx, int T, int k, int E, int cap,
-                           int32_t* chunk_counts, int32_t* chunk_base, int32_t* routed, int32_t* kept,
+                           bool padded, int32_t* chunk_counts, int32_t* chunk_base, int32_t* routed, int32_t* kept,
                            int32_t* offsets, int32_t* dest_row, int32_t* perm_src, void* x_perm,
-                           bool counts_ready, int32_t* status, cudaStream_t s) {
+                           bool counts_ready, bool pdl, int32_t* status, cudaStream_t s) {
+  // the first kernel launches as the caller asks; the later ones always as
+  // programmatic dependents of the one before
+  bool first = pdl;
+  auto next = [&]() {
+    const bool p = first;
+    first = true;
+    return p;
+  };
+  cudaError_t err = cudaSuccess;
   const int n_chunks = (T + kChunkTokens - 1) / kChunkTokens;
   if (n_chunks > 0 && !counts_ready)
-    count_kernel<<<n_chunks, kChunkTokens, 0, s>>>(idx, T, k, E, n_chunks, chunk_counts);
+    err = launch_kernel(count_kernel, dim3(n_chunks), dim3(kChunkTokens), 0, s, next(), 1, idx, T, k, E, n_chunks,
+                        chunk_counts);
+  if (err != cudaSuccess) return err;
   const bool fused = n_chunks > 0 && static_cast<long long>(E) * n_chunks <= kFusedScanMax;
   if (fused) {
-    rank_kernel<true><<<n_chunks, kChunkTokens, 0, s>>>(idx, T, k, E, cap, n_chunks, chunk_counts, nullptr, routed,
-                                                        kept, offsets, dest_row, perm_src, status);
+    err = launch_kernel(rank_kernel<true>, dim3(n_chunks), dim3(kChunkTokens), 0, s, next(), 1, idx, T, k, E, cap,
+                        static_cast<int>(padded), n_chunks, static_cast<const int32_t*>(chunk_counts), static_cast<const int32_t*>(nullptr),
+                        routed, kept, offsets, dest_row, perm_src, status);
   } else {
-    scan_kernel<<<1, 1024, 0, s>>>(chunk_counts, chunk_base, n_chunks, E, cap, routed, kept, offsets);
-    if (n_chunks > 0)
-      rank_kernel<false><<<n_chunks, kChunkTokens, 0, s>>>(idx, T, k, E, cap, n_chunks, chunk_base, offsets,
-                                                           nullptr, nullptr, nullptr, dest_row, perm_src, status);
+    err = launch_kernel(scan_kernel, dim3(1), dim3(1024), 0, s, next(), 1, static_cast<const int32_t*>(chunk_counts),
+                        chunk_base, n_chunks, E, cap, static_cast<int>(padded), routed, kept, offsets);
+    if (err == cudaSuccess && n_chunks > 0)
+      err = launch_kernel(rank_kernel<false>, dim3(n_chunks), dim3(kChunkTokens), 0, s, next(), 1, idx, T, k, E, cap,
+                          static_cast<int>(padded), n_chunks, static_cast<const int32_t*>(chunk_base), static_cast<const int32_t*>(offsets),
+                          static_cast<int32_t*>(nullptr), static_cast<int32_t*>(nullptr),
+                          static_cast<int32_t*>(nullptr), dest_row, perm_src, status);
   }
+  if (err != cudaSuccess) return err;
   if (n_chunks > 0) {
     const int tpc = kCopyTokensPerCta;
     const int piece = static_cast<int>(row_bytes < kCopyPiece ? row_bytes : kCopyPiece);
     const size_t smem = 128 + static_cast<size_t>(kCopyBuffers) * piece + kCopyBuffers * 8 + tpc * k * 4;
-    cudaError_t err = cudaFuncSetAttribute(permute_copy_bulk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                           static_cast<int>(smem));
+    err = cudaFuncSetAttribute(permute_copy_bulk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(smem));
     if (err != cudaSuccess) return err;
-    permute_copy_bulk_kernel<<<(T + tpc - 1) / tpc, 32, smem, s>>>(static_cast<const uint8_t*>(h), dest_row,
-                                                                   static_cast<uint8_t*>(x_perm), T, k,
-                                                                   static_cast<int>(row_bytes), tpc, status);
+    err = launch_kernel(permute_copy_bulk_kernel, dim3((T + tpc - 1) / tpc), dim3(32), smem, s, next(), 1,
+                        static_cast<const uint8_t*>(h), static_cast<const int32_t*>(dest_row),
+                        static_cast<uint8_t*>(x_perm), T, k, static_cast<int>(row_bytes), tpc, status);
+    if (err != cudaSuccess) return err;
+  }
+  if (padded && cap > 0) {
+    const long long rows = static_cast<long long>(E) * cap;
+    const long long want = (rows + 7) / 8;
+    const int grid = static_cast<int>(want < device_sm_count() * 8LL ? want : device_sm_count() * 8LL);
+    err = launch_kernel(pad_rows_kernel, dim3(grid), dim3(256), 0, s, next(), 1, static_cast<const int32_t*>(kept), E,
+                        cap, static_cast<uint4*>(x_perm), static_cast<int>(row_bytes / 16), perm_src);
+    if (err != cudaSuccess) return err;
   }
   return cudaGetLastError();
 }
 
 cudaError_t launch_combine(int dtype, const void* y_perm, const int32_t* dest_row, const float* gate, void* y,
-                           int T, int k, int d, cudaStream_t s) {
+                           int T, int k, int d, bool pdl, cudaStream_t s) {
   if (T == 0) return cudaSuccess;
   const int elem = dtype == MOE_DTYPE_BF16 ? 2 : 4;
   const int vpr = d * elem / 16;
   if (dtype == MOE_DTYPE_BF16)
     return launch_combine_k<MOE_DTYPE_BF16>(static_cast<const uint4*>(y_perm), dest_row, gate,
-                                            static_cast<uint4*>(y), T, k, vpr, warp_grid(T), s);
+                                            static_cast<uint4*>(y), T, k, vpr, warp_grid(T), pdl, s);
   return launch_combine_k<MOE_DTYPE_F32>(static_cast<const uint4*>(y_perm), dest_row, gate, static_cast<uint4*>(y),
-                                         T, k, vpr, warp_grid(T), s);
+                                         T, k, vpr, warp_grid(T), pdl, s);
 }
 
 }  // namespace moe

@@ -117,6 +117,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     tma_prefetch_desc(&tm_a);
     tma_prefetch_desc(&tm_b);
   }
+  pdl_wait();  // offsets and the A rows come from the kernels before this one
   for (int e = threadIdx.x; e <= E; e += blockDim.x) s_off[e] = a.offsets[e];
   __syncthreads();
   if (warp == 0) {
@@ -374,6 +375,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     tma_prefetch_desc(&tm_a);
     tma_prefetch_desc(&tm_b);
   }
+  pdl_wait();  // offsets and the A rows come from the kernels before this one
   for (int e = threadIdx.x; e <= E; e += blockDim.x) s_off[e] = a.offsets[e];
   __syncthreads();
   if (warp == 0) {
@@ -697,7 +699,7 @@ int band_rows(int tile_rows, int K, int lo, int hi) {
 
 cudaError_t launch_grouped_gemm_tc(const CUtensorMap& tm_a, const CUtensorMap& tm_b, bool swiglu,
                                    const int32_t* offsets, int E, int K, int n_per_expert, int n_tiles,
-                                   int out_cols, int ldd, void* D, int32_t* status, cudaStream_t s) {
+                                   int out_cols, int ldd, void* D, int32_t* status, bool pdl, cudaStream_t s) {
   GemmArgs a{offsets, E, K, n_per_expert, n_tiles, out_cols, ldd, static_cast<__nv_bfloat16*>(D), status,
              band_rows(kBM, K, 8, 32)};
   const size_t smem = gemm_smem_bytes();
@@ -707,46 +709,38 @@ cudaError_t launch_grouped_gemm_tc(const CUtensorMap& tm_a, const CUtensorMap& t
     err = cudaFuncSetAttribute(grouped_gemm_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                static_cast<int>(smem));
     if (err != cudaSuccess) return err;
-    grouped_gemm_kernel<true><<<grid, kGemmThreads, smem, s>>>(tm_a, tm_b, a);
+    err = launch_kernel(grouped_gemm_kernel<true>, dim3(grid), dim3(kGemmThreads), smem, s, pdl, 1, tm_a, tm_b, a);
+    if (err != cudaSuccess) return err;
   } else {
     err = cudaFuncSetAttribute(grouped_gemm_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                static_cast<int>(smem));
     if (err != cudaSuccess) return err;
-    grouped_gemm_kernel<false><<<grid, kGemmThreads, smem, s>>>(tm_a, tm_b, a);
+    err = launch_kernel(grouped_gemm_kernel<false>, dim3(grid), dim3(kGemmThreads), smem, s, pdl, 1, tm_a, tm_b, a);
+    if (err != cudaSuccess) return err;
   }
   return cudaGetLastError();
 }
 
 cudaError_t launch_grouped_gemm_pair(const CUtensorMap& tm_a, const CUtensorMap& tm_b, bool swiglu,
                                      const int32_t* offsets, int E, int K, int n_per_expert, int n_tiles, int out_cols,
-                                     int ldd, void* D, int32_t* status, cudaStream_t s) {
+                                     int ldd, void* D, int32_t* status, bool pdl, cudaStream_t s) {
   GemmArgs a{offsets, E, K, n_per_expert, n_tiles, out_cols, ldd, static_cast<__nv_bfloat16*>(D), status,
              band_rows(2 * kBM, K, 4, 16)};
   const size_t smem = pair_smem_bytes();
   const int grid = (device_sm_count() / 2) * 2;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(grid, 1, 1);
-  cfg.blockDim = dim3(kGemmThreads, 1, 1);
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = s;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 2;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
   cudaError_t err;
   if (swiglu) {
     err = cudaFuncSetAttribute(grouped_gemm_pair_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                static_cast<int>(smem));
     if (err != cudaSuccess) return err;
-    err = cudaLaunchKernelEx(&cfg, grouped_gemm_pair_kernel<true>, tm_a, tm_b, a);
+    err = launch_kernel(grouped_gemm_pair_kernel<true>, dim3(grid), dim3(kGemmThreads), smem, s, pdl, 2, tm_a, tm_b,
+                        a);
   } else {
     err = cudaFuncSetAttribute(grouped_gemm_pair_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                static_cast<int>(smem));
     if (err != cudaSuccess) return err;
-    err = cudaLaunchKernelEx(&cfg, grouped_gemm_pair_kernel<false>, tm_a, tm_b, a);
+    err = launch_kernel(grouped_gemm_pair_kernel<false>, dim3(grid), dim3(kGemmThreads), smem, s, pdl, 2, tm_a, tm_b,
+                        a);
   }
   if (err != cudaSuccess) return err;
   return cudaGetLastError();

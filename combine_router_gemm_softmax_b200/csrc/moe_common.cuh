@@ -47,6 +47,17 @@ MOE_DEV void mbar_init(uint64_t* bar, uint32_t count) {
 
 MOE_DEV void fence_mbar_init() { asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory"); }
 
+// Programmatic dependent launch. A kernel launched with programmatic stream
+// serialization may start before the previous kernel on its stream has
+// finished; pdl_wait() blocks until that kernel has completed and its memory
+// is visible (a no-op for an ordinary launch), so it must come before the
+// first access to anything an earlier kernel of the stream writes or reads.
+// No kernel here triggers its dependents early: the trigger is implicit when
+// its blocks exit. (An early trigger let the next kernel's blocks sit in
+// pdl_wait beside a long-running kernel, e.g. the combine beside the down
+// projection GEMM, and on B200 that cost up to 10% of the layer.)
+MOE_DEV void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 MOE_DEV void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
   asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)), "r"(bytes)
                : "memory");
@@ -305,5 +316,35 @@ MOE_DEV uint32_t pack_bf16x2(float lo, float hi) {
 }
 
 MOE_DEV float silu_f(float z) { return z / (1.0f + expf(-z)); }
+
+// Host: launch `kernel` on stream s, optionally as a programmatic dependent
+// launch (the kernel calls pdl_wait() before touching earlier kernels' data)
+// and optionally in clusters of cluster_x CTAs along x.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_kernel(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                                 bool pdl, unsigned cluster_x, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[2];
+  unsigned n = 0;
+  if (pdl) {
+    attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[n].val.programmaticStreamSerializationAllowed = 1;
+    ++n;
+  }
+  if (cluster_x > 1) {
+    attr[n].id = cudaLaunchAttributeClusterDimension;
+    attr[n].val.clusterDim.x = cluster_x;
+    attr[n].val.clusterDim.y = 1;
+    attr[n].val.clusterDim.z = 1;
+    ++n;
+  }
+  cfg.attrs = attr;
+  cfg.numAttrs = n;
+  return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
 
 }  // namespace moe

@@ -33,20 +33,25 @@ cudaError_t launch_router_f32(const float* h, const float* w, int T, int d, int 
                               float* logits, int32_t* idx, float* gate, int32_t* status, cudaStream_t s);
 
 // dispatch.cu
+// padded: every expert owns `cap` rows of x_perm (offsets[e] = e * cap); the
+// rows past its kept count are zero-filled and their perm_src set to -1.
 cudaError_t launch_permute(const void* h, size_t row_bytes, const int32_t* idx, int T, int k, int E, int cap,
-                           int32_t* chunk_counts, int32_t* chunk_base, int32_t* routed, int32_t* kept,
+                           bool padded, int32_t* chunk_counts, int32_t* chunk_base, int32_t* routed, int32_t* kept,
                            int32_t* offsets, int32_t* dest_row, int32_t* perm_src, void* x_perm,
-                           bool counts_ready, int32_t* status, cudaStream_t s);
+                           bool counts_ready, bool pdl, int32_t* status, cudaStream_t s);
 cudaError_t launch_combine(int dtype, const void* y_perm, const int32_t* dest_row, const float* gate, void* y,
-                           int T, int k, int d, cudaStream_t s);
+                           int T, int k, int d, bool pdl, cudaStream_t s);
 
 // grouped_ffn.cu
+// Launch flags `pdl` (here and in launch_permute / launch_combine): launch as
+// a programmatic dependent of the previous kernel on the stream. Only set it
+// when that kernel belongs to the same library call.
 cudaError_t launch_grouped_gemm_tc(const CUtensorMap& tm_a, const CUtensorMap& tm_b, bool swiglu,
                                    const int32_t* offsets, int E, int K, int n_per_expert, int n_tiles,
-                                   int out_cols, int ldd, void* D, int32_t* status, cudaStream_t s);
+                                   int out_cols, int ldd, void* D, int32_t* status, bool pdl, cudaStream_t s);
 cudaError_t launch_grouped_gemm_pair(const CUtensorMap& tm_a, const CUtensorMap& tm_b, bool swiglu,
                                      const int32_t* offsets, int E, int K, int n_per_expert, int n_tiles, int out_cols,
-                                     int ldd, void* D, int32_t* status, cudaStream_t s);
+                                     int ldd, void* D, int32_t* status, bool pdl, cudaStream_t s);
 cudaError_t launch_ffn_f32(const float* x_perm, const int32_t* offsets, const float* w13, const float* wd,
                            float* h_mid, float* y_perm, int rows_max, int d, int F, int E, cudaStream_t s);
 cudaError_t launch_scale_rows(int dtype, int kind, const void* x_perm, const int32_t* offsets, void* y_perm,

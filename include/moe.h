@@ -36,7 +36,7 @@
  *    *status_dev (MOE_STATUS_* bits) when status_dev is not NULL. The caller
  *    zeroes it and reads it when convenient.
  *
- * Limits: 1 <= E <= 256, 1 <= k <= min(E, 8), T >= 0, T*k < 2^31.
+ * Limits: 1 <= E <= 256, 1 <= k <= min(E, 8), T >= 0, T*k < 2^31, E*capacity < 2^31 (PADDED).
  * bf16 path: d and F multiples of 128. fp32 path: d a multiple of 4.
  */
 #ifndef MOE_B200_H
@@ -84,6 +84,19 @@ extern "C" {
 #define MOE_GEMM_TILES_SINGLE 1
 #define MOE_GEMM_TILES_PAIR   2
 
+/* Row layout of the permuted buffers (x_perm, y_perm, perm_src) when a
+ * capacity is set. COMPACT: kept rows only, expert e at [offsets[e],
+ * offsets[e+1]) with offsets the prefix sum of the kept counts; P = T*k rows.
+ * PADDED: every expert owns exactly `capacity` rows, expert e at
+ * [e*capacity, (e+1)*capacity), kept rows first and the rest zero padding
+ * that the grouped FFN computes like any other row; P = E*capacity rows. This
+ * is the padded capacity-based arm that the evaluation in "Dropless MoE Is a
+ * Runtime Problem as Much as a Model Design" compares the dropless grouped
+ * computation against; y is the same in both layouts. PADDED needs
+ * capacity >= 0. */
+#define MOE_LAYOUT_COMPACT 0
+#define MOE_LAYOUT_PADDED  1
+
 #define MOE_OP_ROUTE       0
 #define MOE_OP_PERMUTE     1
 #define MOE_OP_GROUPED_FFN 2
@@ -103,6 +116,7 @@ typedef struct moe_config {
   int32_t expert_kind;  /* MOE_EXPERT_* */
   int32_t capacity;     /* -1: dropless; >= 0: per-expert cap in assignments */
   int32_t gemm_tiles;   /* MOE_GEMM_TILES_*: tile shape of the bf16 grouped GEMMs */
+  int32_t layout;       /* MOE_LAYOUT_*: row layout of the permuted buffers (P rows) */
 } moe_config;
 
 typedef void* moe_stream_t; /* cudaStream_t */
@@ -150,15 +164,18 @@ MOE_API int32_t moe_route(const moe_config* cfg, const void* h, const void* w_ro
  * slot's expert are dropped and flag MOE_STATUS_BAD_ROUTE.
  * rank(t,j) = number of tokens t' < t that picked the same expert. The slot is
  * kept iff capacity < 0 or rank < capacity.
- * Outputs (all written):
+ * Outputs (all written; P rows as given by cfg->layout):
  *   routed_counts [E]  assignments per expert before drops
  *   counts [E]         kept assignments per expert
- *   offsets [E+1]      exclusive prefix sum of counts; offsets[E] = kept total
+ *   offsets [E+1]      COMPACT: exclusive prefix sum of counts, offsets[E] = kept
+ *                      total; PADDED: offsets[e] = e*capacity
  *   dest_row [T, k]    row of x_perm holding slot (t,j), -1 if dropped
- *   perm_src [T*k]     token of each x_perm row (first offsets[E] entries valid)
- *   x_perm [T*k, d]    x_perm[dest_row[t,j]] = h[t], bitwise; rows of expert e
- *                      are [offsets[e], offsets[e+1]) in ascending token order;
- *                      rows past offsets[E] are left untouched. */
+ *   perm_src [P]       token of each x_perm row (COMPACT: first offsets[E]
+ *                      entries valid; PADDED: -1 on padding rows)
+ *   x_perm [P, d]      x_perm[dest_row[t,j]] = h[t], bitwise; the kept rows of
+ *                      expert e start at offsets[e], in ascending token order;
+ *                      COMPACT: rows past offsets[E] are left untouched;
+ *                      PADDED: the padding rows are written as zeros. */
 MOE_API int32_t moe_permute(const moe_config* cfg, const void* h, const int32_t* topk_idx,
                     int32_t* routed_counts, int32_t* counts, int32_t* offsets,
                     int32_t* dest_row, int32_t* perm_src, void* x_perm,
@@ -167,11 +184,11 @@ MOE_API int32_t moe_permute(const moe_config* cfg, const void* h, const int32_t*
 /* moe_grouped_ffn -- all experts over their variable-length row groups in one
  * grouped computation ("Dropless MoE Is a Runtime Problem as Much as a Model
  * Design": one implementation over a collection of expert shapes, no padding).
- * x_perm [T*k, d] and offsets [E+1] as written by moe_permute; the group sizes
+ * x_perm [P, d] and offsets [E+1] as written by moe_permute; the group sizes
  * are read on the device (no host synchronisation).
  * w13_packed [E, 2F, d] from moe_pack_weights, w_down [E, d, F] (SwiGLU only;
  * may be NULL for the identity and scale experts).
- * y_perm [T*k, d]: y_perm[r] = f_e(x_perm[r]) for r in [offsets[e], offsets[e+1]).
+ * y_perm [P, d]: y_perm[r] = f_e(x_perm[r]) for r in [offsets[e], offsets[e+1]).
  * bf16 path: silu(gate) * up is rounded to bf16 before the down projection. */
 MOE_API int32_t moe_grouped_ffn(const moe_config* cfg, const void* x_perm, const int32_t* offsets,
                         const void* w13_packed, const void* w_down, void* y_perm,

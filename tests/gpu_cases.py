@@ -37,6 +37,11 @@ SMALL = {
         name="small_pair_wide", T=2100, d=2048, E=4, k=2, F=640, bias="gauss_0.5", gemm_tiles="pair"),
     "small_skewed_pair": W.get("skewed").with_(
         name="small_skewed_pair", T=777, d=256, E=40, k=4, F=384, gemm_tiles="pair"),
+    # padded capacity layout: capacity 97 is not a multiple of the 128-row
+    # tile, so every expert's last tile is ragged and mixes kept and padding rows
+    "small_skewed_padded": W.get("skewed").with_(
+        name="small_skewed_padded", T=777, d=256, E=40, k=4, F=384,
+        capacity=W.capacity_factor_cap(777, 4, 40), layout="padded"),
 }
 
 
@@ -45,7 +50,7 @@ def workload(name):
 
 
 def cfg_for(wl) -> M.MoeConfig:
-    return M.config(wl.T, wl.d, wl.E, wl.k, wl.F, wl.dtype, wl.expert_kind, wl.capacity, wl.gemm_tiles)
+    return M.config(wl.T, wl.d, wl.E, wl.k, wl.F, wl.dtype, wl.expert_kind, wl.capacity, wl.gemm_tiles, wl.layout)
 
 
 @functools.lru_cache(maxsize=3)

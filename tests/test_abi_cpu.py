@@ -118,3 +118,21 @@ def test_small_workspace_rejected(L):
     p = ctypes.c_void_p(0x1000)
     rc = L.moe_permute(ctypes.byref(cfg), p, p, p, p, p, p, p, p, p, 16, None, None)
     assert rc == M.MOE_ERR_WORKSPACE
+
+
+def test_layout_checked_and_sized(L):
+    """The padded layout needs a capacity and sizes the permuted buffers at
+    E*capacity rows; an unknown layout value is rejected."""
+    bad = M.config(64, 128, 8, 2, 256, layout="padded")          # no capacity
+    assert L.moe_route(ctypes.byref(bad), None, None, None, None, None, None, None, 0, None, None) \
+        == M.MOE_ERR_INVALID_ARG
+    odd = M.config(64, 128, 8, 2, 256, capacity=20)
+    odd.layout = 9
+    assert M.moe_workspace_size(odd, M.MOE_OP_LAYER) == 0
+    compact = M.config(64, 128, 8, 2, 256, capacity=40)
+    padded = M.config(64, 128, 8, 2, 256, capacity=40, layout="padded")
+    assert M.perm_rows(compact) == 128 and M.perm_rows(padded) == 320
+    # h_mid [P, F] bf16 is the whole grouped-FFN workspace
+    assert M.moe_workspace_size(padded, M.MOE_OP_GROUPED_FFN) == 320 * 256 * 2
+    assert M.moe_workspace_size(compact, M.MOE_OP_GROUPED_FFN) == 128 * 256 * 2
+    assert M.moe_workspace_size(padded, M.MOE_OP_LAYER) > M.moe_workspace_size(compact, M.MOE_OP_LAYER)

@@ -19,10 +19,12 @@ from gpu_cases import DEV, DeviceCase, cfg_for, np64, np_, oracle_y, parity_case
 pytestmark = pytest.mark.gpu
 
 LAYER_CASES = ["tiny_f32", "tiny_f32_tagged", "small_ragged", "small_skewed", "small_skewed_capacity",
-               "small_many", "small_pair", "small_pair_wide", "small_skewed_pair", "mixtral_scaled", "skewed", "skewed_capacity", "many_small", "many_small_identity",
-               "mixtral_8x7b"]
+               "small_skewed_padded", "small_many", "small_pair", "small_pair_wide", "small_skewed_pair",
+               "mixtral_scaled", "skewed", "skewed_capacity", "skewed_capacity_padded", "many_small",
+               "many_small_identity", "mixtral_8x7b"]
 FULL_ORACLE = {"tiny_f32", "tiny_f32_tagged", "small_ragged", "small_skewed", "small_skewed_capacity",
-               "small_many", "small_pair", "small_pair_wide", "small_skewed_pair", "many_small_identity"}
+               "small_skewed_padded", "small_many", "small_pair", "small_pair_wide", "small_skewed_pair",
+               "many_small_identity"}
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -198,6 +200,70 @@ def _routes(kind, T, E, k, seed=0):
     ("random", 8320, 256, 2, -1), ("all_to_one", 8320, 256, 3, 70)])
 def test_permute_injected_routes(kind, T, E, k, cap):
     _permute_check(T, 256, E, k, _routes(kind, T, E, k), cap)
+
+
+def _permute_check_padded(T, d, E, k, idx, cap, dtype="bf16", seed=0):
+    tdt = torch.bfloat16 if dtype == "bf16" else torch.float32
+    h = torch.from_numpy(np.random.default_rng(seed).standard_normal((T, d)).astype(np.float32)).to(tdt)
+    cfg = M.config(T, d, E, k, 128, dtype, capacity=cap, layout="padded")
+    assert M.perm_rows(cfg) == E * cap
+    # stale bytes in the output buffers must not survive: padding rows are written
+    out = dict(routed_counts=torch.full((E,), -7, dtype=torch.int32, device=DEV),
+               counts=torch.full((E,), -7, dtype=torch.int32, device=DEV),
+               offsets=torch.full((E + 1,), -7, dtype=torch.int32, device=DEV),
+               dest_row=torch.full((T, k), -7, dtype=torch.int32, device=DEV),
+               perm_src=torch.full((max(E * cap, 1),), 12345, dtype=torch.int32, device=DEV),
+               x_perm=torch.full((max(E * cap, 1), d), 3.0, dtype=tdt, device=DEV))
+    M.moe_permute(cfg, h.to(DEV), torch.from_numpy(np.asarray(idx, np.int32)).to(DEV), out=out)
+    torch.cuda.synchronize()
+    ref = O.dispatch_meta_padded(np.asarray(idx), E, cap)
+    assert np_(out["counts"]).tolist() == ref["kept"].tolist()
+    assert np_(out["routed_counts"]).tolist() == ref["routed"].tolist()
+    assert np_(out["offsets"]).tolist() == ref["offsets"].tolist()
+    assert np.array_equal(np_(out["dest_row"]), ref["dest_row"])
+    ps = np_(out["perm_src"])[:E * cap]
+    assert np.array_equal(ps, ref["perm_src"])
+    xp = out["x_perm"][:E * cap].cpu()
+    bits = torch.int16 if dtype == "bf16" else torch.int32
+    kept_rows = torch.from_numpy(np.nonzero(ref["perm_src"] >= 0)[0])
+    pad_rows = torch.from_numpy(np.nonzero(ref["perm_src"] < 0)[0])
+    assert torch.equal(xp[kept_rows].view(bits), h[torch.from_numpy(ref["perm_src"][ref["perm_src"] >= 0])].view(bits))
+    assert bool((xp[pad_rows] == 0).all())
+
+
+@pytest.mark.parametrize("kind,T,E,k,cap", [
+    ("random", 999, 40, 4, 97), ("all_to_one", 700, 16, 3, 100), ("empty_experts", 513, 32, 4, 64),
+    ("random", 300, 4, 4, 0), ("random", 8320, 256, 3, 70), ("random", 200, 8, 2, 400)])
+def test_permute_padded_layout(kind, T, E, k, cap):
+    """Padded capacity layout: offsets e*C, kept rows at e*C + rank, padding
+    rows zero with perm_src -1 (checked against the oracle's padded layout)."""
+    _permute_check_padded(T, 256, E, k, _routes(kind, T, E, k), cap)
+
+
+def test_permute_padded_fp32_and_zero_tokens():
+    _permute_check_padded(100, 36, 5, 2, _routes("random", 100, 5, 2), 30, dtype="f32")
+    _permute_check_padded(0, 128, 4, 2, np.zeros((0, 2), np.int32), 8)
+
+
+def test_layer_padded_equals_compact():
+    """The padded arm computes the padding rows too but returns the same y,
+    bit for bit, as the compact capacity layout."""
+    a, b = dev_case("small_skewed_capacity"), dev_case("small_skewed_padded")
+    assert (a.wl.T, a.wl.d, a.wl.E, a.wl.k, a.wl.F, a.wl.capacity) == (b.wl.T, b.wl.d, b.wl.E, b.wl.k, b.wl.F,
+                                                                        b.wl.capacity)
+    ya, yb = a.layer()["y"], b.layer()["y"]
+    torch.cuda.synchronize()
+    assert torch.equal(ya.view(torch.int16), yb.view(torch.int16))
+
+
+def test_config_layout_checks():
+    with pytest.raises(M.MoeError):
+        M.moe_layer_forward(M.config(64, 128, 4, 2, 128, layout="padded"),  # padded needs a capacity
+                            torch.zeros((64, 128), dtype=torch.bfloat16, device=DEV),
+                            torch.zeros((4, 128), dtype=torch.bfloat16, device=DEV),
+                            w13_packed=torch.zeros((4, 256, 128), dtype=torch.bfloat16, device=DEV),
+                            w_down=torch.zeros((4, 128, 128), dtype=torch.bfloat16, device=DEV),
+                            ws=torch.zeros(1 << 20, dtype=torch.uint8, device=DEV))
 
 
 def test_permute_fp32_rows():

@@ -60,3 +60,5 @@ def test_launch_count_per_step():
     assert bench.launches(M.config(64, 32, 4, 2, 64, dtype="f32")) == 7
     assert bench.launches(M.config(65536, 128, 256, 2, 128)) == 7      # 256 * 512 chunks: separate scan
     assert bench.launches(M.config(8192, 2048, 128, 8, 768)) == 6      # 128 * 64 chunks: scan inside rank
+    assert bench.launches(M.config(64, 128, 8, 2, 128, capacity=20, layout="padded")) == 7  # + padding fill
+    assert bench.launches(M.config(64, 128, 8, 2, 128, capacity=0, layout="padded")) == 6

@@ -52,6 +52,8 @@ class Workload:
     expert_kind: "swiglu" | "identity" | "scale"
     tagged: identity-tagged tokens h_t = (t+1) * onehot(t mod d).
     gemm_tiles: "auto" | "single" | "pair" (tile shape of the grouped GEMMs).
+    layout: "compact" | "padded" (row layout of the permuted buffers with a
+        capacity: kept rows only, or capacity rows per expert).
     """
 
     name: str
@@ -66,6 +68,7 @@ class Workload:
     expert_kind: str = "swiglu"
     tagged: bool = False
     gemm_tiles: str = "auto"
+    layout: str = "compact"
     note: str = ""
 
     @property
@@ -112,6 +115,9 @@ VARIANTS = {
     "skewed_capacity": WORKLOADS["skewed"].with_(
         name="skewed_capacity", capacity=capacity_factor_cap(16384, 6, 64),
         note="skewed routing with capacity floor(1.25*T*k/E)=1920, overflow dropped in token order"),
+    "skewed_capacity_padded": WORKLOADS["skewed"].with_(
+        name="skewed_capacity_padded", capacity=capacity_factor_cap(16384, 6, 64), layout="padded",
+        note="skewed routing, capacity 1920, padded capacity-based layout: every expert computes 1920 rows"),
     "many_small_identity": WORKLOADS["many_small"].with_(
         name="many_small_identity", expert_kind="identity",
         note="many small experts with identity experts: permute + unpermute only"),
