@@ -90,7 +90,7 @@ extern "C" {
  * PADDED: every expert owns exactly `capacity` rows, expert e at
  * [e*capacity, (e+1)*capacity), kept rows first and the rest zero padding
  * that the grouped FFN computes like any other row; P = E*capacity rows. This
- * is the padded capacity-based arm that the evaluation in "Dropless MoE Is a
+ * is the fixed-capacity padded arm that the evaluation in "Dropless MoE Is a
  * Runtime Problem as Much as a Model Design" compares the dropless grouped
  * computation against; y is the same in both layouts. PADDED needs
  * capacity >= 0. */

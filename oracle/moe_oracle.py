@@ -196,15 +196,16 @@ def dispatch_meta(idx, E, cap=-1):
 
 
 def dispatch_meta_padded(idx, E, cap):
-    """The padded capacity-based layout, the comparison arm of the evaluation
-    the dropless page proposes ("Dropless MoE Is a Runtime Problem as Much as
-    a Model Design": grouped GEMM avoids "padding all experts to a common
-    capacity"; its reproducible-evaluation paragraph compares padded
-    capacity-based against dropless). Every expert owns a buffer of exactly
-    cap rows: expert e's rows are [e*cap, (e+1)*cap). The kept assignments and
-    their ranks are those of the capacity mode (dispatch_meta with the same
-    cap); a kept assignment of rank r goes to row e*cap + r, and the rows past
-    an expert's kept count are padding (perm_src = -1, a zero row in x_perm).
+    """The padded layout with a fixed per-expert capacity: the comparison arm
+    of the evaluation in "Dropless MoE Is a Runtime Problem as Much as a Model
+    Design" (its grouped-GEMM paragraph contrasts one grouped computation with
+    padding every expert up to one shared capacity; its evaluation paragraph
+    lists that padded capacity arm beside the dropless one). Every expert owns
+    a buffer of exactly cap rows: expert e's rows are [e*cap, (e+1)*cap). The
+    kept assignments and their ranks are those of the capacity mode
+    (dispatch_meta with the same cap); a kept assignment of rank r goes to row
+    e*cap + r, and the rows past an expert's kept count are padding
+    (perm_src = -1, a zero row in x_perm).
 
     Returns dispatch_meta's dict with offsets [E+1] = e*cap, dest_row [T,k] and
     perm_src [E*cap] in this layout.

@@ -117,7 +117,7 @@ VARIANTS = {
         note="skewed routing with capacity floor(1.25*T*k/E)=1920, overflow dropped in token order"),
     "skewed_capacity_padded": WORKLOADS["skewed"].with_(
         name="skewed_capacity_padded", capacity=capacity_factor_cap(16384, 6, 64), layout="padded",
-        note="skewed routing, capacity 1920, padded capacity-based layout: every expert computes 1920 rows"),
+        note="skewed routing, capacity 1920, padded layout: every expert computes 1920 rows"),
     "many_small_identity": WORKLOADS["many_small"].with_(
         name="many_small_identity", expert_kind="identity",
         note="many small experts with identity experts: permute + unpermute only"),
