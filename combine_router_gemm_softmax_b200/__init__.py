@@ -14,7 +14,8 @@ tensors into its entry points:
 """
 from ._lib import (  # noqa: F401
     EXPORTED, LIB_PATH, MOE_DTYPE_BF16, MOE_DTYPE_F32, MOE_ERR_CUDA, MOE_ERR_INVALID_ARG, MOE_ERR_NO_DEVICE,
-    MOE_ERR_UNSUPPORTED, MOE_ERR_WORKSPACE, MOE_EXPERT_IDENTITY, MOE_EXPERT_SCALE, MOE_EXPERT_SWIGLU,
+    MOE_DISPATCH_AUTO, MOE_DISPATCH_COPY, MOE_DISPATCH_GATHER, MOE_ERR_UNSUPPORTED, MOE_ERR_WORKSPACE,
+    MOE_EXPERT_IDENTITY, MOE_EXPERT_SCALE, MOE_EXPERT_SWIGLU,
     MOE_GEMM_TILES_AUTO, MOE_GEMM_TILES_PAIR, MOE_GEMM_TILES_SINGLE, MOE_LAYOUT_COMPACT, MOE_LAYOUT_PADDED,
     MOE_MAX_E, MOE_MAX_K, MOE_OK, MOE_OP_GROUPED_FFN, MOE_OP_LAYER, MOE_OP_PERMUTE, MOE_OP_ROUTE, MOE_PACK_BLOCK,
     MOE_STATUS_BAD_ROUTE, MOE_STATUS_NAN_LOGIT, MOE_STATUS_TIMEOUT, MoeConfig, MoeError, config, lib,

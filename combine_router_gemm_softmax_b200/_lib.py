@@ -24,6 +24,7 @@ MOE_EXPERT_SWIGLU, MOE_EXPERT_IDENTITY, MOE_EXPERT_SCALE = 0, 1, 2
 MOE_OP_ROUTE, MOE_OP_PERMUTE, MOE_OP_GROUPED_FFN, MOE_OP_LAYER = 0, 1, 2, 3
 MOE_GEMM_TILES_AUTO, MOE_GEMM_TILES_SINGLE, MOE_GEMM_TILES_PAIR = 0, 1, 2
 MOE_LAYOUT_COMPACT, MOE_LAYOUT_PADDED = 0, 1
+MOE_DISPATCH_AUTO, MOE_DISPATCH_COPY, MOE_DISPATCH_GATHER = 0, 1, 2
 MOE_MAX_E, MOE_MAX_K, MOE_PACK_BLOCK = 256, 8, 128
 
 EXPORTED = ("moe_workspace_size", "moe_status_string", "moe_version", "moe_pack_weights", "moe_route",
@@ -40,7 +41,8 @@ class MoeError(RuntimeError):
 class MoeConfig(ctypes.Structure):
     _fields_ = [("T", ctypes.c_int32), ("d", ctypes.c_int32), ("E", ctypes.c_int32), ("k", ctypes.c_int32),
                 ("d_ff", ctypes.c_int32), ("dtype", ctypes.c_int32), ("expert_kind", ctypes.c_int32),
-                ("capacity", ctypes.c_int32), ("gemm_tiles", ctypes.c_int32), ("layout", ctypes.c_int32)]
+                ("capacity", ctypes.c_int32), ("gemm_tiles", ctypes.c_int32), ("layout", ctypes.c_int32),
+                ("dispatch", ctypes.c_int32)]
 
     def __repr__(self):
         return "MoeConfig(" + ", ".join(f"{n}={getattr(self, n)}" for n, _ in self._fields_) + ")"
@@ -91,13 +93,14 @@ def lib() -> ctypes.CDLL:
 
 
 def config(T, d, E, k, d_ff, dtype="bf16", expert_kind="swiglu", capacity=-1, gemm_tiles="auto",
-           layout="compact") -> MoeConfig:
+           layout="compact", dispatch="auto") -> MoeConfig:
     dt = {"bf16": MOE_DTYPE_BF16, "f32": MOE_DTYPE_F32, torch.bfloat16: MOE_DTYPE_BF16,
           torch.float32: MOE_DTYPE_F32}[dtype]
     kind = {"swiglu": MOE_EXPERT_SWIGLU, "identity": MOE_EXPERT_IDENTITY, "scale": MOE_EXPERT_SCALE}[expert_kind]
     tiles = {"auto": MOE_GEMM_TILES_AUTO, "single": MOE_GEMM_TILES_SINGLE, "pair": MOE_GEMM_TILES_PAIR}[gemm_tiles]
     lay = {"compact": MOE_LAYOUT_COMPACT, "padded": MOE_LAYOUT_PADDED}[layout]
-    return MoeConfig(T, d, E, k, d_ff, dt, kind, capacity, tiles, lay)
+    disp = {"auto": MOE_DISPATCH_AUTO, "copy": MOE_DISPATCH_COPY, "gather": MOE_DISPATCH_GATHER}[dispatch]
+    return MoeConfig(T, d, E, k, d_ff, dt, kind, capacity, tiles, lay, disp)
 
 
 def perm_rows(cfg) -> int:

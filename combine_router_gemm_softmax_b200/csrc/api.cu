@@ -64,6 +64,17 @@ size_t perm_rows(const moe_config& c) {
   return c.layout == MOE_LAYOUT_PADDED ? static_cast<size_t>(c.E) * c.capacity : static_cast<size_t>(c.T) * c.k;
 }
 
+
+// Whether the layer's GEMM1 can gather its A rows from h (no x_perm).
+bool gather_supported(const moe_config& c) {
+  return c.dtype == MOE_DTYPE_BF16 && c.expert_kind == MOE_EXPERT_SWIGLU && c.layout == MOE_LAYOUT_COMPACT &&
+         c.gemm_tiles != MOE_GEMM_TILES_PAIR;
+}
+
+bool layer_gathers(const moe_config& c) {
+  return c.dispatch != MOE_DISPATCH_COPY && gather_supported(c);
+}
+
 int check_cfg(const moe_config* c) {
   if (c == nullptr) return MOE_ERR_INVALID_ARG;
   if (c->T < 0 || c->d <= 0 || c->E <= 0 || c->k <= 0 || c->capacity < -1) return MOE_ERR_INVALID_ARG;
@@ -72,6 +83,8 @@ int check_cfg(const moe_config* c) {
   if (c->gemm_tiles < MOE_GEMM_TILES_AUTO || c->gemm_tiles > MOE_GEMM_TILES_PAIR) return MOE_ERR_INVALID_ARG;
   if (c->layout != MOE_LAYOUT_COMPACT && c->layout != MOE_LAYOUT_PADDED) return MOE_ERR_INVALID_ARG;
   if (c->layout == MOE_LAYOUT_PADDED && c->capacity < 0) return MOE_ERR_INVALID_ARG;
+  if (c->dispatch < MOE_DISPATCH_AUTO || c->dispatch > MOE_DISPATCH_GATHER) return MOE_ERR_INVALID_ARG;
+  if (c->dispatch == MOE_DISPATCH_GATHER && !gather_supported(*c)) return MOE_ERR_UNSUPPORTED;
   if (c->expert_kind == MOE_EXPERT_SWIGLU && c->d_ff <= 0) return MOE_ERR_INVALID_ARG;
   if (c->E > MOE_MAX_E || c->k > MOE_MAX_K || c->k > c->E) return MOE_ERR_UNSUPPORTED;
   if (static_cast<long long>(c->T) * c->k >= (1LL << 31)) return MOE_ERR_UNSUPPORTED;
@@ -137,7 +150,7 @@ LayerBufs carve_layer(const moe_config& c, Carver& w) {
   b.offsets = w.take<int32_t>((c.E + 1) * 4);
   b.dest_row = w.take<int32_t>(A * 4);
   b.perm_src = w.take<int32_t>(P * 4);
-  b.x_perm = w.take<void>(P * row);
+  b.x_perm = layer_gathers(c) ? nullptr : w.take<void>(P * row);  // GEMM1 gathers from h instead
   b.y_perm = c.expert_kind == MOE_EXPERT_IDENTITY ? nullptr : w.take<void>(P * row);
   b.perm = carve_permute(c, w);
   b.h_mid = carve_ffn(c, w);
@@ -187,14 +200,17 @@ int route_impl(const moe_config& c, const void* h, const void* w_router, const f
 // same library call.
 int permute_impl(const moe_config& c, const void* h, const int32_t* idx, int32_t* routed, int32_t* kept,
                  int32_t* offsets, int32_t* dest_row, int32_t* perm_src, void* x_perm, const PermuteScratch& p,
-                 bool counts_ready, bool pdl, int32_t* status, cudaStream_t s) {
+                 bool counts_ready, bool copy_rows, bool pdl, int32_t* status, cudaStream_t s) {
   return cuda_rc(launch_permute(h, static_cast<size_t>(c.d) * elem_bytes(c), idx, c.T, c.k, c.E, c.capacity,
-                                c.layout == MOE_LAYOUT_PADDED, p.chunk_counts, p.chunk_base, routed, kept, offsets,
-                                dest_row, perm_src, x_perm, counts_ready, pdl, status, s));
+                                c.layout == MOE_LAYOUT_PADDED, copy_rows, p.chunk_counts, p.chunk_base, routed, kept,
+                                offsets, dest_row, perm_src, x_perm, counts_ready, pdl, status, s));
 }
 
+// gather_src / gather_rows (bf16 SwiGLU single tiles only; NULL otherwise):
+// GEMM1 reads A row r as gather_src[gather_rows[r]] instead of x_perm[r].
 int ffn_impl(const moe_config& c, const void* x_perm, const int32_t* offsets, const void* w13, const void* w_down,
-             void* y_perm, void* h_mid, bool pdl, int32_t* status, cudaStream_t s) {
+             void* y_perm, void* h_mid, const void* gather_src, const int32_t* gather_rows, bool pdl,
+             int32_t* status, cudaStream_t s) {
   const int rows_max = static_cast<int>(perm_rows(c));
   if (rows_max == 0) return MOE_OK;
   if (c.expert_kind != MOE_EXPERT_SWIGLU)
@@ -208,17 +224,20 @@ int ffn_impl(const moe_config& c, const void* x_perm, const int32_t* offsets, co
   // (256x256, each CTA of the pair stages half of the B tile).
   const bool pair = c.gemm_tiles == MOE_GEMM_TILES_PAIR;
   CUtensorMap a1, b1, a2, b2;
-  int rc = make_map(&a1, x_perm, rows_max, d, kTileM);
+  const bool gather = gather_rows != nullptr && !pair;
+  int rc = gather ? make_map(&a1, gather_src, c.T, d, 1) : make_map(&a1, x_perm, rows_max, d, kTileM);
   if (rc == MOE_OK) rc = make_map(&b1, w13, static_cast<uint64_t>(E) * 2 * F, d, pair ? 128 : kGemmTileN);
   if (rc == MOE_OK) rc = make_map(&a2, h_mid, rows_max, F, kTileM);
   if (rc == MOE_OK) rc = make_map(&b2, w_down, static_cast<uint64_t>(E) * d, F, pair ? 128 : kGemmTileN);
   if (rc != MOE_OK) return rc;
-  cudaError_t e = (pair ? launch_grouped_gemm_pair : launch_grouped_gemm_tc)(a1, b1, true, offsets, E, d, 2 * F,
-                                                                              F / 128, F, F, h_mid, status, pdl, s);
+  cudaError_t e =
+      pair ? launch_grouped_gemm_pair(a1, b1, true, offsets, E, d, 2 * F, F / 128, F, F, h_mid, status, pdl, s)
+           : launch_grouped_gemm_tc(a1, b1, true, offsets, E, d, 2 * F, F / 128, F, F, h_mid,
+                                    gather ? gather_rows : nullptr, status, pdl, s);
   if (e != cudaSuccess) return MOE_ERR_CUDA;
-  e = (pair ? launch_grouped_gemm_pair : launch_grouped_gemm_tc)(a2, b2, false, offsets, E, F, d,
-                                                                  (d + kGemmTileN - 1) / kGemmTileN, d, d, y_perm,
-                                                                  status, true, s);
+  const int n2 = (d + kGemmTileN - 1) / kGemmTileN;
+  e = pair ? launch_grouped_gemm_pair(a2, b2, false, offsets, E, F, d, n2, d, d, y_perm, status, true, s)
+           : launch_grouped_gemm_tc(a2, b2, false, offsets, E, F, d, n2, d, d, y_perm, nullptr, status, true, s);
   return cuda_rc(e);
 }
 
@@ -299,7 +318,7 @@ int32_t moe_permute(const moe_config* cfg, const void* h, const int32_t* topk_id
   Carver w(workspace);
   const PermuteScratch p = carve_permute(*cfg, w);
   return permute_impl(*cfg, h, topk_idx, routed_counts, counts, offsets, dest_row, perm_src, x_perm, p, false,
-                      false, status_dev, static_cast<cudaStream_t>(stream));
+                      true, false, status_dev, static_cast<cudaStream_t>(stream));
 }
 
 int32_t moe_grouped_ffn(const moe_config* cfg, const void* x_perm, const int32_t* offsets, const void* w13_packed,
@@ -317,7 +336,7 @@ int32_t moe_grouped_ffn(const moe_config* cfg, const void* x_perm, const int32_t
   if (ws_bytes < need || (need > 0 && (!workspace || !aligned(workspace, 16)))) return MOE_ERR_WORKSPACE;
   Carver w(workspace);
   void* h_mid = carve_ffn(*cfg, w);
-  return ffn_impl(*cfg, x_perm, offsets, w13_packed, w_down, y_perm, h_mid, false, status_dev,
+  return ffn_impl(*cfg, x_perm, offsets, w13_packed, w_down, y_perm, h_mid, nullptr, nullptr, false, status_dev,
                   static_cast<cudaStream_t>(stream));
 }
 
@@ -378,12 +397,14 @@ int32_t moe_layer_forward_timed(const moe_config* cfg, const void* h, const void
   // after the router, every kernel of the layer launches as a programmatic
   // dependent of the one before it, so its launch and prologue overlap the
   // previous kernel's tail
+  const bool gather = layer_gathers(c);
   rc = permute_impl(c, h, b.idx, b.routed, b.kept, b.offsets, b.dest_row, b.perm_src, b.x_perm, b.perm,
-                    router_counts, true, status_dev, s);
+                    router_counts, !gather, true, status_dev, s);
   if (rc != MOE_OK || (rc = mark(2)) != MOE_OK) return rc;
   const void* y_src = b.x_perm;
   if (c.expert_kind != MOE_EXPERT_IDENTITY) {
-    rc = ffn_impl(c, b.x_perm, b.offsets, w13_packed, w_down, b.y_perm, b.h_mid, true, status_dev, s);
+    rc = ffn_impl(c, b.x_perm, b.offsets, w13_packed, w_down, b.y_perm, b.h_mid, gather ? h : nullptr,
+                  gather ? b.perm_src : nullptr, true, status_dev, s);
     if (rc != MOE_OK) return rc;
     y_src = b.y_perm;
   }

@@ -490,7 +490,8 @@ int warp_grid(int T) {
 }  // namespace
 
 cudaError_t launch_permute(const void* h, size_t row_bytes, const int32_t* idx, int T, int k, int E, int cap,
-                           bool padded, int32_t* chunk_counts, int32_t* chunk_base, int32_t* routed, int32_t* kept,
+                           bool padded, bool copy_rows, int32_t* chunk_counts, int32_t* chunk_base, int32_t* routed,
+                           int32_t* kept,
                            int32_t* offsets, int32_t* dest_row, int32_t* perm_src, void* x_perm,
                            bool counts_ready, bool pdl, int32_t* status, cudaStream_t s) {
   // the first kernel launches as the caller asks; the later ones always as
@@ -522,7 +523,7 @@ cudaError_t launch_permute(const void* h, size_t row_bytes, const int32_t* idx, 
                           static_cast<int32_t*>(nullptr), dest_row, perm_src, status);
   }
   if (err != cudaSuccess) return err;
-  if (n_chunks > 0) {
+  if (n_chunks > 0 && copy_rows) {
     const int tpc = kCopyTokensPerCta;
     const int piece = static_cast<int>(row_bytes < kCopyPiece ? row_bytes : kCopyPiece);
     const size_t smem = 128 + static_cast<size_t>(kCopyBuffers) * piece + kCopyBuffers * 8 + tpc * k * 4;

@@ -40,7 +40,8 @@ constexpr uint32_t kStageBytes = kABytes + kBBytes;
 constexpr uint32_t kTmemCols = 2 * kBN;
 
 constexpr size_t gemm_smem_bytes() {
-  return 1024 + kStages * static_cast<size_t>(kStageBytes) + (2 * kStages + 5) * 8 + 16 + 2 * (kMaxE + 1) * 4;
+  return 1024 + kStages * static_cast<size_t>(kStageBytes) + (2 * kStages + 5) * 8 + 16 + 2 * (kMaxE + 1) * 4 +
+         kBM * 4;
 }
 
 struct GemmArgs {
@@ -54,6 +55,10 @@ struct GemmArgs {
   __nv_bfloat16* D;
   int32_t* status;
   int band;          // row tiles per band of the tile walk
+  // Gather mode (single-CTA kernel only): when set, A row r of the grouped
+  // problem is row gather_rows[r] of the tensor behind tm_a (a box of one
+  // row); rows at or past offsets[E] read row 0 and are never stored.
+  const int32_t* gather_rows;
 };
 
 // tile -> (expert, row tile within the expert, column tile)
@@ -96,6 +101,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   int* consumed_slot = reinterpret_cast<int*>(tmem_slot + 2);
   int* s_off = reinterpret_cast<int*>(tmem_slot + 4);  // [E+1]
   int* prefix = s_off + (kMaxE + 1);                   // [E+1]
+  int* s_rows = prefix + (kMaxE + 1);                  // [128] source rows of the A tile (gather mode)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int E = a.E;
@@ -157,16 +163,28 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
   int issued = 0;
   if (warp == 0) {
-    if (lane == 0) {
-      // ---------------------------------------------------------------- TMA producer
-      int stage = 0;
-      uint32_t phase = 0;
-      bool stop = false;
-      for (long long tile = blockIdx.x; tile < total && !stop; tile += gridDim.x) {
-        int e, m, n;
-        decode_tile(tile, m_total, a.n_tiles, a.band, prefix, E, e, m, n);
-        const int a_row = s_off[e] + m * kBM;
-        const int b_row = e * a.n_per_expert + n * kBN;
+    // ---------------------------------------------------------------- TMA producer
+    // lane 0 issues the loads; in gather mode the whole warp first stages the
+    // tile's 128 source rows in shared memory
+    const bool gather = a.gather_rows != nullptr;
+    const int kept_total = s_off[E];
+    int stage = 0;
+    uint32_t phase = 0;
+    bool stop = false;
+    for (long long tile = blockIdx.x; tile < total && !stop; tile += gridDim.x) {
+      int e, m, n;
+      decode_tile(tile, m_total, a.n_tiles, a.band, prefix, E, e, m, n);
+      const int a_row = s_off[e] + m * kBM;
+      const int b_row = e * a.n_per_expert + n * kBN;
+      if (gather) {
+        __syncwarp();  // the previous tile's rows were read by lane 0's last issue
+        for (int i = lane; i < kBM; i += 32) {
+          const int r = a_row + i;
+          s_rows[i] = r < kept_total ? a.gather_rows[r] : 0;
+        }
+        __syncwarp();
+      }
+      if (lane == 0) {
         for (int kb = 0; kb < nkb; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag)) {
             *abort_flag = 1;
@@ -174,7 +192,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             break;
           }
           mbar_expect_tx(&full[stage], kStageBytes);
-          tma_load_2d(sA + stage * kABytes, &tm_a, &full[stage], kb * kBK, a_row);
+          if (gather) {
+            uint8_t* dst = sA + stage * kABytes;
+#pragma unroll 4
+            for (int i = 0; i < kBM; i += 4)
+              tma_gather4(dst + i * (kBK * 2), &tm_a, &full[stage], kb * kBK, s_rows[i], s_rows[i + 1],
+                          s_rows[i + 2], s_rows[i + 3]);
+          } else {
+            tma_load_2d(sA + stage * kABytes, &tm_a, &full[stage], kb * kBK, a_row);
+          }
           tma_load_2d(sB + stage * kBBytes, &tm_b, &full[stage], kb * kBK, b_row);
           ++issued;
           if (++stage == kStages) {
@@ -183,6 +209,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           }
         }
       }
+      stop = __shfl_sync(0xffffffffu, stop, 0);
     }
   } else if (warp == 1) {
     if (lane == 0) {
@@ -699,9 +726,10 @@ int band_rows(int tile_rows, int K, int lo, int hi) {
 
 cudaError_t launch_grouped_gemm_tc(const CUtensorMap& tm_a, const CUtensorMap& tm_b, bool swiglu,
                                    const int32_t* offsets, int E, int K, int n_per_expert, int n_tiles,
-                                   int out_cols, int ldd, void* D, int32_t* status, bool pdl, cudaStream_t s) {
+                                   int out_cols, int ldd, void* D, const int32_t* gather_rows, int32_t* status,
+                                   bool pdl, cudaStream_t s) {
   GemmArgs a{offsets, E, K, n_per_expert, n_tiles, out_cols, ldd, static_cast<__nv_bfloat16*>(D), status,
-             band_rows(kBM, K, 8, 32)};
+             band_rows(kBM, K, 8, 32), gather_rows};
   const size_t smem = gemm_smem_bytes();
   const int grid = device_sm_count();
   cudaError_t err;
@@ -725,7 +753,7 @@ cudaError_t launch_grouped_gemm_pair(const CUtensorMap& tm_a, const CUtensorMap&
                                      const int32_t* offsets, int E, int K, int n_per_expert, int n_tiles, int out_cols,
                                      int ldd, void* D, int32_t* status, bool pdl, cudaStream_t s) {
   GemmArgs a{offsets, E, K, n_per_expert, n_tiles, out_cols, ldd, static_cast<__nv_bfloat16*>(D), status,
-             band_rows(2 * kBM, K, 4, 16)};
+             band_rows(2 * kBM, K, 4, 16), nullptr};
   const size_t smem = pair_smem_bytes();
   const int grid = (device_sm_count() / 2) * 2;
   cudaError_t err;

@@ -110,6 +110,17 @@ MOE_DEV void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar, int x
       : "memory");
 }
 
+// Row gather: four rows r0..r3 of a 2D tensor map whose box is 64 columns by
+// one row, columns [x, x+64), written to dst as four consecutive 128-byte rows
+// (the map's swizzle applies by shared-memory address, as for a tiled load).
+MOE_DEV void tma_gather4(void* dst, const CUtensorMap* map, uint64_t* bar, int x, int r0, int r1, int r2, int r3) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(smem_addr(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_addr(bar)), "r"(x), "r"(r0), "r"(r1), "r"(r2), "r"(r3)
+      : "memory");
+}
+
 // Untiled bulk copies (TMA engine, no tensor map). Addresses 16-byte aligned,
 // sizes multiples of 16 bytes.
 MOE_DEV void bulk_load(void* smem_dst, const void* gsrc, uint32_t bytes, uint64_t* bar) {

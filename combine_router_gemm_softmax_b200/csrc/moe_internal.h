@@ -35,8 +35,10 @@ cudaError_t launch_router_f32(const float* h, const float* w, int T, int d, int 
 // dispatch.cu
 // padded: every expert owns `cap` rows of x_perm (offsets[e] = e * cap); the
 // rows past its kept count are zero-filled and their perm_src set to -1.
+// copy_rows: false skips the x_perm row copy (the grouped GEMM gathers the
+// rows itself); everything else is still written.
 cudaError_t launch_permute(const void* h, size_t row_bytes, const int32_t* idx, int T, int k, int E, int cap,
-                           bool padded, int32_t* chunk_counts, int32_t* chunk_base, int32_t* routed, int32_t* kept,
+                           bool padded, bool copy_rows, int32_t* chunk_counts, int32_t* chunk_base, int32_t* routed, int32_t* kept,
                            int32_t* offsets, int32_t* dest_row, int32_t* perm_src, void* x_perm,
                            bool counts_ready, bool pdl, int32_t* status, cudaStream_t s);
 cudaError_t launch_combine(int dtype, const void* y_perm, const int32_t* dest_row, const float* gate, void* y,
@@ -46,9 +48,12 @@ cudaError_t launch_combine(int dtype, const void* y_perm, const int32_t* dest_ro
 // Launch flags `pdl` (here and in launch_permute / launch_combine): launch as
 // a programmatic dependent of the previous kernel on the stream. Only set it
 // when that kernel belongs to the same library call.
+// gather_rows (may be NULL): A row r is row gather_rows[r] of the tensor behind
+// tm_a, whose box must then be 64 columns by one row.
 cudaError_t launch_grouped_gemm_tc(const CUtensorMap& tm_a, const CUtensorMap& tm_b, bool swiglu,
                                    const int32_t* offsets, int E, int K, int n_per_expert, int n_tiles,
-                                   int out_cols, int ldd, void* D, int32_t* status, bool pdl, cudaStream_t s);
+                                   int out_cols, int ldd, void* D, const int32_t* gather_rows, int32_t* status,
+                                   bool pdl, cudaStream_t s);
 cudaError_t launch_grouped_gemm_pair(const CUtensorMap& tm_a, const CUtensorMap& tm_b, bool swiglu,
                                      const int32_t* offsets, int E, int K, int n_per_expert, int n_tiles, int out_cols,
                                      int ldd, void* D, int32_t* status, bool pdl, cudaStream_t s);

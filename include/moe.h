@@ -97,6 +97,19 @@ extern "C" {
 #define MOE_LAYOUT_COMPACT 0
 #define MOE_LAYOUT_PADDED  1
 
+/* How moe_layer_forward moves token rows to the grouped FFN. COPY: the
+ * dispatch writes x_perm (a bulk row copy) and GEMM1 reads it. GATHER: no
+ * x_perm; GEMM1's loader fetches each A row straight from h through the
+ * permutation (TMA tile::gather4, four rows per load), the fused dispatch of
+ * "Dropless MoE Is a Runtime Problem as Much as a Model Design" (fusing
+ * dispatch to cut intermediate writes). GATHER needs bf16, SwiGLU experts, the
+ * COMPACT layout and single-CTA tiles; AUTO picks GATHER where it applies,
+ * else COPY. The result is the same bit for bit. The stage entry points
+ * (moe_permute, moe_grouped_ffn) always use x_perm. */
+#define MOE_DISPATCH_AUTO   0
+#define MOE_DISPATCH_COPY   1
+#define MOE_DISPATCH_GATHER 2
+
 #define MOE_OP_ROUTE       0
 #define MOE_OP_PERMUTE     1
 #define MOE_OP_GROUPED_FFN 2
@@ -117,6 +130,7 @@ typedef struct moe_config {
   int32_t capacity;     /* -1: dropless; >= 0: per-expert cap in assignments */
   int32_t gemm_tiles;   /* MOE_GEMM_TILES_*: tile shape of the bf16 grouped GEMMs */
   int32_t layout;       /* MOE_LAYOUT_*: row layout of the permuted buffers (P rows) */
+  int32_t dispatch;     /* MOE_DISPATCH_*: x_perm row copy or gather inside GEMM1 (layer only) */
 } moe_config;
 
 typedef void* moe_stream_t; /* cudaStream_t */

@@ -62,8 +62,11 @@ def test_workspace_sizes(L):
     nc = 4096 // 128
     assert M.moe_workspace_size(cfg, M.MOE_OP_PERMUTE) == 2 * ((nc * 8 * 4 + 255) // 256 * 256)
     assert M.moe_workspace_size(cfg, M.MOE_OP_GROUPED_FFN) == 4096 * 2 * 3584 * 2
+    # the default layer gathers GEMM1's rows from h: y_perm and h_mid, no x_perm
     layer = M.moe_workspace_size(cfg, M.MOE_OP_LAYER)
-    assert layer > 2 * 4096 * 2 * 1024 * 2 + 4096 * 2 * 3584 * 2
+    assert 4096 * 2 * 1024 * 2 + 4096 * 2 * 3584 * 2 < layer < 2 * 4096 * 2 * 1024 * 2 + 4096 * 2 * 3584 * 2
+    copy = M.moe_workspace_size(M.config(4096, 1024, 8, 2, 3584, dispatch="copy"), M.MOE_OP_LAYER)
+    assert copy == layer + 4096 * 2 * 1024 * 2
     ident = M.config(4096, 1024, 8, 2, 3584, expert_kind="identity")
     assert M.moe_workspace_size(ident, M.MOE_OP_GROUPED_FFN) == 0
 
@@ -136,3 +139,19 @@ def test_layout_checked_and_sized(L):
     assert M.moe_workspace_size(padded, M.MOE_OP_GROUPED_FFN) == 320 * 256 * 2
     assert M.moe_workspace_size(compact, M.MOE_OP_GROUPED_FFN) == 128 * 256 * 2
     assert M.moe_workspace_size(padded, M.MOE_OP_LAYER) > M.moe_workspace_size(compact, M.MOE_OP_LAYER)
+
+
+def test_dispatch_mode_checked(L):
+    """GATHER is only for bf16 SwiGLU experts in the compact layout with
+    single-CTA tiles; other values are rejected before any CUDA call."""
+    ok = M.config(64, 128, 8, 2, 256, dispatch="gather")
+    assert M.moe_workspace_size(ok, M.MOE_OP_LAYER) > 0
+    for kw in (dict(dtype="f32"), dict(expert_kind="identity"), dict(gemm_tiles="pair"),
+               dict(capacity=20, layout="padded")):
+        cfg = M.config(64, 128, 8, 2, 256, dispatch="gather", **kw)
+        assert L.moe_route(ctypes.byref(cfg), None, None, None, None, None, None, None, 0, None, None) \
+            == M.MOE_ERR_UNSUPPORTED, kw
+    bad = M.config(64, 128, 8, 2, 256)
+    bad.dispatch = 3
+    assert L.moe_route(ctypes.byref(bad), None, None, None, None, None, None, None, 0, None, None) \
+        == M.MOE_ERR_INVALID_ARG

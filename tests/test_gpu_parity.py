@@ -256,6 +256,22 @@ def test_layer_padded_equals_compact():
     assert torch.equal(ya.view(torch.int16), yb.view(torch.int16))
 
 
+@pytest.mark.parametrize("name", ["small_ragged", "small_skewed", "small_many", "mixtral_scaled"])
+def test_layer_gather_dispatch_equals_copy(name):
+    """GEMM1 gathering its rows from h through the permutation gives the same
+    y, bit for bit, as the row copy into x_perm followed by tiled loads."""
+    dc = dev_case(name)
+    wl = dc.wl
+    base = dict(T=wl.T, d=wl.d, E=wl.E, k=wl.k, d_ff=wl.F, dtype=wl.dtype, expert_kind=wl.expert_kind,
+                capacity=wl.capacity)
+    ys = {}
+    for mode in ("copy", "gather"):
+        cfg = M.config(**base, dispatch=mode)
+        ys[mode] = M.moe_layer_forward(cfg, dc.h, dc.w_router, dc.bias, dc.w13, dc.w_down)
+    torch.cuda.synchronize()
+    assert torch.equal(ys["copy"].view(torch.int16), ys["gather"].view(torch.int16))
+
+
 def test_config_layout_checks():
     with pytest.raises(M.MoeError):
         M.moe_layer_forward(M.config(64, 128, 4, 2, 128, layout="padded"),  # padded needs a capacity
