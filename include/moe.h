@@ -103,9 +103,11 @@ extern "C" {
  * permutation (TMA tile::gather4, four rows per load), the fused dispatch of
  * "Dropless MoE Is a Runtime Problem as Much as a Model Design" (fusing
  * dispatch to cut intermediate writes). GATHER needs bf16, SwiGLU experts, the
- * COMPACT layout and single-CTA tiles; AUTO picks GATHER where it applies,
- * else COPY. The result is the same bit for bit. The stage entry points
- * (moe_permute, moe_grouped_ffn) always use x_perm. */
+ * COMPACT layout and single-CTA tiles. The result is the same bit for bit.
+ * AUTO is COPY: a tile reloads its A rows once per column tile, so the
+ * gather repeats for every column tile, and GATHER measured 2.2-2.4x slower
+ * per layer on B200. The stage entry points (moe_permute, moe_grouped_ffn)
+ * always use x_perm. */
 #define MOE_DISPATCH_AUTO   0
 #define MOE_DISPATCH_COPY   1
 #define MOE_DISPATCH_GATHER 2

@@ -62,11 +62,12 @@ def test_workspace_sizes(L):
     nc = 4096 // 128
     assert M.moe_workspace_size(cfg, M.MOE_OP_PERMUTE) == 2 * ((nc * 8 * 4 + 255) // 256 * 256)
     assert M.moe_workspace_size(cfg, M.MOE_OP_GROUPED_FFN) == 4096 * 2 * 3584 * 2
-    # the default layer gathers GEMM1's rows from h: y_perm and h_mid, no x_perm
+    # the default layer materialises x_perm; with GATHER, GEMM1 reads h directly
     layer = M.moe_workspace_size(cfg, M.MOE_OP_LAYER)
-    assert 4096 * 2 * 1024 * 2 + 4096 * 2 * 3584 * 2 < layer < 2 * 4096 * 2 * 1024 * 2 + 4096 * 2 * 3584 * 2
-    copy = M.moe_workspace_size(M.config(4096, 1024, 8, 2, 3584, dispatch="copy"), M.MOE_OP_LAYER)
-    assert copy == layer + 4096 * 2 * 1024 * 2
+    assert layer > 2 * 4096 * 2 * 1024 * 2 + 4096 * 2 * 3584 * 2
+    assert M.moe_workspace_size(M.config(4096, 1024, 8, 2, 3584, dispatch="copy"), M.MOE_OP_LAYER) == layer
+    gather = M.moe_workspace_size(M.config(4096, 1024, 8, 2, 3584, dispatch="gather"), M.MOE_OP_LAYER)
+    assert gather == layer - 4096 * 2 * 1024 * 2
     ident = M.config(4096, 1024, 8, 2, 3584, expert_kind="identity")
     assert M.moe_workspace_size(ident, M.MOE_OP_GROUPED_FFN) == 0
 
