@@ -141,7 +141,8 @@ def min_adjacent_gap(s, k):
 
 def capacity(T, k, E, factor_num=5, factor_den=4):
     """Per-expert cap in assignments, floor(factor * T * k / E), factor 1.25.
-    [CAPACITY] "factor x (total_tokens / num_experts)", counted in assignments."""
+    [CAPACITY] capacity is a factor times the tokens per expert; counted here in
+    assignments (T*k), the configuration text's reading."""
     return (factor_num * T * k) // (factor_den * E)
 
 
@@ -159,7 +160,7 @@ def valid_slots(idx, E):
 
 def dispatch_meta(idx, E, cap=-1):
     """Per-expert counts, offsets, drop decisions and the permutation.
-    [DISPATCH] "per-expert token counts ... from the routing map", tokens
+    [DISPATCH] counts per expert are derived from the routing map and tokens
     grouped by expert; [REPEAT] capacity resolved in order; [CAPACITY] overflow.
 
     Walks the assignments in token order. rank = number of earlier tokens that
@@ -285,9 +286,9 @@ def layer_forward(h, w_r, bias, k, kind, weights=None, cap=-1, tokens=None):
 
 def remote_assignments(expert_of_token, tokens_per_rank, experts_per_rank):
     """Count assignments whose expert lives on another rank than the token's
-    origin, and their bytes at a given row size. [DISPATCH] "Eight assignments
-    can leave one destination with five" (origin rank r owns tokens
-    r*tokens_per_rank ...). Host-side diagnostic only."""
+    origin, and their bytes at a given row size. [DISPATCH] worked example of the
+    routing maps (an uneven map sends most of eight assignments to one rank;
+    origin rank r owns tokens r*tokens_per_rank ...). Host-side diagnostic only."""
     e = np.asarray(expert_of_token)
     origin = np.arange(e.shape[0]) // tokens_per_rank
     dest = e // experts_per_rank
