@@ -293,3 +293,73 @@ def remote_assignments(expert_of_token, tokens_per_rank, experts_per_rank):
     origin = np.arange(e.shape[0]) // tokens_per_rank
     dest = e // experts_per_rank
     return int((origin != dest).sum())
+
+
+# ---------------------------------------------------------------- backward
+def layer_backward(h, w_r, bias, k, weights, cap, dy):
+    """Gradients of the scalar L = sum_t <dy_t, y_t> for the SwiGLU layer.
+
+    The pages define the forward pass only ([REPEAT] layer formulas) and treat
+    dropless MoE as a training workload ([DROPLESS]); the backward pass is the
+    chain rule through that definition, with the routing decision (which
+    experts, which slots are kept) held fixed, as it is piecewise constant:
+
+      y_t = sum over kept j of g_{t,j} o_{t,j},   o = W_d (silu(a) * u),
+      a = W_g h_t, u = W_u h_t,                  g_j = exp(s_j) / sum_i exp(s_i)
+                                                 over the picked slots i of t
+      dgate_{t,j} = <dy_t, o_{t,j}> (0 for a dropped slot)
+      ds_{t,j}    = g_j (dgate_j - sum_i g_i dgate_i)     (softmax over the picks)
+      do = g_j dy_t;  dW_d += do m^T with m = silu(a) * u;  dm = W_d^T do
+      da = dm * u * silu'(a),  silu'(a) = sig(a) (1 + a (1 - sig(a)));  du = dm * silu(a)
+      dW_g += da h_t^T;  dW_u += du h_t^T;  dh_t += W_g^T da + W_u^T du
+      router: dh_t += sum_j ds_j W_r[e_j];  dW_r[e_j] += ds_j h_t;  db[e_j] += ds_j
+
+    weights(e) -> (w_gate [F,d], w_up [F,d], w_down [d,F]). Returns dict with
+    dh [T,d], dw_router [E,d], dbias [E], dw_gate, dw_up [E,F,d], dw_down
+    [E,d,F], dgate and ds [T,k], all fp64.
+    """
+    h = np.asarray(h, F64)
+    w_r = np.asarray(w_r, F64)
+    dy = np.asarray(dy, F64)
+    T, d = h.shape
+    E = w_r.shape[0]
+    idx, g, _, _ = route(h, w_r, bias, k)
+    meta = dispatch_meta(idx, E, cap)
+    kept = meta["dest_row"] >= 0
+    F = np.asarray(weights(0)[0]).shape[0]
+    dh = np.zeros((T, d))
+    dwg = np.zeros((E, F, d))
+    dwu = np.zeros((E, F, d))
+    dwd = np.zeros((E, d, F))
+    dgate = np.zeros((T, k))
+    for e in range(E):
+        rows, js = np.nonzero(kept & (idx == e))
+        if rows.size == 0:
+            continue
+        wg, wu, wd = (np.asarray(w, F64) for w in weights(e))
+        x = h[rows]
+        a = x @ wg.T
+        u = x @ wu.T
+        with np.errstate(over="ignore"):
+            sg = 1.0 / (1.0 + np.exp(-a))
+        m = a * sg * u
+        o = m @ wd.T
+        dgate[rows, js] = np.sum(dy[rows] * o, axis=1)
+        do = g[rows, js, None] * dy[rows]
+        dwd[e] = do.T @ m
+        dm = do @ wd
+        da = dm * u * (sg * (1.0 + a * (1.0 - sg)))
+        du = dm * a * sg
+        dwg[e] = da.T @ x
+        dwu[e] = du.T @ x
+        dh[rows] += da @ wg + du @ wu          # a token names expert e at most once
+    ds = g * (dgate - np.sum(g * dgate, axis=1, keepdims=True))
+    dwr = np.zeros((E, d))
+    db = np.zeros(E)
+    for j in range(k):
+        e = np.asarray(idx[:, j], np.int64)
+        np.add.at(dwr, e, ds[:, j, None] * h)
+        np.add.at(db, e, ds[:, j])
+        dh += ds[:, j, None] * w_r[e]
+    return dict(dh=dh, dw_router=dwr, dbias=db, dw_gate=dwg, dw_up=dwu, dw_down=dwd, dgate=dgate, ds=ds,
+                idx=idx, gate=g, **{kk: meta[kk] for kk in ("dest_row", "offsets", "kept", "routed")})

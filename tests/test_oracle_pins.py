@@ -366,3 +366,66 @@ def test_skewed_bias_gives_hot_experts_and_empties():
     assert counts[list(W.SKEWED_EMPTY)].sum() == 0
     assert counts.max() >= 5 * counts.mean()
     assert O.dispatch_meta(idx, wl.E, O.capacity(wl.T, wl.k, wl.E))["kept"].max() == 1920
+
+
+# ---------------------------------------------------------------- backward: finite differences
+def _bwd_problem(seed, T=6, d=8, E=4, k=2, F=5):
+    r = np.random.default_rng(seed)
+    h = r.standard_normal((T, d))
+    w_r = r.standard_normal((E, d))
+    bias = r.standard_normal(E) * 0.3
+    wg = r.standard_normal((E, F, d)) / np.sqrt(d)
+    wu = r.standard_normal((E, F, d)) / np.sqrt(d)
+    wd = r.standard_normal((E, d, F)) / np.sqrt(F)
+    dy = r.standard_normal((T, d))
+    return h, w_r, bias, wg, wu, wd, dy
+
+
+@pytest.mark.parametrize("seed,cap", [(1, -1), (2, -1), (3, 2)])
+def test_backward_matches_central_differences(seed, cap):
+    """Every gradient of L = <dy, y> against central differences of the
+    forward definition (eps 1e-6, fp64); the routing decision is checked to
+    be unchanged by each perturbation, and cap=2 drops slots."""
+    h, w_r, bias, wg, wu, wd, dy = _bwd_problem(seed)
+    k, E = 2, w_r.shape[0]
+    s = O.router_logits(h, w_r, bias)
+    assert O.min_adjacent_gap(s, k).min() > 1e-3             # decisions far from any tie
+
+    def loss(h_, w_r_, b_, wg_, wu_, wd_):
+        out = O.layer_forward(h_, w_r_, b_, k, "swiglu", lambda e: (wg_[e], wu_[e], wd_[e]), cap)
+        return float(np.sum(dy * out["y"])), out["idx"], out["dest_row"]
+
+    g = O.layer_backward(h, w_r, bias, k, lambda e: (wg[e], wu[e], wd[e]), cap, dy)
+    base = [h, w_r, bias, wg, wu, wd]
+    names = ["dh", "dw_router", "dbias", "dw_gate", "dw_up", "dw_down"]
+    _, idx0, dest0 = loss(*base)
+    if cap >= 0:
+        assert (dest0 < 0).any()                                  # some slot is dropped
+    eps = 1e-6
+    r = np.random.default_rng(seed + 100)
+    for pi, name in enumerate(names):
+        p = base[pi]
+        flat = p.reshape(-1)
+        picks = r.choice(flat.size, size=min(flat.size, 12), replace=False)
+        for i in picks:
+            args_p = [a.copy() for a in base]
+            args_m = [a.copy() for a in base]
+            args_p[pi].reshape(-1)[i] += eps
+            args_m[pi].reshape(-1)[i] -= eps
+            lp, ip, dp = loss(*args_p)
+            lm, im, dm = loss(*args_m)
+            assert np.array_equal(ip, idx0) and np.array_equal(im, idx0)
+            assert np.array_equal(dp, dest0) and np.array_equal(dm, dest0)
+            fd = (lp - lm) / (2 * eps)
+            an = g[name].reshape(-1)[i]
+            assert abs(fd - an) <= 1e-6 * max(1.0, abs(fd)), (name, i, fd, an)
+
+
+def test_backward_gate_gradient_sums_to_zero():
+    """Softmax over the picks: for every token, sum_j ds_j = 0 (the gates sum
+    to one whatever the scores), so db sums to zero and each token's router
+    gradient lies in the span of the picked rows."""
+    h, w_r, bias, wg, wu, wd, dy = _bwd_problem(5, T=20)
+    g = O.layer_backward(h, w_r, bias, 2, lambda e: (wg[e], wu[e], wd[e]), -1, dy)
+    assert np.allclose(g["ds"].sum(axis=1), 0.0, atol=1e-12)
+    assert abs(g["dbias"].sum()) < 1e-10
