@@ -58,6 +58,8 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--gemm-tiles", choices=["auto", "single", "pair"], default="auto")
+    ap.add_argument("--backward", action="store_true",
+                    help="also time moe_layer_backward (bf16 SwiGLU, compact layout) and report it")
     return ap.parse_args()
 
 
@@ -329,6 +331,9 @@ def main():
     row_bytes = wl.d * wl.elem_bytes
 
     barrier()
+    bwd = run_backward(M, cfg, wl, h, wr, bias, w13, wd, ws, stream, dev, args.steps, args.seed + rank) \
+        if args.backward else None
+    barrier()
 
     if rank == 0:
         pk, pk_kind = peaks()
@@ -351,6 +356,15 @@ def main():
         }
         line["stages"] = stage_report(stages, wl, A_kept, pk, pk_kind)
         line["roofline"] = roofline(stages, wl, A_kept, pk, pk_kind)
+        if bwd is not None:
+            A_kept_b = int(counts.sum().item())
+            flops = 16.0 * A_kept_b * wl.d * wl.F          # incl. the recomputed gate/up GEMM
+            line["backward"] = {"ms_per_step": bwd, "tokens_per_s": wl.T / (bwd / 1e3),
+                                "gemm_tflops": flops / (bwd / 1e3) / 1e12,
+                                "train_step_tokens_per_s": wl.T / ((bwd + ms_max / args.steps) / 1e3),
+                                "note": "moe_layer_backward after one forward, steps back to back; "
+                                        "gemm_tflops counts 16*A*d*F (dgrad, wgrad and the gate/up recompute) "
+                                        "over the whole backward time"}
         line["routing"] = {"routed_counts_max": int(routed.max().item()),
                            "routed_counts_mean": float(routed.float().mean().item()),
                            "empty_experts": int((routed == 0).sum().item()), "kept": A_kept,
@@ -408,6 +422,35 @@ def run_e2e(M, cfg, wl, h_host, h0, y0, wr, bias, w13, wd, ws, stream, dev, step
     e1.record(stream)
     torch.cuda.synchronize()
     return e0.elapsed_time(e1)
+
+
+def run_backward(M, cfg, wl, h, wr, bias, w13, wd, ws, stream, dev, steps, seed):
+    """Device time (ms per call) of moe_layer_backward on the forward state
+    left in ws, CUDA events around `steps` back-to-back calls."""
+    import torch
+
+    import workloads as W
+
+    w13_t, wd_t = M.moe_pack_weights_backward(cfg, w13, wd, stream=stream)
+    dy = W.draw_dy(wl, seed).to(dev)
+    M.moe_layer_forward(cfg, h, wr, bias, w13, wd, ws=ws, stream=stream)
+    bws = M.workspace(cfg, M.MOE_OP_BACKWARD, dev)
+
+    def once():
+        return M.moe_layer_backward(cfg, h, wr, w13, w13_t, wd_t, dy, ws, with_bias=bias is not None, ws=bws,
+                                    stream=stream)
+
+    for _ in range(2):
+        once()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda._sleep(HOST_LEAD_CYCLES)
+    e0.record(stream)
+    for _ in range(steps):
+        once()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / steps
 
 
 def launches(cfg):

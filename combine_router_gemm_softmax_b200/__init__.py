@@ -9,6 +9,7 @@ tensors into its entry points:
     moe_pack_weights       gate/up interleave for the grouped FFN
     moe_grouped_ffn        grouped SwiGLU expert GEMMs over ragged groups
     moe_unpermute_combine  return outputs to their tokens, gate-weighted
+    moe_layer_backward     gradients of the layer (moe_pack_weights_backward first)
     moe_layer_forward      all of the above on one stream (moe_layer_forward_timed
                            with stage events)
 """
@@ -17,7 +18,9 @@ from ._lib import (  # noqa: F401
     MOE_DISPATCH_AUTO, MOE_DISPATCH_COPY, MOE_DISPATCH_GATHER, MOE_ERR_UNSUPPORTED, MOE_ERR_WORKSPACE,
     MOE_EXPERT_IDENTITY, MOE_EXPERT_SCALE, MOE_EXPERT_SWIGLU,
     MOE_GEMM_TILES_AUTO, MOE_GEMM_TILES_PAIR, MOE_GEMM_TILES_SINGLE, MOE_LAYOUT_COMPACT, MOE_LAYOUT_PADDED,
-    MOE_MAX_E, MOE_MAX_K, MOE_OK, MOE_OP_GROUPED_FFN, MOE_OP_LAYER, MOE_OP_PERMUTE, MOE_OP_ROUTE, MOE_PACK_BLOCK,
+    MOE_MAX_E, MOE_MAX_K, MOE_OK, MOE_OP_BACKWARD, MOE_OP_GROUPED_FFN, MOE_OP_LAYER, MOE_OP_PERMUTE, MOE_OP_ROUTE,
+    MOE_PACK_BLOCK,
     MOE_STATUS_BAD_ROUTE, MOE_STATUS_NAN_LOGIT, MOE_STATUS_TIMEOUT, MoeConfig, MoeError, config, lib,
-    moe_grouped_ffn, moe_layer_forward, moe_pack_weights, moe_permute, moe_permute_static_scratch, moe_route,
+    moe_grouped_ffn, moe_layer_backward, moe_layer_forward, moe_pack_weights, moe_pack_weights_backward,
+    moe_permute, moe_permute_static_scratch, moe_route,
     moe_unpermute_combine, moe_workspace_size, perm_rows, workspace)

@@ -21,7 +21,7 @@ MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_WORKSPACE, MOE_ERR_CUD
 MOE_STATUS_NAN_LOGIT, MOE_STATUS_BAD_ROUTE, MOE_STATUS_TIMEOUT = 1, 2, 4
 MOE_DTYPE_BF16, MOE_DTYPE_F32 = 0, 1
 MOE_EXPERT_SWIGLU, MOE_EXPERT_IDENTITY, MOE_EXPERT_SCALE = 0, 1, 2
-MOE_OP_ROUTE, MOE_OP_PERMUTE, MOE_OP_GROUPED_FFN, MOE_OP_LAYER = 0, 1, 2, 3
+MOE_OP_ROUTE, MOE_OP_PERMUTE, MOE_OP_GROUPED_FFN, MOE_OP_LAYER, MOE_OP_BACKWARD = 0, 1, 2, 3, 4
 MOE_GEMM_TILES_AUTO, MOE_GEMM_TILES_SINGLE, MOE_GEMM_TILES_PAIR = 0, 1, 2
 MOE_LAYOUT_COMPACT, MOE_LAYOUT_PADDED = 0, 1
 MOE_DISPATCH_AUTO, MOE_DISPATCH_COPY, MOE_DISPATCH_GATHER = 0, 1, 2
@@ -29,7 +29,8 @@ MOE_MAX_E, MOE_MAX_K, MOE_PACK_BLOCK = 256, 8, 128
 
 EXPORTED = ("moe_workspace_size", "moe_status_string", "moe_version", "moe_pack_weights", "moe_route",
             "moe_permute", "moe_grouped_ffn", "moe_unpermute_combine", "moe_layer_forward",
-            "moe_permute_static_scratch", "moe_layer_forward_timed")
+            "moe_permute_static_scratch", "moe_layer_forward_timed", "moe_pack_weights_backward",
+            "moe_layer_backward")
 
 
 class MoeError(RuntimeError):
@@ -72,6 +73,8 @@ _SIGS = {
     "moe_layer_forward": (I32, [CFG, P, P, P, P, P, P, P, P, P, P, P, SZ, P, P]),
     "moe_permute_static_scratch": (I32, [CFG, P, P, P, P, P, P, P, P, P, P]),
     "moe_layer_forward_timed": (I32, [CFG, P, P, P, P, P, P, P, P, P, P, P, SZ, P, P, P]),
+    "moe_pack_weights_backward": (I32, [CFG, P, P, P, P, P]),
+    "moe_layer_backward": (I32, [CFG, P, P, P, P, P, P, P, P, P, P, P, P, SZ, P, SZ, P, P]),
 }
 
 
@@ -305,4 +308,45 @@ def moe_permute_static_scratch(cfg, h, topk_idx, out=None, status=None, stream=N
         ctypes.byref(cfg), _ptr(h), _ptr(topk_idx), _ptr(out["routed_counts"]), _ptr(out["counts"]),
         _ptr(out["offsets"]), _ptr(out["dest_row"]), _ptr(out["perm_src"]), _ptr(out["x_perm"]), _ptr(status),
         _stream(stream)))
+    return out
+
+
+def moe_pack_weights_backward(cfg, w13_packed, w_down, stream=None):
+    """Per-expert transposes for the backward dgrad GEMMs: returns
+    (w13_t [E, d, 2F], w_down_t [E, F, d])."""
+    dt = cfg.torch_dtype
+    dev = _dev(w13_packed)
+    _check(w13_packed, (cfg.E, 2 * cfg.d_ff, cfg.d), dt, "w13_packed")
+    _check(w_down, (cfg.E, cfg.d, cfg.d_ff), dt, "w_down")
+    w13_t = torch.empty((cfg.E, cfg.d, 2 * cfg.d_ff), dtype=dt, device=dev)
+    w_down_t = torch.empty((cfg.E, cfg.d_ff, cfg.d), dtype=dt, device=dev)
+    _rc("moe_pack_weights_backward", lib().moe_pack_weights_backward(
+        ctypes.byref(cfg), _ptr(w13_packed), _ptr(w_down), _ptr(w13_t), _ptr(w_down_t), _stream(stream)))
+    return w13_t, w_down_t
+
+
+def moe_layer_backward(cfg, h, w_router, w13_packed, w13_t, w_down_t, dy, fwd_ws, with_bias=True, ws=None,
+                       status=None, stream=None):
+    """Gradients of <dy, y> for the moe_layer_forward call that last used
+    fwd_ws. Returns dict dh [T,d] (bf16), dw_router [E,d], dbias [E] (or None),
+    dw13 [E,2F,d] (packed row order), dw_down [E,d,F] (fp32)."""
+    dt = cfg.torch_dtype
+    dev = _dev(h)
+    _check(h, (cfg.T, cfg.d), dt, "h")
+    _check(w_router, (cfg.E, cfg.d), dt, "w_router")
+    _check(w13_packed, (cfg.E, 2 * cfg.d_ff, cfg.d), dt, "w13_packed")
+    _check(w13_t, (cfg.E, cfg.d, 2 * cfg.d_ff), dt, "w13_t")
+    _check(w_down_t, (cfg.E, cfg.d_ff, cfg.d), dt, "w_down_t")
+    _check(dy, (cfg.T, cfg.d), dt, "dy")
+    out = dict(dh=torch.empty((cfg.T, cfg.d), dtype=dt, device=dev),
+               dw_router=torch.empty((cfg.E, cfg.d), dtype=torch.float32, device=dev),
+               dbias=torch.empty(cfg.E, dtype=torch.float32, device=dev) if with_bias else None,
+               dw13=torch.empty((cfg.E, 2 * cfg.d_ff, cfg.d), dtype=torch.float32, device=dev),
+               dw_down=torch.empty((cfg.E, cfg.d, cfg.d_ff), dtype=torch.float32, device=dev))
+    if ws is None:
+        ws = workspace(cfg, MOE_OP_BACKWARD, dev)
+    _rc("moe_layer_backward", lib().moe_layer_backward(
+        ctypes.byref(cfg), _ptr(h), _ptr(w_router), _ptr(w13_packed), _ptr(w13_t), _ptr(w_down_t), _ptr(dy),
+        _ptr(out["dh"]), _ptr(out["dw_router"]), _ptr(out["dbias"]), _ptr(out["dw13"]), _ptr(out["dw_down"]),
+        _ptr(fwd_ws), fwd_ws.numel(), _ptr(ws), ws.numel(), _ptr(status), _stream(stream)))
     return out

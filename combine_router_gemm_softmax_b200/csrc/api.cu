@@ -160,9 +160,51 @@ LayerBufs carve_layer(const moe_config& c, Carver& w) {
   return b;
 }
 
+// Backward scratch. ppad_max bounds the padded column count of the
+// transposed activations: every expert's rows rounded up to 64.
+struct BackwardBufs {
+  void *dy_perm, *dh_mid, *dgu, *dx_perm;
+  float* ds;
+  int32_t* col_off;
+  void *dy_perm_t, *h_mid_t, *dgu_t, *x_perm_t;
+  int ppad_max;
+};
+
+int ppad_max(const moe_config& c) {
+  return static_cast<int>((perm_rows(c) + 63) / 64 * 64 + 64 * static_cast<size_t>(c.E));
+}
+
+BackwardBufs carve_backward(const moe_config& c, Carver& w) {
+  const size_t P = perm_rows(c), A = static_cast<size_t>(c.T) * c.k;
+  const size_t d = c.d, F = c.d_ff;
+  BackwardBufs b;
+  b.ppad_max = ppad_max(c);
+  const size_t pp = b.ppad_max;
+  b.dy_perm = w.take<void>(P * d * 2);
+  b.dh_mid = w.take<void>(P * F * 2);
+  b.dgu = w.take<void>(P * 2 * F * 2);
+  b.dx_perm = w.take<void>(P * d * 2);
+  b.ds = w.take<float>(A * 4);
+  b.col_off = w.take<int32_t>((c.E + 1) * 4);
+  b.dy_perm_t = w.take<void>(d * pp * 2);
+  b.h_mid_t = w.take<void>(F * pp * 2);
+  b.dgu_t = w.take<void>(2 * F * pp * 2);
+  b.x_perm_t = w.take<void>(d * pp * 2);
+  return b;
+}
+
+bool backward_supported(const moe_config& c) {
+  return c.dtype == MOE_DTYPE_BF16 && c.expert_kind == MOE_EXPERT_SWIGLU && c.layout == MOE_LAYOUT_COMPACT &&
+         !layer_gathers(c);
+}
+
 size_t ws_size(const moe_config& c, int op) {
   Carver w(nullptr);
   switch (op) {
+    case MOE_OP_BACKWARD:
+      if (!backward_supported(c)) return 0;
+      carve_backward(c, w);
+      return w.off;
     case MOE_OP_ROUTE:
       return 0;
     case MOE_OP_PERMUTE:
@@ -415,6 +457,100 @@ int32_t moe_layer_forward_timed(const moe_config* cfg, const void* h, const void
   rc = cuda_rc(launch_combine(c.dtype, y_src, b.dest_row, b.gate, y, c.T, c.k, c.d, true, s));
   if (rc != MOE_OK) return rc;
   return mark(4);
+}
+
+int32_t moe_pack_weights_backward(const moe_config* cfg, const void* w13_packed, const void* w_down, void* w13_t,
+                                  void* w_down_t, moe_stream_t stream) {
+  int rc = check_cfg(cfg);
+  if (rc != MOE_OK) return rc;
+  const moe_config& c = *cfg;
+  if (c.dtype != MOE_DTYPE_BF16 || c.expert_kind != MOE_EXPERT_SWIGLU) return MOE_ERR_UNSUPPORTED;
+  if (!w13_packed || !w_down || !w13_t || !w_down_t) return MOE_ERR_INVALID_ARG;
+  if (!aligned(w13_packed, 16) || !aligned(w_down, 16) || !aligned(w13_t, 16) || !aligned(w_down_t, 16))
+    return MOE_ERR_UNSUPPORTED;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = launch_transpose_batched(w13_packed, c.E, 2 * c.d_ff, c.d, w13_t, s);
+  if (e == cudaSuccess) e = launch_transpose_batched(w_down, c.E, c.d, c.d_ff, w_down_t, s);
+  return cuda_rc(e);
+}
+
+int32_t moe_layer_backward(const moe_config* cfg, const void* h, const void* w_router, const void* w13_packed,
+                           const void* w13_t, const void* w_down_t, const void* dy, void* dh, float* dw_router,
+                           float* dbias, float* dw13, float* dw_down, const void* fwd_workspace, size_t fwd_ws_bytes,
+                           void* workspace, size_t ws_bytes, int32_t* status_dev, moe_stream_t stream) {
+  int rc = check_cfg(cfg);
+  if (rc != MOE_OK) return rc;
+  const moe_config& c = *cfg;
+  if (!backward_supported(c)) return MOE_ERR_UNSUPPORTED;
+  if (!w_router || !w13_packed || !w13_t || !w_down_t || !dw_router || !dw13 || !dw_down || !fwd_workspace ||
+      (c.T > 0 && (!h || !dy || !dh)))
+    return MOE_ERR_INVALID_ARG;
+  if (!aligned(h, 16) || !aligned(w_router, 16) || !aligned(w13_packed, 16) || !aligned(w13_t, 16) ||
+      !aligned(w_down_t, 16) || !aligned(dy, 16) || !aligned(dh, 16) || !aligned(dw_router, 16) ||
+      !aligned(dbias, 4) || !aligned(dw13, 16) || !aligned(dw_down, 16) || !aligned(status_dev, 4))
+    return MOE_ERR_UNSUPPORTED;
+  if (fwd_ws_bytes < ws_size(c, MOE_OP_LAYER) || !aligned(fwd_workspace, 16)) return MOE_ERR_WORKSPACE;
+  const size_t need = ws_size(c, MOE_OP_BACKWARD);
+  if (ws_bytes < need || !workspace || !aligned(workspace, 16)) return MOE_ERR_WORKSPACE;
+  Carver fw(const_cast<void*>(fwd_workspace));
+  const LayerBufs f = carve_layer(c, fw);
+  Carver bw(workspace);
+  const BackwardBufs b = carve_backward(c, bw);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int E = c.E, d = c.d, F = c.d_ff, T = c.T, k = c.k;
+  const int P = static_cast<int>(perm_rows(c));
+  cudaError_t e = cudaSuccess;
+  // 1. combine: dy_perm rows and the gate gradient through the softmax over the picks
+  e = launch_combine_bwd(dy, f.y_perm, f.dest_row, f.gate, b.dy_perm, b.ds, T, k, d, s);
+  if (e != cudaSuccess) return MOE_ERR_CUDA;
+  if (P > 0) {
+    CUtensorMap ta, tb;
+    // 2. dh_mid = dy_perm W_down (per expert), B = W_down^T rows
+    rc = make_map(&ta, b.dy_perm, P, d, kTileM);
+    if (rc == MOE_OK) rc = make_map(&tb, w_down_t, static_cast<uint64_t>(E) * F, d, kGemmTileN);
+    if (rc != MOE_OK) return rc;
+    e = launch_grouped_gemm_tc(ta, tb, false, f.offsets, E, d, F, (F + kGemmTileN - 1) / kGemmTileN, F, F, b.dh_mid,
+                               nullptr, status_dev, false, s);
+    if (e != cudaSuccess) return MOE_ERR_CUDA;
+    // 3. gate/up pre-activations recomputed from x_perm; SwiGLU backward in the epilogue
+    rc = make_map(&ta, f.x_perm, P, d, kTileM);
+    if (rc == MOE_OK) rc = make_map(&tb, w13_packed, static_cast<uint64_t>(E) * 2 * F, d, kGemmTileN);
+    if (rc != MOE_OK) return rc;
+    e = launch_grouped_gemm_swiglu_bwd(ta, tb, f.offsets, E, d, F, b.dgu, b.dh_mid, status_dev, false, s);
+    if (e != cudaSuccess) return MOE_ERR_CUDA;
+    // 4. dx_perm = dgu w13 (per expert), B = w13^T rows
+    rc = make_map(&ta, b.dgu, P, 2 * F, kTileM);
+    if (rc == MOE_OK) rc = make_map(&tb, w13_t, static_cast<uint64_t>(E) * d, 2 * F, kGemmTileN);
+    if (rc != MOE_OK) return rc;
+    e = launch_grouped_gemm_tc(ta, tb, false, f.offsets, E, 2 * F, d, (d + kGemmTileN - 1) / kGemmTileN, d, d,
+                               b.dx_perm, nullptr, status_dev, false, s);
+    if (e != cudaSuccess) return MOE_ERR_CUDA;
+  }
+  // 5. dh: expert rows back to their tokens plus the router-score term
+  e = launch_token_grad(b.dx_perm, f.dest_row, f.idx, b.ds, w_router, dh, T, k, d, s);
+  if (e != cudaSuccess) return MOE_ERR_CUDA;
+  // 6. router weights and bias
+  e = launch_router_wgrad(h, f.idx, b.ds, T, k, d, E, dw_router, dbias, s);
+  if (e != cudaSuccess) return MOE_ERR_CUDA;
+  // 7. expert weight gradients: operands transposed to [channels, rows], each
+  //    expert's rows at a 64-aligned column offset, reduced per expert
+  e = launch_col_offsets(f.offsets, E, b.col_off, s);
+  if (e == cudaSuccess) e = launch_transpose_grouped(b.dy_perm, d, f.offsets, b.col_off, E, b.ppad_max, b.dy_perm_t, s);
+  if (e == cudaSuccess) e = launch_transpose_grouped(f.h_mid, F, f.offsets, b.col_off, E, b.ppad_max, b.h_mid_t, s);
+  if (e == cudaSuccess) e = launch_transpose_grouped(b.dgu, 2 * F, f.offsets, b.col_off, E, b.ppad_max, b.dgu_t, s);
+  if (e == cudaSuccess) e = launch_transpose_grouped(f.x_perm, d, f.offsets, b.col_off, E, b.ppad_max, b.x_perm_t, s);
+  if (e != cudaSuccess) return MOE_ERR_CUDA;
+  CUtensorMap ta, tb;
+  rc = make_map(&ta, b.dy_perm_t, d, b.ppad_max, kTileM);
+  if (rc == MOE_OK) rc = make_map(&tb, b.h_mid_t, F, b.ppad_max, kGemmTileN);
+  if (rc != MOE_OK) return rc;
+  e = launch_grouped_gemm_wgrad(ta, tb, b.col_off, E, d, F, dw_down, status_dev, false, s);
+  if (e != cudaSuccess) return MOE_ERR_CUDA;
+  rc = make_map(&ta, b.dgu_t, 2 * F, b.ppad_max, kTileM);
+  if (rc == MOE_OK) rc = make_map(&tb, b.x_perm_t, d, b.ppad_max, kGemmTileN);
+  if (rc != MOE_OK) return rc;
+  e = launch_grouped_gemm_wgrad(ta, tb, b.col_off, E, 2 * F, d, dw13, status_dev, false, s);
+  return cuda_rc(e);
 }
 
 }  // extern "C"

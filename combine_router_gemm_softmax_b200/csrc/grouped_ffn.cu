@@ -59,7 +59,24 @@ struct GemmArgs {
   // problem is row gather_rows[r] of the tensor behind tm_a (a box of one
   // row); rows at or past offsets[E] read row 0 and are never stored.
   const int32_t* gather_rows;
+  // SwiGLU-backward epilogue: the gradient dL/dh_mid [rows, aux_ld] (bf16).
+  const __nv_bfloat16* aux;
+  int aux_ld;
+  // Reduction-grouped mode (weight gradients): offsets are the 64-aligned
+  // column offsets of each expert in the transposed operands, every expert
+  // owns an m_tiles x n_tiles grid of output tiles, and D32 receives the fp32
+  // result [E][m_tiles * 128][out_cols].
+  float* D32;
+  int m_tiles;
 };
+
+// Epilogues and tile groupings of grouped_gemm_kernel.
+constexpr int kEpiStore = 0;       // D (bf16) = accumulator
+constexpr int kEpiSwiGLU = 1;      // D (bf16) = silu(gate) * up, half-width
+constexpr int kEpiSwiGLUBwd = 2;   // D (bf16) = [dgate | dup] from gate, up and aux = dL/dh_mid
+constexpr int kEpiStoreF32 = 3;    // D32 (fp32) = accumulator
+constexpr int kGroupRows = 0;      // groups of rows (experts' token rows), same K for all
+constexpr int kGroupReduce = 1;    // groups along K (experts' token rows are the reduction)
 
 // tile -> (expert, row tile within the expert, column tile)
 MOE_DEV void decode_tile(long long tile, int m_total, int n_tiles, int band_rows, const int* prefix, int E, int& e,
@@ -83,7 +100,7 @@ MOE_DEV void decode_tile(long long tile, int m_total, int n_tiles, int band_rows
   m = gm - prefix[lo];
 }
 
-template <bool kSwiGLU>
+template <int kEpi, int kMode>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
                         const GemmArgs a) {
@@ -158,8 +175,24 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const int m_total = prefix[E];
+  const int m_total = kMode == kGroupRows ? prefix[E] : E * a.m_tiles;
   const long long total = static_cast<long long>(m_total) * a.n_tiles;
+  // tile -> (expert, row tile, column tile) and its K-block range
+  auto coords = [&](long long tile, int& e, int& m, int& n, int& kb0, int& kb1) {
+    if constexpr (kMode == kGroupRows) {
+      decode_tile(tile, m_total, a.n_tiles, a.band, prefix, E, e, m, n);
+      kb0 = 0;
+      kb1 = nkb;
+    } else {
+      const int per = a.m_tiles * a.n_tiles;
+      e = static_cast<int>(tile / per);
+      const int rem = static_cast<int>(tile - static_cast<long long>(e) * per);
+      m = rem % a.m_tiles;
+      n = rem / a.m_tiles;
+      kb0 = s_off[e] / kBK;
+      kb1 = s_off[e + 1] / kBK;
+    }
+  };
 
   int issued = 0;
   if (warp == 0) {
@@ -172,10 +205,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     uint32_t phase = 0;
     bool stop = false;
     for (long long tile = blockIdx.x; tile < total && !stop; tile += gridDim.x) {
-      int e, m, n;
-      decode_tile(tile, m_total, a.n_tiles, a.band, prefix, E, e, m, n);
-      const int a_row = s_off[e] + m * kBM;
-      const int b_row = e * a.n_per_expert + n * kBN;
+      int e, m, n, kb0, kb1;
+      coords(tile, e, m, n, kb0, kb1);
+      const int a_row = kMode == kGroupRows ? s_off[e] + m * kBM : m * kBM;
+      const int b_row = kMode == kGroupRows ? e * a.n_per_expert + n * kBN : n * kBN;
       if (gather) {
         __syncwarp();  // the previous tile's rows were read by lane 0's last issue
         for (int i = lane; i < kBM; i += 32) {
@@ -185,7 +218,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         __syncwarp();
       }
       if (lane == 0) {
-        for (int kb = 0; kb < nkb; ++kb) {
+        for (int kb = kb0; kb < kb1; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag)) {
             *abort_flag = 1;
             stop = true;
@@ -228,7 +261,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
         tc_fence_after();
         const uint32_t d_tmem = tmem + acc * kBN;
-        for (int kb = 0; kb < nkb; ++kb) {
+        int te, tm, tn, kb0, kb1;
+        coords(tile, te, tm, tn, kb0, kb1);
+        for (int kb = kb0; kb < kb1; ++kb) {
           if (!mbar_wait(&full[stage], phase, abort_flag)) {
             *abort_flag = 1;
             stop = true;
@@ -240,7 +275,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 #pragma unroll
           for (int kk = 0; kk < kBK / 16; ++kk)
             umma_bf16(d_tmem, sw128_kmajor_desc(sa + kk * 32), sw128_kmajor_desc(sb + kk * 32), idesc,
-                      (kb | kk) != 0);
+                      (kb != kb0) || (kk != 0));
           umma_commit(&empty[stage]);
           ++consumed;
           if (++stage == kStages) {
@@ -260,8 +295,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const int row = q * 32 + lane;
     int local = 0;
     for (long long tile = blockIdx.x; tile < total; tile += gridDim.x, ++local) {
-      int e, m, n;
-      decode_tile(tile, m_total, a.n_tiles, a.band, prefix, E, e, m, n);
+      int e, m, n, kb0, kb1;
+      coords(tile, e, m, n, kb0, kb1);
       const int acc = local & 1;
       const uint32_t acc_phase = (local >> 1) & 1;
       if (!mbar_wait(&tfull[acc], acc_phase, abort_flag)) {
@@ -269,11 +304,81 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         break;
       }
       tc_fence_after();
+      const uint32_t tbase = tmem + acc * kBN + (static_cast<uint32_t>(q * 32) << 16);
+      if constexpr (kMode == kGroupReduce) {
+        // fp32 weight-gradient tile of expert e; an expert with no rows has no
+        // K blocks, its accumulator was never written and the tile is zero
+        float* out = a.D32 + (static_cast<size_t>(e) * a.m_tiles * kBM + m * kBM + row) * a.ldd + n * kBN;
+        const bool empty_k = kb1 == kb0;
+#pragma unroll 1
+        for (int c = 0; c < kBN; c += 32) {
+          if (n * kBN + c >= a.out_cols) break;
+          uint32_t v[32];
+          if (!empty_k) {
+            tmem_ld32(tbase + c, v);
+            tmem_ld_wait();
+          }
+          float4* dst = reinterpret_cast<float4*>(out + c);
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+            dst[i] = empty_k ? make_float4(0.f, 0.f, 0.f, 0.f)
+                             : make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
+                                           __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]));
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&tempty[acc]);
+        continue;
+      }
       const int rows_valid = min(kBM, s_off[e + 1] - s_off[e] - m * kBM);
       const bool valid = row < rows_valid;
       const size_t grow = static_cast<size_t>(s_off[e] + m * kBM + row);
-      const uint32_t tbase = tmem + acc * kBN + (static_cast<uint32_t>(q * 32) << 16);
-      if constexpr (kSwiGLU) {
+      if constexpr (kEpi == kEpiSwiGLUBwd) {
+        // columns [0,128) of the tile are the gate pre-activations a, [128,256)
+        // the matching up pre-activations u, for channels n*128 + [0,128):
+        // dgate = dh * u * silu'(a), dup = dh * silu(a)
+        __nv_bfloat16* out = a.D + grow * a.ldd + n * kBN;
+        const __nv_bfloat16* dh = a.aux + grow * a.aux_ld + n * (kBN / 2);
+#pragma unroll 1
+        for (int c = 0; c < kBN / 2; c += 32) {
+          uint32_t g[32], u[32];
+          tmem_ld32(tbase + c, g);
+          tmem_ld32(tbase + kBN / 2 + c, u);
+          uint4 dq[4];
+          if (valid) {
+            const uint4* src = reinterpret_cast<const uint4*>(dh + c);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) dq[i] = src[i];
+          }
+          tmem_ld_wait();
+          if (valid) {
+            const __nv_bfloat16* dv = reinterpret_cast<const __nv_bfloat16*>(dq);
+            uint32_t pg[16], pu[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              float dg2[2], du2[2];
+#pragma unroll
+              for (int h2 = 0; h2 < 2; ++h2) {
+                const float av = __uint_as_float(g[2 * i + h2]);
+                const float uv = __uint_as_float(u[2 * i + h2]);
+                const float d0 = __bfloat162float(dv[2 * i + h2]);
+                const float sg = 1.0f / (1.0f + expf(-av));
+                dg2[h2] = d0 * uv * (sg * (1.0f + av * (1.0f - sg)));
+                du2[h2] = d0 * av * sg;
+              }
+              pg[i] = pack_bf16x2(dg2[0], dg2[1]);
+              pu[i] = pack_bf16x2(du2[0], du2[1]);
+            }
+            uint4* dg_dst = reinterpret_cast<uint4*>(out + c);
+            uint4* du_dst = reinterpret_cast<uint4*>(out + kBN / 2 + c);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              dg_dst[i] = make_uint4(pg[4 * i], pg[4 * i + 1], pg[4 * i + 2], pg[4 * i + 3]);
+              du_dst[i] = make_uint4(pu[4 * i], pu[4 * i + 1], pu[4 * i + 2], pu[4 * i + 3]);
+            }
+          }
+        }
+      } else if constexpr (kEpi == kEpiSwiGLU) {
         // columns [0,128) of the tile are gate, [128,256) the matching up
         __nv_bfloat16* out = a.D + grow * a.ldd + n * (kBN / 2);
 #pragma unroll 1
@@ -724,36 +829,52 @@ int band_rows(int tile_rows, int K, int lo, int hi) {
 
 }  // namespace
 
+namespace {
+
+template <int kEpi, int kMode>
+cudaError_t launch_gemm_inst(const CUtensorMap& tm_a, const CUtensorMap& tm_b, const GemmArgs& a, bool pdl,
+                             cudaStream_t s) {
+  const size_t smem = gemm_smem_bytes();
+  cudaError_t err = cudaFuncSetAttribute(grouped_gemm_kernel<kEpi, kMode>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+  if (err != cudaSuccess) return err;
+  err = launch_kernel(grouped_gemm_kernel<kEpi, kMode>, dim3(device_sm_count()), dim3(kGemmThreads), smem, s, pdl, 1,
+                      tm_a, tm_b, a);
+  if (err != cudaSuccess) return err;
+  return cudaGetLastError();
+}
+
+}  // namespace
+
 cudaError_t launch_grouped_gemm_tc(const CUtensorMap& tm_a, const CUtensorMap& tm_b, bool swiglu,
                                    const int32_t* offsets, int E, int K, int n_per_expert, int n_tiles,
                                    int out_cols, int ldd, void* D, const int32_t* gather_rows, int32_t* status,
                                    bool pdl, cudaStream_t s) {
   GemmArgs a{offsets, E, K, n_per_expert, n_tiles, out_cols, ldd, static_cast<__nv_bfloat16*>(D), status,
-             band_rows(kBM, K, 8, 32), gather_rows};
-  const size_t smem = gemm_smem_bytes();
-  const int grid = device_sm_count();
-  cudaError_t err;
-  if (swiglu) {
-    err = cudaFuncSetAttribute(grouped_gemm_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               static_cast<int>(smem));
-    if (err != cudaSuccess) return err;
-    err = launch_kernel(grouped_gemm_kernel<true>, dim3(grid), dim3(kGemmThreads), smem, s, pdl, 1, tm_a, tm_b, a);
-    if (err != cudaSuccess) return err;
-  } else {
-    err = cudaFuncSetAttribute(grouped_gemm_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               static_cast<int>(smem));
-    if (err != cudaSuccess) return err;
-    err = launch_kernel(grouped_gemm_kernel<false>, dim3(grid), dim3(kGemmThreads), smem, s, pdl, 1, tm_a, tm_b, a);
-    if (err != cudaSuccess) return err;
-  }
-  return cudaGetLastError();
+             band_rows(kBM, K, 8, 32), gather_rows, nullptr, 0, nullptr, 0};
+  return swiglu ? launch_gemm_inst<kEpiSwiGLU, kGroupRows>(tm_a, tm_b, a, pdl, s)
+                : launch_gemm_inst<kEpiStore, kGroupRows>(tm_a, tm_b, a, pdl, s);
+}
+
+cudaError_t launch_grouped_gemm_swiglu_bwd(const CUtensorMap& tm_a, const CUtensorMap& tm_b, const int32_t* offsets,
+                                           int E, int K, int F, void* dgu, const void* dh_mid, int32_t* status,
+                                           bool pdl, cudaStream_t s) {
+  GemmArgs a{offsets, E, K, 2 * F, 2 * F / kBN, 2 * F, 2 * F, static_cast<__nv_bfloat16*>(dgu), status,
+             band_rows(kBM, K, 8, 32), nullptr, static_cast<const __nv_bfloat16*>(dh_mid), F, nullptr, 0};
+  return launch_gemm_inst<kEpiSwiGLUBwd, kGroupRows>(tm_a, tm_b, a, pdl, s);
+}
+
+cudaError_t launch_grouped_gemm_wgrad(const CUtensorMap& tm_a, const CUtensorMap& tm_b, const int32_t* col_offsets,
+                                      int E, int M, int N, float* D32, int32_t* status, bool pdl, cudaStream_t s) {
+  GemmArgs a{col_offsets, E, 0, 0, (N + kBN - 1) / kBN, N, N, nullptr, status, 0, nullptr, nullptr, 0, D32, M / kBM};
+  return launch_gemm_inst<kEpiStoreF32, kGroupReduce>(tm_a, tm_b, a, pdl, s);
 }
 
 cudaError_t launch_grouped_gemm_pair(const CUtensorMap& tm_a, const CUtensorMap& tm_b, bool swiglu,
                                      const int32_t* offsets, int E, int K, int n_per_expert, int n_tiles, int out_cols,
                                      int ldd, void* D, int32_t* status, bool pdl, cudaStream_t s) {
   GemmArgs a{offsets, E, K, n_per_expert, n_tiles, out_cols, ldd, static_cast<__nv_bfloat16*>(D), status,
-             band_rows(2 * kBM, K, 4, 16), nullptr};
+             band_rows(2 * kBM, K, 4, 16), nullptr, nullptr, 0, nullptr, 0};
   const size_t smem = pair_smem_bytes();
   const int grid = (device_sm_count() / 2) * 2;
   cudaError_t err;

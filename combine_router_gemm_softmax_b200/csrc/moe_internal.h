@@ -54,6 +54,18 @@ cudaError_t launch_grouped_gemm_tc(const CUtensorMap& tm_a, const CUtensorMap& t
                                    const int32_t* offsets, int E, int K, int n_per_expert, int n_tiles,
                                    int out_cols, int ldd, void* D, const int32_t* gather_rows, int32_t* status,
                                    bool pdl, cudaStream_t s);
+// GEMM1 recomputed with the SwiGLU backward in its epilogue: from the gate and
+// up pre-activations of each row (x_perm rows against w13) and dh_mid [rows, F]
+// it writes dgu [rows, 2F] = [dgate | dup] in w13's interleaved column order.
+cudaError_t launch_grouped_gemm_swiglu_bwd(const CUtensorMap& tm_a, const CUtensorMap& tm_b, const int32_t* offsets,
+                                           int E, int K, int F, void* dgu, const void* dh_mid, int32_t* status,
+                                           bool pdl, cudaStream_t s);
+// Weight gradients: for each expert e, D32[e] [M, N] (fp32) = A_e B_e^T where
+// A [M, cols] and B [N, cols] are transposed activations whose columns
+// [col_offsets[e], col_offsets[e+1]) (multiples of 64, zero padded) belong to
+// expert e. tm_a has boxes of 128 rows, tm_b of 256 rows (64 columns each).
+cudaError_t launch_grouped_gemm_wgrad(const CUtensorMap& tm_a, const CUtensorMap& tm_b, const int32_t* col_offsets,
+                                      int E, int M, int N, float* D32, int32_t* status, bool pdl, cudaStream_t s);
 cudaError_t launch_grouped_gemm_pair(const CUtensorMap& tm_a, const CUtensorMap& tm_b, bool swiglu,
                                      const int32_t* offsets, int E, int K, int n_per_expert, int n_tiles, int out_cols,
                                      int ldd, void* D, int32_t* status, bool pdl, cudaStream_t s);
@@ -63,5 +75,20 @@ cudaError_t launch_scale_rows(int dtype, int kind, const void* x_perm, const int
                               int rows_max, int d, int E, cudaStream_t s);
 cudaError_t launch_pack_w13(const void* w_gate, const void* w_up, void* w13, int E, int F, size_t row_bytes,
                             cudaStream_t s);
+
+// backward.cu
+cudaError_t launch_combine_bwd(const void* dy, const void* y_perm, const int32_t* dest_row, const float* gate,
+                               void* dy_perm, float* ds, int T, int k, int d, cudaStream_t s);
+cudaError_t launch_token_grad(const void* dx_perm, const int32_t* dest_row, const int32_t* idx, const float* ds,
+                              const void* w_router, void* dh, int T, int k, int d, cudaStream_t s);
+cudaError_t launch_router_wgrad(const void* h, const int32_t* idx, const float* ds, int T, int k, int d, int E,
+                                float* dw_router, float* dbias, cudaStream_t s);
+cudaError_t launch_col_offsets(const int32_t* offsets, int E, int32_t* col_off, cudaStream_t s);
+// XT [C, ppad_max] from X [rows, C]: expert e's rows become columns
+// [col_off[e], col_off[e+1]) (multiples of 64), zero padded.
+cudaError_t launch_transpose_grouped(const void* X, int C, const int32_t* offsets, const int32_t* col_off, int E,
+                                     int ppad_max, void* XT, cudaStream_t s);
+// [E][R][C] -> [E][C][R], bf16, R and C multiples of 64.
+cudaError_t launch_transpose_batched(const void* X, int E, int R, int C, void* XT, cudaStream_t s);
 
 }  // namespace moe

@@ -116,6 +116,7 @@ extern "C" {
 #define MOE_OP_PERMUTE     1
 #define MOE_OP_GROUPED_FFN 2
 #define MOE_OP_LAYER       3
+#define MOE_OP_BACKWARD    4
 
 #define MOE_MAX_E 256
 #define MOE_MAX_K 8
@@ -246,6 +247,39 @@ MOE_API int32_t moe_layer_forward_timed(const moe_config* cfg, const void* h, co
                                         int32_t* topk_idx, float* topk_gate, int32_t* routed_counts,
                                         int32_t* counts, void* workspace, size_t ws_bytes,
                                         int32_t* status_dev, moe_stream_t stream, void* const* stage_events);
+
+/* moe_pack_weights_backward -- the transposed expert weights the backward
+ * dgrad GEMMs read (once per weight update, like moe_pack_weights):
+ *   w13_t [E, d, 2F]     w13_t[e] = w13_packed[e]^T (packed column order kept)
+ *   w_down_t [E, F, d]   w_down_t[e] = w_down[e]^T
+ * bf16 only; d and F multiples of 128. */
+MOE_API int32_t moe_pack_weights_backward(const moe_config* cfg, const void* w13_packed, const void* w_down,
+                                          void* w13_t, void* w_down_t, moe_stream_t stream);
+
+/* moe_layer_backward -- gradients of L = sum_t <dy_t, y_t> for the layer
+ * computed by the moe_layer_forward call that last used `fwd_workspace` with
+ * the same cfg, h and weights: the chain rule through the forward
+ * definition ("How Does Mixture-of-Experts Routing Affect LLM
+ * Repeatability?", the token-choice layer) with the routing decision held
+ * fixed. It reads the routing, gates, permutation, x_perm, h_mid and y_perm
+ * that the forward left in fwd_workspace; nothing may touch it in between.
+ *   dy [T, d] (bf16)          upstream gradient
+ *   dh [T, d] (bf16)          through the experts and the router scores
+ *   dw_router [E, d] (fp32)   dL/dW_r;  dbias [E] (fp32, may be NULL)
+ *   dw13 [E, 2F, d] (fp32)    dL/dw13_packed: rows in w13_packed's interleaved
+ *                             order (block b of 128 gate rows, then the
+ *                             matching 128 up rows)
+ *   dw_down [E, d, F] (fp32)  dL/dW_down
+ * Gate gradient: ds_{t,j} = g_j (dgate_j - sum_i g_i dgate_i) over the picked
+ * slots (dgate_j = <dy_t, f_e(h_t)> for kept slots, 0 for dropped ones).
+ * Needs bf16, SwiGLU experts, the COMPACT layout and a forward that wrote
+ * x_perm (dispatch COPY or AUTO); else MOE_ERR_UNSUPPORTED. Scratch:
+ * moe_workspace_size(cfg, MOE_OP_BACKWARD). Deterministic. */
+MOE_API int32_t moe_layer_backward(const moe_config* cfg, const void* h, const void* w_router,
+                                   const void* w13_packed, const void* w13_t, const void* w_down_t,
+                                   const void* dy, void* dh, float* dw_router, float* dbias, float* dw13,
+                                   float* dw_down, const void* fwd_workspace, size_t fwd_ws_bytes,
+                                   void* workspace, size_t ws_bytes, int32_t* status_dev, moe_stream_t stream);
 
 /* moe_permute_static_scratch -- moe_permute for callers that cannot allocate.
  * The paper has no counterpart for this entry point. It is for code that has

@@ -90,3 +90,17 @@ def gate_bound(gate_ref, s_picked_ref):
 def gates_match(gate, gate_ref, logits_ref, idx_ref):
     sp = np.take_along_axis(np.asarray(logits_ref, np.float64), np.asarray(idx_ref, np.int64), axis=1)
     return bool(np.all(np.abs(np.asarray(gate, np.float64) - gate_ref) <= gate_bound(gate_ref, sp)))
+
+
+def matrix_rel_err(got, want):
+    """max |got - want| / max(max |want|, 1e-6) over one matrix. Used for a
+    weight gradient, which is a sum over the tokens routed to one expert: one
+    of its rows can be a near-cancelling sum, or (for an expert with a single
+    token) a rank-one row scaled by a near-zero factor, so a per-row relative
+    error measures rounding of a tiny number; the whole matrix is what an
+    update applies, so it is compared against its own largest element."""
+    got = np.asarray(got, np.float64)
+    want = np.asarray(want, np.float64)
+    if want.size == 0:
+        return 0.0
+    return float(np.abs(got - want).max() / max(np.abs(want).max(), 1e-6))

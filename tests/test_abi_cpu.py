@@ -156,3 +156,24 @@ def test_dispatch_mode_checked(L):
     bad.dispatch = 3
     assert L.moe_route(ctypes.byref(bad), None, None, None, None, None, None, None, 0, None, None) \
         == M.MOE_ERR_INVALID_ARG
+
+
+def test_backward_checked_before_any_cuda_call(L):
+    """The backward needs bf16 SwiGLU experts, the compact layout and x_perm
+    from the forward; its scratch is sized by MOE_OP_BACKWARD."""
+    cfg = M.config(4096, 1024, 8, 2, 3584)
+    need = M.moe_workspace_size(cfg, M.MOE_OP_BACKWARD)
+    P, d, F = 4096 * 2, 1024, 3584
+    assert need >= P * (d + F + 2 * F + d) * 2          # dy_perm, dh_mid, dgu, dx_perm
+    for kw in (dict(dtype="f32"), dict(expert_kind="identity"), dict(dispatch="gather"),
+               dict(capacity=2000, layout="padded")):
+        bad = M.config(4096, 1024, 8, 2, 3584, **kw)
+        assert M.moe_workspace_size(bad, M.MOE_OP_BACKWARD) == 0, kw
+        p = ctypes.c_void_p(0x1000)
+        rc = L.moe_layer_backward(ctypes.byref(bad), p, p, p, p, p, p, p, p, p, p, p, p, 1 << 40, p, 1 << 40,
+                                  None, None)
+        assert rc == M.MOE_ERR_UNSUPPORTED, kw
+    p = ctypes.c_void_p(0x1000)
+    assert L.moe_layer_backward(ctypes.byref(cfg), p, p, p, p, p, p, p, p, p, p, p, p, 16, p, 1 << 40, None,
+                                None) == M.MOE_ERR_WORKSPACE
+    assert L.moe_pack_weights_backward(ctypes.byref(cfg), None, None, None, None, None) == M.MOE_ERR_INVALID_ARG

@@ -1,0 +1,104 @@
+"""GPU parity of the layer backward against the oracle's gradients.
+
+The oracle differentiates the forward definition in fp64 (pinned by central
+differences in test_oracle_pins.py); here every gradient the library returns
+is compared with it row by row on seeded inputs whose routing is away from
+ties, with the same row-relative bound as the forward output."""
+from __future__ import annotations
+
+import functools
+
+import numpy as np
+import pytest
+import torch
+
+import combine_router_gemm_softmax_b200 as M
+import oracle as O
+import workloads as W
+from oracle import cases
+from oracle import check as C
+
+from gpu_cases import DEV, DeviceCase, np64, parity_case
+
+pytestmark = pytest.mark.gpu
+
+# ragged rows and half-width column tiles (d = 384), skewed groups with empty
+# experts, dropped slots under a capacity, 128 experts with k = 8, and a
+# Mixtral-shaped layer at a quarter of its width
+BWD_CASES = ["small_ragged", "small_skewed", "small_skewed_capacity", "small_many", "mixtral_scaled"]
+
+
+@functools.lru_cache(maxsize=2)
+def _dev(name):
+    return DeviceCase(parity_case(name)[0])
+
+
+def _unpack_w13(dw13, F):
+    """Packed rows (block b: 128 gate rows, then the matching 128 up rows) ->
+    (dW_gate, dW_up), each [E, F, d]."""
+    E, _, d = dw13.shape
+    blocks = dw13.reshape(E, F // 128, 2, 128, d)
+    return blocks[:, :, 0].reshape(E, F, d), blocks[:, :, 1].reshape(E, F, d)
+
+
+def _run(name, seed=0):
+    dc = _dev(name)
+    inp, _ = parity_case(name)
+    wl = dc.wl
+    ws = M.workspace(dc.cfg, M.MOE_OP_LAYER, DEV)
+    M.moe_layer_forward(dc.cfg, dc.h, dc.w_router, dc.bias, dc.w13, dc.w_down, ws=ws)
+    w13_t, wd_t = M.moe_pack_weights_backward(dc.cfg, dc.w13, dc.w_down)
+    dy = W.draw_dy(wl, seed)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    g = M.moe_layer_backward(dc.cfg, dc.h, dc.w_router, dc.w13, w13_t, wd_t, dy.to(DEV), ws,
+                             with_bias=dc.bias is not None, status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    return dc, inp, dy, g
+
+
+@pytest.mark.parametrize("name", BWD_CASES)
+def test_layer_backward_matches_oracle(name):
+    dc, inp, dy, g = _run(name)
+    wl = dc.wl
+    ref = O.layer_backward(cases.as64(inp.h), cases.as64(inp.w_router), cases.as64(inp.bias), wl.k,
+                           cases.weights_fn(inp), wl.capacity, cases.as64(dy))
+    tol = C.tol_for(wl.dtype)
+    # dh per token row, like the forward output; weight gradients per expert
+    # matrix against its own largest element (oracle.check.matrix_rel_err)
+    errs = {"dh": C.row_rel_err(np64(g["dh"]), ref["dh"]),
+            "dw_router": C.matrix_rel_err(np64(g["dw_router"]), ref["dw_router"])}
+    dwg, dwu = _unpack_w13(np64(g["dw13"]), wl.F)
+    for key, got in (("dw_gate", dwg), ("dw_up", dwu), ("dw_down", np64(g["dw_down"]))):
+        errs[key] = max(C.matrix_rel_err(got[e], ref[key][e]) for e in range(wl.E))
+    if g["dbias"] is not None:
+        errs["dbias"] = C.matrix_rel_err(np64(g["dbias"]), ref["dbias"])
+    assert all(v <= tol for v in errs.values()), errs
+
+
+def test_layer_backward_is_deterministic():
+    _, _, _, g1 = _run("small_skewed", seed=1)
+    g1 = {k: v.clone() for k, v in g1.items() if v is not None}
+    _, _, _, g2 = _run("small_skewed", seed=1)
+    for k, v in g1.items():
+        assert torch.equal(v.view(torch.int16) if v.dtype == torch.bfloat16 else v.view(torch.int32),
+                           g2[k].view(torch.int16) if g2[k].dtype == torch.bfloat16 else g2[k].view(torch.int32)), k
+
+
+def test_pack_weights_backward_is_a_transpose():
+    dc = _dev("small_ragged")
+    w13_t, wd_t = M.moe_pack_weights_backward(dc.cfg, dc.w13, dc.w_down)
+    torch.cuda.synchronize()
+    assert torch.equal(w13_t, dc.w13.transpose(1, 2))
+    assert torch.equal(wd_t, dc.w_down.transpose(1, 2))
+
+
+def test_backward_rejects_unsupported_configs():
+    dc = _dev("small_ragged")
+    wl = dc.wl
+    for kw in (dict(dispatch="gather"), dict(capacity=100, layout="padded")):
+        cfg = M.config(wl.T, wl.d, wl.E, wl.k, wl.F, wl.dtype, **kw)
+        ws = torch.zeros(1 << 20, dtype=torch.uint8, device=DEV)
+        with pytest.raises(M.MoeError):
+            M.moe_layer_backward(cfg, dc.h, dc.w_router, dc.w13, dc.w13.transpose(1, 2).contiguous(),
+                                 dc.w_down.transpose(1, 2).contiguous(), dc.h, ws, ws=ws)

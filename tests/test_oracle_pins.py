@@ -429,3 +429,13 @@ def test_backward_gate_gradient_sums_to_zero():
     g = O.layer_backward(h, w_r, bias, 2, lambda e: (wg[e], wu[e], wd[e]), -1, dy)
     assert np.allclose(g["ds"].sum(axis=1), 0.0, atol=1e-12)
     assert abs(g["dbias"].sum()) < 1e-10
+
+
+def test_matrix_rel_err_measure():
+    r = np.random.default_rng(0)
+    w = r.standard_normal((5, 7))
+    assert C.matrix_rel_err(w, w) == 0.0
+    bad = w.copy()
+    bad[2, 3] += 0.03 * np.abs(w).max()
+    assert C.matrix_rel_err(bad, w) == pytest.approx(0.03)
+    assert C.matrix_rel_err(np.zeros((3, 3)), np.zeros((3, 3))) == 0.0

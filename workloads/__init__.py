@@ -17,6 +17,7 @@ expert's slice of it, or one token row) can be regenerated on its own:
     stream 5  bias     router bias draws            N(0, 1)
     stream 6  redraw of one token row h_t           key (6, t, attempt)
     stream 7  redraw of one router column W_r[:, c] key (7, c, attempt)
+    stream 8  dy       upstream gradient of y (backward) N(0, 1)
 
 Streams 6 and 7 exist for the test-side pass that keeps every token's top-k
 router scores at least 1e-3 apart (that pass needs the router arithmetic, so
@@ -38,6 +39,7 @@ import torch
 
 STREAM_H, STREAM_WR, STREAM_WG, STREAM_WU, STREAM_WD, STREAM_BIAS = 0, 1, 2, 3, 4, 5
 STREAM_REDRAW_H, STREAM_REDRAW_WR_COL = 6, 7
+STREAM_DY = 8
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 DERIVED_PATH = os.path.join(_HERE, "derived.json")
@@ -162,6 +164,11 @@ def draw_h(wl: Workload, seed: int = 0) -> torch.Tensor:
         h[t, t % wl.d] = (t + 1).astype(np.float32)
         return _to(h, wl.torch_dtype)
     return _to(normal(seed, (STREAM_H,), (wl.T, wl.d)), wl.torch_dtype)
+
+
+def draw_dy(wl: Workload, seed: int = 0) -> torch.Tensor:
+    """Upstream gradient dL/dy [T, d] for the backward pass."""
+    return _to(normal(seed, (STREAM_DY,), (wl.T, wl.d)), wl.torch_dtype)
 
 
 def redraw_h_row(wl: Workload, seed: int, t: int, attempt: int) -> torch.Tensor:
