@@ -167,6 +167,7 @@ struct BackwardBufs {
   float* ds;
   int32_t* col_off;
   void *dy_perm_t, *h_mid_t, *dgu_t, *x_perm_t;
+  float* router_scratch;
   int ppad_max;
 };
 
@@ -190,6 +191,7 @@ BackwardBufs carve_backward(const moe_config& c, Carver& w) {
   b.h_mid_t = w.take<void>(F * pp * 2);
   b.dgu_t = w.take<void>(2 * F * pp * 2);
   b.x_perm_t = w.take<void>(d * pp * 2);
+  b.router_scratch = w.take<float>(router_wgrad_scratch(c.T, c.E, c.d));
   return b;
 }
 
@@ -530,7 +532,7 @@ int32_t moe_layer_backward(const moe_config* cfg, const void* h, const void* w_r
   e = launch_token_grad(b.dx_perm, f.dest_row, f.idx, b.ds, w_router, dh, T, k, d, s);
   if (e != cudaSuccess) return MOE_ERR_CUDA;
   // 6. router weights and bias
-  e = launch_router_wgrad(h, f.idx, b.ds, T, k, d, E, dw_router, dbias, s);
+  e = launch_router_wgrad(h, f.idx, b.ds, T, k, d, E, dw_router, dbias, b.router_scratch, s);
   if (e != cudaSuccess) return MOE_ERR_CUDA;
   // 7. expert weight gradients: operands transposed to [channels, rows], each
   //    expert's rows at a 64-aligned column offset, reduced per expert

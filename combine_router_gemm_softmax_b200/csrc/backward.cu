@@ -15,6 +15,8 @@
 //                 their operands are transposed into [channels, rows] with each
 //                 expert's rows starting at a multiple of 64 (zero padded)
 // All reductions run in a fixed order, so the gradients are deterministic.
+#include <algorithm>
+
 #include "moe_common.cuh"
 #include "moe_internal.h"
 
@@ -136,26 +138,62 @@ __global__ void __launch_bounds__(256) token_grad_kernel(const uint4* __restrict
   }
 }
 
-// CTA (e, column block): each thread owns one column c of dW_r[e] and walks the
-// tokens in order, adding ds_{t,j} h[t, c] for every slot j that picked e.
-// Thread 0 of the first column block also sums db[e].
-__global__ void __launch_bounds__(256) router_wgrad_kernel(const __nv_bfloat16* __restrict__ h,
-                                                           const int32_t* __restrict__ idx,
-                                                           const float* __restrict__ ds, int T, int k, int d,
-                                                           float* __restrict__ dw_router, float* __restrict__ dbias) {
-  const int e = blockIdx.x;
-  const int c = blockIdx.y * blockDim.x + threadIdx.x;
-  float acc = 0.f, accb = 0.f;
-  for (int t = 0; t < T; ++t) {
+// Router weight gradient in two fixed-order passes. Pass 1: CTA (token chunk
+// of kRwChunk tokens, 128 columns) keeps a [E][128] fp32 partial in shared
+// memory, each thread one column, adding ds_{t,j} h[t, c] into row e_j for the
+// chunk's tokens in order (thread 0 also sums ds into a [E] bias partial);
+// it writes the partials out. Pass 2 adds the partials over chunks in chunk
+// order.
+constexpr int kRwChunk = 512;
+constexpr int kRwCols = 128;
+
+__global__ void __launch_bounds__(kRwCols) router_wgrad_partial_kernel(const __nv_bfloat16* __restrict__ h,
+                                                                       const int32_t* __restrict__ idx,
+                                                                       const float* __restrict__ ds, int T, int k,
+                                                                       int d, int E, float* __restrict__ part,
+                                                                       float* __restrict__ part_b) {
+  extern __shared__ float sp[];  // [E][kRwCols], then [E] bias partial
+  float* spb = sp + E * kRwCols;
+  const int chunk = blockIdx.x;
+  const int c = blockIdx.y * kRwCols + threadIdx.x;
+  for (int i = threadIdx.x; i < E * kRwCols; i += blockDim.x) sp[i] = 0.f;
+  for (int i = threadIdx.x; i < E; i += blockDim.x) spb[i] = 0.f;
+  __syncthreads();
+  const int t0 = chunk * kRwChunk, t1 = min(T, t0 + kRwChunk);
+  for (int t = t0; t < t1; ++t) {
+    const float hv = c < d ? __bfloat162float(h[static_cast<size_t>(t) * d + c]) : 0.f;
     for (int j = 0; j < k; ++j) {
-      if (idx[static_cast<size_t>(t) * k + j] != e) continue;
+      const int e = idx[static_cast<size_t>(t) * k + j];
       const float w = ds[static_cast<size_t>(t) * k + j];
-      if (c < d) acc = fmaf(w, __bfloat162float(h[static_cast<size_t>(t) * d + c]), acc);
-      accb += w;
+      sp[e * kRwCols + threadIdx.x] = fmaf(w, hv, sp[e * kRwCols + threadIdx.x]);
+      if (threadIdx.x == 0 && blockIdx.y == 0) spb[e] += w;
     }
   }
-  if (c < d) dw_router[static_cast<size_t>(e) * d + c] = acc;
-  if (dbias != nullptr && blockIdx.y == 0 && threadIdx.x == 0) dbias[e] = accb;
+  __syncthreads();
+  float* out = part + static_cast<size_t>(chunk) * E * d;
+  for (int e = 0; e < E; ++e)
+    if (c < d) out[static_cast<size_t>(e) * d + c] = sp[e * kRwCols + threadIdx.x];
+  if (blockIdx.y == 0)
+    for (int e = threadIdx.x; e < E; e += blockDim.x) part_b[static_cast<size_t>(chunk) * E + e] = spb[e];
+}
+
+__global__ void __launch_bounds__(256) router_wgrad_reduce_kernel(const float* __restrict__ part,
+                                                                  const float* __restrict__ part_b, int n_chunks,
+                                                                  int E, int d, float* __restrict__ dw_router,
+                                                                  float* __restrict__ dbias) {
+  const size_t n = static_cast<size_t>(E) * d;
+  for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n;
+       i += static_cast<size_t>(gridDim.x) * blockDim.x) {
+    float acc = 0.f;
+    for (int ch = 0; ch < n_chunks; ++ch) acc += part[static_cast<size_t>(ch) * n + i];
+    dw_router[i] = acc;
+  }
+  if (dbias != nullptr && blockIdx.x == 0)
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+      float acc = 0.f;
+      for (int ch = 0; ch < n_chunks; ++ch) acc += part_b[static_cast<size_t>(ch) * E + e];
+      dbias[e] = acc;
+    }
 }
 
 // col_off[e] = sum over e' < e of roundup64(offsets[e'+1] - offsets[e']).
@@ -169,16 +207,48 @@ __global__ void col_offsets_kernel(const int32_t* __restrict__ offsets, int E, i
   col_off[E] = run;
 }
 
-constexpr int kTr = 64;  // transpose tile edge
+constexpr int kTr = 64;    // transpose tile edge
+constexpr int kTrLd = 72;  // shared row stride in bf16 (144 bytes: 16-byte aligned, spreads the column reads)
 
-// XT [C, Ppad] from X [rows, C] (bf16): column j of XT in expert e's padded
-// range [col_off[e], col_off[e+1]) is row offsets[e] + (j - col_off[e]) of X,
-// or zero past the expert's rows. One 64 x 64 tile per CTA through shared memory.
+// Fills tile[r][0..63] from 64 bf16 of row r (16-byte loads), rows from `src`
+// (nullptr: a zero row); 256 threads, two 16-byte pieces each.
+MOE_DEV void tr_load(__nv_bfloat16 (*tile)[kTrLd], const __nv_bfloat16* const* src_rows) {
+  for (int i = threadIdx.x; i < kTr * 8; i += blockDim.x) {
+    const int r = i >> 3, seg = i & 7;
+    uint4 v = make_uint4(0, 0, 0, 0);
+    if (src_rows[r] != nullptr) v = *reinterpret_cast<const uint4*>(src_rows[r] + seg * 8);
+    *reinterpret_cast<uint4*>(&tile[r][seg * 8]) = v;
+  }
+}
+
+// Writes column c of the tile (64 values, rows 0..63) as row c of the output:
+// dst_rows[c] + [0, 64), 16-byte stores.
+MOE_DEV void tr_store(__nv_bfloat16 (*tile)[kTrLd], __nv_bfloat16* const* dst_rows) {
+  for (int i = threadIdx.x; i < kTr * 8; i += blockDim.x) {
+    const int c = i >> 3, rseg = i & 7;
+    if (dst_rows[c] == nullptr) continue;
+    uint32_t p[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const uint16_t lo = __bfloat16_as_ushort(tile[rseg * 8 + 2 * q][c]);
+      const uint16_t hi = __bfloat16_as_ushort(tile[rseg * 8 + 2 * q + 1][c]);
+      p[q] = static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16);
+    }
+    *reinterpret_cast<uint4*>(dst_rows[c] + rseg * 8) = make_uint4(p[0], p[1], p[2], p[3]);
+  }
+}
+
+// XT [C, ldt] from X [rows, C] (bf16, C a multiple of 64): column j of XT in
+// expert e's padded range [col_off[e], col_off[e+1]) is row
+// offsets[e] + (j - col_off[e]) of X, or zero past the expert's rows. One 64 x
+// 64 tile per CTA through shared memory.
 __global__ void __launch_bounds__(256) transpose_grouped_kernel(const __nv_bfloat16* __restrict__ X, int C,
                                                                 const int32_t* __restrict__ offsets,
                                                                 const int32_t* __restrict__ col_off, int E,
                                                                 __nv_bfloat16* __restrict__ XT, int ldt) {
-  __shared__ __nv_bfloat16 tile[kTr][kTr + 2];
+  __shared__ __align__(16) __nv_bfloat16 tile[kTr][kTrLd];
+  __shared__ const __nv_bfloat16* src[kTr];
+  __shared__ __nv_bfloat16* dst[kTr];
   const int j0 = blockIdx.x * kTr;  // first padded column (= row of X) of this tile
   const int c0 = blockIdx.y * kTr;  // first channel
   if (j0 >= col_off[E]) return;
@@ -193,34 +263,33 @@ __global__ void __launch_bounds__(256) transpose_grouped_kernel(const __nv_bfloa
   const int e = lo;
   const int i0 = j0 - col_off[e];
   const int rows_e = offsets[e + 1] - offsets[e];
-  for (int i = threadIdx.x; i < kTr * kTr; i += blockDim.x) {
-    const int r = i / kTr, c = i % kTr;  // r: row within the tile (padded column), c: channel
-    const int src = i0 + r;
-    tile[r][c] = (src < rows_e && c0 + c < C) ? X[static_cast<size_t>(offsets[e] + src) * C + c0 + c]
-                                              : __float2bfloat16(0.f);
+  if (threadIdx.x < kTr) {
+    const int r = threadIdx.x;
+    src[r] = i0 + r < rows_e ? X + static_cast<size_t>(offsets[e] + i0 + r) * C + c0 : nullptr;
+    dst[r] = XT + static_cast<size_t>(c0 + r) * ldt + j0;
   }
   __syncthreads();
-  for (int i = threadIdx.x; i < kTr * kTr; i += blockDim.x) {
-    const int c = i / kTr, r = i % kTr;
-    if (c0 + c < C) XT[static_cast<size_t>(c0 + c) * ldt + j0 + r] = tile[r][c];
-  }
+  tr_load(tile, src);
+  __syncthreads();
+  tr_store(tile, dst);
 }
 
 // Per-expert transpose of a weight [E][R][C] into [E][C][R] (R, C multiples of 64).
 __global__ void __launch_bounds__(256) transpose_batched_kernel(const __nv_bfloat16* __restrict__ X, int R, int C,
                                                                 __nv_bfloat16* __restrict__ XT) {
-  __shared__ __nv_bfloat16 tile[kTr][kTr + 2];
+  __shared__ __align__(16) __nv_bfloat16 tile[kTr][kTrLd];
+  __shared__ const __nv_bfloat16* src[kTr];
+  __shared__ __nv_bfloat16* dst[kTr];
   const size_t base = static_cast<size_t>(blockIdx.z) * R * C;
   const int r0 = blockIdx.x * kTr, c0 = blockIdx.y * kTr;
-  for (int i = threadIdx.x; i < kTr * kTr; i += blockDim.x) {
-    const int r = i / kTr, c = i % kTr;
-    tile[r][c] = X[base + static_cast<size_t>(r0 + r) * C + c0 + c];
+  if (threadIdx.x < kTr) {
+    src[threadIdx.x] = X + base + static_cast<size_t>(r0 + threadIdx.x) * C + c0;
+    dst[threadIdx.x] = XT + base + static_cast<size_t>(c0 + threadIdx.x) * R + r0;
   }
   __syncthreads();
-  for (int i = threadIdx.x; i < kTr * kTr; i += blockDim.x) {
-    const int c = i / kTr, r = i % kTr;
-    XT[base + static_cast<size_t>(c0 + c) * R + r0 + r] = tile[r][c];
-  }
+  tr_load(tile, src);
+  __syncthreads();
+  tr_store(tile, dst);
 }
 
 int warp_grid_bwd(int T) {
@@ -287,10 +356,27 @@ cudaError_t launch_token_grad(const void* dx_perm, const int32_t* dest_row, cons
   return cudaGetLastError();
 }
 
+size_t router_wgrad_scratch(int T, int E, int d) {
+  const size_t chunks = (static_cast<size_t>(T) + kRwChunk - 1) / kRwChunk;
+  return chunks * E * (static_cast<size_t>(d) + 1) * 4;
+}
+
 cudaError_t launch_router_wgrad(const void* h, const int32_t* idx, const float* ds, int T, int k, int d, int E,
-                                float* dw_router, float* dbias, cudaStream_t s) {
-  router_wgrad_kernel<<<dim3(E, (d + 255) / 256), 256, 0, s>>>(static_cast<const __nv_bfloat16*>(h), idx, ds, T, k,
-                                                               d, dw_router, dbias);
+                                float* dw_router, float* dbias, float* scratch, cudaStream_t s) {
+  const int chunks = (T + kRwChunk - 1) / kRwChunk;
+  float* part = scratch;
+  float* part_b = scratch + static_cast<size_t>(chunks) * E * d;
+  if (chunks > 0) {
+    const size_t smem = static_cast<size_t>(E) * (kRwCols + 1) * 4;
+    cudaError_t err = cudaFuncSetAttribute(router_wgrad_partial_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           static_cast<int>(smem));
+    if (err != cudaSuccess) return err;
+    router_wgrad_partial_kernel<<<dim3(chunks, (d + kRwCols - 1) / kRwCols), kRwCols, smem, s>>>(
+        static_cast<const __nv_bfloat16*>(h), idx, ds, T, k, d, E, part, part_b);
+  }
+  const long long n = static_cast<long long>(E) * d;
+  const int grid = static_cast<int>(std::min<long long>((n + 255) / 256, device_sm_count() * 8LL));
+  router_wgrad_reduce_kernel<<<grid > 0 ? grid : 1, 256, 0, s>>>(part, part_b, chunks, E, d, dw_router, dbias);
   return cudaGetLastError();
 }
 

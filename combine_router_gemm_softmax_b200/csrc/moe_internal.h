@@ -81,8 +81,10 @@ cudaError_t launch_combine_bwd(const void* dy, const void* y_perm, const int32_t
                                void* dy_perm, float* ds, int T, int k, int d, cudaStream_t s);
 cudaError_t launch_token_grad(const void* dx_perm, const int32_t* dest_row, const int32_t* idx, const float* ds,
                               const void* w_router, void* dh, int T, int k, int d, cudaStream_t s);
+// scratch: router_wgrad_scratch(T, E, d) bytes (per-chunk partial sums).
+size_t router_wgrad_scratch(int T, int E, int d);
 cudaError_t launch_router_wgrad(const void* h, const int32_t* idx, const float* ds, int T, int k, int d, int E,
-                                float* dw_router, float* dbias, cudaStream_t s);
+                                float* dw_router, float* dbias, float* scratch, cudaStream_t s);
 cudaError_t launch_col_offsets(const int32_t* offsets, int E, int32_t* col_off, cudaStream_t s);
 // XT [C, ppad_max] from X [rows, C]: expert e's rows become columns
 // [col_off[e], col_off[e+1]) (multiples of 64), zero padded.
