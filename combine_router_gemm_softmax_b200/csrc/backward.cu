@@ -222,10 +222,12 @@ MOE_DEV void tr_load(__nv_bfloat16 (*tile)[kTrLd], const __nv_bfloat16* const* s
 }
 
 // Writes column c of the tile (64 values, rows 0..63) as row c of the output:
-// dst_rows[c] + [0, 64), 16-byte stores.
+// dst_rows[c] + [0, 64), 16-byte stores. A warp takes 32 consecutive columns
+// of the same 8 rows, so each of its shared-memory reads is one contiguous
+// 64-byte row segment (no bank conflicts).
 MOE_DEV void tr_store(__nv_bfloat16 (*tile)[kTrLd], __nv_bfloat16* const* dst_rows) {
   for (int i = threadIdx.x; i < kTr * 8; i += blockDim.x) {
-    const int c = i >> 3, rseg = i & 7;
+    const int c = i & (kTr - 1), rseg = i >> 6;
     if (dst_rows[c] == nullptr) continue;
     uint32_t p[4];
 #pragma unroll

@@ -77,6 +77,7 @@ constexpr int kEpiSwiGLUBwd = 2;   // D (bf16) = [dgate | dup] from gate, up and
 constexpr int kEpiStoreF32 = 3;    // D32 (fp32) = accumulator
 constexpr int kGroupRows = 0;      // groups of rows (experts' token rows), same K for all
 constexpr int kGroupReduce = 1;    // groups along K (experts' token rows are the reduction)
+constexpr int kReduceBand = 16;    // row tiles per band in the reduction-grouped tile walk
 
 // tile -> (expert, row tile within the expert, column tile)
 MOE_DEV void decode_tile(long long tile, int m_total, int n_tiles, int band_rows, const int* prefix, int E, int& e,
@@ -184,11 +185,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       kb0 = 0;
       kb1 = nkb;
     } else {
+      // within an expert: bands of kReduceBand row tiles, each band sweeping
+      // all column tiles, so a band's A rows stay in L2 while B streams
       const int per = a.m_tiles * a.n_tiles;
       e = static_cast<int>(tile / per);
       const int rem = static_cast<int>(tile - static_cast<long long>(e) * per);
-      m = rem % a.m_tiles;
-      n = rem / a.m_tiles;
+      const int band = rem / (kReduceBand * a.n_tiles);
+      const int m0 = band * kReduceBand;
+      const int rows = min(kReduceBand, a.m_tiles - m0);
+      const int within = rem - band * kReduceBand * a.n_tiles;
+      m = m0 + within % rows;
+      n = within / rows;
       kb0 = s_off[e] / kBK;
       kb1 = s_off[e + 1] / kBK;
     }
