@@ -14,7 +14,8 @@
  * "Follow one documented dispatch and return path": per-expert counts from the
  * routing map, a permutation that groups token rows by expert, the experts,
  * and the return of every output to its original token position. On one GPU
- * the dispatch and the return are on-device permutations.
+ * the dispatch and the return are on-device permutations. moe_layer_backward
+ * differentiates the same layer (bf16, SwiGLU experts).
  *
  * Conventions for every entry point:
  *  - Tensor arguments are DEVICE pointers owned by the caller. The library
