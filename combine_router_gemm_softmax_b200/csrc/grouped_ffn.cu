@@ -22,6 +22,15 @@
 // store it, so the epilogue of tile i overlaps the main loop of tile i+1.
 // Rows past the end of an expert's group are computed on whatever the buffer
 // holds there and never stored.
+//
+// The same kernel, by template arguments, also serves the layer's backward:
+// a plain bf16 store (the down projection and both dgrad GEMMs), the gate/up
+// GEMM recomputed with the SwiGLU backward in its epilogue (it reads dh_mid
+// and writes [dgate | dup]), and a reduction-grouped mode for the weight
+// gradients, where each expert owns a fixed grid of output tiles and its token
+// rows are the K range (operands transposed with 64-aligned per-expert
+// columns), stored in fp32. In gather mode GEMM1's producer loads A rows
+// straight from the token matrix through the permutation (tile::gather4).
 #include "moe_common.cuh"
 #include "moe_internal.h"
 
