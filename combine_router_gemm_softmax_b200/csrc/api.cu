@@ -514,11 +514,15 @@ int32_t moe_layer_backward(const moe_config* cfg, const void* h, const void* w_r
     e = launch_grouped_gemm_tc(ta, tb, false, f.offsets, E, d, F, (F + kGemmTileN - 1) / kGemmTileN, F, F, b.dh_mid,
                                nullptr, status_dev, false, s);
     if (e != cudaSuccess) return MOE_ERR_CUDA;
-    // 3. gate/up pre-activations recomputed from x_perm; SwiGLU backward in the epilogue
+    // 3. gate/up pre-activations recomputed from x_perm; SwiGLU backward in the
+    //    epilogue, which also writes dgu transposed for the weight gradient
+    e = launch_col_offsets(f.offsets, E, b.col_off, s);
+    if (e != cudaSuccess) return MOE_ERR_CUDA;
     rc = make_map(&ta, f.x_perm, P, d, kTileM);
     if (rc == MOE_OK) rc = make_map(&tb, w13_packed, static_cast<uint64_t>(E) * 2 * F, d, kGemmTileN);
     if (rc != MOE_OK) return rc;
-    e = launch_grouped_gemm_swiglu_bwd(ta, tb, f.offsets, E, d, F, b.dgu, b.dh_mid, status_dev, false, s);
+    e = launch_grouped_gemm_swiglu_bwd(ta, tb, f.offsets, E, d, F, b.dgu, b.dh_mid, b.dgu_t, b.col_off, b.ppad_max,
+                                       status_dev, false, s);
     if (e != cudaSuccess) return MOE_ERR_CUDA;
     // 4. dx_perm = dgu w13 (per expert), B = w13^T rows
     rc = make_map(&ta, b.dgu, P, 2 * F, kTileM);
@@ -536,10 +540,9 @@ int32_t moe_layer_backward(const moe_config* cfg, const void* h, const void* w_r
   if (e != cudaSuccess) return MOE_ERR_CUDA;
   // 7. expert weight gradients: operands transposed to [channels, rows], each
   //    expert's rows at a 64-aligned column offset, reduced per expert
-  e = launch_col_offsets(f.offsets, E, b.col_off, s);
+  if (P == 0) e = launch_col_offsets(f.offsets, E, b.col_off, s);  // else done before step 3
   if (e == cudaSuccess) e = launch_transpose_grouped(b.dy_perm, d, f.offsets, b.col_off, E, b.ppad_max, b.dy_perm_t, s);
   if (e == cudaSuccess) e = launch_transpose_grouped(f.h_mid, F, f.offsets, b.col_off, E, b.ppad_max, b.h_mid_t, s);
-  if (e == cudaSuccess) e = launch_transpose_grouped(b.dgu, 2 * F, f.offsets, b.col_off, E, b.ppad_max, b.dgu_t, s);
   if (e == cudaSuccess) e = launch_transpose_grouped(f.x_perm, d, f.offsets, b.col_off, E, b.ppad_max, b.x_perm_t, s);
   if (e != cudaSuccess) return MOE_ERR_CUDA;
   CUtensorMap ta, tb;

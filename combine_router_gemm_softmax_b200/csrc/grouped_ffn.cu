@@ -77,6 +77,12 @@ struct GemmArgs {
   // result [E][m_tiles * 128][out_cols].
   float* D32;
   int m_tiles;
+  // SwiGLU-backward epilogue, optional: also write [dgate | dup] transposed,
+  // DT[column][col_off[e] + row within expert] (ldt columns per row), with
+  // the rows up to col_off[e+1] past the expert's end written as zeros.
+  __nv_bfloat16* DT;
+  const int32_t* col_off;
+  int ldt;
 };
 
 // Epilogues and tile groupings of grouped_gemm_kernel.
@@ -355,6 +361,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         // dgate = dh * u * silu'(a), dup = dh * silu(a)
         __nv_bfloat16* out = a.D + grow * a.ldd + n * kBN;
         const __nv_bfloat16* dh = a.aux + grow * a.aux_ld + n * (kBN / 2);
+        // transposed copy: lanes are consecutive rows, so each 2-byte store of
+        // a warp covers 32 consecutive columns of one DT row
+        const int pcol = a.DT != nullptr ? a.col_off[e] + m * kBM + row : 0;
+        const bool twrite = a.DT != nullptr && pcol < a.col_off[e + 1];
 #pragma unroll 1
         for (int c = 0; c < kBN / 2; c += 32) {
           uint32_t g[32], u[32];
@@ -367,9 +377,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             for (int i = 0; i < 4; ++i) dq[i] = src[i];
           }
           tmem_ld_wait();
+          uint32_t pg[16], pu[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) pg[i] = pu[i] = 0u;
           if (valid) {
             const __nv_bfloat16* dv = reinterpret_cast<const __nv_bfloat16*>(dq);
-            uint32_t pg[16], pu[16];
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
               float dg2[2], du2[2];
@@ -391,6 +403,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             for (int i = 0; i < 4; ++i) {
               dg_dst[i] = make_uint4(pg[4 * i], pg[4 * i + 1], pg[4 * i + 2], pg[4 * i + 3]);
               du_dst[i] = make_uint4(pu[4 * i], pu[4 * i + 1], pu[4 * i + 2], pu[4 * i + 3]);
+            }
+          }
+          if (twrite) {
+            uint16_t* tg = reinterpret_cast<uint16_t*>(a.DT) + static_cast<size_t>(n * kBN + c) * a.ldt + pcol;
+            uint16_t* tu = tg + static_cast<size_t>(kBN / 2) * a.ldt;
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              tg[static_cast<size_t>(2 * i) * a.ldt] = static_cast<uint16_t>(pg[i] & 0xffffu);
+              tg[static_cast<size_t>(2 * i + 1) * a.ldt] = static_cast<uint16_t>(pg[i] >> 16);
+              tu[static_cast<size_t>(2 * i) * a.ldt] = static_cast<uint16_t>(pu[i] & 0xffffu);
+              tu[static_cast<size_t>(2 * i + 1) * a.ldt] = static_cast<uint16_t>(pu[i] >> 16);
             }
           }
         }
@@ -867,22 +890,25 @@ cudaError_t launch_grouped_gemm_tc(const CUtensorMap& tm_a, const CUtensorMap& t
                                    int out_cols, int ldd, void* D, const int32_t* gather_rows, int32_t* status,
                                    bool pdl, cudaStream_t s) {
   GemmArgs a{offsets, E, K, n_per_expert, n_tiles, out_cols, ldd, static_cast<__nv_bfloat16*>(D), status,
-             band_rows(kBM, K, 8, 32), gather_rows, nullptr, 0, nullptr, 0};
+             band_rows(kBM, K, 8, 32), gather_rows, nullptr, 0, nullptr, 0, nullptr, nullptr, 0};
   return swiglu ? launch_gemm_inst<kEpiSwiGLU, kGroupRows>(tm_a, tm_b, a, pdl, s)
                 : launch_gemm_inst<kEpiStore, kGroupRows>(tm_a, tm_b, a, pdl, s);
 }
 
 cudaError_t launch_grouped_gemm_swiglu_bwd(const CUtensorMap& tm_a, const CUtensorMap& tm_b, const int32_t* offsets,
-                                           int E, int K, int F, void* dgu, const void* dh_mid, int32_t* status,
-                                           bool pdl, cudaStream_t s) {
+                                           int E, int K, int F, void* dgu, const void* dh_mid, void* dgu_t,
+                                           const int32_t* col_off, int ldt, int32_t* status, bool pdl,
+                                           cudaStream_t s) {
   GemmArgs a{offsets, E, K, 2 * F, 2 * F / kBN, 2 * F, 2 * F, static_cast<__nv_bfloat16*>(dgu), status,
-             band_rows(kBM, K, 8, 32), nullptr, static_cast<const __nv_bfloat16*>(dh_mid), F, nullptr, 0};
+             band_rows(kBM, K, 8, 32), nullptr, static_cast<const __nv_bfloat16*>(dh_mid), F, nullptr, 0,
+             static_cast<__nv_bfloat16*>(dgu_t), col_off, ldt};
   return launch_gemm_inst<kEpiSwiGLUBwd, kGroupRows>(tm_a, tm_b, a, pdl, s);
 }
 
 cudaError_t launch_grouped_gemm_wgrad(const CUtensorMap& tm_a, const CUtensorMap& tm_b, const int32_t* col_offsets,
                                       int E, int M, int N, float* D32, int32_t* status, bool pdl, cudaStream_t s) {
-  GemmArgs a{col_offsets, E, 0, 0, (N + kBN - 1) / kBN, N, N, nullptr, status, 0, nullptr, nullptr, 0, D32, M / kBM};
+  GemmArgs a{col_offsets, E, 0, 0, (N + kBN - 1) / kBN, N, N, nullptr, status, 0, nullptr, nullptr, 0, D32, M / kBM,
+             nullptr, nullptr, 0};
   return launch_gemm_inst<kEpiStoreF32, kGroupReduce>(tm_a, tm_b, a, pdl, s);
 }
 
@@ -890,7 +916,7 @@ cudaError_t launch_grouped_gemm_pair(const CUtensorMap& tm_a, const CUtensorMap&
                                      const int32_t* offsets, int E, int K, int n_per_expert, int n_tiles, int out_cols,
                                      int ldd, void* D, int32_t* status, bool pdl, cudaStream_t s) {
   GemmArgs a{offsets, E, K, n_per_expert, n_tiles, out_cols, ldd, static_cast<__nv_bfloat16*>(D), status,
-             band_rows(2 * kBM, K, 4, 16), nullptr, nullptr, 0, nullptr, 0};
+             band_rows(2 * kBM, K, 4, 16), nullptr, nullptr, 0, nullptr, 0, nullptr, nullptr, 0};
   const size_t smem = pair_smem_bytes();
   const int grid = (device_sm_count() / 2) * 2;
   cudaError_t err;

@@ -56,10 +56,13 @@ cudaError_t launch_grouped_gemm_tc(const CUtensorMap& tm_a, const CUtensorMap& t
                                    bool pdl, cudaStream_t s);
 // GEMM1 recomputed with the SwiGLU backward in its epilogue: from the gate and
 // up pre-activations of each row (x_perm rows against w13) and dh_mid [rows, F]
-// it writes dgu [rows, 2F] = [dgate | dup] in w13's interleaved column order.
+// it writes dgu [rows, 2F] = [dgate | dup] in w13's interleaved column order,
+// and, when dgu_t is set, the same values transposed: dgu_t [2F, ldt] with
+// expert e's rows at columns col_off[e] + i and zeros up to col_off[e+1].
 cudaError_t launch_grouped_gemm_swiglu_bwd(const CUtensorMap& tm_a, const CUtensorMap& tm_b, const int32_t* offsets,
-                                           int E, int K, int F, void* dgu, const void* dh_mid, int32_t* status,
-                                           bool pdl, cudaStream_t s);
+                                           int E, int K, int F, void* dgu, const void* dh_mid, void* dgu_t,
+                                           const int32_t* col_off, int ldt, int32_t* status, bool pdl,
+                                           cudaStream_t s);
 // Weight gradients: for each expert e, D32[e] [M, N] (fp32) = A_e B_e^T where
 // A [M, cols] and B [N, cols] are transposed activations whose columns
 // [col_offsets[e], col_offsets[e+1]) (multiples of 64, zero padded) belong to
