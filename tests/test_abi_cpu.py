@@ -177,3 +177,18 @@ def test_backward_checked_before_any_cuda_call(L):
     assert L.moe_layer_backward(ctypes.byref(cfg), p, p, p, p, p, p, p, p, p, p, p, p, 16, p, 1 << 40, None,
                                 None) == M.MOE_ERR_WORKSPACE
     assert L.moe_pack_weights_backward(ctypes.byref(cfg), None, None, None, None, None) == M.MOE_ERR_INVALID_ARG
+
+
+def test_backward_workspace_formula(L):
+    """MOE_OP_BACKWARD scratch: four row buffers, ds, the column offsets, four
+    transposed operands over P' = roundup64(P) + 64 E columns, and the router
+    gradient's per-512-token partial sums, each piece 256-byte aligned."""
+    def up(n):
+        return (n + 255) // 256 * 256
+    for T, d, E, k, F in ((4096, 1024, 8, 2, 3584), (777, 256, 40, 4, 384), (8192, 2048, 128, 8, 768)):
+        P = T * k
+        pp = (P + 63) // 64 * 64 + 64 * E
+        chunks = (T + 511) // 512
+        want = (up(P * d * 2) + up(P * F * 2) + up(P * 2 * F * 2) + up(P * d * 2) + up(T * k * 4) + up((E + 1) * 4)
+                + up(d * pp * 2) + up(F * pp * 2) + up(2 * F * pp * 2) + up(d * pp * 2) + up(chunks * E * (d + 1) * 4))
+        assert M.moe_workspace_size(M.config(T, d, E, k, F), M.MOE_OP_BACKWARD) == want
