@@ -1,13 +1,19 @@
 """Benchmark of the MoE layer forward on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+                    [--gemm-tiles auto|single|pair] [--backward] [--no-cpu-baseline]
 
 One step is one whole layer forward (route, permute, grouped SwiGLU FFN,
 unpermute/combine) over one batch of T synthetic tokens, through the C ABI
-entry point moe_layer_forward. Under torchrun each rank runs its own batch on
-its own GPU (token-sharded replicas: weak scaling, no collective on the data
-path); `value` is the tokens of all ranks divided by the slowest rank's
-device time. Rank 0 prints one JSON line.
+entry point moe_layer_forward_timed, which also records a CUDA event between
+the stages so every stage is timed inside the steps. Under torchrun each rank
+runs its own batch on its own GPU (token-sharded replicas: weak scaling, no
+collective on the data path); `value` is the tokens of all ranks divided by
+the slowest rank's device time. Rank 0 prints one JSON line, which also
+carries the end-to-end figure (pinned host buffers, transfers inside the
+timed region), the grouped GEMM's roofline, the SM clocks seen during the
+timed region and a CPU-oracle baseline. --backward adds the time of
+moe_layer_backward.
 
 --impl reference times the CPU oracle (fp64, numpy) on the host cores on a
 bounded token sample of the same workload; under torchrun only rank 0 runs it.
