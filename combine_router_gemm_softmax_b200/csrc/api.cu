@@ -196,8 +196,7 @@ BackwardBufs carve_backward(const moe_config& c, Carver& w) {
 }
 
 bool backward_supported(const moe_config& c) {
-  return c.dtype == MOE_DTYPE_BF16 && c.expert_kind == MOE_EXPERT_SWIGLU && c.layout == MOE_LAYOUT_COMPACT &&
-         !layer_gathers(c);
+  return c.dtype == MOE_DTYPE_BF16 && c.expert_kind == MOE_EXPERT_SWIGLU && !layer_gathers(c);
 }
 
 size_t ws_size(const moe_config& c, int op) {
@@ -502,7 +501,14 @@ int32_t moe_layer_backward(const moe_config* cfg, const void* h, const void* w_r
   const int E = c.E, d = c.d, F = c.d_ff, T = c.T, k = c.k;
   const int P = static_cast<int>(perm_rows(c));
   cudaError_t e = cudaSuccess;
-  // 1. combine: dy_perm rows and the gate gradient through the softmax over the picks
+  // 1. combine: dy_perm rows and the gate gradient through the softmax over the picks.
+  //    In the padded layout the padding rows take part in every expert GEMM
+  //    below (their x_perm and h_mid rows are zero), so their dy_perm rows are
+  //    zeroed first.
+  if (c.layout == MOE_LAYOUT_PADDED && P > 0) {
+    e = cudaMemsetAsync(b.dy_perm, 0, static_cast<size_t>(P) * d * 2, s);
+    if (e != cudaSuccess) return MOE_ERR_CUDA;
+  }
   e = launch_combine_bwd(dy, f.y_perm, f.dest_row, f.gate, b.dy_perm, b.ds, T, k, d, s);
   if (e != cudaSuccess) return MOE_ERR_CUDA;
   if (P > 0) {

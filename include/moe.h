@@ -273,8 +273,9 @@ MOE_API int32_t moe_pack_weights_backward(const moe_config* cfg, const void* w13
  *   dw_down [E, d, F] (fp32)  dL/dW_down
  * Gate gradient: ds_{t,j} = g_j (dgate_j - sum_i g_i dgate_i) over the picked
  * slots (dgate_j = <dy_t, f_e(h_t)> for kept slots, 0 for dropped ones).
- * Needs bf16, SwiGLU experts, the COMPACT layout and a forward that wrote
- * x_perm (dispatch COPY or AUTO); else MOE_ERR_UNSUPPORTED. Scratch:
+ * Needs bf16, SwiGLU experts and a forward that wrote x_perm (dispatch COPY
+ * or AUTO); else MOE_ERR_UNSUPPORTED. Both layouts are supported (in the
+ * PADDED one the padding rows are computed as zero rows). Scratch:
  * moe_workspace_size(cfg, MOE_OP_BACKWARD). Deterministic. */
 MOE_API int32_t moe_layer_backward(const moe_config* cfg, const void* h, const void* w_router,
                                    const void* w13_packed, const void* w13_t, const void* w_down_t,

@@ -165,8 +165,7 @@ def test_backward_checked_before_any_cuda_call(L):
     need = M.moe_workspace_size(cfg, M.MOE_OP_BACKWARD)
     P, d, F = 4096 * 2, 1024, 3584
     assert need >= P * (d + F + 2 * F + d) * 2          # dy_perm, dh_mid, dgu, dx_perm
-    for kw in (dict(dtype="f32"), dict(expert_kind="identity"), dict(dispatch="gather"),
-               dict(capacity=2000, layout="padded")):
+    for kw in (dict(dtype="f32"), dict(expert_kind="identity"), dict(dispatch="gather")):
         bad = M.config(4096, 1024, 8, 2, 3584, **kw)
         assert M.moe_workspace_size(bad, M.MOE_OP_BACKWARD) == 0, kw
         p = ctypes.c_void_p(0x1000)
@@ -177,6 +176,8 @@ def test_backward_checked_before_any_cuda_call(L):
     assert L.moe_layer_backward(ctypes.byref(cfg), p, p, p, p, p, p, p, p, p, p, p, p, 16, p, 1 << 40, None,
                                 None) == M.MOE_ERR_WORKSPACE
     assert L.moe_pack_weights_backward(ctypes.byref(cfg), None, None, None, None, None) == M.MOE_ERR_INVALID_ARG
+    padded = M.config(4096, 1024, 8, 2, 3584, capacity=2000, layout="padded")
+    assert M.moe_workspace_size(padded, M.MOE_OP_BACKWARD) > 0
 
 
 def test_backward_workspace_formula(L):

@@ -23,9 +23,10 @@ from gpu_cases import DEV, DeviceCase, np64, parity_case
 pytestmark = pytest.mark.gpu
 
 # ragged rows and half-width column tiles (d = 384), skewed groups with empty
-# experts, dropped slots under a capacity, 128 experts with k = 8, and a
-# Mixtral-shaped layer at a quarter of its width
-BWD_CASES = ["small_ragged", "small_skewed", "small_skewed_capacity", "small_many", "mixtral_scaled"]
+# experts, dropped slots under a capacity (compact and padded layouts), 128
+# experts with k = 8, and a Mixtral-shaped layer at a quarter of its width
+BWD_CASES = ["small_ragged", "small_skewed", "small_skewed_capacity", "small_skewed_padded", "small_many",
+             "mixtral_scaled"]
 
 
 @functools.lru_cache(maxsize=2)
@@ -96,7 +97,7 @@ def test_pack_weights_backward_is_a_transpose():
 def test_backward_rejects_unsupported_configs():
     dc = _dev("small_ragged")
     wl = dc.wl
-    for kw in (dict(dispatch="gather"), dict(capacity=100, layout="padded")):
+    for kw in (dict(dispatch="gather"), dict(expert_kind="identity")):
         cfg = M.config(wl.T, wl.d, wl.E, wl.k, wl.F, wl.dtype, **kw)
         ws = torch.zeros(1 << 20, dtype=torch.uint8, device=DEV)
         with pytest.raises(M.MoeError):
