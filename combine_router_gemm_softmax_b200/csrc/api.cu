@@ -1,6 +1,7 @@
 // C ABI of the MoE layer: argument checks, workspace carving, TMA descriptor
-// encoding and stage launches. The stage order and the meaning of every
-// argument are documented in include/moe.h.
+// encoding and stage launches, for the forward stages, the whole layer and
+// its backward. The stage order and the meaning of every argument are
+// documented in include/moe.h.
 #include <mutex>
 
 #include "moe_common.cuh"

@@ -17,7 +17,10 @@
 //           expert, from per-warp bitmasks (popc), giving dest_row/perm_src
 //   copy  : TMA bulk copies: each token row is bulk-loaded into shared memory
 //           once and bulk-stored to each kept destination row
+//   pad   : padded layout only: rows past each expert's kept count are zeroed
 // Nothing decides an order with atomics, so the permutation is deterministic.
+// Kernels after the first of a call are launched as programmatic dependents
+// and wait (griddepcontrol.wait) before touching earlier kernels' memory.
 #include "moe_common.cuh"
 #include "moe_internal.h"
 
