@@ -363,3 +363,61 @@ def layer_backward(h, w_r, bias, k, weights, cap, dy):
         dh += ds[:, j, None] * w_r[e]
     return dict(dh=dh, dw_router=dwr, dbias=db, dw_gate=dwg, dw_up=dwu, dw_down=dwd, dgate=dgate, ds=ds,
                 idx=idx, gate=g, **{kk: meta[kk] for kk in ("dest_row", "offsets", "kept", "routed")})
+
+
+def layer_backward_probe(h, w_r, bias, k, weights, cap, dy, tokens, elems):
+    """Selected entries of layer_backward's gradients, computed one by one so
+    that a full-size layer stays within reach (same definitions, same fixed
+    routing decision):
+      dh rows for the listed tokens;
+      for each (e, f, i, j) in elems: dW_down[e][i, f], dW_gate[e][f, j] and
+      dW_up[e][f, j], each a sum over the rows routed to and kept by expert e
+      of one gate/up channel f (the channel's pre-activations a[:, f], u[:, f]
+      and its output gradient dm[:, f] = do . W_down[e][:, f]).
+    Returns dict dh [len(tokens), d] and dw_down, dw_gate, dw_up [len(elems)],
+    plus dw_down_l1, dw_gate_l1, dw_up_l1: the sum of the absolute values of
+    each element's terms, the natural scale of the rounding error of a sum."""
+    h = np.asarray(h, F64)
+    w_r = np.asarray(w_r, F64)
+    dy = np.asarray(dy, F64)
+    E = w_r.shape[0]
+    idx, g, _, _ = route(h, w_r, bias, k)
+    kept = dispatch_meta(idx, E, cap)["dest_row"] >= 0
+    tokens = np.asarray(tokens)
+    dh = np.zeros((len(tokens), h.shape[1]))
+    for n, t in enumerate(tokens):
+        dgate = np.zeros(k)
+        for j in range(k):
+            if not kept[t, j]:
+                continue
+            wg, wu, wd = (np.asarray(w, F64) for w in weights(int(idx[t, j])))
+            x = h[t]
+            a = wg @ x
+            u = wu @ x
+            with np.errstate(over="ignore"):
+                sg = 1.0 / (1.0 + np.exp(-a))
+            o = wd @ (a * sg * u)
+            dgate[j] = dy[t] @ o
+            dm = wd.T @ (g[t, j] * dy[t])
+            dh[n] += wg.T @ (dm * u * sg * (1.0 + a * (1.0 - sg))) + wu.T @ (dm * a * sg)
+        ds = g[t] * (dgate - np.sum(g[t] * dgate))
+        dh[n] += ds @ w_r[np.asarray(idx[t], np.int64)]
+    out = {"dh": dh, "dw_down": [], "dw_gate": [], "dw_up": [], "dw_down_l1": [], "dw_gate_l1": [],
+           "dw_up_l1": []}
+    for e, f, i, j in elems:
+        rows, js = np.nonzero(kept & (idx == e))
+        wg, wu, wd = (np.asarray(w, F64) for w in weights(e))
+        x = h[rows]
+        a = x @ wg[f]
+        u = x @ wu[f]
+        with np.errstate(over="ignore"):
+            sg = 1.0 / (1.0 + np.exp(-a))
+        do = g[rows, js, None] * dy[rows]
+        dm = do @ wd[:, f]
+        terms = {"dw_down": do[:, i] * (a * sg * u),
+                 "dw_gate": (dm * u * sg * (1.0 + a * (1.0 - sg))) * x[:, j],
+                 "dw_up": (dm * a * sg) * x[:, j]}
+        for key, tv in terms.items():
+            out[key].append(float(tv.sum()))
+            out[key + "_l1"].append(float(np.abs(tv).sum()))
+    return {key: np.asarray(v) for key, v in out.items()}

@@ -439,3 +439,20 @@ def test_matrix_rel_err_measure():
     bad[2, 3] += 0.03 * np.abs(w).max()
     assert C.matrix_rel_err(bad, w) == pytest.approx(0.03)
     assert C.matrix_rel_err(np.zeros((3, 3)), np.zeros((3, 3))) == 0.0
+
+
+@pytest.mark.parametrize("cap", [-1, 2])
+def test_backward_probe_equals_full_backward(cap):
+    """The one-by-one entries used at full size agree with the full
+    (finite-difference-pinned) backward."""
+    h, w_r, bias, wg, wu, wd, dy = _bwd_problem(9, T=12)
+    wf = lambda e: (wg[e], wu[e], wd[e])
+    full = O.layer_backward(h, w_r, bias, 2, wf, cap, dy)
+    tokens = np.array([0, 3, 7, 11])
+    elems = [(0, 1, 2, 3), (1, 4, 0, 7), (3, 2, 5, 1), (2, 0, 7, 6)]
+    pr = O.layer_backward_probe(h, w_r, bias, 2, wf, cap, dy, tokens, elems)
+    assert np.allclose(pr["dh"], full["dh"][tokens], rtol=1e-12, atol=1e-12)
+    for n, (e, f, i, j) in enumerate(elems):
+        assert pr["dw_down"][n] == pytest.approx(full["dw_down"][e][i, f], rel=1e-10, abs=1e-12)
+        assert pr["dw_gate"][n] == pytest.approx(full["dw_gate"][e][f, j], rel=1e-10, abs=1e-12)
+        assert pr["dw_up"][n] == pytest.approx(full["dw_up"][e][f, j], rel=1e-10, abs=1e-12)
