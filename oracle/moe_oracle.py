@@ -374,9 +374,10 @@ def layer_backward_probe(h, w_r, bias, k, weights, cap, dy, tokens, elems):
       dW_up[e][f, j], each a sum over the rows routed to and kept by expert e
       of one gate/up channel f (the channel's pre-activations a[:, f], u[:, f]
       and its output gradient dm[:, f] = do . W_down[e][:, f]).
-    Returns dict dh [len(tokens), d] and dw_down, dw_gate, dw_up [len(elems)],
-    plus dw_down_l1, dw_gate_l1, dw_up_l1: the sum of the absolute values of
-    each element's terms, the natural scale of the rounding error of a sum."""
+    Each expert's weights are fetched once. Returns dict dh [len(tokens), d]
+    and dw_down, dw_gate, dw_up [len(elems)], plus dw_down_l1, dw_gate_l1,
+    dw_up_l1: the sum of the absolute values of each element's terms, the
+    natural scale of the rounding error of a sum."""
     h = np.asarray(h, F64)
     w_r = np.asarray(w_r, F64)
     dy = np.asarray(dy, F64)
@@ -385,39 +386,43 @@ def layer_backward_probe(h, w_r, bias, k, weights, cap, dy, tokens, elems):
     kept = dispatch_meta(idx, E, cap)["dest_row"] >= 0
     tokens = np.asarray(tokens)
     dh = np.zeros((len(tokens), h.shape[1]))
-    for n, t in enumerate(tokens):
-        dgate = np.zeros(k)
-        for j in range(k):
-            if not kept[t, j]:
-                continue
-            wg, wu, wd = (np.asarray(w, F64) for w in weights(int(idx[t, j])))
-            x = h[t]
-            a = wg @ x
-            u = wu @ x
+    dgate = np.zeros((len(tokens), k))
+    keys = ("dw_down", "dw_gate", "dw_up")
+    out = {key: np.zeros(len(elems)) for key in keys}
+    out.update({key + "_l1": np.zeros(len(elems)) for key in keys})
+    for e in range(E):
+        pairs = [(n, j) for n, t in enumerate(tokens) for j in range(k) if kept[t, j] and idx[t, j] == e]
+        mine = [(m, el) for m, el in enumerate(elems) if el[0] == e]
+        if not pairs and not mine:
+            continue
+        wg, wu, wd = (np.asarray(w, F64) for w in weights(e))
+        for n, j in pairs:
+            t = tokens[n]
+            a = wg @ h[t]
+            u = wu @ h[t]
             with np.errstate(over="ignore"):
                 sg = 1.0 / (1.0 + np.exp(-a))
-            o = wd @ (a * sg * u)
-            dgate[j] = dy[t] @ o
+            dgate[n, j] = dy[t] @ (wd @ (a * sg * u))
             dm = wd.T @ (g[t, j] * dy[t])
             dh[n] += wg.T @ (dm * u * sg * (1.0 + a * (1.0 - sg))) + wu.T @ (dm * a * sg)
-        ds = g[t] * (dgate - np.sum(g[t] * dgate))
+        if mine:
+            rows, js = np.nonzero(kept & (idx == e))
+            x = h[rows]
+            do = g[rows, js, None] * dy[rows]
+            for m, (_, f, i, j) in mine:
+                a = x @ wg[f]
+                u = x @ wu[f]
+                with np.errstate(over="ignore"):
+                    sg = 1.0 / (1.0 + np.exp(-a))
+                dm = do @ wd[:, f]
+                terms = {"dw_down": do[:, i] * (a * sg * u),
+                         "dw_gate": (dm * u * sg * (1.0 + a * (1.0 - sg))) * x[:, j],
+                         "dw_up": (dm * a * sg) * x[:, j]}
+                for key, tv in terms.items():
+                    out[key][m] = tv.sum()
+                    out[key + "_l1"][m] = np.abs(tv).sum()
+    for n, t in enumerate(tokens):
+        ds = g[t] * (dgate[n] - np.sum(g[t] * dgate[n]))
         dh[n] += ds @ w_r[np.asarray(idx[t], np.int64)]
-    out = {"dh": dh, "dw_down": [], "dw_gate": [], "dw_up": [], "dw_down_l1": [], "dw_gate_l1": [],
-           "dw_up_l1": []}
-    for e, f, i, j in elems:
-        rows, js = np.nonzero(kept & (idx == e))
-        wg, wu, wd = (np.asarray(w, F64) for w in weights(e))
-        x = h[rows]
-        a = x @ wg[f]
-        u = x @ wu[f]
-        with np.errstate(over="ignore"):
-            sg = 1.0 / (1.0 + np.exp(-a))
-        do = g[rows, js, None] * dy[rows]
-        dm = do @ wd[:, f]
-        terms = {"dw_down": do[:, i] * (a * sg * u),
-                 "dw_gate": (dm * u * sg * (1.0 + a * (1.0 - sg))) * x[:, j],
-                 "dw_up": (dm * a * sg) * x[:, j]}
-        for key, tv in terms.items():
-            out[key].append(float(tv.sum()))
-            out[key + "_l1"].append(float(np.abs(tv).sum()))
-    return {key: np.asarray(v) for key, v in out.items()}
+    out["dh"] = dh
+    return out

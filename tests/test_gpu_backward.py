@@ -103,3 +103,29 @@ def test_backward_rejects_unsupported_configs():
         with pytest.raises(M.MoeError):
             M.moe_layer_backward(cfg, dc.h, dc.w_router, dc.w13, dc.w13.transpose(1, 2).contiguous(),
                                  dc.w_down.transpose(1, 2).contiguous(), dc.h, ws, ws=ws)
+
+
+@pytest.mark.parametrize("name", ["mixtral_8x7b", "skewed_capacity", "many_small"])
+def test_layer_backward_full_size_sampled(name):
+    """Full-size layers, in the configuration bench.py --backward times: dh on
+    sampled tokens (row-relative, like the forward) and single elements of
+    dW_down, dW_gate and dW_up, each within 2e-2 of the L1 norm of its terms
+    (the error scale of a sum of rounded products), against the oracle
+    computed entry by entry."""
+    dc, inp, dy, g = _run(name)
+    wl = dc.wl
+    r = np.random.default_rng(11)
+    tokens = np.sort(r.choice(wl.T, size=32, replace=False))
+    elems = [(int(r.integers(wl.E)), int(r.integers(wl.F)), int(r.integers(wl.d)), int(r.integers(wl.d)))
+             for _ in range(8)]
+    ref = O.layer_backward_probe(cases.as64(inp.h), cases.as64(inp.w_router), cases.as64(inp.bias), wl.k,
+                                 cases.weights_fn(inp), wl.capacity, cases.as64(dy), tokens, elems)
+    tol = C.tol_for(wl.dtype)
+    assert C.row_rel_err(np64(g["dh"][torch.from_numpy(tokens).to(DEV)]), ref["dh"]) <= tol
+    for n, (e, f, i, j) in enumerate(elems):
+        gate_row = (f // 128) * 256 + f % 128          # packed w13 row of gate channel f
+        got = {"dw_down": float(g["dw_down"][e, i, f]), "dw_gate": float(g["dw13"][e, gate_row, j]),
+               "dw_up": float(g["dw13"][e, gate_row + 128, j])}
+        for key, v in got.items():
+            bound = tol * max(float(ref[key + "_l1"][n]), 1e-6)
+            assert abs(v - float(ref[key][n])) <= bound, (key, e, f, i, j, v, float(ref[key][n]))
