@@ -104,3 +104,10 @@ def matrix_rel_err(got, want):
     if want.size == 0:
         return 0.0
     return float(np.abs(got - want).max() / max(np.abs(want).max(), 1e-6))
+
+
+def vector_rel_err(got, want):
+    """max |got - want| / max(max |want|, 1e-6) over one vector (a whole row
+    or column of a weight gradient). A wrong sign, a zero or a missing term of
+    the sum changes the vector by the order of its own largest element."""
+    return matrix_rel_err(np.asarray(got, np.float64).reshape(1, -1), np.asarray(want, np.float64).reshape(1, -1))

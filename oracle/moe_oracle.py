@@ -426,3 +426,44 @@ def layer_backward_probe(h, w_r, bias, k, weights, cap, dy, tokens, elems):
         dh[n] += ds @ w_r[np.asarray(idx[t], np.int64)]
     out["dh"] = dh
     return out
+
+
+def layer_backward_channels(h, w_r, bias, k, weights, cap, dy, chans):
+    """Whole gradient rows and columns of layer_backward for chosen (expert,
+    channel) pairs, at O(n_e * d) cost each, so that a full-size layer stays
+    within reach (same definitions, same fixed routing decision).
+
+    For each (e, f) in chans, over the rows routed to and kept by expert e:
+      dw_gate[e][f, :] = sum_r da[r, f] h_r      (row of d entries)
+      dw_up[e][f, :]   = sum_r du[r, f] h_r      (row of d entries)
+      dw_down[e][:, f] = sum_r do_r m[r, f]      (column of d entries)
+    with a = W_gate[e] h, u = W_up[e] h, m = silu(a) * u, do = g * dy and
+    dm[r, f] = do_r . W_down[e][:, f], as in layer_backward. Returns dict
+    dw_gate_rows, dw_up_rows, dw_down_cols, each [len(chans), d]."""
+    h = np.asarray(h, F64)
+    w_r = np.asarray(w_r, F64)
+    dy = np.asarray(dy, F64)
+    E = w_r.shape[0]
+    d = h.shape[1]
+    idx, g, _, _ = route(h, w_r, bias, k)
+    kept = dispatch_meta(idx, E, cap)["dest_row"] >= 0
+    out = {key: np.zeros((len(chans), d)) for key in ("dw_gate_rows", "dw_up_rows", "dw_down_cols")}
+    for e in sorted(set(int(c[0]) for c in chans)):
+        rows, js = np.nonzero(kept & (idx == e))
+        if rows.size == 0:
+            continue
+        wg, wu, wd = (np.asarray(w, F64) for w in weights(e))
+        x = h[rows]
+        do = g[rows, js, None] * dy[rows]
+        for n, (ce, f) in enumerate(chans):
+            if int(ce) != e:
+                continue
+            a = x @ wg[f]
+            u = x @ wu[f]
+            with np.errstate(over="ignore"):
+                sg = 1.0 / (1.0 + np.exp(-a))
+            dm = do @ wd[:, f]
+            out["dw_gate_rows"][n] = (dm * u * sg * (1.0 + a * (1.0 - sg))) @ x
+            out["dw_up_rows"][n] = (dm * a * sg) @ x
+            out["dw_down_cols"][n] = do.T @ (a * sg * u)
+    return out

@@ -456,3 +456,35 @@ def test_backward_probe_equals_full_backward(cap):
         assert pr["dw_down"][n] == pytest.approx(full["dw_down"][e][i, f], rel=1e-10, abs=1e-12)
         assert pr["dw_gate"][n] == pytest.approx(full["dw_gate"][e][f, j], rel=1e-10, abs=1e-12)
         assert pr["dw_up"][n] == pytest.approx(full["dw_up"][e][f, j], rel=1e-10, abs=1e-12)
+
+
+@pytest.mark.parametrize("cap", [-1, 2])
+def test_backward_channels_equal_full_backward(cap):
+    """The whole rows and columns used at full size agree with the full
+    (finite-difference-pinned) backward; an expert with no kept rows gives
+    zero rows."""
+    h, w_r, bias, wg, wu, wd, dy = _bwd_problem(9, T=12)
+    wf = lambda e: (wg[e], wu[e], wd[e])
+    full = O.layer_backward(h, w_r, bias, 2, wf, cap, dy)
+    chans = [(0, 1), (1, 4), (3, 2), (2, 0), (0, 3)]
+    ch = O.layer_backward_channels(h, w_r, bias, 2, wf, cap, dy, chans)
+    for n, (e, f) in enumerate(chans):
+        assert np.allclose(ch["dw_gate_rows"][n], full["dw_gate"][e][f, :], rtol=1e-10, atol=1e-12)
+        assert np.allclose(ch["dw_up_rows"][n], full["dw_up"][e][f, :], rtol=1e-10, atol=1e-12)
+        assert np.allclose(ch["dw_down_cols"][n], full["dw_down"][e][:, f], rtol=1e-10, atol=1e-12)
+
+
+def test_gradient_row_check_rejects_zero_and_sign_flip():
+    """The full-size weight-gradient check compares whole rows against their
+    own largest element at 2e-2; a zeroed row, a sign-flipped row and a row
+    missing one expert row's term all fail it, while bf16-sized rounding of
+    every term passes."""
+    r = np.random.default_rng(4)
+    n, d = 4000, 256
+    terms_a = r.standard_normal((n, 1)) * r.standard_normal((n, d))   # random-sign terms of a sum over rows
+    row = terms_a.sum(axis=0)
+    assert C.vector_rel_err(np.zeros(d), row) > C.TOL_BF16
+    assert C.vector_rel_err(-row, row) > C.TOL_BF16
+    assert C.vector_rel_err(row - terms_a[np.abs(terms_a).sum(axis=1).argmax()], row) > C.TOL_BF16
+    rounded = terms_a * (1.0 + r.uniform(-2.0 ** -8, 2.0 ** -8, size=terms_a.shape))
+    assert C.vector_rel_err(rounded.sum(axis=0), row) < 0.1 * C.TOL_BF16
