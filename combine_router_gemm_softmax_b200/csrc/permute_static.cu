@@ -18,9 +18,14 @@
 //    every entry before the scan reads it), so nothing is cleared. Two calls
 //    that can run at the same time on the GPU (different streams without an
 //    ordering between them) race on the array and give wrong results.
-//  - The first call on each device looks up the array's device address with
-//    cudaGetSymbolAddress while that device is current; make that first call
-//    before any stream capture begins.
+//  - Every call that is not being captured into a CUDA graph looks up the
+//    array's device address with cudaGetSymbolAddress while the stream's
+//    device is current, and remembers it for that device. A call made during
+//    stream capture uses the remembered address (it makes no runtime call that
+//    capture could forbid), so make one call on each device before capturing.
+//    Looking the address up again outside capture means a context torn down
+//    and created again (cudaDeviceReset) cannot leave a stale address behind,
+//    as long as it is not done between a capture and the graph's replay.
 //  - The scratch needs 2 * roundup256(4 * E * ceil(T / 128)) bytes; when that
 //    exceeds 1 MiB (E * ceil(T/128) > 131072, e.g. E = 256 with T > 65536)
 //    the call returns MOE_ERR_WORKSPACE and enqueues nothing.
@@ -39,16 +44,21 @@ static __device__ __align__(256) unsigned char g_permute_scratch[kStaticScratchB
 std::mutex g_mu;
 void* g_scratch_addr[kMaxDevices] = {};
 
-// Device address of g_permute_scratch on the current device (looked up once
-// per device). Host code must not use the symbol itself as a device pointer.
-int scratch_address(void** out) {
+// Device address of g_permute_scratch on the current device: looked up
+// afresh outside stream capture, taken from the per-device record during
+// capture. Host code must not use the symbol itself as a device pointer.
+int scratch_address(cudaStream_t stream, void** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MOE_ERR_NO_DEVICE;
+  cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(stream, &cap) != cudaSuccess) return MOE_ERR_CUDA;
   std::lock_guard<std::mutex> lock(g_mu);
-  if (g_scratch_addr[dev] == nullptr) {
+  if (cap == cudaStreamCaptureStatusNone) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_permute_scratch) != cudaSuccess || p == nullptr) return MOE_ERR_CUDA;
     g_scratch_addr[dev] = p;
+  } else if (g_scratch_addr[dev] == nullptr) {
+    return MOE_ERR_CUDA;  // first call on this device made during capture
   }
   *out = g_scratch_addr[dev];
   return MOE_OK;
@@ -63,7 +73,7 @@ extern "C" int32_t moe_permute_static_scratch(const moe_config* cfg, const void*
   if (cfg == nullptr) return MOE_ERR_INVALID_ARG;
   if (moe_workspace_size(cfg, MOE_OP_PERMUTE) > kStaticScratchBytes) return MOE_ERR_WORKSPACE;
   void* scratch = nullptr;
-  const int rc = scratch_address(&scratch);
+  const int rc = scratch_address(static_cast<cudaStream_t>(stream), &scratch);
   if (rc != MOE_OK) return rc;
   return moe_permute(cfg, h, topk_idx, routed_counts, counts, offsets, dest_row, perm_src, x_perm, scratch,
                      kStaticScratchBytes, status_dev, stream);

@@ -296,9 +296,11 @@ MOE_API int32_t moe_layer_backward(const moe_config* cfg, const void* h, const v
  * return MOE_ERR_WORKSPACE and enqueue nothing.
  * All calls share the array: calls that may overlap on the GPU (streams with
  * no ordering between them) race and give wrong results. Nothing in the array
- * needs to start at zero. The first call on a device looks up the array's
- * address on that device; make it before any stream capture. No cudaMalloc,
- * cudaFree or other allocating call is made. */
+ * needs to start at zero. A call outside stream capture looks up the
+ * array's address on the current device and remembers it; a call made while
+ * `stream` is being captured uses the remembered address, so make one call on
+ * each device before capturing (else MOE_ERR_CUDA). No cudaMalloc, cudaFree
+ * or other allocating call is made. */
 MOE_API int32_t moe_permute_static_scratch(const moe_config* cfg, const void* h, const int32_t* topk_idx,
                                            int32_t* routed_counts, int32_t* counts, int32_t* offsets,
                                            int32_t* dest_row, int32_t* perm_src, void* x_perm,

@@ -1,8 +1,14 @@
 """Parity of the CUDA path with the CPU oracle, called through the C ABI.
 
 Bars: routing indices, counts, offsets, drop decisions, dest_row/perm_src and
-the permuted rows are bit-exact; gates within 1e-5 relative; layer outputs
-within the per-row relative bound (2e-2 for bf16 storage, 1e-4 for fp32).
+the permuted rows are bit-exact; layer outputs within the per-row relative
+bound (2e-2 for bf16 storage, 1e-4 for fp32). Gates here are compared with
+the oracle's gates computed from the oracle's own fp64 scores, so the bound
+is derived from the score tolerance: |g - g_ref| <= g_ref (2 ds_max + 1e-5)
++ 1e-7 with ds_max = 1e-4 + 1e-4 |s| over the token's picks (about 1e-3
+relative for scores near 3; oracle.check.gate_bound). The 1e-5 relative bar
+on the kernel's gate arithmetic itself, given identical scores, is checked
+at full size in test_gpu_dispatch_full.py.
 """
 import numpy as np
 import pytest
