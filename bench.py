@@ -71,6 +71,10 @@ def parse():
     ap.add_argument("--gemm-tiles", choices=["auto", "single", "pair"], default="auto")
     ap.add_argument("--no-backward", action="store_true",
                     help="leave out the moe_layer_backward timing of the headline workload")
+    ap.add_argument("--shape", default="",
+                    help="override workload sizes, e.g. T=8192,E=2 (a smaller slice of the same layer for profiling)")
+    ap.add_argument("--precision", choices=["bf16", "mxfp8"], default="bf16",
+                    help="operands of the expert GEMMs of the timed layer")
     ap.add_argument("--no-sweep", action="store_true",
                     help="leave out the per-workload sweep that follows the headline on one GPU")
     return ap.parse_args()
@@ -223,7 +227,7 @@ SWEEP_STEPS, SWEEP_WARMUP = 10, 3
 class Layer:
     """Device copies of one workload's inputs and the buffers of its steps."""
 
-    def __init__(self, M, W, wl, seed, rank, dev, gemm_tiles="auto", host_h=True):
+    def __init__(self, M, W, wl, seed, rank, dev, gemm_tiles="auto", host_h=True, precision="bf16"):
         import torch
 
         self.wl = wl
@@ -236,7 +240,7 @@ class Layer:
         else:
             self.h = inp.h.to(dev)
         self.cfg = M.config(wl.T, wl.d, wl.E, wl.k, wl.F, wl.dtype, wl.expert_kind, wl.capacity, gemm_tiles,
-                            wl.layout)
+                            wl.layout, precision=precision)
         self.wr = inp.w_router.to(dev)
         self.bias = None if inp.bias is None else inp.bias.to(dev)
         self.w13 = self.wd = None
@@ -245,6 +249,8 @@ class Layer:
             self.w13 = M.moe_pack_weights(self.cfg, wg, wu)
             del wg, wu
             self.wd = inp.w_down.to(dev)
+            if precision == "mxfp8":
+                self.w13, self.wd = M.moe_pack_weights_mxfp8(self.cfg, self.w13, self.wd)
         del inp
         self.y = torch.empty((wl.T, wl.d), dtype=wl.torch_dtype, device=dev)
         self.counts = torch.empty(wl.E, dtype=torch.int32, device=dev)
@@ -313,6 +319,9 @@ def main():
     import workloads as W
 
     wl = W.get(args.workload)
+    if args.shape:
+        kw = {k: int(v) for k, v in (item.split("=") for item in args.shape.split(","))}
+        wl = wl.with_(name=f"{wl.name}[{args.shape}]", **kw)
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
@@ -337,7 +346,7 @@ def main():
 
     # inputs: each rank draws its own batch (seed + rank), weights are the same
     M.lib()
-    L = Layer(M, W, wl, args.seed, rank, dev, args.gemm_tiles)
+    L = Layer(M, W, wl, args.seed, rank, dev, args.gemm_tiles, precision=args.precision)
     stream = torch.cuda.current_stream(dev)
 
     # ------------------------------------------------ timed region (device events)
@@ -359,7 +368,7 @@ def main():
     row_bytes = wl.d * wl.elem_bytes
 
     barrier()
-    do_bwd = not args.no_backward and wl.expert_kind == "swiglu" and wl.dtype == "bf16"
+    do_bwd = not args.no_backward and wl.expert_kind == "swiglu" and wl.dtype == "bf16" and args.precision == "bf16"
     bwd = run_backward(M, L.cfg, wl, L.h, L.wr, L.bias, L.w13, L.wd, L.ws, stream, dev, args.steps,
                        args.seed + rank) if do_bwd else None
     barrier()
@@ -371,9 +380,10 @@ def main():
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": max(args.warmup, 3), "ms_per_step": ms_max / args.steps, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": wl.dtype,
+            "scaling": "weak", "vs_baseline": None, "dtype": wl.dtype if args.precision == "bf16" else "mxfp8",
             "data": "synthetic: seeded N(0,1) tokens, N(0,1/fan_in) random-init weights",
-            "config": {**config_dict(wl, world, flush), "gemm_tiles": args.gemm_tiles},
+            "config": {**config_dict(wl, world, flush), "gemm_tiles": args.gemm_tiles, "precision": args.precision,
+                       "combine": "fused into the down projection" if fused_combine(L.cfg) else "separate kernel"},
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": wl.T * row_bytes,
                     "d2h_bytes_per_step": wl.T * row_bytes, "ms_per_step": e2e_ms / args.steps,
                     "path": "pinned host h -> device, moe_layer_forward, device y -> pinned host; "
@@ -383,8 +393,8 @@ def main():
             "clocks": sampler.summary(),
             "status_word": st,
         }
-        line["stages"] = stage_report(stages, wl, A_kept, pk, pk_kind)
-        line["roofline"] = roofline(stages, wl, A_kept, pk, pk_kind)
+        line["stages"] = stage_report(stages, wl, A_kept, pk, pk_kind, fused_combine(L.cfg), args.precision)
+        line["roofline"] = roofline(stages, wl, A_kept, pk, pk_kind, args.precision)
         if bwd is not None:
             flops = 16.0 * A_kept * wl.d * wl.F          # incl. the recomputed gate/up GEMM
             line["backward"] = {"ms_per_step": bwd, "tokens_per_s": wl.T / (bwd / 1e3),
@@ -399,6 +409,10 @@ def main():
                            "routed_counts_mean": float(L.routed.float().mean().item()),
                            "empty_experts": int((L.routed == 0).sum().item()), "kept": A_kept,
                            "dropped": wl.T * wl.k - A_kept}
+    if rank == 0 and world == 1 and not args.no_sweep:
+        line["combine_separate"] = run_combine_separate(M, L, stream, barrier)
+        if args.precision == "bf16" and wl.expert_kind == "swiglu" and wl.dtype == "bf16":
+            line["mxfp8"] = run_mxfp8(M, L, stream, barrier)
     del L
     torch.cuda.empty_cache()
 
@@ -416,6 +430,69 @@ def main():
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.destroy_process_group()
+
+
+def run_combine_separate(M, L, stream, barrier):
+    """The headline layer again with the combine as its own kernel (the
+    separate dispatch + combine HBM rate), same inputs, SWEEP_STEPS steps."""
+    import copy
+
+    pk, pk_kind = peaks()
+    cfg0 = L.cfg
+    L.cfg = copy.copy(cfg0)
+    L.cfg.combine = M.MOE_COMBINE_SEPARATE
+    try:
+        ms, st, flush = time_steps(L, SWEEP_STEPS, SWEEP_WARMUP, stream, barrier)
+    finally:
+        L.cfg = cfg0
+    A_kept = int(L.counts.sum().item())
+    rep = stage_report(st, L.wl, A_kept, pk, pk_kind)
+    return {"ms_per_step": ms / SWEEP_STEPS, "steps": SWEEP_STEPS, "permute": rep["permute"],
+            "combine": rep["combine"], "dispatch_combine": rep["dispatch_combine"],
+            "grouped_ffn_us": rep["grouped_ffn"]["us"]}
+
+
+def run_mxfp8(M, L, stream, barrier):
+    """The headline workload with MXFP8 expert GEMMs (weights quantised from
+    the same bf16 weights), SWEEP_STEPS steps; GEMM rate against an fp8 peak
+    of twice the measured bf16 one (the nominal ratio)."""
+    import copy
+
+    import torch
+
+    pk, pk_kind = peaks()
+    cfg = copy.copy(L.cfg)
+    cfg.precision = M.MOE_PRECISION_MXFP8
+    cfg.combine = M.MOE_COMBINE_AUTO
+    wcounts = torch.zeros(2, dtype=torch.int32, device=L.dev)
+    w13, wd = M.moe_pack_weights_mxfp8(cfg, L.w13, L.wd, counts=wcounts)
+    ws = M.workspace(cfg, M.MOE_OP_LAYER, L.dev)
+    saved = (L.cfg, L.w13, L.wd, L.ws)
+    L.cfg, L.w13, L.wd, L.ws = cfg, w13, wd, ws
+    gpu_uuid = torch.cuda.get_device_properties(L.dev).uuid
+    sampler = ClockSampler(f"GPU-{gpu_uuid}")
+    try:
+        ms, st, flush = time_steps(L, SWEEP_STEPS, SWEEP_WARMUP, stream, barrier, sampler)
+        counters = M.mx_counters(ws)
+    finally:
+        L.cfg, L.w13, L.wd, L.ws = saved
+    A_kept = int(L.counts.sum().item())
+    del w13, wd, ws
+    torch.cuda.empty_cache()
+    # compact layout: the dispatch stage quantises the rows; padded: it copies
+    # bf16 rows and the expert stage quantises them
+    rep = stage_report(st, L.wl, A_kept, pk, pk_kind, False,
+                       "mxfp8" if L.wl.layout == "compact" else "mxfp8, bf16 dispatch")
+    wl = L.wl
+    return {"ms_per_step": ms / SWEEP_STEPS, "tokens_per_s": wl.T * SWEEP_STEPS / (ms / 1e3), "steps": SWEEP_STEPS,
+            "dtype": "mxfp8 (E4M3 elements, E8M0 scale per 32) with fp32 accumulation, bf16 y",
+            "stages": rep, "gpu_launches_per_step": launches(cfg), "clocks": sampler.summary(),
+            "counts": {"x_saturated": counters[0], "x_underflow": counters[1], "h_mid_saturated": counters[2],
+                       "h_mid_underflow": counters[3], "weights_saturated": int(wcounts[0].item()),
+                       "weights_underflow": int(wcounts[1].item())},
+            "elements": {"x": A_kept * wl.d, "h_mid": A_kept * wl.F, "weights": 3 * wl.E * wl.d * wl.F},
+            "peak_note": "frac_fp8 = TFLOP/s / (2 x bf16_tflops_sustained): the nominal dense fp8:bf16 ratio "
+                         "applied to the measured bf16 peak"}
 
 
 def run_sweep(M, W, names, seed, dev, stream, barrier):
@@ -437,7 +514,11 @@ def run_sweep(M, W, names, seed, dev, stream, barrier):
                  "status_word": int(L.status.item()), "clocks": sampler.summary(),
                  "gpu_launches_per_step": launches(L.cfg)}
         if wl.dtype == "bf16":
-            entry["stages"] = stage_report(stages, wl, A_kept, pk, pk_kind)
+            entry["stages"] = stage_report(stages, wl, A_kept, pk, pk_kind, fused_combine(L.cfg))
+            if wl.expert_kind == "swiglu":
+                mx = run_mxfp8(M, L, stream, barrier)
+                entry["mxfp8"] = {"ms_per_step": mx["ms_per_step"], "tokens_per_s": mx["tokens_per_s"],
+                                  "grouped_ffn": mx["stages"]["grouped_ffn"], "counts": mx["counts"]}
         else:
             entry["stages"] = {k: {"us": 1e3 * v} for k, v in stages.items()}
             entry["note"] = "fp32 SIMT path, sized for correctness, not rooflined"
@@ -520,26 +601,46 @@ def run_backward(M, cfg, wl, h, wr, bias, w13, wd, ws, stream, dev, steps, seed)
     return e0.elapsed_time(e1) / steps
 
 
+def fused_combine(cfg):
+    """Whether moe_layer_forward lets the down projection write y (the rule in
+    include/moe.h at MOE_COMBINE_*)."""
+    return (cfg.combine == 2 and cfg.k <= 2 and cfg.dtype == 0 and cfg.expert_kind == 0 and cfg.gemm_tiles != 2
+            and cfg.precision == 0)
+
+
 def launches(cfg):
     """Kernels one moe_layer_forward launches: router (which also counts the
     experts per 128-token tile on the bf16 path; the fp32 path adds a count
-    kernel), a separate scan only for large E * ceil(T/128), rank, row copy,
-    the zero fill of the padded layout, the expert stage and the combine."""
+    kernel), a separate scan only for large E * ceil(T/128), rank, row copy
+    (in MXFP8 with the compact layout replaced by the dispatch that quantises
+    the rows), the zero fill of the padded layout, the MXFP8 row quantisation
+    of the padded layout, the expert stage and the combine (none when fused
+    into the down projection)."""
     n_chunks = (cfg.T + 127) // 128
     count = 0 if cfg.dtype == 0 else 1
     scan = 0 if cfg.E * n_chunks <= 8192 else 1
     pad = 1 if cfg.layout == 1 and cfg.capacity > 0 else 0
+    copy = 1
     ffn = {0: 2, 1: 0, 2: 1}[cfg.expert_kind]
-    return 1 + count + scan + 1 + 1 + pad + ffn + 1
+    if cfg.precision == 1:
+        ffn += 1                                     # the row quantisation (or the quantising dispatch)
+        copy = 1 if cfg.layout == 1 else 0
+    combine = 0 if fused_combine(cfg) else 1
+    return 1 + count + scan + 1 + copy + pad + ffn + combine
 
 
-def stage_report(st, wl, A_kept, pk, pk_kind):
+def stage_report(st, wl, A_kept, pk, pk_kind, fused=False, precision="bf16"):
+    """Per-stage us and rates of one timed run. fused: the combine ran inside
+    the down projection (its interval is empty and grouped_ffn includes it).
+    precision mxfp8: the expert GEMMs are compared with an fp8 peak taken as
+    twice the measured bf16 one (the nominal dense fp8 : bf16 ratio)."""
     s = wl.elem_bytes
     T, d, E, k, F = wl.T, wl.d, wl.E, wl.k, wl.F
     hbm = pk["hbm_gbs"]
     tf = pk["bf16_tflops_sustained"]
     router_b = T * d * s + E * d * s + T * k * 8
-    permute_b = T * d * s + A_kept * d * s
+    # the dispatch writes bf16 rows, or in MXFP8 E4M3 rows and a scale byte per 32
+    permute_b = T * d * s + (A_kept * d * (1 + 1 / 32) if precision == "mxfp8" else A_kept * d * s)
     combine_b = A_kept * d * s + T * d * s + T * k * 8
     flops = 6.0 * A_kept * d * F if wl.expert_kind == "swiglu" else 0.0
     out = {
@@ -552,24 +653,33 @@ def stage_report(st, wl, A_kept, pk, pk_kind):
         out[key]["frac_hbm"] = out[key]["GB/s"] / hbm
     if flops:
         out["grouped_ffn"]["TFLOP/s"] = flops / st["grouped_ffn"] / 1e9
-        out["grouped_ffn"]["frac_bf16"] = out["grouped_ffn"]["TFLOP/s"] / tf
-    dc = (permute_b + combine_b) / ((st["permute"] + st["combine"]) / 1e3) / 1e9
-    out["dispatch_combine"] = {"GB/s": dc, "frac_hbm": dc / hbm}
+        if precision.startswith("mxfp8"):
+            out["grouped_ffn"]["frac_fp8"] = out["grouped_ffn"]["TFLOP/s"] / (2.0 * tf)
+        else:
+            out["grouped_ffn"]["frac_bf16"] = out["grouped_ffn"]["TFLOP/s"] / tf
+    if fused:
+        out["combine"] = {"us": 1e3 * st["combine"],
+                          "fused": "written by the down projection's epilogue; its time is inside grouped_ffn"}
+        out["dispatch_combine"] = {"note": "combine fused; see the combine_separate object for the separate kernel"}
+    else:
+        dc = (permute_b + combine_b) / ((st["permute"] + st["combine"]) / 1e3) / 1e9
+        out["dispatch_combine"] = {"GB/s": dc, "frac_hbm": dc / hbm}
     out["peaks"] = {"hbm_gbs": hbm, "bf16_tflops_sustained": tf, "source": f"{pk_kind} (MEASURED_PEAKS.json)"
                     if pk_kind == "measured" else "fallback"}
     return out
 
 
-def roofline(st, wl, A_kept, pk, pk_kind):
+def roofline(st, wl, A_kept, pk, pk_kind, precision="bf16"):
     if wl.expert_kind == "swiglu":
         flops = 6.0 * A_kept * wl.d * wl.F
         ach = flops / (st["grouped_ffn"] / 1e3) / 1e12
-        peak = pk["bf16_tflops_sustained"]
+        peak = pk["bf16_tflops_sustained"] * (2.0 if precision == "mxfp8" else 1.0)
         return {"bound": "tensor", "kernel": "grouped_gemm (SwiGLU GEMM1 + GEMM2, one call)", "achieved": ach,
                 "peak": peak, "unit": "TFLOP/s", "frac": ach / peak, "traffic": None,
                 "traffic_note": "DRAM bytes come from ncu captures kept as summaries under profiles/; "
                                 "this run does not measure them",
-                "peak_source": f"bf16_tflops_sustained, {pk_kind}"}
+                "peak_source": (f"2 x bf16_tflops_sustained (nominal fp8:bf16 ratio), {pk_kind}"
+                                if precision == "mxfp8" else f"bf16_tflops_sustained, {pk_kind}")}
     s = wl.elem_bytes
     b = wl.T * wl.d * s + A_kept * wl.d * s
     ach = b / (st["permute"] / 1e3) / 1e9

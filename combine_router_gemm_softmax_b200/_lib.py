@@ -19,6 +19,9 @@ LIB_PATH = os.path.join(_HERE, "libmoe_b200.so")
 
 MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_WORKSPACE, MOE_ERR_CUDA, MOE_ERR_NO_DEVICE = range(6)
 MOE_STATUS_NAN_LOGIT, MOE_STATUS_BAD_ROUTE, MOE_STATUS_TIMEOUT = 1, 2, 4
+MOE_STATUS_MX_SATURATED, MOE_STATUS_MX_UNDERFLOW = 8, 16
+MOE_PRECISION_BF16, MOE_PRECISION_MXFP8 = 0, 1
+MOE_COMBINE_AUTO, MOE_COMBINE_SEPARATE, MOE_COMBINE_FUSED = 0, 1, 2
 MOE_DTYPE_BF16, MOE_DTYPE_F32 = 0, 1
 MOE_EXPERT_SWIGLU, MOE_EXPERT_IDENTITY, MOE_EXPERT_SCALE = 0, 1, 2
 MOE_OP_ROUTE, MOE_OP_PERMUTE, MOE_OP_GROUPED_FFN, MOE_OP_LAYER, MOE_OP_BACKWARD = 0, 1, 2, 3, 4
@@ -30,7 +33,8 @@ MOE_MAX_E, MOE_MAX_K, MOE_PACK_BLOCK = 256, 8, 128
 EXPORTED = ("moe_workspace_size", "moe_status_string", "moe_version", "moe_pack_weights", "moe_route",
             "moe_permute", "moe_grouped_ffn", "moe_unpermute_combine", "moe_layer_forward",
             "moe_permute_static_scratch", "moe_layer_forward_timed", "moe_pack_weights_backward",
-            "moe_layer_backward")
+            "moe_layer_backward", "moe_mxfp8_quantize", "moe_mxfp8_weights_size", "moe_pack_weights_mxfp8",
+            "moe_debug_stall_next_gemms")
 
 
 class MoeError(RuntimeError):
@@ -43,7 +47,7 @@ class MoeConfig(ctypes.Structure):
     _fields_ = [("T", ctypes.c_int32), ("d", ctypes.c_int32), ("E", ctypes.c_int32), ("k", ctypes.c_int32),
                 ("d_ff", ctypes.c_int32), ("dtype", ctypes.c_int32), ("expert_kind", ctypes.c_int32),
                 ("capacity", ctypes.c_int32), ("gemm_tiles", ctypes.c_int32), ("layout", ctypes.c_int32),
-                ("dispatch", ctypes.c_int32)]
+                ("dispatch", ctypes.c_int32), ("precision", ctypes.c_int32), ("combine", ctypes.c_int32)]
 
     def __repr__(self):
         return "MoeConfig(" + ", ".join(f"{n}={getattr(self, n)}" for n, _ in self._fields_) + ")"
@@ -75,6 +79,10 @@ _SIGS = {
     "moe_layer_forward_timed": (I32, [CFG, P, P, P, P, P, P, P, P, P, P, P, SZ, P, P, P]),
     "moe_pack_weights_backward": (I32, [CFG, P, P, P, P, P]),
     "moe_layer_backward": (I32, [CFG, P, P, P, P, P, P, P, P, P, P, P, P, SZ, P, SZ, P, P]),
+    "moe_mxfp8_quantize": (I32, [P, I32, I32, P, P, P, P, P]),
+    "moe_mxfp8_weights_size": (SZ, [CFG, I32]),
+    "moe_pack_weights_mxfp8": (I32, [CFG, P, P, P, P, P, P]),
+    "moe_debug_stall_next_gemms": (I32, [I32]),
 }
 
 
@@ -96,14 +104,16 @@ def lib() -> ctypes.CDLL:
 
 
 def config(T, d, E, k, d_ff, dtype="bf16", expert_kind="swiglu", capacity=-1, gemm_tiles="auto",
-           layout="compact", dispatch="auto") -> MoeConfig:
+           layout="compact", dispatch="auto", precision="bf16", combine="auto") -> MoeConfig:
     dt = {"bf16": MOE_DTYPE_BF16, "f32": MOE_DTYPE_F32, torch.bfloat16: MOE_DTYPE_BF16,
           torch.float32: MOE_DTYPE_F32}[dtype]
     kind = {"swiglu": MOE_EXPERT_SWIGLU, "identity": MOE_EXPERT_IDENTITY, "scale": MOE_EXPERT_SCALE}[expert_kind]
     tiles = {"auto": MOE_GEMM_TILES_AUTO, "single": MOE_GEMM_TILES_SINGLE, "pair": MOE_GEMM_TILES_PAIR}[gemm_tiles]
     lay = {"compact": MOE_LAYOUT_COMPACT, "padded": MOE_LAYOUT_PADDED}[layout]
     disp = {"auto": MOE_DISPATCH_AUTO, "copy": MOE_DISPATCH_COPY, "gather": MOE_DISPATCH_GATHER}[dispatch]
-    return MoeConfig(T, d, E, k, d_ff, dt, kind, capacity, tiles, lay, disp)
+    prec = {"bf16": MOE_PRECISION_BF16, "mxfp8": MOE_PRECISION_MXFP8}[precision]
+    comb = {"auto": MOE_COMBINE_AUTO, "separate": MOE_COMBINE_SEPARATE, "fused": MOE_COMBINE_FUSED}[combine]
+    return MoeConfig(T, d, E, k, d_ff, dt, kind, capacity, tiles, lay, disp, prec, comb)
 
 
 def perm_rows(cfg) -> int:
@@ -145,6 +155,17 @@ def _rc(fn, code):
 
 def _dev(ref):
     return ref.device
+
+
+def _check_expert_weights(cfg, w13, w_down):
+    """bf16: w13_packed [E, 2F, d] and w_down [E, d, F]; MXFP8: the two uint8
+    blobs of moe_pack_weights_mxfp8."""
+    if cfg.precision == MOE_PRECISION_MXFP8:
+        _check(w13, (moe_mxfp8_weights_size(cfg, 0),), torch.uint8, "w13 MXFP8 blob")
+        _check(w_down, (moe_mxfp8_weights_size(cfg, 1),), torch.uint8, "w_down MXFP8 blob")
+    else:
+        _check(w13, (cfg.E, 2 * cfg.d_ff, cfg.d), cfg.torch_dtype, "w13_packed")
+        _check(w_down, (cfg.E, cfg.d, cfg.d_ff), cfg.torch_dtype, "w_down")
 
 
 def moe_workspace_size(cfg: MoeConfig, op: int) -> int:
@@ -219,8 +240,7 @@ def moe_grouped_ffn(cfg, x_perm, offsets, w13_packed=None, w_down=None, y_perm=N
         raise ValueError("x_perm needs perm_rows(cfg) rows")
     _check(offsets, (cfg.E + 1,), torch.int32, "offsets")
     if cfg.expert_kind == MOE_EXPERT_SWIGLU:
-        _check(w13_packed, (cfg.E, 2 * cfg.d_ff, cfg.d), dt, "w13_packed")
-        _check(w_down, (cfg.E, cfg.d, cfg.d_ff), dt, "w_down")
+        _check_expert_weights(cfg, w13_packed, w_down)
     if y_perm is None:
         y_perm = torch.empty((rows, cfg.d), dtype=dt, device=dev)
     if ws is None:
@@ -255,8 +275,7 @@ def moe_layer_forward(cfg, h, w_router, bias=None, w13_packed=None, w_down=None,
     _check(w_router, (cfg.E, cfg.d), dt, "w_router")
     _check(bias, (cfg.E,), torch.float32, "bias")
     if cfg.expert_kind == MOE_EXPERT_SWIGLU:
-        _check(w13_packed, (cfg.E, 2 * cfg.d_ff, cfg.d), dt, "w13_packed")
-        _check(w_down, (cfg.E, cfg.d, cfg.d_ff), dt, "w_down")
+        _check_expert_weights(cfg, w13_packed, w_down)
     _check(topk_idx, (cfg.T, cfg.k), torch.int32, "topk_idx")
     _check(topk_gate, (cfg.T, cfg.k), torch.float32, "topk_gate")
     _check(routed_counts, (cfg.E,), torch.int32, "routed_counts")
@@ -350,3 +369,55 @@ def moe_layer_backward(cfg, h, w_router, w13_packed, w13_t, w_down_t, dy, fwd_ws
         _ptr(out["dh"]), _ptr(out["dw_router"]), _ptr(out["dbias"]), _ptr(out["dw13"]), _ptr(out["dw_down"]),
         _ptr(fwd_ws), fwd_ws.numel(), _ptr(ws), ws.numel(), _ptr(status), _stream(stream)))
     return out
+
+
+def moe_mxfp8_weights_size(cfg, which: int) -> int:
+    """Bytes of the MXFP8 weight blob: which 0 = w13, 1 = w_down."""
+    return int(lib().moe_mxfp8_weights_size(ctypes.byref(cfg), which))
+
+
+def mxfp8_scale_bytes(rows, cols) -> int:
+    """Bytes of the scale atoms moe_mxfp8_quantize writes for [rows, cols]."""
+    return (cols // 128) * ((rows + 127) // 128) * 512
+
+
+def moe_mxfp8_quantize(x, q=None, sf=None, counts=None, status=None, stream=None):
+    """MXFP8 quantisation of a bf16 matrix [rows, cols] along its rows.
+    Returns (q [rows, cols] uint8 E4M3 bytes, sf uint8 scale atoms);
+    counts (uint32 [2], may be None) receives the saturated and underflowed
+    element counts added."""
+    if x.dim() != 2 or x.dtype != torch.bfloat16:
+        raise ValueError("x must be a 2-D bf16 tensor")
+    rows, cols = x.shape
+    dev = _dev(x)
+    if q is None:
+        q = torch.empty((rows, cols), dtype=torch.uint8, device=dev)
+    if sf is None:
+        sf = torch.zeros(max(mxfp8_scale_bytes(rows, cols), 1), dtype=torch.uint8, device=dev)
+    _check(q, (rows, cols), torch.uint8, "q")
+    if sf.numel() < mxfp8_scale_bytes(rows, cols) or sf.dtype != torch.uint8:
+        raise ValueError("sf too small")
+    if counts is not None and (counts.dtype != torch.int32 or counts.numel() < 2):
+        raise ValueError("counts must be int32 with 2 entries (read as uint32)")
+    _rc("moe_mxfp8_quantize", lib().moe_mxfp8_quantize(_ptr(x), rows, cols, _ptr(q), _ptr(sf), _ptr(counts),
+                                                       _ptr(status), _stream(stream)))
+    return q, sf
+
+
+def moe_pack_weights_mxfp8(cfg, w13_packed, w_down, counts=None, stream=None):
+    """Quantise the expert weights for MOE_PRECISION_MXFP8. Returns the two
+    uint8 blobs (w13_mx, w_down_mx)."""
+    _check(w13_packed, (cfg.E, 2 * cfg.d_ff, cfg.d), torch.bfloat16, "w13_packed")
+    _check(w_down, (cfg.E, cfg.d, cfg.d_ff), torch.bfloat16, "w_down")
+    dev = _dev(w13_packed)
+    a = torch.empty(moe_mxfp8_weights_size(cfg, 0), dtype=torch.uint8, device=dev)
+    b = torch.empty(moe_mxfp8_weights_size(cfg, 1), dtype=torch.uint8, device=dev)
+    _rc("moe_pack_weights_mxfp8", lib().moe_pack_weights_mxfp8(ctypes.byref(cfg), _ptr(w13_packed), _ptr(w_down),
+                                                               _ptr(a), _ptr(b), _ptr(counts), _stream(stream)))
+    return a, b
+
+
+def mx_counters(ws):
+    """The four uint32 counters an MXFP8 call leaves at the start of its
+    workspace: x saturated, x underflowed, h_mid saturated, h_mid underflowed."""
+    return ws[:16].view(torch.int32).cpu().tolist()

@@ -55,6 +55,21 @@ int make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uin
   return r == CUDA_SUCCESS ? MOE_OK : MOE_ERR_CUDA;
 }
 
+// Row-major byte matrix [rows, cols] (E4M3 elements), box of box_rows x 128
+// columns, 128-byte swizzle.
+int make_map_u8(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (enc == nullptr) return MOE_ERR_NO_DEVICE;
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {cols};
+  const cuuint32_t box[2] = {128, box_rows};
+  const cuuint32_t es[2] = {1, 1};
+  const CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, es,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? MOE_OK : MOE_ERR_CUDA;
+}
+
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
 
 int elem_bytes(const moe_config& c) { return c.dtype == MOE_DTYPE_BF16 ? 2 : 4; }
@@ -66,11 +81,48 @@ size_t perm_rows(const moe_config& c) {
 }
 
 
+bool is_mx(const moe_config& c) { return c.precision == MOE_PRECISION_MXFP8; }
+
+// The layer's MXFP8 dispatch writes the quantised rows straight from h.
+bool mx_dispatch_fused(const moe_config& c) { return is_mx(c) && c.layout == MOE_LAYOUT_COMPACT; }
+
 // Whether the layer's GEMM1 can gather its A rows from h (no x_perm).
 bool gather_supported(const moe_config& c) {
   return c.dtype == MOE_DTYPE_BF16 && c.expert_kind == MOE_EXPERT_SWIGLU && c.layout == MOE_LAYOUT_COMPACT &&
-         c.gemm_tiles != MOE_GEMM_TILES_PAIR;
+         c.gemm_tiles != MOE_GEMM_TILES_PAIR && !is_mx(c);
 }
+
+size_t round256(size_t n) { return (n + 255) & ~static_cast<size_t>(255); }
+
+// MXFP8 weight blob: E4M3 bytes [rows, cols], then the scale atoms with one
+// extra 128-row block per 128-column slice (a 256-row B tile that ends one
+// block past the last expert reads it).
+struct MxBlob {
+  size_t rows, cols, q_bytes, sf_bytes;
+  int row_blocks;  // including the extra one
+};
+
+MxBlob mx_blob(const moe_config& c, int which) {
+  MxBlob b;
+  b.rows = which == 0 ? static_cast<size_t>(c.E) * 2 * c.d_ff : static_cast<size_t>(c.E) * c.d;
+  b.cols = which == 0 ? static_cast<size_t>(c.d) : static_cast<size_t>(c.d_ff);
+  b.row_blocks = static_cast<int>(b.rows / 128 + 1);
+  b.q_bytes = round256(b.rows * b.cols);
+  b.sf_bytes = (b.cols / 128) * static_cast<size_t>(b.row_blocks) * 512;
+  return b;
+}
+
+// Whether the layer's down projection also writes y (the combine fused into
+// its epilogue): k <= 2, bf16 SwiGLU experts on single-CTA bf16 tiles.
+bool combine_fusable(const moe_config& c) {
+  return c.k <= 2 && c.dtype == MOE_DTYPE_BF16 && c.expert_kind == MOE_EXPERT_SWIGLU &&
+         c.gemm_tiles != MOE_GEMM_TILES_PAIR && !is_mx(c);
+}
+
+// AUTO keeps the separate combine: fusing it measured 1-3% slower per layer
+// on B200 (the down projection's epilogue re-reads both rows of a token and
+// competes with the GEMM; the separate kernel streams them at HBM rate).
+bool layer_fuses_combine(const moe_config& c) { return c.combine == MOE_COMBINE_FUSED && combine_fusable(c); }
 
 // AUTO copies: gathering costs one four-row TMA gather per 512 bytes of A
 // every time a tile reloads its A rows (once per column tile), and measured
@@ -93,6 +145,13 @@ int check_cfg(const moe_config* c) {
   if (c->E > MOE_MAX_E || c->k > MOE_MAX_K || c->k > c->E) return MOE_ERR_UNSUPPORTED;
   if (static_cast<long long>(c->T) * c->k >= (1LL << 31)) return MOE_ERR_UNSUPPORTED;
   if (c->layout == MOE_LAYOUT_PADDED && static_cast<long long>(c->E) * c->capacity >= (1LL << 31))
+    return MOE_ERR_UNSUPPORTED;
+  if (c->precision != MOE_PRECISION_BF16 && c->precision != MOE_PRECISION_MXFP8) return MOE_ERR_INVALID_ARG;
+  if (c->combine < MOE_COMBINE_AUTO || c->combine > MOE_COMBINE_FUSED) return MOE_ERR_INVALID_ARG;
+  if (c->combine == MOE_COMBINE_FUSED && !combine_fusable(*c)) return MOE_ERR_UNSUPPORTED;
+  if (c->precision == MOE_PRECISION_MXFP8 &&
+      (c->dtype != MOE_DTYPE_BF16 || c->expert_kind != MOE_EXPERT_SWIGLU || c->gemm_tiles == MOE_GEMM_TILES_PAIR ||
+       c->dispatch == MOE_DISPATCH_GATHER))
     return MOE_ERR_UNSUPPORTED;
   if (c->dtype == MOE_DTYPE_BF16) {
     if (c->d % 128 != 0) return MOE_ERR_UNSUPPORTED;
@@ -131,15 +190,43 @@ PermuteScratch carve_permute(const moe_config& c, Carver& w) {
 }
 
 void* carve_ffn(const moe_config& c, Carver& w) {
-  if (c.expert_kind != MOE_EXPERT_SWIGLU) return nullptr;
+  if (c.expert_kind != MOE_EXPERT_SWIGLU || is_mx(c)) return nullptr;
   return w.take<void>(perm_rows(c) * c.d_ff * elem_bytes(c));
 }
+
+// MXFP8 scratch (first in the workspace of the grouped FFN and the layer):
+// the call's four counters, then the quantised token rows and h_mid in the
+// padded layout (each expert's rows from a 128-row boundary) with their scale
+// atoms. The padded rows are at most P + 127 E.
+struct MxBufs {
+  uint32_t* counters;  // [4]: x saturated, x underflowed, h_mid saturated, h_mid underflowed
+  uint8_t *xq, *xsf, *hq, *hsf;
+  int pad_rows, row_blocks;
+};
+
+MxBufs carve_mx(const moe_config& c, Carver& w) {
+  MxBufs m{};
+  m.pad_rows = static_cast<int>((perm_rows(c) + 127) / 128 * 128 + 128 * static_cast<size_t>(c.E));
+  m.row_blocks = m.pad_rows / 128;
+  const size_t d = c.d, F = c.d_ff, R = m.pad_rows;
+  m.counters = w.take<uint32_t>(16);
+  m.xq = w.take<uint8_t>(R * d);
+  m.xsf = w.take<uint8_t>((d / 128) * m.row_blocks * 512);
+  m.hq = w.take<uint8_t>(R * F);
+  m.hsf = w.take<uint8_t>((F / 128) * m.row_blocks * 512);
+  return m;
+}
+
+// Counters of the fused combine per token: one per 256-column tile of the
+// down projection and per half of it (two epilogue warps share a tile row).
+int pair_entries(const moe_config& c) { return 2 * ((c.d + kGemmTileN - 1) / kGemmTileN); }
 
 struct LayerBufs {
   int32_t *idx, *routed, *kept, *offsets, *dest_row, *perm_src;
   float* gate;
   void *x_perm, *y_perm, *h_mid;
   PermuteScratch perm;
+  int32_t* pair_cnt;  // [T][pair_entries(c)] when the combine is fused, else NULL
 };
 
 LayerBufs carve_layer(const moe_config& c, Carver& w) {
@@ -154,10 +241,13 @@ LayerBufs carve_layer(const moe_config& c, Carver& w) {
   b.offsets = w.take<int32_t>((c.E + 1) * 4);
   b.dest_row = w.take<int32_t>(A * 4);
   b.perm_src = w.take<int32_t>(P * 4);
-  b.x_perm = layer_gathers(c) ? nullptr : w.take<void>(P * row);  // GEMM1 gathers from h instead
+  // no x_perm when GEMM1 gathers from h, or when the MXFP8 dispatch quantises h straight into its
+  // layout (compact rows; the padded capacity layout keeps the bf16 copy, whose padding rows are zeroed)
+  b.x_perm = layer_gathers(c) || mx_dispatch_fused(c) ? nullptr : w.take<void>(P * row);
   b.y_perm = c.expert_kind == MOE_EXPERT_IDENTITY ? nullptr : w.take<void>(P * row);
   b.perm = carve_permute(c, w);
   b.h_mid = carve_ffn(c, w);
+  b.pair_cnt = layer_fuses_combine(c) ? w.take<int32_t>(static_cast<size_t>(c.T) * pair_entries(c) * 4) : nullptr;
   return b;
 }
 
@@ -197,7 +287,7 @@ BackwardBufs carve_backward(const moe_config& c, Carver& w) {
 }
 
 bool backward_supported(const moe_config& c) {
-  return c.dtype == MOE_DTYPE_BF16 && c.expert_kind == MOE_EXPERT_SWIGLU && !layer_gathers(c);
+  return c.dtype == MOE_DTYPE_BF16 && c.expert_kind == MOE_EXPERT_SWIGLU && !layer_gathers(c) && !is_mx(c);
 }
 
 size_t ws_size(const moe_config& c, int op) {
@@ -213,9 +303,11 @@ size_t ws_size(const moe_config& c, int op) {
       carve_permute(c, w);
       return w.off;
     case MOE_OP_GROUPED_FFN:
+      if (is_mx(c)) carve_mx(c, w);
       carve_ffn(c, w);
       return w.off;
     case MOE_OP_LAYER:
+      if (is_mx(c)) carve_mx(c, w);
       carve_layer(c, w);
       return w.off;
     default:
@@ -247,19 +339,77 @@ int route_impl(const moe_config& c, const void* h, const void* w_router, const f
 // same library call.
 int permute_impl(const moe_config& c, const void* h, const int32_t* idx, int32_t* routed, int32_t* kept,
                  int32_t* offsets, int32_t* dest_row, int32_t* perm_src, void* x_perm, const PermuteScratch& p,
-                 bool counts_ready, bool copy_rows, bool pdl, int32_t* status, cudaStream_t s) {
+                 bool counts_ready, bool copy_rows, bool pdl, int32_t* status, cudaStream_t s,
+                 int32_t* pair_cnt = nullptr, void* y_zero = nullptr) {
   return cuda_rc(launch_permute(h, static_cast<size_t>(c.d) * elem_bytes(c), idx, c.T, c.k, c.E, c.capacity,
                                 c.layout == MOE_LAYOUT_PADDED, copy_rows, p.chunk_counts, p.chunk_base, routed, kept,
-                                offsets, dest_row, perm_src, x_perm, counts_ready, pdl, status, s));
+                                offsets, dest_row, perm_src, x_perm, counts_ready, pdl, status, s, pair_cnt,
+                                pair_cnt != nullptr ? pair_entries(c) : 0, y_zero));
 }
+
+// The combine done by the down projection (launch_grouped_gemm_combine).
+struct FusedCombine {
+  const int32_t* perm_src;
+  const int32_t* dest_row;
+  const float* gate;
+  int32_t* pair_cnt;
+  void* y;
+};
 
 // gather_src / gather_rows (bf16 SwiGLU single tiles only; NULL otherwise):
 // GEMM1 reads A row r as gather_src[gather_rows[r]] instead of x_perm[r].
+// MXFP8 experts: quantise the permuted rows into the padded layout, GEMM1
+// with SwiGLU and the MXFP8 quantisation of h_mid in its epilogue, GEMM2 to
+// bf16 y_perm. w13 and w_down are the blobs of moe_pack_weights_mxfp8; the
+// counters were zeroed by the caller.
+// The layer's MXFP8 dispatch: the token rows go from h straight into the
+// padded quantised layout (no bf16 x_perm).
+struct MxDispatch {
+  const void* h;
+  const int32_t* idx;
+  const int32_t* dest_row;
+};
+
+// The layer's quantising dispatch (part of its dispatch stage).
+int mx_dispatch_impl(const moe_config& c, const MxDispatch& md, const int32_t* offsets, const MxBufs& m,
+                     int32_t* status, cudaStream_t s) {
+  return cuda_rc(launch_mx_dispatch(md.h, c.T, c.d, c.k, md.idx, md.dest_row, offsets, c.E, m.xq, m.xsf,
+                                    m.row_blocks, m.counters, status, true, s));
+}
+
+// x_quantized: the token rows are already in m.xq (the layer's quantising
+// dispatch ran); else x_perm is quantised first.
+int ffn_mx_impl(const moe_config& c, const void* x_perm, const int32_t* offsets, const void* w13, const void* w_down,
+                void* y_perm, const MxBufs& m, bool pdl, int32_t* status, cudaStream_t s, bool x_quantized) {
+  const int F = c.d_ff, d = c.d, E = c.E;
+  const MxBlob b13 = mx_blob(c, 0), bd = mx_blob(c, 1);
+  const uint8_t* w13q = static_cast<const uint8_t*>(w13);
+  const uint8_t* wdq = static_cast<const uint8_t*>(w_down);
+  cudaError_t e = cudaSuccess;
+  if (!x_quantized)
+    e = launch_mx_quantize(x_perm, m.pad_rows, d, offsets, E, m.xq, m.xsf, m.row_blocks, m.counters, status, pdl, s);
+  if (e != cudaSuccess) return MOE_ERR_CUDA;
+  CUtensorMap a1, b1, a2, b2;
+  int rc = make_map_u8(&a1, m.xq, m.pad_rows, d, 128);
+  if (rc == MOE_OK) rc = make_map_u8(&b1, w13q, b13.rows, d, 256);
+  if (rc == MOE_OK) rc = make_map_u8(&a2, m.hq, m.pad_rows, F, 128);
+  if (rc == MOE_OK) rc = make_map_u8(&b2, wdq, bd.rows, F, 256);
+  if (rc != MOE_OK) return rc;
+  e = launch_grouped_gemm_mx(a1, b1, true, offsets, E, d, 2 * F, F, m.xsf, m.row_blocks, w13q + b13.q_bytes, m.hq,
+                             m.hsf, F, m.counters + 2, nullptr, 0, status, true, s);
+  if (e != cudaSuccess) return MOE_ERR_CUDA;
+  e = launch_grouped_gemm_mx(a2, b2, false, offsets, E, F, d, d, m.hsf, m.row_blocks, wdq + bd.q_bytes, nullptr,
+                             nullptr, 0, nullptr, y_perm, d, status, true, s);
+  return cuda_rc(e);
+}
+
 int ffn_impl(const moe_config& c, const void* x_perm, const int32_t* offsets, const void* w13, const void* w_down,
              void* y_perm, void* h_mid, const void* gather_src, const int32_t* gather_rows, bool pdl,
-             int32_t* status, cudaStream_t s) {
+             int32_t* status, cudaStream_t s, const MxBufs* mx = nullptr, const FusedCombine* fc = nullptr,
+             bool mx_x_quantized = false) {
   const int rows_max = static_cast<int>(perm_rows(c));
   if (rows_max == 0) return MOE_OK;
+  if (is_mx(c)) return ffn_mx_impl(c, x_perm, offsets, w13, w_down, y_perm, *mx, pdl, status, s, mx_x_quantized);
   if (c.expert_kind != MOE_EXPERT_SWIGLU)
     return cuda_rc(launch_scale_rows(c.dtype, c.expert_kind, x_perm, offsets, y_perm, rows_max, c.d, c.E, s));
   if (c.dtype == MOE_DTYPE_F32)
@@ -283,8 +433,12 @@ int ffn_impl(const moe_config& c, const void* x_perm, const int32_t* offsets, co
                                     gather ? gather_rows : nullptr, status, pdl, s);
   if (e != cudaSuccess) return MOE_ERR_CUDA;
   const int n2 = (d + kGemmTileN - 1) / kGemmTileN;
-  e = pair ? launch_grouped_gemm_pair(a2, b2, false, offsets, E, F, d, n2, d, d, y_perm, status, true, s)
-           : launch_grouped_gemm_tc(a2, b2, false, offsets, E, F, d, n2, d, d, y_perm, nullptr, status, true, s);
+  if (fc != nullptr)
+    e = launch_grouped_gemm_combine(a2, b2, offsets, E, F, d, y_perm, fc->perm_src, fc->dest_row, fc->gate,
+                                    fc->pair_cnt, fc->y, c.k, status, true, s);
+  else
+    e = pair ? launch_grouped_gemm_pair(a2, b2, false, offsets, E, F, d, n2, d, d, y_perm, status, true, s)
+             : launch_grouped_gemm_tc(a2, b2, false, offsets, E, F, d, n2, d, d, y_perm, nullptr, status, true, s);
   return cuda_rc(e);
 }
 
@@ -295,7 +449,7 @@ using namespace moe;
 
 extern "C" {
 
-int32_t moe_version(void) { return (1 << 16) | 0; }
+int32_t moe_version(void) { return (1 << 16) | 1; }
 
 const char* moe_status_string(int32_t code) {
   switch (code) {
@@ -382,9 +536,15 @@ int32_t moe_grouped_ffn(const moe_config* cfg, const void* x_perm, const int32_t
   const size_t need = ws_size(*cfg, MOE_OP_GROUPED_FFN);
   if (ws_bytes < need || (need > 0 && (!workspace || !aligned(workspace, 16)))) return MOE_ERR_WORKSPACE;
   Carver w(workspace);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  MxBufs mx{};
+  if (is_mx(*cfg)) {
+    mx = carve_mx(*cfg, w);
+    if (cudaMemsetAsync(mx.counters, 0, 16, s) != cudaSuccess) return MOE_ERR_CUDA;
+  }
   void* h_mid = carve_ffn(*cfg, w);
-  return ffn_impl(*cfg, x_perm, offsets, w13_packed, w_down, y_perm, h_mid, nullptr, nullptr, false, status_dev,
-                  static_cast<cudaStream_t>(stream));
+  return ffn_impl(*cfg, x_perm, offsets, w13_packed, w_down, y_perm, h_mid, nullptr, nullptr, false, status_dev, s,
+                  &mx);
 }
 
 int32_t moe_unpermute_combine(const moe_config* cfg, const void* y_perm, const int32_t* dest_row,
@@ -393,11 +553,12 @@ int32_t moe_unpermute_combine(const moe_config* cfg, const void* y_perm, const i
   int rc = check_cfg(cfg);
   if (rc != MOE_OK) return rc;
   if (cfg->T > 0 && (!y_perm || !dest_row || !topk_gate || !y)) return MOE_ERR_INVALID_ARG;
-  if (!aligned(y_perm, 16) || !aligned(y, 16) || !aligned(dest_row, 4) || !aligned(topk_gate, 4))
+  if (!aligned(y_perm, 16) || !aligned(y, 16) || !aligned(dest_row, 4) || !aligned(topk_gate, 4) ||
+      !aligned(status_dev, 4))
     return MOE_ERR_UNSUPPORTED;
   return cuda_rc(
       launch_combine(cfg->dtype, y_perm, dest_row, topk_gate, y, cfg->T, cfg->k, cfg->d, false,
-                     static_cast<cudaStream_t>(stream)));
+                     static_cast<cudaStream_t>(stream), status_dev));
 }
 
 int32_t moe_layer_forward(const moe_config* cfg, const void* h, const void* w_router, const float* bias,
@@ -425,6 +586,8 @@ int32_t moe_layer_forward_timed(const moe_config* cfg, const void* h, const void
   const size_t need = ws_size(c, MOE_OP_LAYER);
   if (ws_bytes < need || (need > 0 && (!workspace || !aligned(workspace, 16)))) return MOE_ERR_WORKSPACE;
   Carver w(workspace);
+  MxBufs mx{};
+  if (is_mx(c)) mx = carve_mx(c, w);
   LayerBufs b = carve_layer(c, w);
   if (topk_idx) b.idx = topk_idx;
   if (topk_gate) b.gate = topk_gate;
@@ -435,6 +598,7 @@ int32_t moe_layer_forward_timed(const moe_config* cfg, const void* h, const void
     if (stage_events == nullptr || stage_events[i] == nullptr) return MOE_OK;
     return cuda_rc(cudaEventRecord(static_cast<cudaEvent_t>(stage_events[i]), s));
   };
+  if (is_mx(c) && cudaMemsetAsync(mx.counters, 0, 16, s) != cudaSuccess) return MOE_ERR_CUDA;
   if ((rc = mark(0)) != MOE_OK) return rc;
   // the bf16 router also writes the per-tile expert histogram the dispatch needs
   const bool router_counts = c.dtype == MOE_DTYPE_BF16;
@@ -445,20 +609,76 @@ int32_t moe_layer_forward_timed(const moe_config* cfg, const void* h, const void
   // dependent of the one before it, so its launch and prologue overlap the
   // previous kernel's tail
   const bool gather = layer_gathers(c);
+  const bool fused = b.pair_cnt != nullptr;
   rc = permute_impl(c, h, b.idx, b.routed, b.kept, b.offsets, b.dest_row, b.perm_src, b.x_perm, b.perm,
-                    router_counts, !gather, true, status_dev, s);
+                    router_counts, b.x_perm != nullptr, true, status_dev, s, b.pair_cnt, fused ? y : nullptr);
+  // MXFP8 (compact): the rows go from h straight into the quantised layout, as part of the dispatch
+  const bool mx_disp = mx_dispatch_fused(c) && perm_rows(c) > 0;
+  if (rc == MOE_OK && mx_disp) rc = mx_dispatch_impl(c, MxDispatch{h, b.idx, b.dest_row}, b.offsets, mx, status_dev, s);
   if (rc != MOE_OK || (rc = mark(2)) != MOE_OK) return rc;
   const void* y_src = b.x_perm;
+  const FusedCombine fc{b.perm_src, b.dest_row, b.gate, b.pair_cnt, y};
   if (c.expert_kind != MOE_EXPERT_IDENTITY) {
     rc = ffn_impl(c, b.x_perm, b.offsets, w13_packed, w_down, b.y_perm, b.h_mid, gather ? h : nullptr,
-                  gather ? b.perm_src : nullptr, true, status_dev, s);
+                  gather ? b.perm_src : nullptr, true, status_dev, s, &mx, fused ? &fc : nullptr, mx_disp);
     if (rc != MOE_OK) return rc;
     y_src = b.y_perm;
   }
   if ((rc = mark(3)) != MOE_OK) return rc;
-  rc = cuda_rc(launch_combine(c.dtype, y_src, b.dest_row, b.gate, y, c.T, c.k, c.d, true, s));
-  if (rc != MOE_OK) return rc;
+  if (!fused) {
+    rc = cuda_rc(launch_combine(c.dtype, y_src, b.dest_row, b.gate, y, c.T, c.k, c.d, true, s, status_dev));
+    if (rc != MOE_OK) return rc;
+  }
   return mark(4);
+}
+
+int32_t moe_debug_stall_next_gemms(int32_t n) {
+  if (n < 0) return MOE_ERR_INVALID_ARG;
+  debug_stall_next_gemms(n);
+  return MOE_OK;
+}
+
+int32_t moe_mxfp8_quantize(const void* x, int32_t rows, int32_t cols, void* q, void* sf, uint32_t* counts,
+                           int32_t* status_dev, moe_stream_t stream) {
+  if (rows < 0 || cols <= 0) return MOE_ERR_INVALID_ARG;
+  if (cols % 128 != 0) return MOE_ERR_UNSUPPORTED;
+  if (rows > 0 && (!x || !q || !sf)) return MOE_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(q, 16) || !aligned(counts, 4) || !aligned(status_dev, 4))
+    return MOE_ERR_UNSUPPORTED;
+  return cuda_rc(launch_mx_quantize(x, rows, cols, nullptr, 0, q, sf, (rows + 127) / 128, counts, status_dev, false,
+                                    static_cast<cudaStream_t>(stream)));
+}
+
+size_t moe_mxfp8_weights_size(const moe_config* cfg, int32_t which) {
+  if (check_cfg(cfg) != MOE_OK || cfg->dtype != MOE_DTYPE_BF16 || cfg->expert_kind != MOE_EXPERT_SWIGLU ||
+      (which != 0 && which != 1))
+    return 0;
+  const MxBlob b = mx_blob(*cfg, which);
+  return b.q_bytes + b.sf_bytes;
+}
+
+int32_t moe_pack_weights_mxfp8(const moe_config* cfg, const void* w13_packed, const void* w_down, void* w13_mx,
+                               void* w_down_mx, uint32_t* counts, moe_stream_t stream) {
+  int rc = check_cfg(cfg);
+  if (rc != MOE_OK) return rc;
+  const moe_config& c = *cfg;
+  if (c.dtype != MOE_DTYPE_BF16 || c.expert_kind != MOE_EXPERT_SWIGLU) return MOE_ERR_UNSUPPORTED;
+  if (!w13_packed || !w_down || !w13_mx || !w_down_mx) return MOE_ERR_INVALID_ARG;
+  if (!aligned(w13_packed, 16) || !aligned(w_down, 16) || !aligned(w13_mx, 256) || !aligned(w_down_mx, 256) ||
+      !aligned(counts, 4))
+    return MOE_ERR_UNSUPPORTED;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const void* src[2] = {w13_packed, w_down};
+  void* dst[2] = {w13_mx, w_down_mx};
+  for (int which = 0; which < 2; ++which) {
+    const MxBlob b = mx_blob(c, which);
+    uint8_t* q = static_cast<uint8_t*>(dst[which]);
+    if (cudaMemsetAsync(q + b.q_bytes, 0, b.sf_bytes, s) != cudaSuccess) return MOE_ERR_CUDA;
+    const cudaError_t e = launch_mx_quantize(src[which], static_cast<int>(b.rows), static_cast<int>(b.cols), nullptr,
+                                             0, q, q + b.q_bytes, b.row_blocks, counts, nullptr, false, s);
+    if (e != cudaSuccess) return MOE_ERR_CUDA;
+  }
+  return MOE_OK;
 }
 
 int32_t moe_pack_weights_backward(const moe_config* cfg, const void* w13_packed, const void* w_down, void* w13_t,

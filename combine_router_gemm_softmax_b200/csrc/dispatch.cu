@@ -153,7 +153,7 @@ __global__ void __launch_bounds__(kChunkTokens) rank_kernel(
     const int32_t* __restrict__ chunk_table,  // counts [n_chunks][E] (fused) or bases [n_chunks][E]
     const int32_t* __restrict__ offsets_in, int32_t* __restrict__ routed_out, int32_t* __restrict__ kept_out,
     int32_t* __restrict__ offsets_out, int32_t* __restrict__ dest_row, int32_t* __restrict__ perm_src,
-    int32_t* status) {
+    int32_t* status, int32_t* __restrict__ pair_cnt, int pair_tiles, uint4* __restrict__ y_zero, int y_vpr) {
   constexpr int kWarps = kChunkTokens / 32;
   __shared__ uint32_t mask[kWarps][kMaxE];
   __shared__ int wbase[kWarps][kMaxE];
@@ -253,6 +253,7 @@ __global__ void __launch_bounds__(kChunkTokens) rank_kernel(
   __syncthreads();
   if (t < T) {
     const uint32_t lt = lanemask_lt();
+    int n_kept = 0;
 #pragma unroll
     for (int j = 0; j < kMaxK; ++j) {
       if (j >= k) break;
@@ -263,11 +264,19 @@ __global__ void __launch_bounds__(kChunkTokens) rank_kernel(
         if (cap < 0 || r < cap) {
           dest = s_off[e] + r;
           perm_src[dest] = t;
+          ++n_kept;
         }
       }
       dest_row[static_cast<size_t>(t) * k + j] = dest;
     }
     if (valid != ((1u << k) - 1u)) report_status(status, MOE_STATUS_BAD_ROUTE);
+    // combine fused into the down projection: this call's per-token counters
+    // start at zero, and a token with no kept slot gets its zero output row
+    // here (no expert row will write it)
+    if (pair_cnt != nullptr)
+      for (int i = 0; i < pair_tiles; ++i) pair_cnt[static_cast<size_t>(t) * pair_tiles + i] = 0;
+    if (y_zero != nullptr && n_kept == 0)
+      for (int v = 0; v < y_vpr; ++v) y_zero[static_cast<size_t>(t) * y_vpr + v] = make_uint4(0, 0, 0, 0);
   }
 }
 
@@ -297,6 +306,7 @@ constexpr int kCopyPiece = 8192;    // bytes per bulk transfer
 // Tokens per CTA: small blocks give many CTAs per SM and the most row loads in
 // flight (measured on B200 for 4-8 KiB rows and k = 2..8).
 constexpr int kCopyTokensPerCta = 4;
+static_assert(kCopyTokensPerCta <= 32, "one lane stages the active-token list");
 
 // Row copy with the TMA engine. Each CTA owns a contiguous block of tokens and
 // stages their dest_row entries in shared memory; one thread then runs a
@@ -327,14 +337,23 @@ __global__ void __launch_bounds__(32) permute_copy_bulk_kernel(const uint8_t* __
   __syncwarp();
   if (lane != 0) return;
 
-  const int n = nt * n_pieces;
+  // tokens of this block that keep at least one slot (a token whose slots
+  // were all dropped is not read)
+  int act[kCopyTokensPerCta];
+  int n_act = 0;
+  for (int tl = 0; tl < nt; ++tl) {
+    bool any = false;
+    for (int j = 0; j < k; ++j) any = any || dests[tl * k + j] >= 0;
+    if (any) act[n_act++] = tl;
+  }
+  const int n = n_act * n_pieces;
   int issued = 0;
   auto issue = [&](int m) {
     const int b = m % kCopyBuffers;
     const int off = (m % n_pieces) * piece;
     const uint32_t bytes = static_cast<uint32_t>(min(piece, rb - off));
     mbar_expect_tx(&bars[b], bytes);
-    bulk_load(buf + b * piece, h + static_cast<size_t>(t0 + m / n_pieces) * rb + off, bytes, &bars[b]);
+    bulk_load(buf + b * piece, h + static_cast<size_t>(t0 + act[m / n_pieces]) * rb + off, bytes, &bars[b]);
     ++issued;
   };
   for (int m = 0; m < kCopyLead && m < n; ++m) issue(m);
@@ -345,7 +364,7 @@ __global__ void __launch_bounds__(32) permute_copy_bulk_kernel(const uint8_t* __
       report_status(status, MOE_STATUS_TIMEOUT);
       break;
     }
-    const int tl = m / n_pieces;
+    const int tl = act[m / n_pieces];
     const int off = (m % n_pieces) * piece;
     const uint32_t bytes = static_cast<uint32_t>(min(piece, rb - off));
     for (int j = 0; j < k; ++j) {
@@ -405,56 +424,87 @@ struct Vec<MOE_DTYPE_F32> {
   }
 };
 
+// y[t] from the token's NK kept rows (slot order), one warp: all NK rows of U
+// 16-byte segments per lane are loaded before any is used, so NK * U loads
+// per lane are in flight (about 16 whatever NK is).
+template <int DT, int NK, int U, int K>
+MOE_DEV void combine_rows(const uint4* __restrict__ y_perm, const int (&dst)[K], const float (&g)[K],
+                          uint4* __restrict__ yrow, int vpr, int lane) {
+  using V = Vec<DT>;
+  for (int v0 = 0; v0 < vpr; v0 += 32 * U) {
+    uint4 q[NK][U];
+#pragma unroll
+    for (int j = 0; j < NK; ++j)
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int v = v0 + u * 32 + lane;
+        q[j][u] = v < vpr ? __ldg(y_perm + static_cast<size_t>(dst[j]) * vpr + v) : make_uint4(0, 0, 0, 0);
+      }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      float acc[V::N];
+#pragma unroll
+      for (int i = 0; i < V::N; ++i) acc[i] = 0.f;
+#pragma unroll
+      for (int j = 0; j < NK; ++j) {
+        float f[V::N];
+        V::load(q[j][u], f);
+#pragma unroll
+        for (int i = 0; i < V::N; ++i) acc[i] = fmaf(g[j], f[i], acc[i]);
+      }
+      const int v = v0 + u * 32 + lane;
+      if (v < vpr) yrow[v] = V::store(acc);
+    }
+  }
+}
+
 // One warp per token: y[t] = sum_j gate[t,j] * y_perm[dest_row[t,j]] in fp32,
-// slots in order 0..k-1, dropped slots skipped. All k rows of U segments are
-// loaded before any of them is used, so k*U 16-byte loads per lane are in
-// flight (k*U = 8 for k <= 8).
+// slots in order 0..k-1, dropped slots skipped. The kept slots are listed
+// first (in slot order) and the loads are batched by their number, so a token
+// that kept few of its k slots still has about 16 loads per lane in flight.
 template <int DT, int K>
 __global__ void __launch_bounds__(256) combine_kernel(const uint4* __restrict__ y_perm,
                                                       const int32_t* __restrict__ dest_row,
                                                       const float* __restrict__ gate, uint4* __restrict__ y, int T,
                                                       int vpr) {
-  using V = Vec<DT>;
-  constexpr int U = K >= 8 ? 1 : 8 / K;
   pdl_wait();
   const int lane = threadIdx.x & 31;
   const int nw = gridDim.x * (blockDim.x >> 5);
   for (int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); t < T; t += nw) {
     const int my_dest = lane < K ? dest_row[static_cast<size_t>(t) * K + lane] : -1;
     const float my_gate = lane < K ? gate[static_cast<size_t>(t) * K + lane] : 0.f;
+    const uint32_t kept = __ballot_sync(0xffffffffu, my_dest >= 0);
+    // kept slots in slot order: the j-th set bit of `kept`
     int dst[K];
     float g[K];
+    uint32_t rest = kept;
 #pragma unroll
     for (int j = 0; j < K; ++j) {
-      dst[j] = __shfl_sync(0xffffffffu, my_dest, j);
-      g[j] = __shfl_sync(0xffffffffu, my_gate, j);
+      const int src = rest ? __ffs(rest) - 1 : 0;
+      rest &= rest - 1;
+      dst[j] = __shfl_sync(0xffffffffu, my_dest, src);
+      g[j] = __shfl_sync(0xffffffffu, my_gate, src);
     }
-    for (int v0 = 0; v0 < vpr; v0 += 32 * U) {
-      uint4 q[K][U];
-#pragma unroll
-      for (int j = 0; j < K; ++j)
-#pragma unroll
-        for (int u = 0; u < U; ++u) {
-          const int v = v0 + u * 32 + lane;
-          q[j][u] = (dst[j] >= 0 && v < vpr) ? __ldg(y_perm + static_cast<size_t>(dst[j]) * vpr + v)
-                                             : make_uint4(0, 0, 0, 0);
-        }
-#pragma unroll
-      for (int u = 0; u < U; ++u) {
-        float acc[V::N];
-#pragma unroll
-        for (int i = 0; i < V::N; ++i) acc[i] = 0.f;
-#pragma unroll
-        for (int j = 0; j < K; ++j) {
-          if (dst[j] < 0) continue;
-          float f[V::N];
-          V::load(q[j][u], f);
-#pragma unroll
-          for (int i = 0; i < V::N; ++i) acc[i] = fmaf(g[j], f[i], acc[i]);
-        }
-        const int v = v0 + u * 32 + lane;
-        if (v < vpr) y[static_cast<size_t>(t) * vpr + v] = V::store(acc);
-      }
+    uint4* yrow = y + static_cast<size_t>(t) * vpr;
+    switch (__popc(kept)) {
+      case 0:
+        for (int v = lane; v < vpr; v += 32) yrow[v] = make_uint4(0, 0, 0, 0);
+        break;
+#define MOE_COMBINE_NK(NKK)                                                              \
+  case NKK:                                                                              \
+    if constexpr (NKK <= K) combine_rows<DT, NKK, (16 / NKK > 1 ? 16 / NKK : 1), K>(y_perm, dst, g, yrow, vpr, lane); \
+    break;
+      MOE_COMBINE_NK(1)
+      MOE_COMBINE_NK(2)
+      MOE_COMBINE_NK(3)
+      MOE_COMBINE_NK(4)
+      MOE_COMBINE_NK(5)
+      MOE_COMBINE_NK(6)
+      MOE_COMBINE_NK(7)
+      MOE_COMBINE_NK(8)
+#undef MOE_COMBINE_NK
+      default:
+        break;
     }
   }
 }
@@ -496,7 +546,9 @@ cudaError_t launch_permute(const void* h, size_t row_bytes, const int32_t* idx, 
                            bool padded, bool copy_rows, int32_t* chunk_counts, int32_t* chunk_base, int32_t* routed,
                            int32_t* kept,
                            int32_t* offsets, int32_t* dest_row, int32_t* perm_src, void* x_perm,
-                           bool counts_ready, bool pdl, int32_t* status, cudaStream_t s) {
+                           bool counts_ready, bool pdl, int32_t* status, cudaStream_t s, int32_t* pair_cnt,
+                           int pair_tiles, void* y_zero) {
+  const int y_vpr = static_cast<int>(row_bytes / 16);
   // the first kernel launches as the caller asks; the later ones always as
   // programmatic dependents of the one before
   bool first = pdl;
@@ -515,7 +567,8 @@ cudaError_t launch_permute(const void* h, size_t row_bytes, const int32_t* idx, 
   if (fused) {
     err = launch_kernel(rank_kernel<true>, dim3(n_chunks), dim3(kChunkTokens), 0, s, next(), 1, idx, T, k, E, cap,
                         static_cast<int>(padded), n_chunks, static_cast<const int32_t*>(chunk_counts), static_cast<const int32_t*>(nullptr),
-                        routed, kept, offsets, dest_row, perm_src, status);
+                        routed, kept, offsets, dest_row, perm_src, status, pair_cnt, pair_tiles,
+                        static_cast<uint4*>(y_zero), y_vpr);
   } else {
     err = launch_kernel(scan_kernel, dim3(1), dim3(1024), 0, s, next(), 1, static_cast<const int32_t*>(chunk_counts),
                         chunk_base, n_chunks, E, cap, static_cast<int>(padded), routed, kept, offsets);
@@ -523,7 +576,8 @@ cudaError_t launch_permute(const void* h, size_t row_bytes, const int32_t* idx, 
       err = launch_kernel(rank_kernel<false>, dim3(n_chunks), dim3(kChunkTokens), 0, s, next(), 1, idx, T, k, E, cap,
                           static_cast<int>(padded), n_chunks, static_cast<const int32_t*>(chunk_base), static_cast<const int32_t*>(offsets),
                           static_cast<int32_t*>(nullptr), static_cast<int32_t*>(nullptr),
-                          static_cast<int32_t*>(nullptr), dest_row, perm_src, status);
+                          static_cast<int32_t*>(nullptr), dest_row, perm_src, status, pair_cnt, pair_tiles,
+                          static_cast<uint4*>(y_zero), y_vpr);
   }
   if (err != cudaSuccess) return err;
   if (n_chunks > 0 && copy_rows) {
@@ -550,7 +604,8 @@ cudaError_t launch_permute(const void* h, size_t row_bytes, const int32_t* idx, 
 }
 
 cudaError_t launch_combine(int dtype, const void* y_perm, const int32_t* dest_row, const float* gate, void* y,
-                           int T, int k, int d, bool pdl, cudaStream_t s) {
+                           int T, int k, int d, bool pdl, cudaStream_t s, int32_t* status) {
+  (void)status;  // the combine has no wait that could time out
   if (T == 0) return cudaSuccess;
   const int elem = dtype == MOE_DTYPE_BF16 ? 2 : 4;
   const int vpr = d * elem / 16;

@@ -31,6 +31,8 @@
 // rows are the K range (operands transposed with 64-aligned per-expert
 // columns), stored in fp32. In gather mode GEMM1's producer loads A rows
 // straight from the token matrix through the permutation (tile::gather4).
+#include <atomic>
+
 #include "moe_common.cuh"
 #include "moe_internal.h"
 
@@ -42,7 +44,12 @@ constexpr int kBM = kTileM;       // 128
 constexpr int kBN = kGemmTileN;   // 256
 constexpr int kBK = 64;
 constexpr int kStages = 4;
-constexpr int kGemmThreads = 192;
+// warp 0: TMA producer, warp 1: TMEM allocation and MMA issue, warps 2..9:
+// epilogue, two warps per TMEM lane quadrant, each draining half of a
+// tile's columns (the SwiGLU epilogue is as long as a short-K main loop)
+constexpr int kGemmThreads = 320;
+constexpr int kEpiWarps = 8;
+constexpr int kPairThreads = 192;
 constexpr uint32_t kABytes = kBM * kBK * 2;
 constexpr uint32_t kBBytes = kBN * kBK * 2;
 constexpr uint32_t kStageBytes = kABytes + kBBytes;
@@ -83,6 +90,22 @@ struct GemmArgs {
   __nv_bfloat16* DT;
   const int32_t* col_off;
   int ldt;
+  // Combine fused into the down projection (k <= 2, kEpiStoreCombine): every
+  // row is stored to D (y_perm) as usual; a token with one kept slot gets
+  // y[t] = gate * row written at once; for a token with two kept slots the
+  // epilogue that finishes the second of its rows in this column tile (a
+  // counter per token and column tile decides which) reads both rows back
+  // and writes y[t] in slot order, bit-identical to the separate combine.
+  const int32_t* perm_src;
+  const int32_t* dest_row;
+  const float* gate;
+  int32_t* pair_cnt;  // [T][n_tiles][2 column halves], zeroed by the rank kernel of the same call
+  __nv_bfloat16* Y;
+  int k;
+  // Testing hook (moe_debug_stall_next_gemms): the MMA issuer first waits on a
+  // barrier that nothing signals, so its bounded wait runs out and the
+  // kernel takes its timeout path.
+  int stall;
 };
 
 // Epilogues and tile groupings of grouped_gemm_kernel.
@@ -90,6 +113,7 @@ constexpr int kEpiStore = 0;       // D (bf16) = accumulator
 constexpr int kEpiSwiGLU = 1;      // D (bf16) = silu(gate) * up, half-width
 constexpr int kEpiSwiGLUBwd = 2;   // D (bf16) = [dgate | dup] from gate, up and aux = dL/dh_mid
 constexpr int kEpiStoreF32 = 3;    // D32 (fp32) = accumulator
+constexpr int kEpiStoreCombine = 4;  // D (bf16) = accumulator, and the combine into Y for k <= 2
 constexpr int kGroupRows = 0;      // groups of rows (experts' token rows), same K for all
 constexpr int kGroupReduce = 1;    // groups along K (experts' token rows are the reduction)
 constexpr int kReduceBand = 16;    // row tiles per band in the reduction-grouped tile walk
@@ -147,7 +171,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&tfull[i], 1);
-      mbar_init(&tempty[i], 4);
+      mbar_init(&tempty[i], kEpiWarps);
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -274,6 +298,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       uint32_t phase = 0;
       int consumed = 0, local = 0;
       bool stop = false;
+      if (a.stall && !mbar_wait(drain, 0, abort_flag)) {  // nothing arrives on `drain` before the end
+        *abort_flag = 1;
+        stop = true;
+      }
       for (long long tile = blockIdx.x; tile < total && !stop; tile += gridDim.x, ++local) {
         const int acc = local & 1;
         const uint32_t acc_phase = (local >> 1) & 1;
@@ -313,7 +341,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
   } else {
     // ---------------------------------------------------------------- epilogue
-    const int q = warp & 3;  // TMEM lane quadrant this warp may read
+    const int q = warp & 3;            // TMEM lane quadrant this warp may read
+    const int half = (warp - 2) >> 2;  // which half of the tile's columns it drains
     const int row = q * 32 + lane;
     int local = 0;
     for (long long tile = blockIdx.x; tile < total; tile += gridDim.x, ++local) {
@@ -333,7 +362,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         float* out = a.D32 + (static_cast<size_t>(e) * a.m_tiles * kBM + m * kBM + row) * a.ldd + n * kBN;
         const bool empty_k = kb1 == kb0;
 #pragma unroll 1
-        for (int c = 0; c < kBN; c += 32) {
+        for (int c = half * (kBN / 2); c < (half + 1) * (kBN / 2); c += 32) {
           if (n * kBN + c >= a.out_cols) break;
           uint32_t v[32];
           if (!empty_k) {
@@ -366,7 +395,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         const int pcol = a.DT != nullptr ? a.col_off[e] + m * kBM + row : 0;
         const bool twrite = a.DT != nullptr && pcol < a.col_off[e + 1];
 #pragma unroll 1
-        for (int c = 0; c < kBN / 2; c += 32) {
+        for (int c = half * (kBN / 4); c < (half + 1) * (kBN / 4); c += 32) {
           uint32_t g[32], u[32];
           tmem_ld32(tbase + c, g);
           tmem_ld32(tbase + kBN / 2 + c, u);
@@ -421,7 +450,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         // columns [0,128) of the tile are gate, [128,256) the matching up
         __nv_bfloat16* out = a.D + grow * a.ldd + n * (kBN / 2);
 #pragma unroll 1
-        for (int c = 0; c < kBN / 2; c += 32) {
+        for (int c = half * (kBN / 4); c < (half + 1) * (kBN / 4); c += 32) {
           uint32_t g[32], u[32];
           tmem_ld32(tbase + c, g);
           tmem_ld32(tbase + kBN / 2 + c, u);
@@ -439,10 +468,88 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             for (int i = 0; i < 4; ++i) dst[i] = make_uint4(p[4 * i], p[4 * i + 1], p[4 * i + 2], p[4 * i + 3]);
           }
         }
+      } else if constexpr (kEpi == kEpiStoreCombine) {
+        __nv_bfloat16* out = a.D + grow * a.ldd + n * kBN;
+        // this row's token, its slot, its gate and the token's other kept row
+        int t = -1, slot = 0, other = -1;
+        float g_own = 0.f, g_other = 0.f;
+        if (valid) {
+          t = a.perm_src[grow];
+          if (t >= 0) {
+            slot = a.dest_row[static_cast<size_t>(t) * a.k] == static_cast<int>(grow) ? 0 : 1;
+            g_own = a.gate[static_cast<size_t>(t) * a.k + slot];
+            if (a.k == 2) {
+              other = a.dest_row[static_cast<size_t>(t) * 2 + (1 - slot)];
+              if (other >= 0) g_other = a.gate[static_cast<size_t>(t) * 2 + (1 - slot)];
+            }
+          }
+        }
+        __nv_bfloat16* yrow = a.Y + static_cast<size_t>(t < 0 ? 0 : t) * a.ldd + n * kBN;
+#pragma unroll 1
+        for (int c = half * (kBN / 2); c < (half + 1) * (kBN / 2); c += 32) {
+          if (n * kBN + c >= a.out_cols) break;
+          uint32_t v[32];
+          tmem_ld32(tbase + c, v);
+          tmem_ld_wait();
+          if (valid) {
+            uint32_t p[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) p[i] = pack_bf16x2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
+            uint4* dst = reinterpret_cast<uint4*>(out + c);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) dst[i] = make_uint4(p[4 * i], p[4 * i + 1], p[4 * i + 2], p[4 * i + 3]);
+            if (t >= 0 && other < 0) {
+              // the token's only kept slot: y = gate * row (the row rounded to bf16 first)
+              uint32_t yq[16];
+#pragma unroll
+              for (int i = 0; i < 16; ++i) {
+                const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&p[i]));
+                yq[i] = pack_bf16x2(fmaf(g_own, f.x, 0.f), fmaf(g_own, f.y, 0.f));
+              }
+              uint4* ydst = reinterpret_cast<uint4*>(yrow + c);
+#pragma unroll
+              for (int i = 0; i < 4; ++i)
+                ydst[i] = make_uint4(yq[4 * i], yq[4 * i + 1], yq[4 * i + 2], yq[4 * i + 3]);
+            }
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&tempty[acc]);
+        if (t >= 0 && other >= 0) {
+          // both rows of this column tile stored: the later of the two adds them
+          __threadfence();
+          const int prev = atomicAdd(a.pair_cnt + (static_cast<size_t>(t) * a.n_tiles + n) * 2 + half, 1);
+          if (prev == 1) {
+            __threadfence();
+            const size_t r0 = slot == 0 ? grow : static_cast<size_t>(other);
+            const size_t r1 = slot == 0 ? static_cast<size_t>(other) : grow;
+            const float g0 = slot == 0 ? g_own : g_other, g1 = slot == 0 ? g_other : g_own;
+            const int c0 = half * (kBN / 2);
+            const uint4* s0 = reinterpret_cast<const uint4*>(a.D + r0 * a.ldd + n * kBN + c0);
+            const uint4* s1 = reinterpret_cast<const uint4*>(a.D + r1 * a.ldd + n * kBN + c0);
+            uint4* ydst = reinterpret_cast<uint4*>(yrow + c0);
+            const int vcols = max(0, min(kBN / 2, a.out_cols - n * kBN - c0)) / 8;
+#pragma unroll 4
+            for (int v8 = 0; v8 < vcols; ++v8) {
+              const uint4 q0 = __ldcg(s0 + v8), q1 = __ldcg(s1 + v8);
+              const __nv_bfloat162* h0 = reinterpret_cast<const __nv_bfloat162*>(&q0);
+              const __nv_bfloat162* h1 = reinterpret_cast<const __nv_bfloat162*>(&q1);
+              uint32_t o[4];
+#pragma unroll
+              for (int i = 0; i < 4; ++i) {
+                const float2 f0 = __bfloat1622float2(h0[i]), f1 = __bfloat1622float2(h1[i]);
+                o[i] = pack_bf16x2(fmaf(g1, f1.x, fmaf(g0, f0.x, 0.f)), fmaf(g1, f1.y, fmaf(g0, f0.y, 0.f)));
+              }
+              ydst[v8] = make_uint4(o[0], o[1], o[2], o[3]);
+            }
+          }
+        }
+        continue;
       } else {
         __nv_bfloat16* out = a.D + grow * a.ldd + n * kBN;
 #pragma unroll 1
-        for (int c = 0; c < kBN; c += 32) {
+        for (int c = half * (kBN / 2); c < (half + 1) * (kBN / 2); c += 32) {
           if (n * kBN + c >= a.out_cols) break;
           uint32_t v[32];
           tmem_ld32(tbase + c, v);
@@ -501,7 +608,7 @@ constexpr size_t pair_smem_bytes() {
 }
 
 template <bool kSwiGLU>
-__global__ void __launch_bounds__(kGemmThreads, 1)
+__global__ void __launch_bounds__(kPairThreads, 1)
     grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
                              const GemmArgs a) {
   extern __shared__ uint8_t smem_raw[];
@@ -870,9 +977,15 @@ int band_rows(int tile_rows, int K, int lo, int hi) {
 
 namespace {
 
+std::atomic<int> g_stall_gemms{0};
+
 template <int kEpi, int kMode>
-cudaError_t launch_gemm_inst(const CUtensorMap& tm_a, const CUtensorMap& tm_b, const GemmArgs& a, bool pdl,
+cudaError_t launch_gemm_inst(const CUtensorMap& tm_a, const CUtensorMap& tm_b, GemmArgs a, bool pdl,
                              cudaStream_t s) {
+  int left = g_stall_gemms.load();
+  while (left > 0 && !g_stall_gemms.compare_exchange_weak(left, left - 1)) {
+  }
+  a.stall = left > 0 ? 1 : 0;
   const size_t smem = gemm_smem_bytes();
   cudaError_t err = cudaFuncSetAttribute(grouped_gemm_kernel<kEpi, kMode>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
@@ -893,6 +1006,23 @@ cudaError_t launch_grouped_gemm_tc(const CUtensorMap& tm_a, const CUtensorMap& t
              band_rows(kBM, K, 8, 32), gather_rows, nullptr, 0, nullptr, 0, nullptr, nullptr, 0};
   return swiglu ? launch_gemm_inst<kEpiSwiGLU, kGroupRows>(tm_a, tm_b, a, pdl, s)
                 : launch_gemm_inst<kEpiStore, kGroupRows>(tm_a, tm_b, a, pdl, s);
+}
+
+void debug_stall_next_gemms(int n) { g_stall_gemms.store(n > 0 ? n : 0); }
+
+cudaError_t launch_grouped_gemm_combine(const CUtensorMap& tm_a, const CUtensorMap& tm_b, const int32_t* offsets, int E,
+                                        int K, int d, void* y_perm, const int32_t* perm_src, const int32_t* dest_row,
+                                        const float* gate, int32_t* pair_cnt, void* y, int k, int32_t* status, bool pdl,
+                                        cudaStream_t s) {
+  GemmArgs a{offsets, E, K, d, (d + kBN - 1) / kBN, d, d, static_cast<__nv_bfloat16*>(y_perm), status,
+             band_rows(kBM, K, 8, 32), nullptr, nullptr, 0, nullptr, 0, nullptr, nullptr, 0};
+  a.perm_src = perm_src;
+  a.dest_row = dest_row;
+  a.gate = gate;
+  a.pair_cnt = pair_cnt;
+  a.Y = static_cast<__nv_bfloat16*>(y);
+  a.k = k;
+  return launch_gemm_inst<kEpiStoreCombine, kGroupRows>(tm_a, tm_b, a, pdl, s);
 }
 
 cudaError_t launch_grouped_gemm_swiglu_bwd(const CUtensorMap& tm_a, const CUtensorMap& tm_b, const int32_t* offsets,
@@ -924,13 +1054,13 @@ cudaError_t launch_grouped_gemm_pair(const CUtensorMap& tm_a, const CUtensorMap&
     err = cudaFuncSetAttribute(grouped_gemm_pair_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                static_cast<int>(smem));
     if (err != cudaSuccess) return err;
-    err = launch_kernel(grouped_gemm_pair_kernel<true>, dim3(grid), dim3(kGemmThreads), smem, s, pdl, 2, tm_a, tm_b,
+    err = launch_kernel(grouped_gemm_pair_kernel<true>, dim3(grid), dim3(kPairThreads), smem, s, pdl, 2, tm_a, tm_b,
                         a);
   } else {
     err = cudaFuncSetAttribute(grouped_gemm_pair_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                static_cast<int>(smem));
     if (err != cudaSuccess) return err;
-    err = launch_kernel(grouped_gemm_pair_kernel<false>, dim3(grid), dim3(kGemmThreads), smem, s, pdl, 2, tm_a, tm_b,
+    err = launch_kernel(grouped_gemm_pair_kernel<false>, dim3(grid), dim3(kPairThreads), smem, s, pdl, 2, tm_a, tm_b,
                         a);
   }
   if (err != cudaSuccess) return err;

@@ -138,6 +138,10 @@ MOE_DEV void bulk_store(void* gdst, const void* smem_src, uint32_t bytes) {
 
 MOE_DEV void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 
+// Orders this thread's earlier generic-proxy accesses of shared memory before
+// its later async-proxy (bulk copy, TMA) accesses.
+MOE_DEV void fence_proxy_async_shared() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
 // Wait until at most N committed bulk groups still read shared memory.
 template <int N>
 MOE_DEV void bulk_wait_read() {

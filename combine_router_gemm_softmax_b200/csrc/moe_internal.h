@@ -37,12 +37,16 @@ cudaError_t launch_router_f32(const float* h, const float* w, int T, int d, int 
 // rows past its kept count are zero-filled and their perm_src set to -1.
 // copy_rows: false skips the x_perm row copy (the grouped GEMM gathers the
 // rows itself); everything else is still written.
+// pair_cnt / pair_tiles / y_zero (the combine fused into the down projection;
+// NULL / 0 / NULL otherwise): the rank kernel zeroes pair_cnt [T][pair_tiles]
+// and the y rows (row_bytes each) of tokens that keep no slot.
 cudaError_t launch_permute(const void* h, size_t row_bytes, const int32_t* idx, int T, int k, int E, int cap,
                            bool padded, bool copy_rows, int32_t* chunk_counts, int32_t* chunk_base, int32_t* routed, int32_t* kept,
                            int32_t* offsets, int32_t* dest_row, int32_t* perm_src, void* x_perm,
-                           bool counts_ready, bool pdl, int32_t* status, cudaStream_t s);
+                           bool counts_ready, bool pdl, int32_t* status, cudaStream_t s, int32_t* pair_cnt = nullptr,
+                           int pair_tiles = 0, void* y_zero = nullptr);
 cudaError_t launch_combine(int dtype, const void* y_perm, const int32_t* dest_row, const float* gate, void* y,
-                           int T, int k, int d, bool pdl, cudaStream_t s);
+                           int T, int k, int d, bool pdl, cudaStream_t s, int32_t* status = nullptr);
 
 // grouped_ffn.cu
 // Launch flags `pdl` (here and in launch_permute / launch_combine): launch as
@@ -54,6 +58,18 @@ cudaError_t launch_grouped_gemm_tc(const CUtensorMap& tm_a, const CUtensorMap& t
                                    const int32_t* offsets, int E, int K, int n_per_expert, int n_tiles,
                                    int out_cols, int ldd, void* D, const int32_t* gather_rows, int32_t* status,
                                    bool pdl, cudaStream_t s);
+// The down projection with the combine fused into its epilogue (k <= 2): y_perm
+// rows as launch_grouped_gemm_tc, and y [T, d] = sum over each token's kept
+// slots, in slot order, of gate * bf16 row (bit-identical to launch_combine).
+// pair_cnt [T][2 * ceil(d/256)] must be zero and the y rows of tokens that keep
+// no slot written beforehand (launch_permute does both).
+cudaError_t launch_grouped_gemm_combine(const CUtensorMap& tm_a, const CUtensorMap& tm_b, const int32_t* offsets, int E,
+                                        int K, int d, void* y_perm, const int32_t* perm_src, const int32_t* dest_row,
+                                        const float* gate, int32_t* pair_cnt, void* y, int k, int32_t* status, bool pdl,
+                                        cudaStream_t s);
+// Testing hook: the next n launches of the bf16 grouped GEMM kernel stall their
+// MMA issuer on a barrier nothing signals until the bounded wait gives up.
+void debug_stall_next_gemms(int n);
 // GEMM1 recomputed with the SwiGLU backward in its epilogue: from the gate and
 // up pre-activations of each row (x_perm rows against w13) and dh_mid [rows, F]
 // it writes dgu [rows, 2F] = [dgate | dup] in w13's interleaved column order,
@@ -78,6 +94,29 @@ cudaError_t launch_scale_rows(int dtype, int kind, const void* x_perm, const int
                               int rows_max, int d, int E, cudaStream_t s);
 cudaError_t launch_pack_w13(const void* w_gate, const void* w_up, void* w13, int E, int F, size_t row_bytes,
                             cudaStream_t s);
+
+// grouped_ffn_mx.cu (MXFP8: E4M3 elements, one E8M0 scale per 32 along the
+// reduction axis; scales in 512-byte atoms per 128 rows x 128 columns)
+// Quantises rows of a bf16 matrix. offsets != NULL: grouped mode, the output
+// rows are the padded layout (every expert's rows start on a 128-row
+// boundary, rows past its count are zeros) and `rows` only bounds the grid.
+// sf_row_blocks: 128-row blocks per 128-column slice of the atom array.
+cudaError_t launch_mx_quantize(const void* src, int rows, int cols, const int32_t* offsets, int E, void* q, void* sf,
+                               int sf_row_blocks, uint32_t* counts, int32_t* status, bool pdl, cudaStream_t s);
+// The layer's dispatch fused with the quantisation: token rows of h [T, d]
+// straight to the padded quantised layout (every kept slot's destination from
+// dest_row, idx and offsets), padding rows zeroed.
+cudaError_t launch_mx_dispatch(const void* h, int T, int d, int k, const int32_t* idx, const int32_t* dest_row,
+                               const int32_t* offsets, int E, void* q, void* sf, int sf_row_blocks, uint32_t* counts,
+                               int32_t* status, bool pdl, cudaStream_t s);
+// Block-scaled grouped GEMM over the padded groups. swiglu_quant: GEMM1, D is
+// the quantised silu(gate) * up in the padded layout (q_out, sf_out with
+// ra_blocks row blocks, ldq = F); else GEMM2, bf16 D in the compact layout.
+// sfb: the B scale atoms with rb_blocks + 1 row blocks per slice.
+cudaError_t launch_grouped_gemm_mx(const CUtensorMap& tm_a, const CUtensorMap& tm_b, bool swiglu_quant,
+                                   const int32_t* offsets, int E, int K, int n_per_expert, int out_cols,
+                                   const void* sfa, int ra_blocks, const void* sfb, void* q_out, void* sf_out, int ldq,
+                                   uint32_t* counts, void* D, int ldd, int32_t* status, bool pdl, cudaStream_t s);
 
 // backward.cu
 cudaError_t launch_combine_bwd(const void* dy, const void* y_perm, const int32_t* dest_row, const float* gate,

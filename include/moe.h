@@ -68,6 +68,11 @@ extern "C" {
 #define MOE_STATUS_NAN_LOGIT 1  /* a router logit was NaN (treated as -inf) */
 #define MOE_STATUS_BAD_ROUTE 2  /* an index out of [0,E) or repeated within a token (slot dropped) */
 #define MOE_STATUS_TIMEOUT   4  /* a bounded on-chip wait gave up (output invalid) */
+/* MXFP8 precision only, informational (the output is valid): */
+#define MOE_STATUS_MX_SATURATED 8   /* an element was clamped to +-448 when quantised; the OCP scale
+                                       rule does this whenever a block's largest magnitude has a
+                                       mantissa above 1.75, so it is expected on most calls */
+#define MOE_STATUS_MX_UNDERFLOW 16  /* a non-zero element was quantised to 0 */
 
 #define MOE_DTYPE_BF16 0
 #define MOE_DTYPE_F32  1
@@ -113,6 +118,42 @@ extern "C" {
 #define MOE_DISPATCH_COPY   1
 #define MOE_DISPATCH_GATHER 2
 
+/* Arithmetic of the grouped expert GEMMs (moe_grouped_ffn, moe_layer_forward).
+ * BF16: bf16 operands (the default).
+ * MXFP8: block-scaled 8-bit operands, the MXFP8 variant of "Dropless MoE Is a
+ * Runtime Problem as Much as a Model Design" (its MXFP8 paragraph), with the
+ * format of the OCP Microscaling specification: every 32 consecutive
+ * elements along the reduction axis of a row share one scale 2^E (an E8M0
+ * byte E + 127), E = floor(log2 max|v|) - 8 clamped to [-127, 127], and every
+ * element is FP8 E4M3 of v / 2^E, rounded to nearest even and clamped at
+ * +-448. The permuted token rows are quantised along d, the weights along
+ * their reduction axis (moe_pack_weights_mxfp8), and silu(gate) * up along F
+ * in GEMM1's epilogue before GEMM2; accumulation is fp32 and y_perm, y stay
+ * bf16. Routing, dispatch and combine are unchanged. Needs bf16 storage,
+ * SwiGLU experts, single-CTA tiles and the COPY dispatch; the backward is
+ * bf16 only. In this precision the w13_packed and w_down arguments of
+ * moe_grouped_ffn and moe_layer_forward are the two blobs written by
+ * moe_pack_weights_mxfp8, and the first 16 bytes of their workspace receive
+ * four uint32 counters of the call: token-row elements saturated and
+ * underflowed (once per permuted row), then h_mid elements saturated and
+ * underflowed. */
+#define MOE_PRECISION_BF16  0
+#define MOE_PRECISION_MXFP8 1
+
+/* Where moe_layer_forward applies the combine. SEPARATE: its own kernel reads
+ * y_perm back and writes y. FUSED (k <= 2 only): the down projection's
+ * epilogue writes y itself: a token with one kept slot gets gate * row at
+ * once, and for a token with two the epilogue that stores the later of its
+ * two rows of a column tile (a per-token counter decides) reads both back
+ * from y_perm and writes y in slot order. y is bit-identical either way, and
+ * y_perm is still written (the backward reads it). Needs bf16 SwiGLU
+ * experts, single-CTA tiles and bf16 precision. AUTO is SEPARATE: on B200
+ * the fused form measured 1-3% slower per layer (its epilogue re-reads both
+ * rows of a token while the GEMM runs), so it is opt-in. */
+#define MOE_COMBINE_AUTO     0
+#define MOE_COMBINE_SEPARATE 1
+#define MOE_COMBINE_FUSED    2
+
 #define MOE_OP_ROUTE       0
 #define MOE_OP_PERMUTE     1
 #define MOE_OP_GROUPED_FFN 2
@@ -135,6 +176,8 @@ typedef struct moe_config {
   int32_t gemm_tiles;   /* MOE_GEMM_TILES_*: tile shape of the bf16 grouped GEMMs */
   int32_t layout;       /* MOE_LAYOUT_*: row layout of the permuted buffers (P rows) */
   int32_t dispatch;     /* MOE_DISPATCH_*: x_perm row copy or gather inside GEMM1 (layer only) */
+  int32_t precision;    /* MOE_PRECISION_*: operands of the grouped expert GEMMs */
+  int32_t combine;      /* MOE_COMBINE_*: separate combine kernel or fused into the down projection (layer only) */
 } moe_config;
 
 typedef void* moe_stream_t; /* cudaStream_t */
@@ -282,6 +325,47 @@ MOE_API int32_t moe_layer_backward(const moe_config* cfg, const void* h, const v
                                    const void* dy, void* dh, float* dw_router, float* dbias, float* dw13,
                                    float* dw_down, const void* fwd_workspace, size_t fwd_ws_bytes,
                                    void* workspace, size_t ws_bytes, int32_t* status_dev, moe_stream_t stream);
+
+/* moe_mxfp8_quantize -- MXFP8 quantisation of a bf16 matrix along its rows
+ * (the format described at MOE_PRECISION_MXFP8).
+ * x [rows, cols] bf16, cols a multiple of 128. q [rows, cols]: one E4M3 byte
+ * per element. sf: the E8M0 scale bytes in the order the block-scaled tensor
+ * cores read them: for every 128-row block R and 128-column slice kt one
+ * 512-byte atom at (kt * ceil(rows/128) + R) * 512, in which the scale of row
+ * r (within the block) and 32-column block j (within the slice) is byte
+ * (r % 32) * 16 + (r / 32) * 4 + j; (cols/128) * ceil(rows/128) * 512 bytes.
+ * Bytes of the last atom row that belong to rows past `rows` are left
+ * untouched. counts [2] uint32 (may be NULL): saturated and underflowed
+ * elements are ADDED to counts[0] and counts[1]. status_dev as elsewhere
+ * (MOE_STATUS_MX_* bits). */
+MOE_API int32_t moe_mxfp8_quantize(const void* x, int32_t rows, int32_t cols, void* q, void* sf, uint32_t* counts,
+                                   int32_t* status_dev, moe_stream_t stream);
+
+/* Bytes of the MXFP8 weight blobs for cfg: which = 0 for w13 (GEMM1's B,
+ * [E*2F, d]), 1 for w_down (GEMM2's B, [E*d, F]). A blob holds the E4M3
+ * bytes [rows, cols], then at the next 256-byte boundary the scale atoms of
+ * moe_mxfp8_quantize's layout with one extra (zero) 128-row block per
+ * 128-column slice: (cols/128) * (rows/128 + 1) * 512 bytes. 0 on an
+ * invalid cfg. */
+MOE_API size_t moe_mxfp8_weights_size(const moe_config* cfg, int32_t which);
+
+/* moe_pack_weights_mxfp8 -- quantise the expert weights once for
+ * MOE_PRECISION_MXFP8: w13_packed [E, 2F, d] (from moe_pack_weights) along d
+ * into w13_mx, and w_down [E, d, F] along F into w_down_mx (blobs sized by
+ * moe_mxfp8_weights_size). counts [2] (may be NULL): saturated and
+ * underflowed weight elements are added. bf16, SwiGLU experts. */
+MOE_API int32_t moe_pack_weights_mxfp8(const moe_config* cfg, const void* w13_packed, const void* w_down,
+                                       void* w13_mx, void* w_down_mx, uint32_t* counts, moe_stream_t stream);
+
+/* moe_debug_stall_next_gemms -- testing hook for the timeout path. The pages
+ * have no counterpart. The next n launches (process-wide, any stream) of the
+ * bf16 grouped GEMM kernel make their MMA-issuing thread first wait on a
+ * barrier that nothing signals. That wait gives up after the library's
+ * on-chip limit (2 s), the kernel unwinds as after any timeout (no MMA was
+ * issued; the operand loads already issued are waited for and TMEM is freed)
+ * and MOE_STATUS_TIMEOUT is OR-ed into the status word; that call's outputs
+ * are invalid and the context stays usable. n = 0 cancels. */
+MOE_API int32_t moe_debug_stall_next_gemms(int32_t n);
 
 /* moe_permute_static_scratch -- moe_permute for callers that cannot allocate.
  * The paper has no counterpart for this entry point. It is for code that has

@@ -1,0 +1,197 @@
+"""MXFP8 grouped expert FFN against the MXFP8 oracle (GPU, through the C ABI).
+
+* moe_mxfp8_quantize is bit-exact: every E4M3 byte, every scale byte (read
+  back from the tensor-core atom layout) and the saturated / underflowed
+  counts equal oracle.mxfp8.mx_quantize on the same bf16 inputs (both sides
+  scale by an exact power of two and round to nearest even).
+* moe_pack_weights_mxfp8 writes exactly the oracle's quantised weights.
+* moe_grouped_ffn and moe_layer_forward in MXFP8 precision match the oracle's
+  MXFP8 expert (x and weights quantised along their reduction axis, the
+  SwiGLU product quantised along F) within the bf16 output bar (2e-2 of each
+  row's largest magnitude). The kernel accumulates in fp32 where the oracle
+  is exact, so an element of h_mid next to an E4M3 rounding boundary may
+  round the other way; one such flip moves an output row by about
+  ulp/sqrt(F) of its magnitude, far inside the bar. The same outputs differ
+  from the exact bf16 expert by the format's own rounding (several per cent),
+  which shows the path really computes in MXFP8.
+"""
+import numpy as np
+import pytest
+import torch
+
+import combine_router_gemm_softmax_b200 as M
+import oracle as O
+from oracle import cases
+from oracle import check as C
+from oracle import mxfp8 as X
+
+from gpu_cases import DEV, DeviceCase, np64, np_, parity_case, workload
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _device():
+    assert torch.cuda.is_available(), "these tests need a CUDA device"
+    torch.cuda.set_device(0)
+    M.lib()
+
+
+def decode_scales(sf, rows, cols, row_blocks):
+    """Scale exponents [rows, cols/32] from the atom layout: byte
+    (r % 32) * 16 + (r / 32) * 4 + j of atom (kt, R) is row 128 R + r, block
+    4 kt + j."""
+    a = np.asarray(sf)[: (cols // 128) * row_blocks * 512].reshape(cols // 128, row_blocks, 32, 4, 4)
+    e = a.transpose(1, 3, 2, 0, 4).reshape(row_blocks * 128, cols // 32)
+    return e[:rows].astype(np.int64) - 127
+
+
+def e4m3_values(q):
+    return q.view(torch.float8_e4m3fn).double().cpu().numpy()
+
+
+def test_quantize_bit_exact():
+    r = np.random.default_rng(0)
+    rows, cols = 300, 512
+    x = r.standard_normal((rows, cols)) * np.exp2(r.integers(-20, 20, size=(rows, 1)))
+    x[5] = 0.0                                             # all-zero blocks
+    x[7, :64] = 1e-30                                      # underflow to zero
+    x[9, ::32] = 1.99 * np.exp2(r.integers(-3, 3, size=16))  # block maxima that saturate
+    xb = torch.from_numpy(x).to(torch.bfloat16)
+    counts = torch.zeros(2, dtype=torch.int32, device=DEV)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    q, sf = M.moe_mxfp8_quantize(xb.to(DEV), counts=counts, status=status)
+    torch.cuda.synchronize()
+    ref = X.mx_quantize(xb.double().numpy())
+    assert np.array_equal(e4m3_values(q), ref["q"])
+    assert np.array_equal(decode_scales(np_(sf), rows, cols, (rows + 127) // 128), ref["exp"])
+    assert np_(counts).tolist() == [ref["saturated"], ref["underflow"]]
+    assert ref["saturated"] > 0 and ref["underflow"] > 0
+    assert int(status.item()) == M.MOE_STATUS_MX_SATURATED | M.MOE_STATUS_MX_UNDERFLOW
+
+
+def test_pack_weights_mxfp8_is_the_oracle_quantisation():
+    dc = DeviceCase(parity_case("small_ragged")[0])
+    cfg = M.config(dc.wl.T, dc.wl.d, dc.wl.E, dc.wl.k, dc.wl.F, precision="mxfp8")
+    w13_mx, wd_mx = M.moe_pack_weights_mxfp8(cfg, dc.w13, dc.w_down)
+    torch.cuda.synchronize()
+    for blob, w in ((w13_mx, dc.w13), (wd_mx, dc.w_down)):
+        E, R, K = w.shape
+        rows = E * R
+        qbytes = (rows * K + 255) // 256 * 256
+        ref = X.mx_quantize(w.reshape(rows, K).double().cpu().numpy())
+        assert np.array_equal(e4m3_values(blob[:rows * K].view(rows, K)), ref["q"])
+        sf = np_(blob[qbytes:])
+        assert np.array_equal(decode_scales(sf, rows, K, rows // 128 + 1), ref["exp"])
+
+
+def _mx_weights(inp):
+    def f(e):
+        return cases.as64(inp.w_gate[e]), cases.as64(inp.w_up[e]), cases.as64(inp.w_down[e])
+    return f
+
+
+@pytest.mark.parametrize("name", ["small_ragged", "small_skewed", "small_many", "small_skewed_padded",
+                                  "mixtral_scaled"])
+def test_grouped_ffn_mxfp8_matches_oracle(name):
+    inp, ref = parity_case(name)
+    dc = DeviceCase(inp)
+    wl = dc.wl
+    cfg = M.config(wl.T, wl.d, wl.E, wl.k, wl.F, capacity=wl.capacity, layout=wl.layout, precision="mxfp8")
+    P = M.perm_rows(cfg)
+    padded = wl.layout == "padded"
+    meta = O.dispatch_meta_padded(ref["idx"], wl.E, wl.capacity) if padded else ref
+    x_perm = torch.zeros((max(P, 1), wl.d), dtype=torch.bfloat16)
+    kept = np.nonzero(meta["perm_src"] >= 0)[0]
+    x_perm[kept] = inp.h[meta["perm_src"][kept]]
+    offsets = torch.from_numpy(meta["offsets"].astype(np.int32))
+    w13_mx, wd_mx = M.moe_pack_weights_mxfp8(cfg, dc.w13, dc.w_down)
+    ws = M.workspace(cfg, M.MOE_OP_GROUPED_FFN, DEV)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    y_perm = M.moe_grouped_ffn(cfg, x_perm.to(DEV), offsets.to(DEV), w13_mx, wd_mx, ws=ws, status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) & M.MOE_STATUS_TIMEOUT == 0
+    n = int(meta["offsets"][-1])
+    rows = np.linspace(0, n - 1, min(n, 1024)).astype(np.int64)
+    xs = cases.as64(x_perm)
+    wf = _mx_weights(inp)
+    want = np.zeros((len(rows), wl.d))
+    exact = np.zeros((len(rows), wl.d))
+    for e in range(wl.E):
+        sel = np.nonzero((rows >= meta["offsets"][e]) & (rows < meta["offsets"][e + 1]))[0]
+        if sel.size:
+            want[sel], _, _ = X.mx_swiglu_expert(xs[rows[sel]], *wf(e))
+            exact[sel] = O.swiglu_expert(xs[rows[sel]], *wf(e))
+    live = np.abs(want).max(axis=1) > 0                        # padding rows of the padded layout are zero
+    got = np64(y_perm[torch.from_numpy(rows).to(DEV)])
+    assert C.row_rel_err(got[live], want[live]) <= C.TOL_BF16
+    assert not got[~live].any()
+    # MXFP8, not bf16: the format's rounding (E4M3 keeps 3 mantissa bits) puts
+    # the result several per cent away from the exact expert, where the bf16
+    # path stays within a few tenths of a per cent
+    dev_exact = C.row_rel_err(got[live], exact[live])
+    assert 0.01 < dev_exact < 0.25, dev_exact
+    cnt = M.mx_counters(ws)
+    assert cnt[2] > 0                                          # h_mid block maxima saturate under the OCP rule
+
+
+# the compact layouts go through the fused dispatch (token rows quantised
+# straight from h); the padded capacity layout through x_perm and the row
+# quantiser
+MX_LAYER_CASES = ["small_ragged", "small_skewed", "small_skewed_capacity", "small_skewed_padded", "small_many",
+                  "mixtral_scaled", "skewed_capacity", "many_small", "mixtral_8x7b"]
+MX_FULL_ORACLE = {"small_ragged", "small_skewed", "small_skewed_capacity", "small_skewed_padded", "small_many"}
+
+
+@pytest.mark.parametrize("name", MX_LAYER_CASES)
+def test_layer_mxfp8_matches_oracle(name):
+    inp, ref = parity_case(name)
+    dc = DeviceCase(inp)
+    wl = dc.wl
+    cfg = M.config(wl.T, wl.d, wl.E, wl.k, wl.F, capacity=wl.capacity, layout=wl.layout, precision="mxfp8")
+    w13_mx, wd_mx = M.moe_pack_weights_mxfp8(cfg, dc.w13, dc.w_down)
+    ws = M.workspace(cfg, M.MOE_OP_LAYER, DEV)
+    idx = torch.empty((wl.T, wl.k), dtype=torch.int32, device=DEV)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    y = M.moe_layer_forward(cfg, dc.h, dc.w_router, dc.bias, w13_mx, wd_mx, topk_idx=idx, ws=ws, status=status)
+    torch.cuda.synchronize()
+    assert np.array_equal(np_(idx), ref["idx"])
+    assert int(status.item()) & (M.MOE_STATUS_TIMEOUT | M.MOE_STATUS_BAD_ROUTE | M.MOE_STATUS_NAN_LOGIT) == 0
+    tokens = None if name in MX_FULL_ORACLE else cases.sample_tokens(ref["idx"], ref["dest_row"], 256)
+    want = X.mx_combine(cases.as64(inp.h), ref["idx"], ref["gate"], ref["dest_row"], _mx_weights(inp), tokens)
+    got = np64(y) if tokens is None else np64(y[torch.from_numpy(tokens).to(DEV)])
+    assert C.row_rel_err(got, want) <= C.TOL_BF16
+    cnt = M.mx_counters(ws)
+    assert cnt[2] > 0
+    assert bool(int(status.item()) & M.MOE_STATUS_MX_SATURATED)
+
+
+def test_layer_mxfp8_is_deterministic_and_counters_reset():
+    inp, _ = parity_case("small_skewed")
+    dc = DeviceCase(inp)
+    wl = dc.wl
+    cfg = M.config(wl.T, wl.d, wl.E, wl.k, wl.F, precision="mxfp8")
+    w13_mx, wd_mx = M.moe_pack_weights_mxfp8(cfg, dc.w13, dc.w_down)
+    ws = M.workspace(cfg, M.MOE_OP_LAYER, DEV)
+    a = M.moe_layer_forward(cfg, dc.h, dc.w_router, dc.bias, w13_mx, wd_mx, ws=ws).clone()
+    c1 = M.mx_counters(ws)
+    b = M.moe_layer_forward(cfg, dc.h, dc.w_router, dc.bias, w13_mx, wd_mx, ws=ws)
+    c2 = M.mx_counters(ws)
+    torch.cuda.synchronize()
+    assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+    assert c1 == c2                                            # zeroed by every call, not accumulated
+
+
+def test_mxfp8_rejects_unsupported_configs():
+    h = torch.zeros((64, 128), dtype=torch.bfloat16, device=DEV)
+    for kw in (dict(dispatch="gather"), dict(gemm_tiles="pair"), dict(expert_kind="identity")):
+        cfg = M.config(64, 128, 4, 2, 128, precision="mxfp8", **kw)
+        assert M.moe_workspace_size(cfg, M.MOE_OP_LAYER) == 0, kw
+    cfg = M.config(64, 128, 4, 2, 128, precision="mxfp8")
+    ws = M.workspace(cfg, M.MOE_OP_LAYER, DEV)
+    with pytest.raises(M.MoeError):                            # the backward is bf16 only
+        M.moe_layer_backward(cfg, h, torch.zeros((4, 128), dtype=torch.bfloat16, device=DEV),
+                             torch.zeros((4, 256, 128), dtype=torch.bfloat16, device=DEV),
+                             torch.zeros((4, 128, 256), dtype=torch.bfloat16, device=DEV),
+                             torch.zeros((4, 128, 128), dtype=torch.bfloat16, device=DEV), h, ws,
+                             ws=torch.zeros(1 << 20, dtype=torch.uint8, device=DEV))

@@ -478,3 +478,44 @@ def test_layer_stage_events_time_the_same_layer():
     assert torch.equal(y0.view(torch.int16), y2.view(torch.int16))
     with pytest.raises(ValueError):
         M.moe_layer_forward(dc.cfg, dc.h, dc.w_router, dc.bias, dc.w13, dc.w_down, ws=ws, stage_events=ev[:3])
+
+
+@pytest.mark.parametrize("name,kw", [("small_ragged", {}), ("mixtral_scaled", {}),
+                                     ("small_ragged", dict(capacity=150)), ("small_ragged", dict(k=1)),
+                                     ("mixtral_8x7b", {})])
+def test_layer_fused_combine_equals_separate(name, kw):
+    """The combine done by the down projection's epilogue (k <= 2) gives y bit
+    for bit equal to the separate combine kernel, with every slot kept, with
+    capacity drops (tokens keeping one slot or none) and with k = 1; y_perm,
+    which the backward reads, is written the same way."""
+    dc = dev_case(name)
+    wl = dc.wl.with_(**kw) if kw else dc.wl
+    h = dc.h
+    if "k" in kw:
+        inp = W.draw(wl, 5)
+        inp = cases.enforce_margin(inp, 5)
+        dc = DeviceCase(inp)
+        h = dc.h
+    base = dict(T=wl.T, d=wl.d, E=wl.E, k=wl.k, d_ff=wl.F, dtype=wl.dtype, expert_kind=wl.expert_kind,
+                capacity=wl.capacity)
+    ys = {}
+    for mode in ("separate", "fused"):
+        cfg = M.config(**base, combine=mode)
+        ws = M.workspace(cfg, M.MOE_OP_LAYER, DEV)
+        y = torch.full((wl.T, wl.d), 7.0, dtype=torch.bfloat16, device=DEV)      # stale bytes must not survive
+        ys[mode] = M.moe_layer_forward(cfg, h, dc.w_router, dc.bias, dc.w13, dc.w_down, y=y, ws=ws)
+        torch.cuda.synchronize()
+    assert torch.equal(ys["separate"].view(torch.int16), ys["fused"].view(torch.int16))
+    if wl.capacity >= 0:
+        cfg = M.config(**base)
+        counts = torch.empty(wl.E, dtype=torch.int32, device=DEV)
+        M.moe_layer_forward(cfg, h, dc.w_router, dc.bias, dc.w13, dc.w_down, counts=counts)
+        assert int(counts.sum().item()) < wl.T * wl.k                            # drops happened
+
+
+def test_fused_combine_rejected_where_it_does_not_apply():
+    for kw in (dict(k=4, E=8), dict(gemm_tiles="pair"), dict(expert_kind="identity"), dict(precision="mxfp8")):
+        base = dict(T=64, d=128, E=4, k=2, d_ff=128)
+        base.update(kw)
+        cfg = M.config(**base, combine="fused")
+        assert M.moe_workspace_size(cfg, M.MOE_OP_LAYER) == 0, kw

@@ -55,10 +55,14 @@ def test_launch_count_per_step():
     import bench
     import combine_router_gemm_softmax_b200 as M
     assert bench.launches(M.config(64, 128, 8, 2, 128)) == 6
+    # combine fused into the down projection (opt-in): no combine kernel
+    assert bench.launches(M.config(64, 128, 8, 2, 128, combine="fused")) == 5
+    # MXFP8: the row copy is replaced by the dispatch that quantises the rows
+    assert bench.launches(M.config(64, 128, 8, 2, 128, precision="mxfp8")) == 6
     assert bench.launches(M.config(64, 128, 8, 2, 128, expert_kind="identity")) == 4
     assert bench.launches(M.config(64, 128, 8, 2, 128, expert_kind="scale")) == 5
     assert bench.launches(M.config(64, 32, 4, 2, 64, dtype="f32")) == 7
     assert bench.launches(M.config(65536, 128, 256, 2, 128)) == 7      # 256 * 512 chunks: separate scan
     assert bench.launches(M.config(8192, 2048, 128, 8, 768)) == 6      # 128 * 64 chunks: scan inside rank
-    assert bench.launches(M.config(64, 128, 8, 2, 128, capacity=20, layout="padded")) == 7  # + padding fill
-    assert bench.launches(M.config(64, 128, 8, 2, 128, capacity=0, layout="padded")) == 6
+    assert bench.launches(M.config(64, 128, 8, 4, 128, capacity=20, layout="padded")) == 7  # + padding fill
+    assert bench.launches(M.config(64, 128, 8, 4, 128, capacity=0, layout="padded")) == 6
