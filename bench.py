@@ -181,12 +181,15 @@ def run_reference(args, wl, rank):
         times.append(dt)
     total = sum(times)
     value = inp.wl.T * args.steps / total
-    sample = f"first {inp.wl.T} tokens of {wl.name} as their own batch per step, {args.steps} steps"
+    sample = (f"first {inp.wl.T} tokens of {wl.name} as their own batch per step, {args.steps} steps; the oracle "
+              f"batches tokens per expert, so its rate grows with the sample size (the cpu_baseline of the GPU "
+              f"arm uses a larger sample)")
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic (seeded)", "config": config_dict(wl, args.gpus),
-            "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": sample},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": os.cpu_count(), "blas_threads": threads,
+                             "kind": "oracle", "sample": sample},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
@@ -397,6 +400,7 @@ def main():
         line["roofline"] = roofline(stages, wl, A_kept, pk, pk_kind, args.precision)
         if bwd is not None:
             flops = 16.0 * A_kept * wl.d * wl.F          # incl. the recomputed gate/up GEMM
+            bwd, bwd_saved, fwd_saving = bwd
             line["backward"] = {"ms_per_step": bwd, "tokens_per_s": wl.T / (bwd / 1e3),
                                 "gemm_tflops": flops / (bwd / 1e3) / 1e12,
                                 "frac_bf16": flops / (bwd / 1e3) / 1e12 / pk["bf16_tflops_sustained"],
@@ -404,7 +408,14 @@ def main():
                                 "steps": args.steps,
                                 "note": "moe_layer_backward after one forward, steps back to back; "
                                         "gemm_tflops counts 16*A*d*F (dgrad, wgrad and the gate/up recompute) "
-                                        "over the whole backward time"}
+                                        "over the whole backward time",
+                                "saved_preact": {
+                                    "ms_per_step": bwd_saved, "forward_ms_per_step": fwd_saving,
+                                    "gemm_tflops": 12.0 * A_kept * wl.d * wl.F / (bwd_saved / 1e3) / 1e12,
+                                    "train_step_tokens_per_s": wl.T / ((bwd_saved + fwd_saving) / 1e3),
+                                    "note": "forward keeps the gate/up pre-activations (MOE_PREACT_SAVE), the "
+                                            "backward skips their recompute; gemm_tflops counts 12*A*d*F; "
+                                            "forward_ms_per_step is that forward, 5 steps back to back"}}
         line["routing"] = {"routed_counts_max": int(L.routed.max().item()),
                            "routed_counts_mean": float(L.routed.float().mean().item()),
                            "empty_experts": int((L.routed == 0).sum().item()), "kept": A_kept,
@@ -574,31 +585,48 @@ def run_e2e(M, cfg, wl, h_host, h0, y0, wr, bias, w13, wd, ws, stream, dev, step
 
 def run_backward(M, cfg, wl, h, wr, bias, w13, wd, ws, stream, dev, steps, seed):
     """Device time (ms per call) of moe_layer_backward on the forward state
-    left in ws, CUDA events around `steps` back-to-back calls."""
+    left in ws, CUDA events around `steps` back-to-back calls. Returns
+    (recompute ms, saved-pre-activation ms, forward ms with the
+    pre-activations kept): the second form runs on a forward that kept
+    them (MOE_PREACT_SAVE), timed the same way."""
+    import copy
+
     import torch
 
     import workloads as W
 
     w13_t, wd_t = M.moe_pack_weights_backward(cfg, w13, wd, stream=stream)
     dy = W.draw_dy(wl, seed).to(dev)
-    M.moe_layer_forward(cfg, h, wr, bias, w13, wd, ws=ws, stream=stream)
-    bws = M.workspace(cfg, M.MOE_OP_BACKWARD, dev)
 
-    def once():
-        return M.moe_layer_backward(cfg, h, wr, w13, w13_t, wd_t, dy, ws, with_bias=bias is not None, ws=bws,
-                                    stream=stream)
+    def timed(fn, n):
+        for _ in range(2):
+            fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda._sleep(HOST_LEAD_CYCLES)
+        e0.record(stream)
+        for _ in range(n):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / n
 
-    for _ in range(2):
-        once()
-    torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    torch.cuda._sleep(HOST_LEAD_CYCLES)
-    e0.record(stream)
-    for _ in range(steps):
-        once()
-    e1.record(stream)
-    torch.cuda.synchronize()
-    return e0.elapsed_time(e1) / steps
+    out = []
+    for preact in (M.MOE_PREACT_RECOMPUTE, M.MOE_PREACT_SAVE):
+        c = copy.copy(cfg)
+        c.preact = preact
+        fws = ws if preact == M.MOE_PREACT_RECOMPUTE else M.workspace(c, M.MOE_OP_LAYER, dev)
+        fwd_ms = timed(lambda: M.moe_layer_forward(c, h, wr, bias, w13, wd, ws=fws, stream=stream), 5)
+        bws = M.workspace(c, M.MOE_OP_BACKWARD, dev)
+        out.append(timed(lambda: M.moe_layer_backward(c, h, wr, w13, w13_t, wd_t, dy, fws, with_bias=bias is not None,
+                                                      ws=bws, stream=stream), steps))
+        if preact == M.MOE_PREACT_SAVE:
+            out.append(fwd_ms)
+        del bws
+        if fws is not ws:
+            del fws
+        torch.cuda.empty_cache()
+    return tuple(out)
 
 
 def fused_combine(cfg):

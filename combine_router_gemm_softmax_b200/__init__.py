@@ -23,7 +23,7 @@ from ._lib import (  # noqa: F401
     MOE_GEMM_TILES_AUTO, MOE_GEMM_TILES_PAIR, MOE_GEMM_TILES_SINGLE, MOE_LAYOUT_COMPACT, MOE_LAYOUT_PADDED,
     MOE_MAX_E, MOE_MAX_K, MOE_OK, MOE_OP_BACKWARD, MOE_OP_GROUPED_FFN, MOE_OP_LAYER, MOE_OP_PERMUTE, MOE_OP_ROUTE,
     MOE_PACK_BLOCK,
-    MOE_COMBINE_AUTO, MOE_COMBINE_FUSED, MOE_COMBINE_SEPARATE, MOE_PRECISION_BF16, MOE_PRECISION_MXFP8, MOE_STATUS_MX_SATURATED, MOE_STATUS_MX_UNDERFLOW,
+    MOE_COMBINE_AUTO, MOE_COMBINE_FUSED, MOE_COMBINE_SEPARATE, MOE_PREACT_RECOMPUTE, MOE_PREACT_SAVE, MOE_PRECISION_BF16, MOE_PRECISION_MXFP8, MOE_STATUS_MX_SATURATED, MOE_STATUS_MX_UNDERFLOW,
     MOE_STATUS_BAD_ROUTE, MOE_STATUS_NAN_LOGIT, MOE_STATUS_TIMEOUT, MoeConfig, MoeError, config, lib,
     moe_grouped_ffn, moe_layer_backward, moe_layer_forward, moe_pack_weights, moe_pack_weights_backward,
     moe_permute, moe_permute_static_scratch, moe_route,

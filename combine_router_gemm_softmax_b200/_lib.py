@@ -22,6 +22,7 @@ MOE_STATUS_NAN_LOGIT, MOE_STATUS_BAD_ROUTE, MOE_STATUS_TIMEOUT = 1, 2, 4
 MOE_STATUS_MX_SATURATED, MOE_STATUS_MX_UNDERFLOW = 8, 16
 MOE_PRECISION_BF16, MOE_PRECISION_MXFP8 = 0, 1
 MOE_COMBINE_AUTO, MOE_COMBINE_SEPARATE, MOE_COMBINE_FUSED = 0, 1, 2
+MOE_PREACT_RECOMPUTE, MOE_PREACT_SAVE = 0, 1
 MOE_DTYPE_BF16, MOE_DTYPE_F32 = 0, 1
 MOE_EXPERT_SWIGLU, MOE_EXPERT_IDENTITY, MOE_EXPERT_SCALE = 0, 1, 2
 MOE_OP_ROUTE, MOE_OP_PERMUTE, MOE_OP_GROUPED_FFN, MOE_OP_LAYER, MOE_OP_BACKWARD = 0, 1, 2, 3, 4
@@ -47,7 +48,8 @@ class MoeConfig(ctypes.Structure):
     _fields_ = [("T", ctypes.c_int32), ("d", ctypes.c_int32), ("E", ctypes.c_int32), ("k", ctypes.c_int32),
                 ("d_ff", ctypes.c_int32), ("dtype", ctypes.c_int32), ("expert_kind", ctypes.c_int32),
                 ("capacity", ctypes.c_int32), ("gemm_tiles", ctypes.c_int32), ("layout", ctypes.c_int32),
-                ("dispatch", ctypes.c_int32), ("precision", ctypes.c_int32), ("combine", ctypes.c_int32)]
+                ("dispatch", ctypes.c_int32), ("precision", ctypes.c_int32), ("combine", ctypes.c_int32),
+                ("preact", ctypes.c_int32)]
 
     def __repr__(self):
         return "MoeConfig(" + ", ".join(f"{n}={getattr(self, n)}" for n, _ in self._fields_) + ")"
@@ -104,7 +106,7 @@ def lib() -> ctypes.CDLL:
 
 
 def config(T, d, E, k, d_ff, dtype="bf16", expert_kind="swiglu", capacity=-1, gemm_tiles="auto",
-           layout="compact", dispatch="auto", precision="bf16", combine="auto") -> MoeConfig:
+           layout="compact", dispatch="auto", precision="bf16", combine="auto", preact="recompute") -> MoeConfig:
     dt = {"bf16": MOE_DTYPE_BF16, "f32": MOE_DTYPE_F32, torch.bfloat16: MOE_DTYPE_BF16,
           torch.float32: MOE_DTYPE_F32}[dtype]
     kind = {"swiglu": MOE_EXPERT_SWIGLU, "identity": MOE_EXPERT_IDENTITY, "scale": MOE_EXPERT_SCALE}[expert_kind]
@@ -113,7 +115,8 @@ def config(T, d, E, k, d_ff, dtype="bf16", expert_kind="swiglu", capacity=-1, ge
     disp = {"auto": MOE_DISPATCH_AUTO, "copy": MOE_DISPATCH_COPY, "gather": MOE_DISPATCH_GATHER}[dispatch]
     prec = {"bf16": MOE_PRECISION_BF16, "mxfp8": MOE_PRECISION_MXFP8}[precision]
     comb = {"auto": MOE_COMBINE_AUTO, "separate": MOE_COMBINE_SEPARATE, "fused": MOE_COMBINE_FUSED}[combine]
-    return MoeConfig(T, d, E, k, d_ff, dt, kind, capacity, tiles, lay, disp, prec, comb)
+    pre = {"recompute": MOE_PREACT_RECOMPUTE, "save": MOE_PREACT_SAVE}[preact]
+    return MoeConfig(T, d, E, k, d_ff, dt, kind, capacity, tiles, lay, disp, prec, comb, pre)
 
 
 def perm_rows(cfg) -> int:

@@ -122,6 +122,14 @@ bool combine_fusable(const moe_config& c) {
 // AUTO keeps the separate combine: fusing it measured 1-3% slower per layer
 // on B200 (the down projection's epilogue re-reads both rows of a token and
 // competes with the GEMM; the separate kernel streams them at HBM rate).
+// Whether the layer keeps the gate/up pre-activations for the backward.
+bool preact_savable(const moe_config& c) {
+  return c.dtype == MOE_DTYPE_BF16 && c.expert_kind == MOE_EXPERT_SWIGLU && c.gemm_tiles != MOE_GEMM_TILES_PAIR &&
+         !is_mx(c) && c.dispatch != MOE_DISPATCH_GATHER;
+}
+
+bool layer_saves_preact(const moe_config& c) { return c.preact == MOE_PREACT_SAVE && preact_savable(c); }
+
 bool layer_fuses_combine(const moe_config& c) { return c.combine == MOE_COMBINE_FUSED && combine_fusable(c); }
 
 // AUTO copies: gathering costs one four-row TMA gather per 512 bytes of A
@@ -149,6 +157,8 @@ int check_cfg(const moe_config* c) {
   if (c->precision != MOE_PRECISION_BF16 && c->precision != MOE_PRECISION_MXFP8) return MOE_ERR_INVALID_ARG;
   if (c->combine < MOE_COMBINE_AUTO || c->combine > MOE_COMBINE_FUSED) return MOE_ERR_INVALID_ARG;
   if (c->combine == MOE_COMBINE_FUSED && !combine_fusable(*c)) return MOE_ERR_UNSUPPORTED;
+  if (c->preact != MOE_PREACT_RECOMPUTE && c->preact != MOE_PREACT_SAVE) return MOE_ERR_INVALID_ARG;
+  if (c->preact == MOE_PREACT_SAVE && !preact_savable(*c)) return MOE_ERR_UNSUPPORTED;
   if (c->precision == MOE_PRECISION_MXFP8 &&
       (c->dtype != MOE_DTYPE_BF16 || c->expert_kind != MOE_EXPERT_SWIGLU || c->gemm_tiles == MOE_GEMM_TILES_PAIR ||
        c->dispatch == MOE_DISPATCH_GATHER))
@@ -227,6 +237,7 @@ struct LayerBufs {
   void *x_perm, *y_perm, *h_mid;
   PermuteScratch perm;
   int32_t* pair_cnt;  // [T][pair_entries(c)] when the combine is fused, else NULL
+  void* preact;       // [P, 2F] bf16 gate/up pre-activations when kept for the backward, else NULL
 };
 
 LayerBufs carve_layer(const moe_config& c, Carver& w) {
@@ -248,6 +259,7 @@ LayerBufs carve_layer(const moe_config& c, Carver& w) {
   b.perm = carve_permute(c, w);
   b.h_mid = carve_ffn(c, w);
   b.pair_cnt = layer_fuses_combine(c) ? w.take<int32_t>(static_cast<size_t>(c.T) * pair_entries(c) * 4) : nullptr;
+  b.preact = layer_saves_preact(c) ? w.take<void>(P * 2 * static_cast<size_t>(c.d_ff) * 2) : nullptr;
   return b;
 }
 
@@ -406,7 +418,7 @@ int ffn_mx_impl(const moe_config& c, const void* x_perm, const int32_t* offsets,
 int ffn_impl(const moe_config& c, const void* x_perm, const int32_t* offsets, const void* w13, const void* w_down,
              void* y_perm, void* h_mid, const void* gather_src, const int32_t* gather_rows, bool pdl,
              int32_t* status, cudaStream_t s, const MxBufs* mx = nullptr, const FusedCombine* fc = nullptr,
-             bool mx_x_quantized = false) {
+             bool mx_x_quantized = false, void* preact = nullptr) {
   const int rows_max = static_cast<int>(perm_rows(c));
   if (rows_max == 0) return MOE_OK;
   if (is_mx(c)) return ffn_mx_impl(c, x_perm, offsets, w13, w_down, y_perm, *mx, pdl, status, s, mx_x_quantized);
@@ -430,7 +442,7 @@ int ffn_impl(const moe_config& c, const void* x_perm, const int32_t* offsets, co
   cudaError_t e =
       pair ? launch_grouped_gemm_pair(a1, b1, true, offsets, E, d, 2 * F, F / 128, F, F, h_mid, status, pdl, s)
            : launch_grouped_gemm_tc(a1, b1, true, offsets, E, d, 2 * F, F / 128, F, F, h_mid,
-                                    gather ? gather_rows : nullptr, status, pdl, s);
+                                    gather ? gather_rows : nullptr, status, pdl, s, preact);
   if (e != cudaSuccess) return MOE_ERR_CUDA;
   const int n2 = (d + kGemmTileN - 1) / kGemmTileN;
   if (fc != nullptr)
@@ -620,7 +632,8 @@ int32_t moe_layer_forward_timed(const moe_config* cfg, const void* h, const void
   const FusedCombine fc{b.perm_src, b.dest_row, b.gate, b.pair_cnt, y};
   if (c.expert_kind != MOE_EXPERT_IDENTITY) {
     rc = ffn_impl(c, b.x_perm, b.offsets, w13_packed, w_down, b.y_perm, b.h_mid, gather ? h : nullptr,
-                  gather ? b.perm_src : nullptr, true, status_dev, s, &mx, fused ? &fc : nullptr, mx_disp);
+                  gather ? b.perm_src : nullptr, true, status_dev, s, &mx, fused ? &fc : nullptr, mx_disp,
+                  b.preact);
     if (rc != MOE_OK) return rc;
     y_src = b.y_perm;
   }
@@ -734,23 +747,32 @@ int32_t moe_layer_backward(const moe_config* cfg, const void* h, const void* w_r
   if (e != cudaSuccess) return MOE_ERR_CUDA;
   if (P > 0) {
     CUtensorMap ta, tb;
-    // 2. dh_mid = dy_perm W_down (per expert), B = W_down^T rows
+    e = launch_col_offsets(f.offsets, E, b.col_off, s);
+    if (e != cudaSuccess) return MOE_ERR_CUDA;
     rc = make_map(&ta, b.dy_perm, P, d, kTileM);
     if (rc == MOE_OK) rc = make_map(&tb, w_down_t, static_cast<uint64_t>(E) * F, d, kGemmTileN);
     if (rc != MOE_OK) return rc;
-    e = launch_grouped_gemm_tc(ta, tb, false, f.offsets, E, d, F, (F + kGemmTileN - 1) / kGemmTileN, F, F, b.dh_mid,
-                               nullptr, status_dev, false, s);
-    if (e != cudaSuccess) return MOE_ERR_CUDA;
-    // 3. gate/up pre-activations recomputed from x_perm; SwiGLU backward in the
-    //    epilogue, which also writes dgu transposed for the weight gradient
-    e = launch_col_offsets(f.offsets, E, b.col_off, s);
-    if (e != cudaSuccess) return MOE_ERR_CUDA;
-    rc = make_map(&ta, f.x_perm, P, d, kTileM);
-    if (rc == MOE_OK) rc = make_map(&tb, w13_packed, static_cast<uint64_t>(E) * 2 * F, d, kGemmTileN);
-    if (rc != MOE_OK) return rc;
-    e = launch_grouped_gemm_swiglu_bwd(ta, tb, f.offsets, E, d, F, b.dgu, b.dh_mid, b.dgu_t, b.col_off, b.ppad_max,
-                                       status_dev, false, s);
-    if (e != cudaSuccess) return MOE_ERR_CUDA;
+    if (f.preact != nullptr) {
+      // 2+3. dL/dh_mid = dy_perm W_down (per expert) with the SwiGLU backward in
+      //      the epilogue, from the pre-activations the forward kept: writes
+      //      dgu and its transposed copy; no recompute of the gate/up GEMM
+      e = launch_grouped_gemm_dh_swiglu_bwd(ta, tb, f.offsets, E, d, F, f.preact, b.dgu, b.dgu_t, b.col_off,
+                                            b.ppad_max, status_dev, false, s);
+      if (e != cudaSuccess) return MOE_ERR_CUDA;
+    } else {
+      // 2. dh_mid = dy_perm W_down (per expert), B = W_down^T rows
+      e = launch_grouped_gemm_tc(ta, tb, false, f.offsets, E, d, F, (F + kGemmTileN - 1) / kGemmTileN, F, F,
+                                 b.dh_mid, nullptr, status_dev, false, s);
+      if (e != cudaSuccess) return MOE_ERR_CUDA;
+      // 3. gate/up pre-activations recomputed from x_perm; SwiGLU backward in the
+      //    epilogue, which also writes dgu transposed for the weight gradient
+      rc = make_map(&ta, f.x_perm, P, d, kTileM);
+      if (rc == MOE_OK) rc = make_map(&tb, w13_packed, static_cast<uint64_t>(E) * 2 * F, d, kGemmTileN);
+      if (rc != MOE_OK) return rc;
+      e = launch_grouped_gemm_swiglu_bwd(ta, tb, f.offsets, E, d, F, b.dgu, b.dh_mid, b.dgu_t, b.col_off,
+                                         b.ppad_max, status_dev, false, s);
+      if (e != cudaSuccess) return MOE_ERR_CUDA;
+    }
     // 4. dx_perm = dgu w13 (per expert), B = w13^T rows
     rc = make_map(&ta, b.dgu, P, 2 * F, kTileM);
     if (rc == MOE_OK) rc = make_map(&tb, w13_t, static_cast<uint64_t>(E) * d, 2 * F, kGemmTileN);

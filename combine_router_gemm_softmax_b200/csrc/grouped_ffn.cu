@@ -106,6 +106,11 @@ struct GemmArgs {
   // barrier that nothing signals, so its bounded wait runs out and the
   // kernel takes its timeout path.
   int stall;
+  // Gate/up pre-activations [rows, preact_ld] (bf16, w13's interleaved column
+  // order): written by the SwiGLU epilogue when set (kept for the backward),
+  // read by the kEpiDhSwiGLUBwd epilogue.
+  __nv_bfloat16* preact;
+  int preact_ld;
 };
 
 // Epilogues and tile groupings of grouped_gemm_kernel.
@@ -114,6 +119,11 @@ constexpr int kEpiSwiGLU = 1;      // D (bf16) = silu(gate) * up, half-width
 constexpr int kEpiSwiGLUBwd = 2;   // D (bf16) = [dgate | dup] from gate, up and aux = dL/dh_mid
 constexpr int kEpiStoreF32 = 3;    // D32 (fp32) = accumulator
 constexpr int kEpiStoreCombine = 4;  // D (bf16) = accumulator, and the combine into Y for k <= 2
+// The dh_mid GEMM of the backward with the SwiGLU backward in its epilogue,
+// from saved pre-activations: the accumulator is dL/dh_mid for 256 channels;
+// D (bf16) = [dgate | dup] in w13's interleaved order, from the accumulator
+// and the saved a, u (preact), and optionally the transposed copy DT.
+constexpr int kEpiDhSwiGLUBwd = 5;
 constexpr int kGroupRows = 0;      // groups of rows (experts' token rows), same K for all
 constexpr int kGroupReduce = 1;    // groups along K (experts' token rows are the reduction)
 constexpr int kReduceBand = 16;    // row tiles per band in the reduction-grouped tile walk
@@ -466,6 +476,87 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             uint4* dst = reinterpret_cast<uint4*>(out + c);
 #pragma unroll
             for (int i = 0; i < 4; ++i) dst[i] = make_uint4(p[4 * i], p[4 * i + 1], p[4 * i + 2], p[4 * i + 3]);
+            if (a.preact != nullptr) {  // the pre-activations themselves, for the backward
+              uint32_t pg[16], pu[16];
+#pragma unroll
+              for (int i = 0; i < 16; ++i) {
+                pg[i] = pack_bf16x2(__uint_as_float(g[2 * i]), __uint_as_float(g[2 * i + 1]));
+                pu[i] = pack_bf16x2(__uint_as_float(u[2 * i]), __uint_as_float(u[2 * i + 1]));
+              }
+              uint4* pgd = reinterpret_cast<uint4*>(a.preact + grow * a.preact_ld + n * kBN + c);
+              uint4* pud = reinterpret_cast<uint4*>(a.preact + grow * a.preact_ld + n * kBN + kBN / 2 + c);
+#pragma unroll
+              for (int i = 0; i < 4; ++i) {
+                pgd[i] = make_uint4(pg[4 * i], pg[4 * i + 1], pg[4 * i + 2], pg[4 * i + 3]);
+                pud[i] = make_uint4(pu[4 * i], pu[4 * i + 1], pu[4 * i + 2], pu[4 * i + 3]);
+              }
+            }
+          }
+        }
+      } else if constexpr (kEpi == kEpiDhSwiGLUBwd) {
+        // this half of the tile's 256 channels is pack block b of w13: its
+        // gate pre-activations at columns [256 b, 256 b + 128) of preact and
+        // of the output, the up ones at [256 b + 128, 256 b + 256)
+        const int b = 2 * n + half;
+        const bool live = b * MOE_PACK_BLOCK < a.out_cols;
+        const int pcol = a.DT != nullptr ? a.col_off[e] + m * kBM + row : 0;
+        const bool twrite = live && a.DT != nullptr && pcol < a.col_off[e + 1];
+        const __nv_bfloat16* pre = a.preact + grow * a.preact_ld + b * kBN;
+        __nv_bfloat16* out = a.D + grow * a.ldd + b * kBN;
+#pragma unroll 1
+        for (int c = 0; c < kBN / 2 && live; c += 32) {
+          uint32_t dh[32];
+          tmem_ld32(tbase + half * (kBN / 2) + c, dh);
+          uint4 ga[4], ua[4];
+          if (valid) {
+            const uint4* gsrc = reinterpret_cast<const uint4*>(pre + c);
+            const uint4* usrc = reinterpret_cast<const uint4*>(pre + kBN / 2 + c);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              ga[i] = gsrc[i];
+              ua[i] = usrc[i];
+            }
+          }
+          tmem_ld_wait();
+          uint32_t pg[16], pu[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) pg[i] = pu[i] = 0u;
+          if (valid) {
+            const __nv_bfloat16* av = reinterpret_cast<const __nv_bfloat16*>(ga);
+            const __nv_bfloat16* uv = reinterpret_cast<const __nv_bfloat16*>(ua);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              float dg2[2], du2[2];
+#pragma unroll
+              for (int h2 = 0; h2 < 2; ++h2) {
+                const float av1 = __bfloat162float(av[2 * i + h2]);
+                const float uv1 = __bfloat162float(uv[2 * i + h2]);
+                const float d0 = __uint_as_float(dh[2 * i + h2]);
+                const float sg = 1.0f / (1.0f + expf(-av1));
+                dg2[h2] = d0 * uv1 * (sg * (1.0f + av1 * (1.0f - sg)));
+                du2[h2] = d0 * av1 * sg;
+              }
+              pg[i] = pack_bf16x2(dg2[0], dg2[1]);
+              pu[i] = pack_bf16x2(du2[0], du2[1]);
+            }
+            uint4* dg_dst = reinterpret_cast<uint4*>(out + c);
+            uint4* du_dst = reinterpret_cast<uint4*>(out + kBN / 2 + c);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              dg_dst[i] = make_uint4(pg[4 * i], pg[4 * i + 1], pg[4 * i + 2], pg[4 * i + 3]);
+              du_dst[i] = make_uint4(pu[4 * i], pu[4 * i + 1], pu[4 * i + 2], pu[4 * i + 3]);
+            }
+          }
+          if (twrite) {
+            uint16_t* tg = reinterpret_cast<uint16_t*>(a.DT) + static_cast<size_t>(b * kBN + c) * a.ldt + pcol;
+            uint16_t* tu = tg + static_cast<size_t>(kBN / 2) * a.ldt;
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              tg[static_cast<size_t>(2 * i) * a.ldt] = static_cast<uint16_t>(pg[i] & 0xffffu);
+              tg[static_cast<size_t>(2 * i + 1) * a.ldt] = static_cast<uint16_t>(pg[i] >> 16);
+              tu[static_cast<size_t>(2 * i) * a.ldt] = static_cast<uint16_t>(pu[i] & 0xffffu);
+              tu[static_cast<size_t>(2 * i + 1) * a.ldt] = static_cast<uint16_t>(pu[i] >> 16);
+            }
           }
         }
       } else if constexpr (kEpi == kEpiStoreCombine) {
@@ -1001,9 +1092,11 @@ cudaError_t launch_gemm_inst(const CUtensorMap& tm_a, const CUtensorMap& tm_b, G
 cudaError_t launch_grouped_gemm_tc(const CUtensorMap& tm_a, const CUtensorMap& tm_b, bool swiglu,
                                    const int32_t* offsets, int E, int K, int n_per_expert, int n_tiles,
                                    int out_cols, int ldd, void* D, const int32_t* gather_rows, int32_t* status,
-                                   bool pdl, cudaStream_t s) {
+                                   bool pdl, cudaStream_t s, void* preact) {
   GemmArgs a{offsets, E, K, n_per_expert, n_tiles, out_cols, ldd, static_cast<__nv_bfloat16*>(D), status,
              band_rows(kBM, K, 8, 32), gather_rows, nullptr, 0, nullptr, 0, nullptr, nullptr, 0};
+  a.preact = static_cast<__nv_bfloat16*>(preact);
+  a.preact_ld = n_per_expert;
   return swiglu ? launch_gemm_inst<kEpiSwiGLU, kGroupRows>(tm_a, tm_b, a, pdl, s)
                 : launch_gemm_inst<kEpiStore, kGroupRows>(tm_a, tm_b, a, pdl, s);
 }
@@ -1023,6 +1116,18 @@ cudaError_t launch_grouped_gemm_combine(const CUtensorMap& tm_a, const CUtensorM
   a.Y = static_cast<__nv_bfloat16*>(y);
   a.k = k;
   return launch_gemm_inst<kEpiStoreCombine, kGroupRows>(tm_a, tm_b, a, pdl, s);
+}
+
+cudaError_t launch_grouped_gemm_dh_swiglu_bwd(const CUtensorMap& tm_a, const CUtensorMap& tm_b,
+                                              const int32_t* offsets, int E, int K, int F, const void* preact,
+                                              void* dgu, void* dgu_t, const int32_t* col_off, int ldt, int32_t* status,
+                                              bool pdl, cudaStream_t s) {
+  GemmArgs a{offsets, E, K, F, (F + kBN - 1) / kBN, F, 2 * F, static_cast<__nv_bfloat16*>(dgu), status,
+             band_rows(kBM, K, 8, 32), nullptr, nullptr, 0, nullptr, 0, static_cast<__nv_bfloat16*>(dgu_t), col_off,
+             ldt};
+  a.preact = static_cast<__nv_bfloat16*>(const_cast<void*>(preact));
+  a.preact_ld = 2 * F;
+  return launch_gemm_inst<kEpiDhSwiGLUBwd, kGroupRows>(tm_a, tm_b, a, pdl, s);
 }
 
 cudaError_t launch_grouped_gemm_swiglu_bwd(const CUtensorMap& tm_a, const CUtensorMap& tm_b, const int32_t* offsets,

@@ -54,10 +54,20 @@ cudaError_t launch_combine(int dtype, const void* y_perm, const int32_t* dest_ro
 // when that kernel belongs to the same library call.
 // gather_rows (may be NULL): A row r is row gather_rows[r] of the tensor behind
 // tm_a, whose box must then be 64 columns by one row.
+// preact (swiglu only, may be NULL): also store the gate/up pre-activations
+// [rows, n_per_expert] bf16 in w13's interleaved column order.
 cudaError_t launch_grouped_gemm_tc(const CUtensorMap& tm_a, const CUtensorMap& tm_b, bool swiglu,
                                    const int32_t* offsets, int E, int K, int n_per_expert, int n_tiles,
                                    int out_cols, int ldd, void* D, const int32_t* gather_rows, int32_t* status,
-                                   bool pdl, cudaStream_t s);
+                                   bool pdl, cudaStream_t s, void* preact = nullptr);
+// The backward's dh_mid GEMM (dy_perm rows against W_down^T rows, K = d) with
+// the SwiGLU backward in its epilogue from the saved pre-activations
+// preact [rows, 2F]: writes dgu [rows, 2F] = [dgate | dup] (interleaved) and
+// its transposed copy dgu_t as launch_grouped_gemm_swiglu_bwd does.
+cudaError_t launch_grouped_gemm_dh_swiglu_bwd(const CUtensorMap& tm_a, const CUtensorMap& tm_b,
+                                              const int32_t* offsets, int E, int K, int F, const void* preact,
+                                              void* dgu, void* dgu_t, const int32_t* col_off, int ldt, int32_t* status,
+                                              bool pdl, cudaStream_t s);
 // The down projection with the combine fused into its epilogue (k <= 2): y_perm
 // rows as launch_grouped_gemm_tc, and y [T, d] = sum over each token's kept
 // slots, in slot order, of gate * bf16 row (bit-identical to launch_combine).

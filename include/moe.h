@@ -154,6 +154,19 @@ extern "C" {
 #define MOE_COMBINE_SEPARATE 1
 #define MOE_COMBINE_FUSED    2
 
+/* What moe_layer_forward keeps for moe_layer_backward. RECOMPUTE: nothing
+ * extra; the backward recomputes the gate/up pre-activations with a grouped
+ * GEMM (4 A d F flops) and applies the SwiGLU backward in its epilogue. SAVE:
+ * GEMM1's epilogue also stores the pre-activations a = x W_gate^T and
+ * u = x W_up^T as bf16 [P, 2F] in the layer workspace (w13's interleaved
+ * column order), and the backward applies the SwiGLU backward in the epilogue
+ * of its dh_mid GEMM from them, with no recompute. The forward then writes
+ * 4 P F more bytes; the backward's gradients use the bf16-rounded a and u.
+ * SAVE needs bf16 SwiGLU experts, single-CTA tiles, bf16 precision and the
+ * COPY dispatch. */
+#define MOE_PREACT_RECOMPUTE 0
+#define MOE_PREACT_SAVE      1
+
 #define MOE_OP_ROUTE       0
 #define MOE_OP_PERMUTE     1
 #define MOE_OP_GROUPED_FFN 2
@@ -178,6 +191,7 @@ typedef struct moe_config {
   int32_t dispatch;     /* MOE_DISPATCH_*: x_perm row copy or gather inside GEMM1 (layer only) */
   int32_t precision;    /* MOE_PRECISION_*: operands of the grouped expert GEMMs */
   int32_t combine;      /* MOE_COMBINE_*: separate combine kernel or fused into the down projection (layer only) */
+  int32_t preact;       /* MOE_PREACT_*: gate/up pre-activations recomputed or kept for the backward (layer only) */
 } moe_config;
 
 typedef void* moe_stream_t; /* cudaStream_t */

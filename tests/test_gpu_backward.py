@@ -42,25 +42,39 @@ def _unpack_w13(dw13, F):
     return blocks[:, :, 0].reshape(E, F, d), blocks[:, :, 1].reshape(E, F, d)
 
 
-def _run(name, seed=0):
+def _cfg(dc, preact):
+    if preact == "recompute":
+        return dc.cfg
+    wl = dc.wl
+    return M.config(wl.T, wl.d, wl.E, wl.k, wl.F, wl.dtype, wl.expert_kind, wl.capacity, wl.gemm_tiles, wl.layout,
+                    preact=preact)
+
+
+def _run(name, seed=0, preact="recompute"):
     dc = _dev(name)
     inp, _ = parity_case(name)
     wl = dc.wl
-    ws = M.workspace(dc.cfg, M.MOE_OP_LAYER, DEV)
-    M.moe_layer_forward(dc.cfg, dc.h, dc.w_router, dc.bias, dc.w13, dc.w_down, ws=ws)
-    w13_t, wd_t = M.moe_pack_weights_backward(dc.cfg, dc.w13, dc.w_down)
+    cfg = _cfg(dc, preact)
+    ws = M.workspace(cfg, M.MOE_OP_LAYER, DEV)
+    M.moe_layer_forward(cfg, dc.h, dc.w_router, dc.bias, dc.w13, dc.w_down, ws=ws)
+    w13_t, wd_t = M.moe_pack_weights_backward(cfg, dc.w13, dc.w_down)
     dy = W.draw_dy(wl, seed)
     status = torch.zeros(1, dtype=torch.int32, device=DEV)
-    g = M.moe_layer_backward(dc.cfg, dc.h, dc.w_router, dc.w13, w13_t, wd_t, dy.to(DEV), ws,
+    g = M.moe_layer_backward(cfg, dc.h, dc.w_router, dc.w13, w13_t, wd_t, dy.to(DEV), ws,
                              with_bias=dc.bias is not None, status=status)
     torch.cuda.synchronize()
     assert int(status.item()) == 0
     return dc, inp, dy, g
 
 
-@pytest.mark.parametrize("name", BWD_CASES)
-def test_layer_backward_matches_oracle(name):
-    dc, inp, dy, g = _run(name)
+@pytest.mark.parametrize("name,preact", [(n, "recompute") for n in BWD_CASES] +
+                         [(n, "save") for n in ("small_ragged", "small_skewed_capacity", "small_skewed_padded",
+                                                "small_many")])
+def test_layer_backward_matches_oracle(name, preact):
+    """preact "save": the forward keeps the gate/up pre-activations (bf16) and
+    the backward applies the SwiGLU backward in the dh_mid GEMM's epilogue
+    instead of recomputing them; same bounds."""
+    dc, inp, dy, g = _run(name, preact=preact)
     wl = dc.wl
     ref = O.layer_backward(cases.as64(inp.h), cases.as64(inp.w_router), cases.as64(inp.bias), wl.k,
                            cases.weights_fn(inp), wl.capacity, cases.as64(dy))
@@ -139,3 +153,45 @@ def test_layer_backward_full_size_sampled(name):
             assert np.abs(ref[key][n]).max() > 0, (key, e, f)           # a live expert has a non-zero row
             errs[(key, e, f)] = C.vector_rel_err(v, ref[key][n])
     assert max(errs.values()) <= tol, errs
+
+
+def test_saving_preactivations_leaves_the_forward_unchanged():
+    """The forward that keeps its pre-activations returns the same y, bit for
+    bit, and the two backward forms agree to bf16 rounding."""
+    dc = _dev("small_skewed")
+    outs = {}
+    for preact in ("recompute", "save"):
+        cfg = _cfg(dc, preact)
+        outs[preact] = M.moe_layer_forward(cfg, dc.h, dc.w_router, dc.bias, dc.w13, dc.w_down)
+    torch.cuda.synchronize()
+    assert torch.equal(outs["recompute"].view(torch.int16), outs["save"].view(torch.int16))
+    _, _, _, g_r = _run("small_skewed", seed=2)
+    g_r = {k: v.clone() for k, v in g_r.items() if v is not None}
+    _, _, _, g_s = _run("small_skewed", seed=2, preact="save")
+    for key in ("dh", "dw13", "dw_down", "dw_router"):
+        a, b = np64(g_r[key]), np64(g_s[key])
+        assert np.abs(a - b).max() <= 2e-2 * np.abs(a).max(), key
+
+
+@pytest.mark.parametrize("name", ["mixtral_8x7b"])
+def test_layer_backward_full_size_saved_preact(name):
+    """The Mixtral 8x7B layer with saved pre-activations, in the configuration
+    bench.py times: dh on sampled tokens and whole dW rows and columns, as
+    test_layer_backward_full_size_sampled."""
+    dc, inp, dy, g = _run(name, preact="save")
+    wl = dc.wl
+    r = np.random.default_rng(12)
+    e0 = int(r.integers(wl.E))
+    chans = [(e0, int(f)) for f in r.choice(wl.F, size=2, replace=False)]
+    tokens = np.sort(r.choice(wl.T, size=16, replace=False))
+    probe = O.layer_backward_probe(cases.as64(inp.h), cases.as64(inp.w_router), cases.as64(inp.bias), wl.k,
+                                   cases.weights_fn(inp), wl.capacity, cases.as64(dy), tokens, [])
+    tol = C.tol_for(wl.dtype)
+    assert C.row_rel_err(np64(g["dh"][torch.from_numpy(tokens).to(DEV)]), probe["dh"]) <= tol
+    ref = O.layer_backward_channels(cases.as64(inp.h), cases.as64(inp.w_router), cases.as64(inp.bias), wl.k,
+                                    cases.weights_fn(inp), wl.capacity, cases.as64(dy), chans)
+    for n, (e, f) in enumerate(chans):
+        gate_row = (f // 128) * 256 + f % 128
+        assert C.vector_rel_err(np64(g["dw13"][e, gate_row]), ref["dw_gate_rows"][n]) <= tol
+        assert C.vector_rel_err(np64(g["dw13"][e, gate_row + 128]), ref["dw_up_rows"][n]) <= tol
+        assert C.vector_rel_err(np64(g["dw_down"][e, :, f]), ref["dw_down_cols"][n]) <= tol
