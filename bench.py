@@ -422,6 +422,8 @@ def main():
                            "dropped": wl.T * wl.k - A_kept}
     if rank == 0 and world == 1 and not args.no_sweep:
         line["combine_separate"] = run_combine_separate(M, L, stream, barrier)
+        if L.input_bytes() >= 2 * L2_BYTES:
+            line["ops_alone"] = run_ops_alone(M, L, stream, barrier)
         if args.precision == "bf16" and wl.expert_kind == "swiglu" and wl.dtype == "bf16":
             line["mxfp8"] = run_mxfp8(M, L, stream, barrier)
     del L
@@ -461,6 +463,62 @@ def run_combine_separate(M, L, stream, barrier):
     return {"ms_per_step": ms / SWEEP_STEPS, "steps": SWEEP_STEPS, "permute": rep["permute"],
             "combine": rep["combine"], "dispatch_combine": rep["dispatch_combine"],
             "grouped_ffn_us": rep["grouped_ffn"]["us"]}
+
+
+def run_ops_alone(M, L, stream, barrier, reps=20):
+    """The three HBM-bound entry points of the headline layer, each called
+    alone: 3 warm-up calls, then `reps` calls back to back on one stream
+    between two events. Inside a layer step the router also pays for writing
+    back the previous step's combine output (up to L2's 126 MB of dirty
+    lines), and the combine leaves part of its own output in L2; called back
+    to back, each op pays for its own writes."""
+    import torch
+
+    pk, pk_kind = peaks()
+    cfg, wl = L.cfg, L.wl
+    s = wl.elem_bytes
+    T, d, E, k = wl.T, wl.d, wl.E, wl.k
+    dev = L.dev
+    idx = torch.empty((T, k), dtype=torch.int32, device=dev)
+    gates = torch.empty((T, k), dtype=torch.float32, device=dev)
+    st = torch.zeros(1, dtype=torch.int32, device=dev)
+    ws = M.workspace(cfg, M.MOE_OP_PERMUTE, dev)
+    M.moe_route(cfg, L.h, L.wr, L.bias, topk_idx=idx, topk_gate=gates, status=st, stream=stream)
+    out = M.moe_permute(cfg, L.h, idx, ws=ws, status=st, stream=stream)
+    A_kept = int(out["counts"].sum().item())
+    y = torch.empty_like(L.y)
+    calls = {
+        "route": (lambda: M.moe_route(cfg, L.h, L.wr, L.bias, topk_idx=idx, topk_gate=gates, status=st,
+                                      stream=stream),
+                  T * d * s + E * d * s + T * k * 8),
+        "permute": (lambda: M.moe_permute(cfg, L.h, idx, out=out, ws=ws, status=st, stream=stream),
+                    T * k * 4 + T * d * s + A_kept * d * s),
+        "combine": (lambda: M.moe_unpermute_combine(cfg, out["x_perm"], out["dest_row"], gates, y=y, status=st,
+                                                    stream=stream),
+                    A_kept * d * s + T * d * s + T * k * 8),
+    }
+    res = {}
+    for name, (fn, nbytes) in calls.items():
+        for _ in range(3):
+            fn()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        barrier()
+        torch.cuda._sleep(HOST_LEAD_CYCLES)
+        e0.record(stream)
+        for _ in range(reps):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        us = 1e3 * e0.elapsed_time(e1) / reps
+        res[name] = {"us": us, "GB/s": nbytes / us / 1e3, "frac_hbm": nbytes / us / 1e3 / pk["hbm_gbs"],
+                     "bytes": nbytes}
+    if int(st.item()) & ~(M.MOE_STATUS_MX_SATURATED | M.MOE_STATUS_MX_UNDERFLOW):
+        raise RuntimeError(f"ops alone: status word {int(st.item())}")
+    res["reps"] = reps
+    res["note"] = ("each entry point alone (moe_route; moe_permute with its own count kernel; "
+                   "moe_unpermute_combine of x_perm as y_perm), calls back to back, inputs larger than L2")
+    return res
 
 
 def run_mxfp8(M, L, stream, barrier):

@@ -165,6 +165,12 @@ __global__ void __launch_bounds__(kChunkTokens) rank_kernel(
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int chunk = blockIdx.x;
   for (int i = threadIdx.x; i < kWarps * kMaxE; i += blockDim.x) (&mask[0][0])[i] = 0u;
+  // this thread's token's route, loaded first so that its latency overlaps
+  // the count-table pass below
+  const int t = chunk * kChunkTokens + threadIdx.x;
+  int ev[kMaxK];
+  uint32_t valid = 0;
+  if (t < T) valid = load_route(idx, t, k, E, ev);
 
   if constexpr (kFusedScan) {
     // The whole counts matrix (at most kFusedScanMax entries, 32 KB) comes
@@ -179,7 +185,7 @@ __global__ void __launch_bounds__(kChunkTokens) rank_kernel(
       const int n4 = n >> 2;
       const int4* src4 = reinterpret_cast<const int4*>(chunk_table);
       int4* dst4 = reinterpret_cast<int4*>(s_tab);
-#pragma unroll 4
+#pragma unroll 16
       for (int i = threadIdx.x; i < n4; i += blockDim.x) dst4[i] = src4[i];
       for (int i = 4 * n4 + threadIdx.x; i < n; i += blockDim.x) s_tab[i] = chunk_table[i];
       __syncthreads();
@@ -245,11 +251,7 @@ __global__ void __launch_bounds__(kChunkTokens) rank_kernel(
   }
   __syncthreads();
 
-  const int t = chunk * kChunkTokens + threadIdx.x;
-  int ev[kMaxK];
-  uint32_t valid = 0;
   if (t < T) {
-    valid = load_route(idx, t, k, E, ev);
 #pragma unroll
     for (int j = 0; j < kMaxK; ++j)
       if (valid & (1u << j)) atomicOr(&mask[warp][ev[j]], 1u << lane);
@@ -323,9 +325,12 @@ static_assert(kCopyTokensPerCta <= 32, "one lane stages the active-token list");
 
 // Row copy with the TMA engine. Each CTA owns a contiguous block of tokens and
 // stages their dest_row entries in shared memory; one thread then runs a
-// pipeline: bulk-load a row (or a piece of it) into one of 8 buffers, and when
-// it lands, bulk-store it to every kept destination row. Each row is read from
-// HBM once; a few instructions move a whole row.
+// pipeline: bulk-load a row (or a piece of it) into one of up to 8 buffers,
+// and when it lands, bulk-store it to every kept destination row. Each row is
+// read from HBM once; a few instructions move a whole row. A block reserves
+// only the buffers its rows can use (4 tokens of one piece: 4 buffers), so
+// twice as many blocks fit on an SM as with 8 (A/B on B200: the Mixtral 8x7B
+// dispatch 152 -> 139 us, skewed with capacity 39.6 -> 33.8 us).
 __global__ void __launch_bounds__(32) permute_copy_bulk_kernel(const uint8_t* __restrict__ h,
                                                                const int32_t* __restrict__ dest_row,
                                                                uint8_t* __restrict__ x_perm, int T, int k, int rb,
@@ -335,8 +340,9 @@ __global__ void __launch_bounds__(32) permute_copy_bulk_kernel(const uint8_t* __
   uint8_t* smem = smem_raw + ((128u - (smem_addr(smem_raw) & 127u)) & 127u);
   const int piece = rb < kCopyPiece ? rb : kCopyPiece;
   const int n_pieces = (rb + piece - 1) / piece;
-  uint8_t* buf = smem;                                                    // kCopyBuffers x piece
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kCopyBuffers * piece);
+  const int nbuf = min(kCopyBuffers, tokens_per_cta * n_pieces);
+  uint8_t* buf = smem;                                                    // nbuf x piece
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + nbuf * piece);
   int* dests = reinterpret_cast<int*>(bars + kCopyBuffers);               // tokens_per_cta x k
   const int lane = threadIdx.x;
   const int t0 = blockIdx.x * tokens_per_cta;
@@ -445,6 +451,16 @@ struct Vec<MOE_DTYPE_F32> {
 constexpr int combine_batch(int nk) {
   return nk == 1 ? 16 : nk == 2 ? 8 : nk == 3 ? 5 : nk == 4 ? 4 : nk <= 6 ? 2 : 1;
 }
+// Resident CTAs per SM the register budget is sized for: three (80 registers
+// a thread) up to k = 6, four (64) for k = 7 and 8, where the loads in flight
+// per lane are capped at 8 so that the budget holds without spills. Against
+// two CTAs per SM, A/B runs on B200 gave 5-13% faster combines at k = 6 and 8,
+// the same at k = 2.
+template <int K>
+constexpr int kCombineCtasPerSm = K >= 7 ? 4 : 3;
+constexpr int combine_batch_k(int nk, int k) {
+  return k >= 7 && combine_batch(nk) * nk > 8 ? (8 / nk > 0 ? 8 / nk : 1) : combine_batch(nk);
+}
 
 // y[t] from the token's NK kept rows (slot order), one warp: all NK rows of U
 // 16-byte segments per lane are loaded before any is used.
@@ -484,7 +500,7 @@ MOE_DEV void combine_rows(const uint4* __restrict__ y_perm, const int (&dst)[K],
 // first (in slot order) and the loads are batched by their number, so a token
 // that kept few of its k slots still has about 16 loads per lane in flight.
 template <int DT, int K>
-__global__ void __launch_bounds__(256) combine_kernel(const uint4* __restrict__ y_perm,
+__global__ void __launch_bounds__(256, kCombineCtasPerSm<K>) combine_kernel(const uint4* __restrict__ y_perm,
                                                       const int32_t* __restrict__ dest_row,
                                                       const float* __restrict__ gate, uint4* __restrict__ y, int T,
                                                       int vpr) {
@@ -513,7 +529,7 @@ __global__ void __launch_bounds__(256) combine_kernel(const uint4* __restrict__ 
         break;
 #define MOE_COMBINE_NK(NKK)                                                              \
   case NKK:                                                                              \
-    if constexpr (NKK <= K) combine_rows<DT, NKK, combine_batch(NKK), K>(y_perm, dst, g, yrow, vpr, lane); \
+    if constexpr (NKK <= K) combine_rows<DT, NKK, combine_batch_k(NKK, K), K>(y_perm, dst, g, yrow, vpr, lane); \
     break;
       MOE_COMBINE_NK(1)
       MOE_COMBINE_NK(2)
@@ -604,7 +620,9 @@ cudaError_t launch_permute(const void* h, size_t row_bytes, const int32_t* idx, 
   if (n_chunks > 0 && copy_rows) {
     const int tpc = kCopyTokensPerCta;
     const int piece = static_cast<int>(row_bytes < kCopyPiece ? row_bytes : kCopyPiece);
-    const size_t smem = 128 + static_cast<size_t>(kCopyBuffers) * piece + kCopyBuffers * 8 + tpc * k * 4;
+    const int n_pieces = static_cast<int>((row_bytes + piece - 1) / piece);
+    const int nbuf = tpc * n_pieces < kCopyBuffers ? tpc * n_pieces : kCopyBuffers;
+    const size_t smem = 128 + static_cast<size_t>(nbuf) * piece + kCopyBuffers * 8 + tpc * k * 4;
     err = cudaFuncSetAttribute(permute_copy_bulk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                static_cast<int>(smem));
     if (err != cudaSuccess) return err;
