@@ -136,12 +136,6 @@ __global__ void __launch_bounds__(1024) scan_kernel(const int32_t* __restrict__ 
 // larger ones go through scan_kernel first.
 constexpr int kFusedScanMax = 8192;
 
-MOE_DEV int warp_sum(int v) {
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
-  return v;
-}
-
 // Ranks of one 128-token chunk: rank(t,j) = tokens before t (in earlier
 // chunks, then in earlier warps of this chunk, then in lower lanes) that
 // picked the same expert. With kFusedScan the chunk bases and offsets are
@@ -319,8 +313,10 @@ constexpr int kCopyBuffers = 8;     // shared-memory row buffers per CTA
 constexpr int kCopyLead = 4;        // row loads kept in flight ahead of the stores
 constexpr int kCopyPiece = 8192;    // bytes per bulk transfer
 // Tokens per CTA: small blocks give many CTAs per SM and the most row loads in
-// flight (measured on B200 for 4-8 KiB rows and k = 2..8).
-constexpr int kCopyTokensPerCta = 4;
+// flight. With buffers reserved per block, 2 tokens (2 buffers for rows of up
+// to 8 KiB, about 26 CTAs per SM) beat 4 in A/B runs on B200: many_small
+// 65.6 -> 57.9 us, skewed 85.0 -> 82.2 us, Mixtral 8x7B unchanged.
+constexpr int kCopyTokensPerCta = 2;
 static_assert(kCopyTokensPerCta <= 32, "one lane stages the active-token list");
 
 // Row copy with the TMA engine. Each CTA owns a contiguous block of tokens and
@@ -328,9 +324,10 @@ static_assert(kCopyTokensPerCta <= 32, "one lane stages the active-token list");
 // pipeline: bulk-load a row (or a piece of it) into one of up to 8 buffers,
 // and when it lands, bulk-store it to every kept destination row. Each row is
 // read from HBM once; a few instructions move a whole row. A block reserves
-// only the buffers its rows can use (4 tokens of one piece: 4 buffers), so
-// twice as many blocks fit on an SM as with 8 (A/B on B200: the Mixtral 8x7B
-// dispatch 152 -> 139 us, skewed with capacity 39.6 -> 33.8 us).
+// only the buffers its rows can use (2 tokens of one piece: 2 buffers), so
+// many more blocks fit on an SM than with 8 (A/B on B200, 4 tokens and 4
+// buffers against 8 buffers: the Mixtral 8x7B dispatch 152 -> 139 us, skewed
+// with capacity 39.6 -> 33.8 us).
 __global__ void __launch_bounds__(32) permute_copy_bulk_kernel(const uint8_t* __restrict__ h,
                                                                const int32_t* __restrict__ dest_row,
                                                                uint8_t* __restrict__ x_perm, int T, int k, int rb,

@@ -292,6 +292,17 @@ def test_permute_fp32_rows():
     _permute_check(100, 36, 5, 2, _routes("random", 100, 5, 2), dtype="f32")
 
 
+@pytest.mark.parametrize("T,d,E,k,cap,dtype", [
+    (301, 6144, 8, 2, -1, "bf16"),    # 12 KB rows: an 8 KB piece and a 4 KB piece
+    (257, 8192, 16, 4, 40, "bf16"),   # 16 KB rows, two full pieces, with drops
+    (129, 3000, 8, 3, -1, "f32"),     # 12000-byte rows: 8192 + 3808
+])
+def test_permute_multi_piece_rows(T, d, E, k, cap, dtype):
+    """Rows longer than one bulk transfer move in pieces; every kept row still
+    lands bit for bit, including the ragged last piece."""
+    _permute_check(T, d, E, k, _routes("random", T, E, k, seed=d), cap, dtype=dtype)
+
+
 def test_permute_zero_tokens():
     cfg = M.config(0, 128, 8, 2, 128)
     out = M.moe_permute(cfg, torch.empty((0, 128), dtype=torch.bfloat16, device=DEV),
