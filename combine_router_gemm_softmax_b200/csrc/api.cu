@@ -55,6 +55,21 @@ int make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uin
   return r == CUDA_SUCCESS ? MOE_OK : MOE_ERR_CUDA;
 }
 
+// Row-major bf16 matrix [rows, cols] written by TMA stores: boxes of 32 rows x
+// 32 columns (64 bytes), 64-byte swizzle (the GEMM epilogue's staging layout).
+int make_map_store(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols) {
+  EncodeTiledFn enc = encode_fn();
+  if (enc == nullptr) return MOE_ERR_NO_DEVICE;
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {cols * 2};
+  const cuuint32_t box[2] = {32, 32};
+  const cuuint32_t es[2] = {1, 1};
+  const CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
+                         CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? MOE_OK : MOE_ERR_CUDA;
+}
+
 // Row-major byte matrix [rows, cols] (E4M3 elements), box of box_rows x 128
 // columns, 128-byte swizzle.
 int make_map_u8(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows) {
@@ -432,17 +447,19 @@ int ffn_impl(const moe_config& c, const void* x_perm, const int32_t* offsets, co
   // Tile shape: single-CTA 128x256 tiles unless the caller asks for CTA pairs
   // (256x256, each CTA of the pair stages half of the B tile).
   const bool pair = c.gemm_tiles == MOE_GEMM_TILES_PAIR;
-  CUtensorMap a1, b1, a2, b2;
+  CUtensorMap a1, b1, a2, b2, d1, d2;
   const bool gather = gather_rows != nullptr && !pair;
   int rc = gather ? make_map(&a1, gather_src, c.T, d, 1) : make_map(&a1, x_perm, rows_max, d, kTileM);
   if (rc == MOE_OK) rc = make_map(&b1, w13, static_cast<uint64_t>(E) * 2 * F, d, pair ? 128 : kGemmTileN);
   if (rc == MOE_OK) rc = make_map(&a2, h_mid, rows_max, F, kTileM);
   if (rc == MOE_OK) rc = make_map(&b2, w_down, static_cast<uint64_t>(E) * d, F, pair ? 128 : kGemmTileN);
+  if (rc == MOE_OK) rc = make_map_store(&d1, h_mid, rows_max, F);
+  if (rc == MOE_OK) rc = make_map_store(&d2, y_perm, rows_max, d);
   if (rc != MOE_OK) return rc;
   cudaError_t e =
       pair ? launch_grouped_gemm_pair(a1, b1, true, offsets, E, d, 2 * F, F / 128, F, F, h_mid, status, pdl, s)
            : launch_grouped_gemm_tc(a1, b1, true, offsets, E, d, 2 * F, F / 128, F, F, h_mid,
-                                    gather ? gather_rows : nullptr, status, pdl, s, preact);
+                                    gather ? gather_rows : nullptr, status, pdl, s, preact, &d1);
   if (e != cudaSuccess) return MOE_ERR_CUDA;
   const int n2 = (d + kGemmTileN - 1) / kGemmTileN;
   if (fc != nullptr)
@@ -450,7 +467,8 @@ int ffn_impl(const moe_config& c, const void* x_perm, const int32_t* offsets, co
                                     fc->pair_cnt, fc->y, c.k, status, true, s);
   else
     e = pair ? launch_grouped_gemm_pair(a2, b2, false, offsets, E, F, d, n2, d, d, y_perm, status, true, s)
-             : launch_grouped_gemm_tc(a2, b2, false, offsets, E, F, d, n2, d, d, y_perm, nullptr, status, true, s);
+             : launch_grouped_gemm_tc(a2, b2, false, offsets, E, F, d, n2, d, d, y_perm, nullptr, status, true, s,
+                                      nullptr, &d2);
   return cuda_rc(e);
 }
 

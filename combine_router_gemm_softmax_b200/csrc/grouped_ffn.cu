@@ -55,10 +55,15 @@ constexpr uint32_t kBBytes = kBN * kBK * 2;
 constexpr uint32_t kStageBytes = kABytes + kBBytes;
 constexpr uint32_t kTmemCols = 2 * kBN;
 
+// Epilogue store staging: one 32-row x 32-column bf16 block (2 KB) per
+// epilogue warp, in the 64-byte-swizzled layout of the store tensor map's box.
+constexpr uint32_t kStgBytes = 32 * 32 * 2;
+
 constexpr size_t gemm_smem_bytes() {
-  return 1024 + kStages * static_cast<size_t>(kStageBytes) + (2 * kStages + 5) * 8 + 16 + 2 * (kMaxE + 1) * 4 +
-         kBM * 4;
+  return 1024 + kStages * static_cast<size_t>(kStageBytes) + kEpiWarps * kStgBytes + (2 * kStages + 5) * 8 + 16 +
+         2 * (kMaxE + 1) * 4 + kBM * 4;
 }
+static_assert(gemm_smem_bytes() <= 227 * 1024, "shared memory");
 
 struct GemmArgs {
   const int32_t* offsets;
@@ -111,6 +116,11 @@ struct GemmArgs {
   // read by the kEpiDhSwiGLUBwd epilogue.
   __nv_bfloat16* preact;
   int preact_ld;
+  // kEpiSwiGLU / kEpiStore: D is also described by the kernel's tm_d (bf16,
+  // boxes of 32 rows x 32 columns, 64-byte swizzle). A warp whose 32 rows of
+  // the tile all belong to the expert stores each 32-column block through its
+  // staging buffer with one TMA store; other warps store row by row.
+  int tma_store;
 };
 
 // Epilogues and tile groupings of grouped_gemm_kernel.
@@ -150,15 +160,36 @@ MOE_DEV void decode_tile(long long tile, int m_total, int n_tiles, int band_rows
   m = gm - prefix[lo];
 }
 
+// One warp's 32 rows x 32 bf16 columns (p: this lane's row, 64 bytes) to D
+// through the warp's staging buffer and a TMA store at (x, y). The previous
+// store from the buffer must have read it first; lane 0 owns the warp's
+// bulk groups.
+MOE_DEV void stage_store(uint8_t* stg, const uint32_t (&p)[16], int lane, const CUtensorMap* tm_d, int x, int y) {
+  if (lane == 0) bulk_wait_read<0>();
+  __syncwarp();
+  uint8_t* rowp = stg + lane * 64;
+  const int sw = (lane >> 1) & 3;  // 64-byte swizzle: 16-byte chunk j of row r sits at chunk j ^ ((r >> 1) & 3)
+#pragma unroll
+  for (int j = 0; j < 4; ++j)
+    *reinterpret_cast<uint4*>(rowp + ((j ^ sw) << 4)) = make_uint4(p[4 * j], p[4 * j + 1], p[4 * j + 2], p[4 * j + 3]);
+  fence_proxy_async_shared();
+  __syncwarp();
+  if (lane == 0) {
+    tma_store_2d(tm_d, stg, x, y);
+    bulk_commit();
+  }
+}
+
 template <int kEpi, int kMode>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
-                        const GemmArgs a) {
+                        const __grid_constant__ CUtensorMap tm_d, const GemmArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align_1024(smem_raw);
   uint8_t* sA = smem;
   uint8_t* sB = smem + kStages * kABytes;
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kStages * kStageBytes);
+  uint8_t* stg_all = smem + kStages * kStageBytes;  // kEpiWarps x kStgBytes, 1024-aligned
+  uint64_t* full = reinterpret_cast<uint64_t*>(stg_all + kEpiWarps * kStgBytes);
   uint64_t* empty = full + kStages;
   uint64_t* tfull = empty + kStages;
   uint64_t* tempty = tfull + 2;
@@ -189,6 +220,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     fence_mbar_init();
     tma_prefetch_desc(&tm_a);
     tma_prefetch_desc(&tm_b);
+    if (a.tma_store) tma_prefetch_desc(&tm_d);
   }
   pdl_wait();  // offsets and the A rows come from the kernels before this one
   for (int e = threadIdx.x; e <= E; e += blockDim.x) s_off[e] = a.offsets[e];
@@ -354,6 +386,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const int q = warp & 3;            // TMEM lane quadrant this warp may read
     const int half = (warp - 2) >> 2;  // which half of the tile's columns it drains
     const int row = q * 32 + lane;
+    uint8_t* stg = stg_all + (warp - 2) * kStgBytes;
     int local = 0;
     for (long long tile = blockIdx.x; tile < total; tile += gridDim.x, ++local) {
       int e, m, n, kb0, kb1;
@@ -394,6 +427,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       const int rows_valid = min(kBM, s_off[e + 1] - s_off[e] - m * kBM);
       const bool valid = row < rows_valid;
       const size_t grow = static_cast<size_t>(s_off[e] + m * kBM + row);
+      // this warp's 32 rows all belong to the expert: stage and TMA-store them
+      const bool staged = a.tma_store != 0 && q * 32 + 32 <= rows_valid;
+      const int srow = s_off[e] + m * kBM + q * 32;
       if constexpr (kEpi == kEpiSwiGLUBwd) {
         // columns [0,128) of the tile are the gate pre-activations a, [128,256)
         // the matching up pre-activations u, for channels n*128 + [0,128):
@@ -473,9 +509,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
               const float h1 = silu_f(__uint_as_float(g[2 * i + 1])) * __uint_as_float(u[2 * i + 1]);
               p[i] = pack_bf16x2(h0, h1);
             }
-            uint4* dst = reinterpret_cast<uint4*>(out + c);
+            if (staged) {
+              stage_store(stg, p, lane, &tm_d, n * (kBN / 2) + c, srow);
+            } else {
+              uint4* dst = reinterpret_cast<uint4*>(out + c);
 #pragma unroll
-            for (int i = 0; i < 4; ++i) dst[i] = make_uint4(p[4 * i], p[4 * i + 1], p[4 * i + 2], p[4 * i + 3]);
+              for (int i = 0; i < 4; ++i) dst[i] = make_uint4(p[4 * i], p[4 * i + 1], p[4 * i + 2], p[4 * i + 3]);
+            }
             if (a.preact != nullptr) {  // the pre-activations themselves, for the backward
               uint32_t pg[16], pu[16];
 #pragma unroll
@@ -649,9 +689,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             uint32_t p[16];
 #pragma unroll
             for (int i = 0; i < 16; ++i) p[i] = pack_bf16x2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
-            uint4* dst = reinterpret_cast<uint4*>(out + c);
+            if (staged) {
+              stage_store(stg, p, lane, &tm_d, n * kBN + c, srow);
+            } else {
+              uint4* dst = reinterpret_cast<uint4*>(out + c);
 #pragma unroll
-            for (int i = 0; i < 4; ++i) dst[i] = make_uint4(p[4 * i], p[4 * i + 1], p[4 * i + 2], p[4 * i + 3]);
+              for (int i = 0; i < 4; ++i) dst[i] = make_uint4(p[4 * i], p[4 * i + 1], p[4 * i + 2], p[4 * i + 3]);
+            }
           }
         }
       }
@@ -661,6 +705,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
   }
   __syncwarp();
+  if (warp >= 2 && lane == 0) bulk_wait_all();  // the epilogue's staged stores have completed
 
   tc_fence_before();
   __syncthreads();
@@ -1072,7 +1117,8 @@ std::atomic<int> g_stall_gemms{0};
 
 template <int kEpi, int kMode>
 cudaError_t launch_gemm_inst(const CUtensorMap& tm_a, const CUtensorMap& tm_b, GemmArgs a, bool pdl,
-                             cudaStream_t s) {
+                             cudaStream_t s, const CUtensorMap* tm_d = nullptr) {
+  a.tma_store = tm_d != nullptr ? 1 : 0;
   int left = g_stall_gemms.load();
   while (left > 0 && !g_stall_gemms.compare_exchange_weak(left, left - 1)) {
   }
@@ -1082,7 +1128,7 @@ cudaError_t launch_gemm_inst(const CUtensorMap& tm_a, const CUtensorMap& tm_b, G
                                          static_cast<int>(smem));
   if (err != cudaSuccess) return err;
   err = launch_kernel(grouped_gemm_kernel<kEpi, kMode>, dim3(device_sm_count()), dim3(kGemmThreads), smem, s, pdl, 1,
-                      tm_a, tm_b, a);
+                      tm_a, tm_b, tm_d != nullptr ? *tm_d : tm_a, a);
   if (err != cudaSuccess) return err;
   return cudaGetLastError();
 }
@@ -1092,13 +1138,13 @@ cudaError_t launch_gemm_inst(const CUtensorMap& tm_a, const CUtensorMap& tm_b, G
 cudaError_t launch_grouped_gemm_tc(const CUtensorMap& tm_a, const CUtensorMap& tm_b, bool swiglu,
                                    const int32_t* offsets, int E, int K, int n_per_expert, int n_tiles,
                                    int out_cols, int ldd, void* D, const int32_t* gather_rows, int32_t* status,
-                                   bool pdl, cudaStream_t s, void* preact) {
+                                   bool pdl, cudaStream_t s, void* preact, const CUtensorMap* tm_d) {
   GemmArgs a{offsets, E, K, n_per_expert, n_tiles, out_cols, ldd, static_cast<__nv_bfloat16*>(D), status,
              band_rows(kBM, K, 8, 32), gather_rows, nullptr, 0, nullptr, 0, nullptr, nullptr, 0};
   a.preact = static_cast<__nv_bfloat16*>(preact);
   a.preact_ld = n_per_expert;
-  return swiglu ? launch_gemm_inst<kEpiSwiGLU, kGroupRows>(tm_a, tm_b, a, pdl, s)
-                : launch_gemm_inst<kEpiStore, kGroupRows>(tm_a, tm_b, a, pdl, s);
+  return swiglu ? launch_gemm_inst<kEpiSwiGLU, kGroupRows>(tm_a, tm_b, a, pdl, s, tm_d)
+                : launch_gemm_inst<kEpiStore, kGroupRows>(tm_a, tm_b, a, pdl, s, tm_d);
 }
 
 void debug_stall_next_gemms(int n) { g_stall_gemms.store(n > 0 ? n : 0); }

@@ -121,6 +121,16 @@ MOE_DEV void tma_gather4(void* dst, const CUtensorMap* map, uint64_t* bar, int x
       : "memory");
 }
 
+// 2-D tile store shared -> global, tracked in this thread's bulk async-group
+// (bulk_commit / bulk_wait_read / bulk_wait_all). Coordinates are not
+// negative; x * element size is a multiple of 16 bytes.
+MOE_DEV void tma_store_2d(const CUtensorMap* map, const void* src, int x, int y) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(smem_addr(src)), "r"(x), "r"(y)
+               : "memory");
+}
+
 // Untiled bulk copies (TMA engine, no tensor map). Addresses 16-byte aligned,
 // sizes multiples of 16 bytes.
 MOE_DEV void bulk_load(void* smem_dst, const void* gsrc, uint32_t bytes, uint64_t* bar) {

@@ -56,10 +56,14 @@ cudaError_t launch_combine(int dtype, const void* y_perm, const int32_t* dest_ro
 // tm_a, whose box must then be 64 columns by one row.
 // preact (swiglu only, may be NULL): also store the gate/up pre-activations
 // [rows, n_per_expert] bf16 in w13's interleaved column order.
+// tm_d (may be NULL): D as a store tensor map (make_map_store: bf16, 32 x 32
+// boxes, 64-byte swizzle); the epilogue then writes whole 32-row blocks of
+// the tile with TMA stores.
 cudaError_t launch_grouped_gemm_tc(const CUtensorMap& tm_a, const CUtensorMap& tm_b, bool swiglu,
                                    const int32_t* offsets, int E, int K, int n_per_expert, int n_tiles,
                                    int out_cols, int ldd, void* D, const int32_t* gather_rows, int32_t* status,
-                                   bool pdl, cudaStream_t s, void* preact = nullptr);
+                                   bool pdl, cudaStream_t s, void* preact = nullptr,
+                                   const CUtensorMap* tm_d = nullptr);
 // The backward's dh_mid GEMM (dy_perm rows against W_down^T rows, K = d) with
 // the SwiGLU backward in its epilogue from the saved pre-activations
 // preact [rows, 2F]: writes dgu [rows, 2F] = [dgate | dup] (interleaved) and
