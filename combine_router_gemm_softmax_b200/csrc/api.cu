@@ -70,6 +70,21 @@ int make_map_store(CUtensorMap* m, const void* base, uint64_t rows, uint64_t col
   return r == CUDA_SUCCESS ? MOE_OK : MOE_ERR_CUDA;
 }
 
+// Row-major byte matrix [rows, cols] written by TMA stores: boxes of 32 rows x
+// 32 bytes, 32-byte swizzle (the MXFP8 GEMM epilogue's staging layout).
+int make_map_store_u8(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols) {
+  EncodeTiledFn enc = encode_fn();
+  if (enc == nullptr) return MOE_ERR_NO_DEVICE;
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {cols};
+  const cuuint32_t box[2] = {32, 32};
+  const cuuint32_t es[2] = {1, 1};
+  const CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, es,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_32B,
+                         CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? MOE_OK : MOE_ERR_CUDA;
+}
+
 // Row-major byte matrix [rows, cols] (E4M3 elements), box of box_rows x 128
 // columns, 128-byte swizzle.
 int make_map_u8(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows) {
@@ -416,17 +431,19 @@ int ffn_mx_impl(const moe_config& c, const void* x_perm, const int32_t* offsets,
   if (!x_quantized)
     e = launch_mx_quantize(x_perm, m.pad_rows, d, offsets, E, m.xq, m.xsf, m.row_blocks, m.counters, status, pdl, s);
   if (e != cudaSuccess) return MOE_ERR_CUDA;
-  CUtensorMap a1, b1, a2, b2;
+  CUtensorMap a1, b1, a2, b2, d1, d2;
   int rc = make_map_u8(&a1, m.xq, m.pad_rows, d, 128);
   if (rc == MOE_OK) rc = make_map_u8(&b1, w13q, b13.rows, d, 256);
   if (rc == MOE_OK) rc = make_map_u8(&a2, m.hq, m.pad_rows, F, 128);
   if (rc == MOE_OK) rc = make_map_u8(&b2, wdq, bd.rows, F, 256);
+  if (rc == MOE_OK) rc = make_map_store_u8(&d1, m.hq, m.pad_rows, F);
+  if (rc == MOE_OK) rc = make_map_store(&d2, y_perm, perm_rows(c), d);
   if (rc != MOE_OK) return rc;
   e = launch_grouped_gemm_mx(a1, b1, true, offsets, E, d, 2 * F, F, m.xsf, m.row_blocks, w13q + b13.q_bytes, m.hq,
-                             m.hsf, F, m.counters + 2, nullptr, 0, status, true, s);
+                             m.hsf, F, m.counters + 2, nullptr, 0, status, true, s, &d1);
   if (e != cudaSuccess) return MOE_ERR_CUDA;
   e = launch_grouped_gemm_mx(a2, b2, false, offsets, E, F, d, d, m.hsf, m.row_blocks, wdq + bd.q_bytes, nullptr,
-                             nullptr, 0, nullptr, y_perm, d, status, true, s);
+                             nullptr, 0, nullptr, y_perm, d, status, true, s, &d2);
   return cuda_rc(e);
 }
 
@@ -779,8 +796,11 @@ int32_t moe_layer_backward(const moe_config* cfg, const void* h, const void* w_r
       if (e != cudaSuccess) return MOE_ERR_CUDA;
     } else {
       // 2. dh_mid = dy_perm W_down (per expert), B = W_down^T rows
+      CUtensorMap td;
+      rc = make_map_store(&td, b.dh_mid, P, F);
+      if (rc != MOE_OK) return rc;
       e = launch_grouped_gemm_tc(ta, tb, false, f.offsets, E, d, F, (F + kGemmTileN - 1) / kGemmTileN, F, F,
-                                 b.dh_mid, nullptr, status_dev, false, s);
+                                 b.dh_mid, nullptr, status_dev, false, s, nullptr, &td);
       if (e != cudaSuccess) return MOE_ERR_CUDA;
       // 3. gate/up pre-activations recomputed from x_perm; SwiGLU backward in the
       //    epilogue, which also writes dgu transposed for the weight gradient
@@ -792,11 +812,13 @@ int32_t moe_layer_backward(const moe_config* cfg, const void* h, const void* w_r
       if (e != cudaSuccess) return MOE_ERR_CUDA;
     }
     // 4. dx_perm = dgu w13 (per expert), B = w13^T rows
+    CUtensorMap tdx;
     rc = make_map(&ta, b.dgu, P, 2 * F, kTileM);
     if (rc == MOE_OK) rc = make_map(&tb, w13_t, static_cast<uint64_t>(E) * d, 2 * F, kGemmTileN);
+    if (rc == MOE_OK) rc = make_map_store(&tdx, b.dx_perm, P, d);
     if (rc != MOE_OK) return rc;
     e = launch_grouped_gemm_tc(ta, tb, false, f.offsets, E, 2 * F, d, (d + kGemmTileN - 1) / kGemmTileN, d, d,
-                               b.dx_perm, nullptr, status_dev, false, s);
+                               b.dx_perm, nullptr, status_dev, false, s, nullptr, &tdx);
     if (e != cudaSuccess) return MOE_ERR_CUDA;
   }
   // 5. dh: expert rows back to their tokens plus the router-score term

@@ -160,24 +160,12 @@ MOE_DEV void decode_tile(long long tile, int m_total, int n_tiles, int band_rows
   m = gm - prefix[lo];
 }
 
-// One warp's 32 rows x 32 bf16 columns (p: this lane's row, 64 bytes) to D
-// through the warp's staging buffer and a TMA store at (x, y). The previous
-// store from the buffer must have read it first; lane 0 owns the warp's
-// bulk groups.
+// One warp's 32 rows x 32 bf16 columns (p: this lane's row) to D with a TMA
+// store through the warp's staging buffer.
 MOE_DEV void stage_store(uint8_t* stg, const uint32_t (&p)[16], int lane, const CUtensorMap* tm_d, int x, int y) {
-  if (lane == 0) bulk_wait_read<0>();
-  __syncwarp();
-  uint8_t* rowp = stg + lane * 64;
-  const int sw = (lane >> 1) & 3;  // 64-byte swizzle: 16-byte chunk j of row r sits at chunk j ^ ((r >> 1) & 3)
-#pragma unroll
-  for (int j = 0; j < 4; ++j)
-    *reinterpret_cast<uint4*>(rowp + ((j ^ sw) << 4)) = make_uint4(p[4 * j], p[4 * j + 1], p[4 * j + 2], p[4 * j + 3]);
-  fence_proxy_async_shared();
-  __syncwarp();
-  if (lane == 0) {
-    tma_store_2d(tm_d, stg, x, y);
-    bulk_commit();
-  }
+  const uint4 v[4] = {make_uint4(p[0], p[1], p[2], p[3]), make_uint4(p[4], p[5], p[6], p[7]),
+                      make_uint4(p[8], p[9], p[10], p[11]), make_uint4(p[12], p[13], p[14], p[15])};
+  stage_store_rows<64>(stg, v, lane, tm_d, x, y);
 }
 
 template <int kEpi, int kMode>

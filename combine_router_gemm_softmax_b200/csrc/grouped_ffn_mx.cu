@@ -73,10 +73,15 @@ constexpr uint32_t kSfaCol = 448;
 constexpr uint32_t kSfbCol = 452;
 constexpr uint32_t kMxTmemCols = 512;
 
+// Epilogue store staging: one 2 KB block per epilogue warp (32 rows x 32 bf16
+// for GEMM2, 32 rows x 32 E4M3 bytes for GEMM1).
+constexpr uint32_t kMxStgBytes = 2048;
+
 constexpr size_t mx_smem_bytes() {
   return 1024 + kMxStages * static_cast<size_t>(kMxABytes + kMxBBytes + kSfaBytes + kSfbBytes) +
-         (2 * kMxStages + 4) * 8 + 16 + 2 * (kMaxE + 1) * 4;
+         kMxEpiWarps * kMxStgBytes + (2 * kMxStages + 4) * 8 + 16 + 2 * (kMaxE + 1) * 4;
 }
+static_assert(mx_smem_bytes() <= 227 * 1024, "shared memory");
 
 // ------------------------------------------------------------------ quantisation
 // E of the shared scale from the block's largest magnitude: floor(log2 amax) - 8
@@ -315,6 +320,10 @@ struct MxGemmArgs {
   __nv_bfloat16* D;
   int ldd;
   int32_t* status;
+  // The output (q_out for GEMM1, D for GEMM2) is also the kernel's tm_d: a
+  // warp whose 32 rows of the tile are all to be written stores each
+  // 32-column block with one TMA store through its staging buffer.
+  int tma_store;
 };
 
 // tile -> (expert, row tile within the expert, column tile); bands of row tiles
@@ -342,12 +351,13 @@ MOE_DEV void mx_decode_tile(long long tile, int m_total, int n_tiles, int band_r
 template <bool kSwiGLUQuant>
 __global__ void __launch_bounds__(kMxThreads, 1)
     grouped_gemm_mx_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
-                           const MxGemmArgs a) {
+                           const __grid_constant__ CUtensorMap tm_d, const MxGemmArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align_1024(smem_raw);
   uint8_t* sA = smem;
   uint8_t* sB = sA + kMxStages * kMxABytes;
-  uint8_t* sSFA = sB + kMxStages * kMxBBytes;
+  uint8_t* stg_all = sB + kMxStages * kMxBBytes;  // kMxEpiWarps x kMxStgBytes, 1024-aligned
+  uint8_t* sSFA = stg_all + kMxEpiWarps * kMxStgBytes;
   uint8_t* sSFB = sSFA + kMxStages * kSfaBytes;
   uint64_t* full = reinterpret_cast<uint64_t*>(sSFB + kMxStages * kSfbBytes);
   uint64_t* empty = full + kMxStages;
@@ -378,6 +388,7 @@ __global__ void __launch_bounds__(kMxThreads, 1)
     fence_mbar_init();
     tma_prefetch_desc(&tm_a);
     tma_prefetch_desc(&tm_b);
+    if (a.tma_store) tma_prefetch_desc(&tm_d);
   }
   pdl_wait();  // offsets and the A rows come from the kernels before this one
   for (int e = threadIdx.x; e <= E; e += blockDim.x) s_off[e] = a.offsets[e];
@@ -481,6 +492,7 @@ __global__ void __launch_bounds__(kMxThreads, 1)
     const int q = warp & 3;            // TMEM lane quadrant this warp may read
     const int half = (warp - 2) >> 2;  // chunks half, half + 2, ... of the tile's column order
     const int row = q * 32 + lane;
+    uint8_t* stg = stg_all + (warp - 2) * kMxStgBytes;
     int local = 0;
     int n_sat = 0, n_under = 0;
     for (long long tile = blockIdx.x; tile < total; tile += gridDim.x, ++local) {
@@ -520,14 +532,19 @@ __global__ void __launch_bounds__(kMxThreads, 1)
           for (int j = 0; j < 32; ++j) h[j] = silu_mx(__uint_as_float(g[j])) * __uint_as_float(u[j]);
           uint4 out[2];
           const uint32_t byte = mx_quantize_block(h, out, n_sat, n_under);
-          uint4* dst = reinterpret_cast<uint4*>(qout + c);
-          dst[0] = out[0];
-          dst[1] = out[1];
+          if (a.tma_store) {
+            stage_store_rows<32>(stg, out, lane, &tm_d, n * (kMxBN / 2) + c, static_cast<int>(prow - lane));
+          } else {
+            uint4* dst = reinterpret_cast<uint4*>(qout + c);
+            dst[0] = out[0];
+            dst[1] = out[1];
+          }
           sfo[c >> 5] = static_cast<uint8_t>(byte);
         }
       } else {
         const int rows_valid = min(kMxBM, s_off[e + 1] - s_off[e] - m * kMxBM);
         const bool valid = row < rows_valid;
+        const bool staged = a.tma_store != 0 && q * 32 + 32 <= rows_valid;
         __nv_bfloat16* out = a.D + static_cast<size_t>(s_off[e] + m * kMxBM + row) * a.ldd + n * kMxBN;
 #pragma unroll 1
         for (int i = half; i < 8; i += 2) {
@@ -542,9 +559,15 @@ __global__ void __launch_bounds__(kMxThreads, 1)
 #pragma unroll
               for (int j = 0; j < 16; ++j)
                 p[j] = pack_bf16x2(__uint_as_float(v[2 * j]), __uint_as_float(v[2 * j + 1]));
-              uint4* dst = reinterpret_cast<uint4*>(out + c);
+              const uint4 pv[4] = {make_uint4(p[0], p[1], p[2], p[3]), make_uint4(p[4], p[5], p[6], p[7]),
+                                   make_uint4(p[8], p[9], p[10], p[11]), make_uint4(p[12], p[13], p[14], p[15])};
+              if (staged) {
+                stage_store_rows<64>(stg, pv, lane, &tm_d, n * kMxBN + c, s_off[e] + m * kMxBM + q * 32);
+              } else {
+                uint4* dst = reinterpret_cast<uint4*>(out + c);
 #pragma unroll
-              for (int j = 0; j < 4; ++j) dst[j] = make_uint4(p[4 * j], p[4 * j + 1], p[4 * j + 2], p[4 * j + 3]);
+                for (int j = 0; j < 4; ++j) dst[j] = pv[j];
+              }
             }
           }
           if (i < 2) {  // this warp's chunk of the shared columns is drained
@@ -556,6 +579,7 @@ __global__ void __launch_bounds__(kMxThreads, 1)
       }
     }
     if constexpr (kSwiGLUQuant) mx_report(n_sat, n_under, a.counts, a.status);
+    if (lane == 0) bulk_wait_all();  // this warp's staged stores have completed
   }
   __syncwarp();
 
@@ -725,8 +749,10 @@ cudaError_t launch_mx_dispatch(const void* h, int T, int d, int k, const int32_t
 cudaError_t launch_grouped_gemm_mx(const CUtensorMap& tm_a, const CUtensorMap& tm_b, bool swiglu_quant,
                                    const int32_t* offsets, int E, int K, int n_per_expert, int out_cols,
                                    const void* sfa, int ra_blocks, const void* sfb, void* q_out, void* sf_out, int ldq,
-                                   uint32_t* counts, void* D, int ldd, int32_t* status, bool pdl, cudaStream_t s) {
+                                   uint32_t* counts, void* D, int ldd, int32_t* status, bool pdl, cudaStream_t s,
+                                   const CUtensorMap* tm_d) {
   MxGemmArgs a{};
+  a.tma_store = tm_d != nullptr ? 1 : 0;
   a.offsets = offsets;
   a.E = E;
   a.K = K;
@@ -752,13 +778,13 @@ cudaError_t launch_grouped_gemm_mx(const CUtensorMap& tm_a, const CUtensorMap& t
                                static_cast<int>(smem));
     if (err == cudaSuccess)
       err = launch_kernel(grouped_gemm_mx_kernel<true>, dim3(device_sm_count()), dim3(kMxThreads), smem, s, pdl, 1,
-                          tm_a, tm_b, a);
+                          tm_a, tm_b, tm_d != nullptr ? *tm_d : tm_a, a);
   } else {
     err = cudaFuncSetAttribute(grouped_gemm_mx_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                static_cast<int>(smem));
     if (err == cudaSuccess)
       err = launch_kernel(grouped_gemm_mx_kernel<false>, dim3(device_sm_count()), dim3(kMxThreads), smem, s, pdl, 1,
-                          tm_a, tm_b, a);
+                          tm_a, tm_b, tm_d != nullptr ? *tm_d : tm_a, a);
   }
   return err != cudaSuccess ? err : cudaGetLastError();
 }

@@ -161,6 +161,31 @@ MOE_DEV void bulk_wait_read() {
 // Wait until every committed bulk group has completed.
 MOE_DEV void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
+// One warp's block of 32 rows x kRowBytes (64: 32 bf16, or 32: 32 bytes) to
+// global memory with a TMA store at (x, y): lane r writes its row v into the
+// warp's staging buffer `stg` in the swizzled layout of the store map's box
+// (64-byte swizzle: 16-byte chunk j of row r at chunk j ^ ((r >> 1) & 3);
+// 32-byte swizzle: at j ^ ((r >> 2) & 1)), then lane 0 issues the store. The
+// buffer (512-byte aligned) is rewritten only after the previous store from
+// it has read it; lane 0 owns the warp's bulk groups.
+template <int kRowBytes>
+MOE_DEV void stage_store_rows(uint8_t* stg, const uint4 (&v)[kRowBytes / 16], int lane, const CUtensorMap* tm, int x,
+                              int y) {
+  static_assert(kRowBytes == 64 || kRowBytes == 32, "row bytes");
+  if (lane == 0) bulk_wait_read<0>();
+  __syncwarp();
+  uint8_t* rowp = stg + lane * kRowBytes;
+  const int sw = kRowBytes == 64 ? (lane >> 1) & 3 : (lane >> 2) & 1;
+#pragma unroll
+  for (int j = 0; j < kRowBytes / 16; ++j) *reinterpret_cast<uint4*>(rowp + ((j ^ sw) << 4)) = v[j];
+  fence_proxy_async_shared();
+  __syncwarp();
+  if (lane == 0) {
+    tma_store_2d(tm, stg, x, y);
+    bulk_commit();
+  }
+}
+
 // ------------------------------------------------------------------ tcgen05
 MOE_DEV void tmem_alloc(uint32_t* dst_smem, uint32_t ncols) {  // whole warp
   asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_addr(dst_smem)),

@@ -130,7 +130,8 @@ cudaError_t launch_mx_dispatch(const void* h, int T, int d, int k, const int32_t
 cudaError_t launch_grouped_gemm_mx(const CUtensorMap& tm_a, const CUtensorMap& tm_b, bool swiglu_quant,
                                    const int32_t* offsets, int E, int K, int n_per_expert, int out_cols,
                                    const void* sfa, int ra_blocks, const void* sfb, void* q_out, void* sf_out, int ldq,
-                                   uint32_t* counts, void* D, int ldd, int32_t* status, bool pdl, cudaStream_t s);
+                                   uint32_t* counts, void* D, int ldd, int32_t* status, bool pdl, cudaStream_t s,
+                                   const CUtensorMap* tm_d = nullptr);
 
 // backward.cu
 cudaError_t launch_combine_bwd(const void* dy, const void* y_perm, const int32_t* dest_row, const float* gate,
