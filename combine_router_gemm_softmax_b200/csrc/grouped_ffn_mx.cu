@@ -60,8 +60,10 @@ constexpr int kMxBN = 256;
 constexpr int kMxBK = 128;  // elements (= bytes) of K per stage
 constexpr int kMxStages = 4;
 // warp 0: TMA producer, warp 1: TMEM allocation and MMA issue, warps 2..9:
-// epilogue, two per TMEM lane quadrant, each draining half of a tile
-constexpr int kMxThreads = 320;
+// epilogue, two per TMEM lane quadrant, each draining half of a tile, warp
+// 10: copies each stage's scale atoms into TMEM (a ring of four column sets)
+// and signals the MMA thread through sf_full when they have landed
+constexpr int kMxThreads = 352;
 constexpr int kMxEpiWarps = 8;
 constexpr uint32_t kMxABytes = kMxBM * kMxBK;   // 16 KB
 constexpr uint32_t kMxBBytes = kMxBN * kMxBK;   // 32 KB
@@ -69,9 +71,9 @@ constexpr uint32_t kSfaBytes = 512;
 constexpr uint32_t kSfbBytes = 1024;
 constexpr uint32_t kMxStageTx = kMxABytes + kMxBBytes + kSfaBytes + kSfbBytes;
 constexpr uint32_t kAcc1Col = 192;   // second accumulator; [192, 256) is shared
-constexpr uint32_t kSfaCol = 448;
-constexpr uint32_t kSfbCol = 452;
+constexpr uint32_t kSfaCol = 448;    // stage s: SFA at 448 + 12 s, SFB at 452 + 12 s (8 columns)
 constexpr uint32_t kMxTmemCols = 512;
+static_assert(kSfaCol + 12 * kMxStages <= kMxTmemCols, "scale ring");
 
 // Epilogue store staging: one 2 KB block per epilogue warp (32 rows x 32 bf16
 // for GEMM2, 32 rows x 32 E4M3 bytes for GEMM1).
@@ -79,7 +81,7 @@ constexpr uint32_t kMxStgBytes = 2048;
 
 constexpr size_t mx_smem_bytes() {
   return 1024 + kMxStages * static_cast<size_t>(kMxABytes + kMxBBytes + kSfaBytes + kSfbBytes) +
-         kMxEpiWarps * kMxStgBytes + (2 * kMxStages + 4) * 8 + 16 + 2 * (kMaxE + 1) * 4;
+         kMxEpiWarps * kMxStgBytes + (3 * kMxStages + 5) * 8 + 16 + 2 * (kMaxE + 1) * 4;
 }
 static_assert(mx_smem_bytes() <= 227 * 1024, "shared memory");
 
@@ -364,7 +366,9 @@ __global__ void __launch_bounds__(kMxThreads, 1)
   uint64_t* tfull = empty + kMxStages;
   uint64_t* ovl = tfull + 2;
   uint64_t* drain = ovl + 1;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* sf_full = drain + 1;
+  uint64_t* cp_drain = sf_full + kMxStages;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(cp_drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   int* consumed_slot = reinterpret_cast<int*>(tmem_slot + 2);
   int* s_off = reinterpret_cast<int*>(tmem_slot + 4);  // [E+1]
@@ -383,6 +387,8 @@ __global__ void __launch_bounds__(kMxThreads, 1)
     mbar_init(&tfull[1], 1);
     mbar_init(ovl, kMxEpiWarps);
     mbar_init(drain, 1);
+    for (int s = 0; s < kMxStages; ++s) mbar_init(&sf_full[s], 1);
+    mbar_init(cp_drain, 1);
     *abort_flag = 0;
     *consumed_slot = 0;
     fence_mbar_init();
@@ -463,16 +469,19 @@ __global__ void __launch_bounds__(kMxThreads, 1)
             stop = true;
             break;
           }
+          if (!mbar_wait(&sf_full[stage], phase, abort_flag)) {
+            *abort_flag = 1;
+            stop = true;
+            break;
+          }
           tc_fence_after();
-          tmem_cp_32x128_x4(tmem + kSfaCol, sf_copy_desc(smem_addr(sSFA + stage * kSfaBytes)));
-          tmem_cp_32x128_x4(tmem + kSfbCol, sf_copy_desc(smem_addr(sSFB + stage * kSfbBytes)));
-          tmem_cp_32x128_x4(tmem + kSfbCol + 4, sf_copy_desc(smem_addr(sSFB + stage * kSfbBytes + 512)));
+          const uint32_t sf_a = tmem + kSfaCol + 12u * stage, sf_b = sf_a + 4;
           const uint32_t sa = smem_addr(sA + stage * kMxABytes);
           const uint32_t sb = smem_addr(sB + stage * kMxBBytes);
 #pragma unroll
           for (uint32_t kk = 0; kk < kMxBK / 32; ++kk)
             umma_mxf8(d_tmem, sw128_kmajor_desc(sa + kk * 32), sw128_kmajor_desc(sb + kk * 32),
-                      idesc_mxf8(kMxBM, kMxBN, kk), (tmem + kSfaCol) | (kk << 30), (tmem + kSfbCol) | (kk << 30),
+                      idesc_mxf8(kMxBM, kMxBN, kk), sf_a | (kk << 30), sf_b | (kk << 30),
                       (kt | kk) != 0);
           umma_commit(&empty[stage]);
           ++consumed;
@@ -486,6 +495,34 @@ __global__ void __launch_bounds__(kMxThreads, 1)
       *consumed_slot = consumed;
       umma_commit(drain);
       mbar_wait(drain, 0, nullptr);
+    }
+  } else if (warp == 2 + kMxEpiWarps) {
+    if (lane == 0) {
+      // ---------------------------------------------------------------- scale copier
+      int stage = 0;
+      uint32_t phase = 0;
+      bool stop = false;
+      for (long long tile = blockIdx.x; tile < total && !stop; tile += gridDim.x) {
+        for (int kt = 0; kt < nkt; ++kt) {
+          if (!mbar_wait(&full[stage], phase, abort_flag)) {
+            *abort_flag = 1;
+            stop = true;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sf_a = tmem + kSfaCol + 12u * stage, sf_b = sf_a + 4;
+          tmem_cp_32x128_x4(sf_a, sf_copy_desc(smem_addr(sSFA + stage * kSfaBytes)));
+          tmem_cp_32x128_x4(sf_b, sf_copy_desc(smem_addr(sSFB + stage * kSfbBytes)));
+          tmem_cp_32x128_x4(sf_b + 4, sf_copy_desc(smem_addr(sSFB + stage * kSfbBytes + 512)));
+          umma_commit(&sf_full[stage]);
+          if (++stage == kMxStages) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+      }
+      umma_commit(cp_drain);
+      mbar_wait(cp_drain, 0, nullptr);
     }
   } else {
     // ---------------------------------------------------------------- epilogue
