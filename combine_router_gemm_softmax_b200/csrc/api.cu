@@ -791,8 +791,11 @@ int32_t moe_layer_backward(const moe_config* cfg, const void* h, const void* w_r
       // 2+3. dL/dh_mid = dy_perm W_down (per expert) with the SwiGLU backward in
       //      the epilogue, from the pre-activations the forward kept: writes
       //      dgu and its transposed copy; no recompute of the gate/up GEMM
+      CUtensorMap tdg;
+      rc = make_map_store(&tdg, b.dgu, P, 2 * F);
+      if (rc != MOE_OK) return rc;
       e = launch_grouped_gemm_dh_swiglu_bwd(ta, tb, f.offsets, E, d, F, f.preact, b.dgu, b.dgu_t, b.col_off,
-                                            b.ppad_max, status_dev, false, s);
+                                            b.ppad_max, status_dev, false, s, &tdg);
       if (e != cudaSuccess) return MOE_ERR_CUDA;
     } else {
       // 2. dh_mid = dy_perm W_down (per expert), B = W_down^T rows
@@ -807,8 +810,11 @@ int32_t moe_layer_backward(const moe_config* cfg, const void* h, const void* w_r
       rc = make_map(&ta, f.x_perm, P, d, kTileM);
       if (rc == MOE_OK) rc = make_map(&tb, w13_packed, static_cast<uint64_t>(E) * 2 * F, d, kGemmTileN);
       if (rc != MOE_OK) return rc;
+      CUtensorMap tdg;
+      if (rc == MOE_OK) rc = make_map_store(&tdg, b.dgu, P, 2 * F);
+      if (rc != MOE_OK) return rc;
       e = launch_grouped_gemm_swiglu_bwd(ta, tb, f.offsets, E, d, F, b.dgu, b.dh_mid, b.dgu_t, b.col_off,
-                                         b.ppad_max, status_dev, false, s);
+                                         b.ppad_max, status_dev, false, s, &tdg);
       if (e != cudaSuccess) return MOE_ERR_CUDA;
     }
     // 4. dx_perm = dgu w13 (per expert), B = w13^T rows

@@ -460,12 +460,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
               pg[i] = pack_bf16x2(dg2[0], dg2[1]);
               pu[i] = pack_bf16x2(du2[0], du2[1]);
             }
-            uint4* dg_dst = reinterpret_cast<uint4*>(out + c);
-            uint4* du_dst = reinterpret_cast<uint4*>(out + kBN / 2 + c);
+            if (staged) {
+              stage_store(stg, pg, lane, &tm_d, n * kBN + c, srow);
+              stage_store(stg, pu, lane, &tm_d, n * kBN + kBN / 2 + c, srow);
+            } else {
+              uint4* dg_dst = reinterpret_cast<uint4*>(out + c);
+              uint4* du_dst = reinterpret_cast<uint4*>(out + kBN / 2 + c);
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              dg_dst[i] = make_uint4(pg[4 * i], pg[4 * i + 1], pg[4 * i + 2], pg[4 * i + 3]);
-              du_dst[i] = make_uint4(pu[4 * i], pu[4 * i + 1], pu[4 * i + 2], pu[4 * i + 3]);
+              for (int i = 0; i < 4; ++i) {
+                dg_dst[i] = make_uint4(pg[4 * i], pg[4 * i + 1], pg[4 * i + 2], pg[4 * i + 3]);
+                du_dst[i] = make_uint4(pu[4 * i], pu[4 * i + 1], pu[4 * i + 2], pu[4 * i + 3]);
+              }
             }
           }
           if (twrite) {
@@ -567,12 +572,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
               pg[i] = pack_bf16x2(dg2[0], dg2[1]);
               pu[i] = pack_bf16x2(du2[0], du2[1]);
             }
-            uint4* dg_dst = reinterpret_cast<uint4*>(out + c);
-            uint4* du_dst = reinterpret_cast<uint4*>(out + kBN / 2 + c);
+            if (staged) {
+              stage_store(stg, pg, lane, &tm_d, b * kBN + c, srow);
+              stage_store(stg, pu, lane, &tm_d, b * kBN + kBN / 2 + c, srow);
+            } else {
+              uint4* dg_dst = reinterpret_cast<uint4*>(out + c);
+              uint4* du_dst = reinterpret_cast<uint4*>(out + kBN / 2 + c);
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              dg_dst[i] = make_uint4(pg[4 * i], pg[4 * i + 1], pg[4 * i + 2], pg[4 * i + 3]);
-              du_dst[i] = make_uint4(pu[4 * i], pu[4 * i + 1], pu[4 * i + 2], pu[4 * i + 3]);
+              for (int i = 0; i < 4; ++i) {
+                dg_dst[i] = make_uint4(pg[4 * i], pg[4 * i + 1], pg[4 * i + 2], pg[4 * i + 3]);
+                du_dst[i] = make_uint4(pu[4 * i], pu[4 * i + 1], pu[4 * i + 2], pu[4 * i + 3]);
+              }
             }
           }
           if (twrite) {
@@ -1155,23 +1165,23 @@ cudaError_t launch_grouped_gemm_combine(const CUtensorMap& tm_a, const CUtensorM
 cudaError_t launch_grouped_gemm_dh_swiglu_bwd(const CUtensorMap& tm_a, const CUtensorMap& tm_b,
                                               const int32_t* offsets, int E, int K, int F, const void* preact,
                                               void* dgu, void* dgu_t, const int32_t* col_off, int ldt, int32_t* status,
-                                              bool pdl, cudaStream_t s) {
+                                              bool pdl, cudaStream_t s, const CUtensorMap* tm_d) {
   GemmArgs a{offsets, E, K, F, (F + kBN - 1) / kBN, F, 2 * F, static_cast<__nv_bfloat16*>(dgu), status,
              band_rows(kBM, K, 8, 32), nullptr, nullptr, 0, nullptr, 0, static_cast<__nv_bfloat16*>(dgu_t), col_off,
              ldt};
   a.preact = static_cast<__nv_bfloat16*>(const_cast<void*>(preact));
   a.preact_ld = 2 * F;
-  return launch_gemm_inst<kEpiDhSwiGLUBwd, kGroupRows>(tm_a, tm_b, a, pdl, s);
+  return launch_gemm_inst<kEpiDhSwiGLUBwd, kGroupRows>(tm_a, tm_b, a, pdl, s, tm_d);
 }
 
 cudaError_t launch_grouped_gemm_swiglu_bwd(const CUtensorMap& tm_a, const CUtensorMap& tm_b, const int32_t* offsets,
                                            int E, int K, int F, void* dgu, const void* dh_mid, void* dgu_t,
                                            const int32_t* col_off, int ldt, int32_t* status, bool pdl,
-                                           cudaStream_t s) {
+                                           cudaStream_t s, const CUtensorMap* tm_d) {
   GemmArgs a{offsets, E, K, 2 * F, 2 * F / kBN, 2 * F, 2 * F, static_cast<__nv_bfloat16*>(dgu), status,
              band_rows(kBM, K, 8, 32), nullptr, static_cast<const __nv_bfloat16*>(dh_mid), F, nullptr, 0,
              static_cast<__nv_bfloat16*>(dgu_t), col_off, ldt};
-  return launch_gemm_inst<kEpiSwiGLUBwd, kGroupRows>(tm_a, tm_b, a, pdl, s);
+  return launch_gemm_inst<kEpiSwiGLUBwd, kGroupRows>(tm_a, tm_b, a, pdl, s, tm_d);
 }
 
 cudaError_t launch_grouped_gemm_wgrad(const CUtensorMap& tm_a, const CUtensorMap& tm_b, const int32_t* col_offsets,

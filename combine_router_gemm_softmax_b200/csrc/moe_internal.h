@@ -71,7 +71,8 @@ cudaError_t launch_grouped_gemm_tc(const CUtensorMap& tm_a, const CUtensorMap& t
 cudaError_t launch_grouped_gemm_dh_swiglu_bwd(const CUtensorMap& tm_a, const CUtensorMap& tm_b,
                                               const int32_t* offsets, int E, int K, int F, const void* preact,
                                               void* dgu, void* dgu_t, const int32_t* col_off, int ldt, int32_t* status,
-                                              bool pdl, cudaStream_t s);
+                                              bool pdl, cudaStream_t s,
+                                              const CUtensorMap* tm_d = nullptr);
 // The down projection with the combine fused into its epilogue (k <= 2): y_perm
 // rows as launch_grouped_gemm_tc, and y [T, d] = sum over each token's kept
 // slots, in slot order, of gate * bf16 row (bit-identical to launch_combine).
@@ -92,7 +93,8 @@ void debug_stall_next_gemms(int n);
 cudaError_t launch_grouped_gemm_swiglu_bwd(const CUtensorMap& tm_a, const CUtensorMap& tm_b, const int32_t* offsets,
                                            int E, int K, int F, void* dgu, const void* dh_mid, void* dgu_t,
                                            const int32_t* col_off, int ldt, int32_t* status, bool pdl,
-                                           cudaStream_t s);
+                                           cudaStream_t s,
+                                           const CUtensorMap* tm_d = nullptr);
 // Weight gradients: for each expert e, D32[e] [M, N] (fp32) = A_e B_e^T where
 // A [M, cols] and B [N, cols] are transposed activations whose columns
 // [col_offsets[e], col_offsets[e+1]) (multiples of 64, zero padded) belong to
