@@ -19,6 +19,7 @@ import oracle as O
 import workloads as W
 from oracle import cases
 from oracle import check as C
+from oracle import mxfp8 as X
 
 from gpu_cases import DEV, DeviceCase, cfg_for, np64, np_, oracle_y, parity_case, workload
 
@@ -530,3 +531,45 @@ def test_fused_combine_rejected_where_it_does_not_apply():
         base.update(kw)
         cfg = M.config(**base, combine="fused")
         assert M.moe_workspace_size(cfg, M.MOE_OP_LAYER) == 0, kw
+
+
+@pytest.mark.parametrize("precision", ["bf16", "mxfp8"])
+def test_grouped_ffn_expert_boundaries_inside_tiles(precision):
+    """Experts whose row counts fall on and next to the 32-row blocks the
+    epilogue stores whole (0, 1, 31, 32, 33, 64, 96, 128, 160, 255 rows):
+    every row of every expert equals the oracle's expert output, and the rows
+    past the last expert are left as they were."""
+    counts = [32, 64, 96, 128, 31, 33, 0, 1, 160, 255]
+    E, d, F, k = len(counts), 256, 256, 2
+    n = sum(counts)
+    T = n // k + 50                      # 100 rows past the last expert
+    cfg = M.config(T, d, E, k, F, precision=precision)
+    r = np.random.default_rng(11)
+    x = r.standard_normal((T * k, d)).astype(np.float32)
+    wg = (r.standard_normal((E, F, d)) / np.sqrt(d)).astype(np.float32)
+    wu = (r.standard_normal((E, F, d)) / np.sqrt(d)).astype(np.float32)
+    wd = (r.standard_normal((E, d, F)) / np.sqrt(F)).astype(np.float32)
+    xb, wgb, wub, wdb = (torch.from_numpy(a).to(torch.bfloat16) for a in (x, wg, wu, wd))
+    offsets = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
+    w13 = M.moe_pack_weights(M.config(T, d, E, k, F), wgb.to(DEV), wub.to(DEV))
+    wdd = wdb.to(DEV)
+    if precision == "mxfp8":
+        w13, wdd = M.moe_pack_weights_mxfp8(cfg, w13, wdd)
+    y_perm = torch.full((T * k, d), 7.0, dtype=torch.bfloat16, device=DEV)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    M.moe_grouped_ffn(cfg, xb.to(DEV), torch.from_numpy(offsets).to(DEV), w13, wdd, y_perm=y_perm, status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) & (M.MOE_STATUS_TIMEOUT | M.MOE_STATUS_BAD_ROUTE) == 0
+    got = np64(y_perm)
+    xs = cases.as64(xb)
+    want = np.zeros((n, d))
+    for e in range(E):
+        lo, hi = int(offsets[e]), int(offsets[e + 1])
+        if hi > lo:
+            ws = (cases.as64(wgb[e]), cases.as64(wub[e]), cases.as64(wdb[e]))
+            want[lo:hi] = X.mx_swiglu_expert(xs[lo:hi], *ws)[0] if precision == "mxfp8" else O.swiglu_expert(xs[lo:hi], *ws)
+    for e in range(E):
+        lo, hi = int(offsets[e]), int(offsets[e + 1])
+        if hi > lo:
+            assert C.row_rel_err(got[lo:hi], want[lo:hi]) <= C.TOL_BF16, f"expert {e} ({hi - lo} rows)"
+    assert bool((got[n:] == 7.0).all())
