@@ -55,9 +55,8 @@ int make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uin
   return r == CUDA_SUCCESS ? MOE_OK : MOE_ERR_CUDA;
 }
 
-// Row-major bf16 matrix [rows, cols] written (or, in the SwiGLU-backward
-// epilogues, read) by the GEMM epilogue's TMA copies: boxes of 32 rows x 32
-// columns (64 bytes), 64-byte swizzle (the epilogue's staging layout).
+// Row-major bf16 matrix [rows, cols] written by TMA stores: boxes of 32 rows x
+// 32 columns (64 bytes), 64-byte swizzle (the GEMM epilogue's staging layout).
 int make_map_store(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols) {
   EncodeTiledFn enc = encode_fn();
   if (enc == nullptr) return MOE_ERR_NO_DEVICE;
@@ -792,12 +791,11 @@ int32_t moe_layer_backward(const moe_config* cfg, const void* h, const void* w_r
       // 2+3. dL/dh_mid = dy_perm W_down (per expert) with the SwiGLU backward in
       //      the epilogue, from the pre-activations the forward kept: writes
       //      dgu and its transposed copy; no recompute of the gate/up GEMM
-      CUtensorMap tdg, tpre;
+      CUtensorMap tdg;
       rc = make_map_store(&tdg, b.dgu, P, 2 * F);
-      if (rc == MOE_OK) rc = make_map_store(&tpre, f.preact, P, 2 * F);
       if (rc != MOE_OK) return rc;
       e = launch_grouped_gemm_dh_swiglu_bwd(ta, tb, f.offsets, E, d, F, f.preact, b.dgu, b.dgu_t, b.col_off,
-                                            b.ppad_max, status_dev, false, s, &tdg, &tpre);
+                                            b.ppad_max, status_dev, false, s, &tdg);
       if (e != cudaSuccess) return MOE_ERR_CUDA;
     } else {
       // 2. dh_mid = dy_perm W_down (per expert), B = W_down^T rows
@@ -812,12 +810,11 @@ int32_t moe_layer_backward(const moe_config* cfg, const void* h, const void* w_r
       rc = make_map(&ta, f.x_perm, P, d, kTileM);
       if (rc == MOE_OK) rc = make_map(&tb, w13_packed, static_cast<uint64_t>(E) * 2 * F, d, kGemmTileN);
       if (rc != MOE_OK) return rc;
-      CUtensorMap tdg, tdh;
+      CUtensorMap tdg;
       if (rc == MOE_OK) rc = make_map_store(&tdg, b.dgu, P, 2 * F);
-      if (rc == MOE_OK) rc = make_map_store(&tdh, b.dh_mid, P, F);
       if (rc != MOE_OK) return rc;
       e = launch_grouped_gemm_swiglu_bwd(ta, tb, f.offsets, E, d, F, b.dgu, b.dh_mid, b.dgu_t, b.col_off,
-                                         b.ppad_max, status_dev, false, s, &tdg, &tdh);
+                                         b.ppad_max, status_dev, false, s, &tdg);
       if (e != cudaSuccess) return MOE_ERR_CUDA;
     }
     // 4. dx_perm = dgu w13 (per expert), B = w13^T rows

@@ -60,8 +60,8 @@ constexpr uint32_t kTmemCols = 2 * kBN;
 constexpr uint32_t kStgBytes = 32 * 32 * 2;
 
 constexpr size_t gemm_smem_bytes() {
-  return 1024 + kStages * static_cast<size_t>(kStageBytes) + kEpiWarps * kStgBytes +
-         (2 * kStages + 5 + kEpiWarps) * 8 + 16 + 2 * (kMaxE + 1) * 4 + kBM * 4;
+  return 1024 + kStages * static_cast<size_t>(kStageBytes) + kEpiWarps * kStgBytes + (2 * kStages + 5) * 8 + 16 +
+         2 * (kMaxE + 1) * 4 + kBM * 4;
 }
 static_assert(gemm_smem_bytes() <= 227 * 1024, "shared memory");
 
@@ -121,10 +121,6 @@ struct GemmArgs {
   // the tile all belong to the expert stores each 32-column block through its
   // staging buffer with one TMA store; other warps store row by row.
   int tma_store;
-  // SwiGLU-backward epilogues: the rows they read (aux, or preact) are also
-  // described by tm_e (same box format); such a warp then loads each 32 x 32
-  // block with one TMA load into its staging buffer instead of row by row.
-  int tma_aux;
 };
 
 // Epilogues and tile groupings of grouped_gemm_kernel.
@@ -175,8 +171,7 @@ MOE_DEV void stage_store(uint8_t* stg, const uint32_t (&p)[16], int lane, const 
 template <int kEpi, int kMode>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
-                        const __grid_constant__ CUtensorMap tm_d, const __grid_constant__ CUtensorMap tm_e,
-                        const GemmArgs a) {
+                        const __grid_constant__ CUtensorMap tm_d, const GemmArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align_1024(smem_raw);
   uint8_t* sA = smem;
@@ -187,8 +182,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   uint64_t* tfull = empty + kStages;
   uint64_t* tempty = tfull + 2;
   uint64_t* drain = tempty + 2;
-  uint64_t* ld_bar = drain + 1;  // [kEpiWarps] epilogue warps' TMA loads of aux / preact blocks
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ld_bar + kEpiWarps);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   int* consumed_slot = reinterpret_cast<int*>(tmem_slot + 2);
   int* s_off = reinterpret_cast<int*>(tmem_slot + 4);  // [E+1]
@@ -209,14 +203,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       mbar_init(&tempty[i], kEpiWarps);
     }
     mbar_init(drain, 1);
-    for (int w = 0; w < kEpiWarps; ++w) mbar_init(&ld_bar[w], 1);
     *abort_flag = 0;
     *consumed_slot = 0;
     fence_mbar_init();
     tma_prefetch_desc(&tm_a);
     tma_prefetch_desc(&tm_b);
     if (a.tma_store) tma_prefetch_desc(&tm_d);
-    if (a.tma_aux) tma_prefetch_desc(&tm_e);
   }
   pdl_wait();  // offsets and the A rows come from the kernels before this one
   for (int e = threadIdx.x; e <= E; e += blockDim.x) s_off[e] = a.offsets[e];
@@ -383,9 +375,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const int half = (warp - 2) >> 2;  // which half of the tile's columns it drains
     const int row = q * 32 + lane;
     uint8_t* stg = stg_all + (warp - 2) * kStgBytes;
-    uint64_t* my_ld = &ld_bar[warp - 2];
-    uint32_t ld_phase = 0;
-    bool ld_pending = false;  // a TMA load into stg may still be in flight (its wait gave up)
     int local = 0;
     for (long long tile = blockIdx.x; tile < total; tile += gridDim.x, ++local) {
       int e, m, n, kb0, kb1;
@@ -445,13 +434,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           tmem_ld32(tbase + c, g);
           tmem_ld32(tbase + kBN / 2 + c, u);
           uint4 dq[4];
-          if (staged && a.tma_aux) {
-            if (!stage_load_rows64(stg, my_ld, ld_phase, lane, &tm_e, n * (kBN / 2) + c, srow, dq, abort_flag)) {
-              tmem_ld_wait();
-              ld_pending = true;
-              break;
-            }
-          } else if (valid) {
+          if (valid) {
             const uint4* src = reinterpret_cast<const uint4*>(dh + c);
 #pragma unroll
             for (int i = 0; i < 4; ++i) dq[i] = src[i];
@@ -558,14 +541,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           uint32_t dh[32];
           tmem_ld32(tbase + half * (kBN / 2) + c, dh);
           uint4 ga[4], ua[4];
-          if (staged && a.tma_aux) {
-            if (!stage_load_rows64(stg, my_ld, ld_phase, lane, &tm_e, b * kBN + c, srow, ga, abort_flag) ||
-                !stage_load_rows64(stg, my_ld, ld_phase, lane, &tm_e, b * kBN + kBN / 2 + c, srow, ua, abort_flag)) {
-              tmem_ld_wait();
-              ld_pending = true;
-              break;
-            }
-          } else if (valid) {
+          if (valid) {
             const uint4* gsrc = reinterpret_cast<const uint4*>(pre + c);
             const uint4* usrc = reinterpret_cast<const uint4*>(pre + kBN / 2 + c);
 #pragma unroll
@@ -721,16 +697,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           }
         }
       }
-      if (ld_pending) {  // a staged load's wait gave up: stop (the other roles see the flag)
-        *abort_flag = 1;
-        break;
-      }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&tempty[acc]);
     }
-    // a load whose wait gave up must land before the buffer goes away
-    if (ld_pending && lane == 0) mbar_wait(my_ld, ld_phase, nullptr);
   }
   __syncwarp();
   if (warp >= 2 && lane == 0) bulk_wait_all();  // the epilogue's staged stores have completed
@@ -1145,9 +1115,8 @@ std::atomic<int> g_stall_gemms{0};
 
 template <int kEpi, int kMode>
 cudaError_t launch_gemm_inst(const CUtensorMap& tm_a, const CUtensorMap& tm_b, GemmArgs a, bool pdl,
-                             cudaStream_t s, const CUtensorMap* tm_d = nullptr, const CUtensorMap* tm_e = nullptr) {
+                             cudaStream_t s, const CUtensorMap* tm_d = nullptr) {
   a.tma_store = tm_d != nullptr ? 1 : 0;
-  a.tma_aux = tm_e != nullptr ? 1 : 0;
   int left = g_stall_gemms.load();
   while (left > 0 && !g_stall_gemms.compare_exchange_weak(left, left - 1)) {
   }
@@ -1157,7 +1126,7 @@ cudaError_t launch_gemm_inst(const CUtensorMap& tm_a, const CUtensorMap& tm_b, G
                                          static_cast<int>(smem));
   if (err != cudaSuccess) return err;
   err = launch_kernel(grouped_gemm_kernel<kEpi, kMode>, dim3(device_sm_count()), dim3(kGemmThreads), smem, s, pdl, 1,
-                      tm_a, tm_b, tm_d != nullptr ? *tm_d : tm_a, tm_e != nullptr ? *tm_e : tm_a, a);
+                      tm_a, tm_b, tm_d != nullptr ? *tm_d : tm_a, a);
   if (err != cudaSuccess) return err;
   return cudaGetLastError();
 }
@@ -1196,24 +1165,23 @@ cudaError_t launch_grouped_gemm_combine(const CUtensorMap& tm_a, const CUtensorM
 cudaError_t launch_grouped_gemm_dh_swiglu_bwd(const CUtensorMap& tm_a, const CUtensorMap& tm_b,
                                               const int32_t* offsets, int E, int K, int F, const void* preact,
                                               void* dgu, void* dgu_t, const int32_t* col_off, int ldt, int32_t* status,
-                                              bool pdl, cudaStream_t s, const CUtensorMap* tm_d,
-                                              const CUtensorMap* tm_e) {
+                                              bool pdl, cudaStream_t s, const CUtensorMap* tm_d) {
   GemmArgs a{offsets, E, K, F, (F + kBN - 1) / kBN, F, 2 * F, static_cast<__nv_bfloat16*>(dgu), status,
              band_rows(kBM, K, 8, 32), nullptr, nullptr, 0, nullptr, 0, static_cast<__nv_bfloat16*>(dgu_t), col_off,
              ldt};
   a.preact = static_cast<__nv_bfloat16*>(const_cast<void*>(preact));
   a.preact_ld = 2 * F;
-  return launch_gemm_inst<kEpiDhSwiGLUBwd, kGroupRows>(tm_a, tm_b, a, pdl, s, tm_d, tm_d != nullptr ? tm_e : nullptr);
+  return launch_gemm_inst<kEpiDhSwiGLUBwd, kGroupRows>(tm_a, tm_b, a, pdl, s, tm_d);
 }
 
 cudaError_t launch_grouped_gemm_swiglu_bwd(const CUtensorMap& tm_a, const CUtensorMap& tm_b, const int32_t* offsets,
                                            int E, int K, int F, void* dgu, const void* dh_mid, void* dgu_t,
                                            const int32_t* col_off, int ldt, int32_t* status, bool pdl,
-                                           cudaStream_t s, const CUtensorMap* tm_d, const CUtensorMap* tm_e) {
+                                           cudaStream_t s, const CUtensorMap* tm_d) {
   GemmArgs a{offsets, E, K, 2 * F, 2 * F / kBN, 2 * F, 2 * F, static_cast<__nv_bfloat16*>(dgu), status,
              band_rows(kBM, K, 8, 32), nullptr, static_cast<const __nv_bfloat16*>(dh_mid), F, nullptr, 0,
              static_cast<__nv_bfloat16*>(dgu_t), col_off, ldt};
-  return launch_gemm_inst<kEpiSwiGLUBwd, kGroupRows>(tm_a, tm_b, a, pdl, s, tm_d, tm_d != nullptr ? tm_e : nullptr);
+  return launch_gemm_inst<kEpiSwiGLUBwd, kGroupRows>(tm_a, tm_b, a, pdl, s, tm_d);
 }
 
 cudaError_t launch_grouped_gemm_wgrad(const CUtensorMap& tm_a, const CUtensorMap& tm_b, const int32_t* col_offsets,

@@ -186,33 +186,6 @@ MOE_DEV void stage_store_rows(uint8_t* stg, const uint4 (&v)[kRowBytes / 16], in
   }
 }
 
-// One warp's 32 rows x 32 bf16 columns at (x, y) of the tensor behind tm into
-// v (lane r gets row r): lane 0 issues a TMA load into the warp's staging
-// buffer (after any store from it has read it), every lane waits on the
-// warp's barrier `bar` (phase `phase`, flipped here) and reads its row back
-// from the 64-byte-swizzled box. Returns the same verdict in every lane:
-// false if the wait gave up (timeout or *abort); the load may then still be
-// in flight, and the caller waits for it before the buffer goes away.
-MOE_DEV bool stage_load_rows64(uint8_t* stg, uint64_t* bar, uint32_t& phase, int lane, const CUtensorMap* tm, int x,
-                               int y, uint4 (&v)[4], volatile int* abort) {
-  if (lane == 0) {
-    bulk_wait_read<0>();
-    mbar_expect_tx(bar, 32 * 64);
-    tma_load_2d(stg, tm, bar, x, y);
-  }
-  __syncwarp();
-  const bool ok = __all_sync(0xffffffffu, mbar_wait(bar, phase, abort));
-  if (!ok) return false;
-  phase ^= 1;
-  const uint8_t* rowp = stg + lane * 64;
-  const int sw = (lane >> 1) & 3;
-#pragma unroll
-  for (int j = 0; j < 4; ++j) v[j] = *reinterpret_cast<const uint4*>(rowp + ((j ^ sw) << 4));
-  fence_proxy_async_shared();  // these reads before the next TMA write of the buffer
-  __syncwarp();
-  return true;
-}
-
 // ------------------------------------------------------------------ tcgen05
 MOE_DEV void tmem_alloc(uint32_t* dst_smem, uint32_t ncols) {  // whole warp
   asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_addr(dst_smem)),

@@ -58,9 +58,7 @@ cudaError_t launch_combine(int dtype, const void* y_perm, const int32_t* dest_ro
 // [rows, n_per_expert] bf16 in w13's interleaved column order.
 // tm_d (may be NULL): D as a store tensor map (make_map_store: bf16, 32 x 32
 // boxes, 64-byte swizzle); the epilogue then writes whole 32-row blocks of
-// the tile with TMA stores. The SwiGLU-backward launchers also take tm_e, the
-// rows their epilogue reads (dh_mid, or the saved pre-activations) in the same
-// format, used only together with tm_d.
+// the tile with TMA stores.
 cudaError_t launch_grouped_gemm_tc(const CUtensorMap& tm_a, const CUtensorMap& tm_b, bool swiglu,
                                    const int32_t* offsets, int E, int K, int n_per_expert, int n_tiles,
                                    int out_cols, int ldd, void* D, const int32_t* gather_rows, int32_t* status,
@@ -74,7 +72,7 @@ cudaError_t launch_grouped_gemm_dh_swiglu_bwd(const CUtensorMap& tm_a, const CUt
                                               const int32_t* offsets, int E, int K, int F, const void* preact,
                                               void* dgu, void* dgu_t, const int32_t* col_off, int ldt, int32_t* status,
                                               bool pdl, cudaStream_t s,
-                                              const CUtensorMap* tm_d = nullptr, const CUtensorMap* tm_e = nullptr);
+                                              const CUtensorMap* tm_d = nullptr);
 // The down projection with the combine fused into its epilogue (k <= 2): y_perm
 // rows as launch_grouped_gemm_tc, and y [T, d] = sum over each token's kept
 // slots, in slot order, of gate * bf16 row (bit-identical to launch_combine).
@@ -96,7 +94,7 @@ cudaError_t launch_grouped_gemm_swiglu_bwd(const CUtensorMap& tm_a, const CUtens
                                            int E, int K, int F, void* dgu, const void* dh_mid, void* dgu_t,
                                            const int32_t* col_off, int ldt, int32_t* status, bool pdl,
                                            cudaStream_t s,
-                                           const CUtensorMap* tm_d = nullptr, const CUtensorMap* tm_e = nullptr);
+                                           const CUtensorMap* tm_d = nullptr);
 // Weight gradients: for each expert e, D32[e] [M, N] (fp32) = A_e B_e^T where
 // A [M, cols] and B [N, cols] are transposed activations whose columns
 // [col_offsets[e], col_offsets[e+1]) (multiples of 64, zero padded) belong to
