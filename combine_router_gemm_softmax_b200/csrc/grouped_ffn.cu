@@ -498,8 +498,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             uint32_t p[16];
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
-              const float h0 = silu_f(__uint_as_float(g[2 * i])) * __uint_as_float(u[2 * i]);
-              const float h1 = silu_f(__uint_as_float(g[2 * i + 1])) * __uint_as_float(u[2 * i + 1]);
+              const float h0 = silu_fast(__uint_as_float(g[2 * i])) * __uint_as_float(u[2 * i]);
+              const float h1 = silu_fast(__uint_as_float(g[2 * i + 1])) * __uint_as_float(u[2 * i + 1]);
               p[i] = pack_bf16x2(h0, h1);
             }
             if (staged) {
@@ -931,8 +931,8 @@ __global__ void __launch_bounds__(kPairThreads, 1)
             uint32_t p[16];
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
-              const float h0 = silu_f(__uint_as_float(g[2 * i])) * __uint_as_float(u[2 * i]);
-              const float h1 = silu_f(__uint_as_float(g[2 * i + 1])) * __uint_as_float(u[2 * i + 1]);
+              const float h0 = silu_fast(__uint_as_float(g[2 * i])) * __uint_as_float(u[2 * i]);
+              const float h1 = silu_fast(__uint_as_float(g[2 * i + 1])) * __uint_as_float(u[2 * i + 1]);
               p[i] = pack_bf16x2(h0, h1);
             }
             uint4* dst = reinterpret_cast<uint4*>(out + c);

@@ -136,11 +136,6 @@ MOE_DEV uint32_t mx_quantize_block(const float (&v)[32], uint4 (&out)[2], int& n
   return static_cast<uint32_t>(E + 127);
 }
 
-// silu(z) = z / (1 + e^-z) with the fast exponential and division intrinsics
-// (about 2 ulp in fp32). Its result is rounded to E4M3 (3 mantissa bits)
-// next, so their error does not show; the bf16 path keeps the IEEE forms.
-MOE_DEV float silu_mx(float z) { return __fdividef(z, 1.0f + __expf(-z)); }
-
 // Byte offset of the scale of (row, 32-element block b) in the atom layout.
 MOE_DEV size_t mx_sf_offset(long long row, int b, int row_blocks) {
   const int kt = b >> 2, j = b & 3;
@@ -566,7 +561,7 @@ __global__ void __launch_bounds__(kMxThreads, 1)
           }
           float h[32];
 #pragma unroll
-          for (int j = 0; j < 32; ++j) h[j] = silu_mx(__uint_as_float(g[j])) * __uint_as_float(u[j]);
+          for (int j = 0; j < 32; ++j) h[j] = silu_fast(__uint_as_float(g[j])) * __uint_as_float(u[j]);
           uint4 out[2];
           const uint32_t byte = mx_quantize_block(h, out, n_sat, n_under);
           if (a.tma_store) {
