@@ -59,17 +59,20 @@ constexpr int kMxBM = 128;
 constexpr int kMxBN = 256;
 constexpr int kMxBK = 128;  // elements (= bytes) of K per stage
 constexpr int kMxStages = 4;
-// warp 0: TMA producer, warp 1: TMEM allocation and MMA issue, warps 2..9:
-// epilogue, two per TMEM lane quadrant, each draining half of a tile, warp
-// 10: copies each stage's scale atoms into TMEM (a ring of four column sets)
-// and signals the MMA thread through sf_full when they have landed
-constexpr int kMxThreads = 352;
+// warp 0: TMA producer of the operand tiles, warp 1: TMEM allocation and MMA
+// issue, warps 2..9: epilogue, two per TMEM lane quadrant, each draining half
+// of a tile, warp 10: copies each stage's scale atoms into TMEM (a ring of
+// four column sets) and signals the MMA thread through sf_full, warp 11:
+// loads the scale atoms into shared memory (sf_loaded), so the producer
+// issues two copies per stage, as in the bf16 kernel
+constexpr int kMxThreads = 384;
 constexpr int kMxEpiWarps = 8;
 constexpr uint32_t kMxABytes = kMxBM * kMxBK;   // 16 KB
 constexpr uint32_t kMxBBytes = kMxBN * kMxBK;   // 32 KB
 constexpr uint32_t kSfaBytes = 512;
 constexpr uint32_t kSfbBytes = 1024;
-constexpr uint32_t kMxStageTx = kMxABytes + kMxBBytes + kSfaBytes + kSfbBytes;
+constexpr uint32_t kMxStageTx = kMxABytes + kMxBBytes;
+constexpr uint32_t kMxSfTx = kSfaBytes + kSfbBytes;
 constexpr uint32_t kAcc1Col = 192;   // second accumulator; [192, 256) is shared
 constexpr uint32_t kSfaCol = 448;    // stage s: SFA at 448 + 12 s, SFB at 452 + 12 s (8 columns)
 constexpr uint32_t kMxTmemCols = 512;
@@ -81,7 +84,7 @@ constexpr uint32_t kMxStgBytes = 2048;
 
 constexpr size_t mx_smem_bytes() {
   return 1024 + kMxStages * static_cast<size_t>(kMxABytes + kMxBBytes + kSfaBytes + kSfbBytes) +
-         kMxEpiWarps * kMxStgBytes + (3 * kMxStages + 5) * 8 + 16 + 2 * (kMaxE + 1) * 4;
+         kMxEpiWarps * kMxStgBytes + (4 * kMxStages + 5) * 8 + 16 + 2 * (kMaxE + 1) * 4;
 }
 static_assert(mx_smem_bytes() <= 227 * 1024, "shared memory");
 
@@ -363,7 +366,8 @@ __global__ void __launch_bounds__(kMxThreads, 1)
   uint64_t* drain = ovl + 1;
   uint64_t* sf_full = drain + 1;
   uint64_t* cp_drain = sf_full + kMxStages;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(cp_drain + 1);
+  uint64_t* sf_loaded = cp_drain + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sf_loaded + kMxStages);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   int* consumed_slot = reinterpret_cast<int*>(tmem_slot + 2);
   int* s_off = reinterpret_cast<int*>(tmem_slot + 4);  // [E+1]
@@ -384,6 +388,7 @@ __global__ void __launch_bounds__(kMxThreads, 1)
     mbar_init(drain, 1);
     for (int s = 0; s < kMxStages; ++s) mbar_init(&sf_full[s], 1);
     mbar_init(cp_drain, 1);
+    for (int s = 0; s < kMxStages; ++s) mbar_init(&sf_loaded[s], 1);
     *abort_flag = 0;
     *consumed_slot = 0;
     fence_mbar_init();
@@ -428,11 +433,6 @@ __global__ void __launch_bounds__(kMxThreads, 1)
           mbar_expect_tx(&full[stage], kMxStageTx);
           tma_load_2d(sA + stage * kMxABytes, &tm_a, &full[stage], kt * kMxBK, a_row);
           tma_load_2d(sB + stage * kMxBBytes, &tm_b, &full[stage], kt * kMxBK, b_row);
-          bulk_load(sSFA + stage * kSfaBytes, a.sfa + (static_cast<size_t>(kt) * a.ra_blocks + a_row / 128) * 512,
-                    kSfaBytes, &full[stage]);
-          bulk_load(sSFB + stage * kSfbBytes,
-                    a.sfb + (static_cast<size_t>(kt) * (a.rb_blocks + 1) + b_row / 128) * 512, kSfbBytes,
-                    &full[stage]);
           ++issued;
           if (++stage == kMxStages) {
             stage = 0;
@@ -499,7 +499,7 @@ __global__ void __launch_bounds__(kMxThreads, 1)
       bool stop = false;
       for (long long tile = blockIdx.x; tile < total && !stop; tile += gridDim.x) {
         for (int kt = 0; kt < nkt; ++kt) {
-          if (!mbar_wait(&full[stage], phase, abort_flag)) {
+          if (!mbar_wait(&sf_loaded[stage], phase, abort_flag)) {
             *abort_flag = 1;
             stop = true;
             break;
@@ -518,6 +518,44 @@ __global__ void __launch_bounds__(kMxThreads, 1)
       }
       umma_commit(cp_drain);
       mbar_wait(cp_drain, 0, nullptr);
+    }
+  } else if (warp == 3 + kMxEpiWarps) {
+    if (lane == 0) {
+      // ---------------------------------------------------------------- scale loader
+      int stage = 0;
+      uint32_t phase = 0;
+      bool stop = false;
+      int sf_issued = 0;
+      for (long long tile = blockIdx.x; tile < total && !stop; tile += gridDim.x) {
+        int e, m, n;
+        mx_decode_tile(tile, m_total, a.n_tiles, a.band, prefix, E, e, m, n);
+        const int a_row = (prefix[e] + m) * kMxBM;
+        const int b_row = e * a.n_per_expert + n * kMxBN;
+        for (int kt = 0; kt < nkt; ++kt) {
+          // the stage's MMAs of the previous round are done, and with them the
+          // copy of its scales into TMEM
+          if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag)) {
+            *abort_flag = 1;
+            stop = true;
+            break;
+          }
+          mbar_expect_tx(&sf_loaded[stage], kMxSfTx);
+          bulk_load(sSFA + stage * kSfaBytes, a.sfa + (static_cast<size_t>(kt) * a.ra_blocks + a_row / 128) * 512,
+                    kSfaBytes, &sf_loaded[stage]);
+          bulk_load(sSFB + stage * kSfbBytes,
+                    a.sfb + (static_cast<size_t>(kt) * (a.rb_blocks + 1) + b_row / 128) * 512, kSfbBytes,
+                    &sf_loaded[stage]);
+          ++sf_issued;
+          if (++stage == kMxStages) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+      }
+      // each stage holds at most one load that nobody may have waited for:
+      // let it land before the CTA leaves
+      for (int i = sf_issued > kMxStages ? sf_issued - kMxStages : 0; i < sf_issued; ++i)
+        mbar_wait(&sf_loaded[i % kMxStages], (i / kMxStages) & 1, nullptr);
     }
   } else {
     // ---------------------------------------------------------------- epilogue
