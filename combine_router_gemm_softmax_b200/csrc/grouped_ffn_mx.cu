@@ -33,8 +33,9 @@
 //                             to each of its kept rows of the padded layout
 //   grouped_gemm_mx_kernel    persistent warp-specialised GEMM over the
 //                             padded groups: TMA for the operand tiles, bulk
-//                             copies for the scale atoms, tcgen05.cp of the
-//                             scales into TMEM and tcgen05.mma
+//                             copies for the scale atoms (a warp of their
+//                             own), tcgen05.cp of the scales into TMEM (another
+//                             warp) and tcgen05.mma
 //                             kind::mxf8f6f4.block_scale (128 x 256 x 32) by
 //                             one thread. GEMM1 forms silu(gate) * up in its
 //                             epilogue and quantises it straight to MXFP8 for
