@@ -44,9 +44,11 @@
 // TMEM: the two accumulators overlap. Tile i uses columns [0, 256) when i is
 // even and [192, 448) when odd; the epilogue drains the shared columns
 // [192, 256) first and signals, so the next tile's MMAs start while it drains
-// the rest. Columns [448, 460) hold the current k-slice's scales. The scale
-// copy for a k-slice is issued by the MMA thread right before that slice's
-// MMAs; tcgen05 copies and MMAs issued by one thread execute in issue order.
+// the rest. Columns [448, 496) hold the scales of the four k-slices in flight
+// (12 columns each: 4 for A, 8 for B). A slice's scales are copied into its
+// column set by the scale-copy warp, which commits the copies to the slice's
+// sf_full barrier; the MMA thread waits for that barrier before the slice's
+// MMAs, and a column set is rewritten only after its previous MMAs are done.
 #include <cuda_fp8.h>
 
 #include "moe_common.cuh"
