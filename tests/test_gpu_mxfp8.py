@@ -195,3 +195,33 @@ def test_mxfp8_rejects_unsupported_configs():
                              torch.zeros((4, 128, 256), dtype=torch.bfloat16, device=DEV),
                              torch.zeros((4, 128, 128), dtype=torch.bfloat16, device=DEV), h, ws,
                              ws=torch.zeros(1 << 20, dtype=torch.uint8, device=DEV))
+
+
+@pytest.mark.parametrize("T,E,k,cap", [(0, 8, 2, -1), (1, 8, 2, -1), (129, 1, 1, -1), (200, 8, 8, -1),
+                                       (300, 8, 2, 0)])
+def test_layer_mxfp8_edge_cases(T, E, k, cap):
+    """The MXFP8 layer on the layer's edge cases: no tokens, one token, one
+    expert, k = E, and a capacity of zero (every assignment dropped)."""
+    import workloads as W
+
+    wl = W.Workload("edge", T=T, d=128, E=E, k=k, F=128, bias="none", capacity=cap)
+    inp = W.draw(wl, 3)
+    if T:
+        inp = cases.enforce_margin(inp, 3)
+    dc = DeviceCase(inp)
+    cfg = M.config(T, 128, E, k, 128, capacity=cap, precision="mxfp8")
+    w13_mx, wd_mx = M.moe_pack_weights_mxfp8(cfg, dc.w13, dc.w_down)
+    idx = torch.empty((T, k), dtype=torch.int32, device=DEV)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    y = M.moe_layer_forward(cfg, dc.h, dc.w_router, dc.bias, w13_mx, wd_mx, topk_idx=idx, status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) & (M.MOE_STATUS_TIMEOUT | M.MOE_STATUS_BAD_ROUTE | M.MOE_STATUS_NAN_LOGIT) == 0
+    if T == 0:
+        assert y.numel() == 0
+        return
+    ref = O.layer_forward(cases.as64(inp.h), cases.as64(inp.w_router), None, k, "swiglu", cases.weights_fn(inp), cap)
+    assert np.array_equal(np_(idx), ref["idx"])
+    want = X.mx_combine(cases.as64(inp.h), ref["idx"], ref["gate"], ref["dest_row"], _mx_weights(inp), None)
+    assert C.row_rel_err(np64(y), want) <= C.TOL_BF16
+    if cap == 0:
+        assert not y.any()
