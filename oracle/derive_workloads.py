@@ -11,7 +11,6 @@ Run:  python -m oracle.derive_workloads
 from __future__ import annotations
 
 import json
-import os
 
 import numpy as np
 

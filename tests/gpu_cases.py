@@ -5,7 +5,6 @@ from __future__ import annotations
 
 import functools
 
-import numpy as np
 import torch
 
 import combine_router_gemm_softmax_b200 as M

@@ -25,7 +25,7 @@ from oracle import cases
 from oracle import check as C
 from oracle import mxfp8 as X
 
-from gpu_cases import DEV, DeviceCase, np64, np_, parity_case, workload
+from gpu_cases import DEV, DeviceCase, np64, np_, parity_case
 
 pytestmark = pytest.mark.gpu
 

@@ -21,7 +21,7 @@ from oracle import cases
 from oracle import check as C
 from oracle import mxfp8 as X
 
-from gpu_cases import DEV, DeviceCase, cfg_for, np64, np_, oracle_y, parity_case, workload
+from gpu_cases import DEV, DeviceCase, cfg_for, np64, np_, oracle_y, parity_case
 
 pytestmark = pytest.mark.gpu
 

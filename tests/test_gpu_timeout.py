@@ -12,7 +12,7 @@ import torch
 
 import combine_router_gemm_softmax_b200 as M
 
-from gpu_cases import DEV, DeviceCase, parity_case
+from gpu_cases import DeviceCase, parity_case
 
 pytestmark = pytest.mark.gpu
 

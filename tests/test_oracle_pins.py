@@ -10,7 +10,6 @@ that the comparison rules catch them.
 """
 import itertools
 import json
-import math
 import os
 
 import numpy as np

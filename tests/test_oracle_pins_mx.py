@@ -13,7 +13,6 @@
   conversion as the element quantiser.
 """
 import numpy as np
-import pytest
 import torch
 
 import oracle as O
