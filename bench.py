@@ -209,6 +209,12 @@ def combine_ranks(ms_local, tokens_per_rank, steps, world, device=None):
     return ms, tokens_per_rank * world * steps / (ms / 1e3)
 
 
+def tiles_used(M, cfg):
+    """Tile shape the grouped GEMMs take for cfg (AUTO resolved by the library)."""
+    return {M.MOE_GEMM_TILES_SINGLE: "single (128x256)", M.MOE_GEMM_TILES_PAIR: "pair (256x256, 2 SMs)"}[
+        M.moe_gemm_tiles_used(cfg)]
+
+
 def config_dict(wl, n, flush=None):
     c = {"workload": wl.name, "T": wl.T, "d": wl.d, "E": wl.E, "k": wl.k, "d_ff": wl.F, "dtype": wl.dtype,
          "expert_kind": wl.expert_kind, "capacity": wl.capacity, "layout": wl.layout, "global_batch": wl.T * n,
@@ -409,7 +415,8 @@ def main():
             "warmup": max(args.warmup, 3), "ms_per_step": ms_max / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": wl.dtype if args.precision == "bf16" else "mxfp8",
             "data": "synthetic: seeded N(0,1) tokens, N(0,1/fan_in) random-init weights",
-            "config": {**config_dict(wl, world, flush), "gemm_tiles": args.gemm_tiles, "precision": args.precision,
+            "config": {**config_dict(wl, world, flush), "gemm_tiles": args.gemm_tiles,
+                       "gemm_tiles_used": tiles_used(M, L.cfg), "precision": args.precision,
                        "combine": "fused into the down projection" if fused_combine(L.cfg) else "separate kernel"},
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": wl.T * row_bytes,
                     "d2h_bytes_per_step": wl.T * row_bytes, "ms_per_step": e2e_ms / args.steps,
@@ -605,7 +612,8 @@ def run_sweep(M, W, names, seed, dev, stream, barrier):
         ms, stages, flush = time_steps(L, SWEEP_STEPS, SWEEP_WARMUP, stream, barrier, sampler)
         A_kept = int(L.counts.sum().item())
         entry = {"ms_per_step": ms / SWEEP_STEPS, "tokens_per_s": wl.T * SWEEP_STEPS / (ms / 1e3),
-                 "steps": SWEEP_STEPS, "config": config_dict(wl, 1, flush), "kept": A_kept,
+                 "steps": SWEEP_STEPS, "config": {**config_dict(wl, 1, flush), "gemm_tiles_used": tiles_used(M, L.cfg)},
+                 "kept": A_kept,
                  "status_word": int(L.status.item()), "clocks": sampler.summary(),
                  "gpu_launches_per_step": launches(L.cfg)}
         if wl.dtype == "bf16":

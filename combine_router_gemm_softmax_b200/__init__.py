@@ -27,5 +27,5 @@ from ._lib import (  # noqa: F401
     MOE_STATUS_BAD_ROUTE, MOE_STATUS_NAN_LOGIT, MOE_STATUS_TIMEOUT, MoeConfig, MoeError, config, lib,
     moe_grouped_ffn, moe_layer_backward, moe_layer_forward, moe_pack_weights, moe_pack_weights_backward,
     moe_permute, moe_permute_static_scratch, moe_route,
-    moe_unpermute_combine, moe_workspace_size, perm_rows, workspace,
+    moe_unpermute_combine, moe_workspace_size, moe_gemm_tiles_used, perm_rows, workspace,
     moe_mxfp8_quantize, moe_mxfp8_weights_size, moe_pack_weights_mxfp8, mx_counters, mxfp8_scale_bytes)

@@ -35,7 +35,7 @@ EXPORTED = ("moe_workspace_size", "moe_status_string", "moe_version", "moe_pack_
             "moe_permute", "moe_grouped_ffn", "moe_unpermute_combine", "moe_layer_forward",
             "moe_permute_static_scratch", "moe_layer_forward_timed", "moe_pack_weights_backward",
             "moe_layer_backward", "moe_mxfp8_quantize", "moe_mxfp8_weights_size", "moe_pack_weights_mxfp8",
-            "moe_debug_stall_next_gemms")
+            "moe_debug_stall_next_gemms", "moe_gemm_tiles_used")
 
 
 class MoeError(RuntimeError):
@@ -71,6 +71,7 @@ _SIGS = {
     "moe_workspace_size": (SZ, [CFG, I32]),
     "moe_status_string": (ctypes.c_char_p, [I32]),
     "moe_version": (I32, []),
+    "moe_gemm_tiles_used": (I32, [CFG]),
     "moe_pack_weights": (I32, [CFG, P, P, P, P]),
     "moe_route": (I32, [CFG, P, P, P, P, P, P, P, SZ, P, P]),
     "moe_permute": (I32, [CFG, P, P, P, P, P, P, P, P, P, SZ, P, P]),
@@ -173,6 +174,15 @@ def _check_expert_weights(cfg, w13, w_down):
 
 def moe_workspace_size(cfg: MoeConfig, op: int) -> int:
     return int(lib().moe_workspace_size(ctypes.byref(cfg), op))
+
+
+def moe_gemm_tiles_used(cfg: MoeConfig) -> int:
+    """MOE_GEMM_TILES_SINGLE or MOE_GEMM_TILES_PAIR: the grouped GEMMs' tile
+    shape for cfg with AUTO resolved (host only)."""
+    r = int(lib().moe_gemm_tiles_used(ctypes.byref(cfg)))
+    if r < 0:
+        _rc("moe_gemm_tiles_used", r)
+    return r
 
 
 def workspace(cfg: MoeConfig, op: int, device) -> torch.Tensor:

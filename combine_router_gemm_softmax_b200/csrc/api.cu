@@ -2,6 +2,7 @@
 // encoding and stage launches, for the forward stages, the whole layer and
 // its backward. The stage order and the meaning of every argument are
 // documented in include/moe.h.
+#include <algorithm>
 #include <mutex>
 
 #include "moe_common.cuh"
@@ -149,9 +150,6 @@ bool combine_fusable(const moe_config& c) {
          c.gemm_tiles != MOE_GEMM_TILES_PAIR && !is_mx(c);
 }
 
-// AUTO keeps the separate combine: fusing it measured 1-3% slower per layer
-// on B200 (the down projection's epilogue re-reads both rows of a token and
-// competes with the GEMM; the separate kernel streams them at HBM rate).
 // Whether the layer keeps the gate/up pre-activations for the backward.
 bool preact_savable(const moe_config& c) {
   return c.dtype == MOE_DTYPE_BF16 && c.expert_kind == MOE_EXPERT_SWIGLU && c.gemm_tiles != MOE_GEMM_TILES_PAIR &&
@@ -160,6 +158,9 @@ bool preact_savable(const moe_config& c) {
 
 bool layer_saves_preact(const moe_config& c) { return c.preact == MOE_PREACT_SAVE && preact_savable(c); }
 
+// AUTO keeps the separate combine: fusing it measured 1-3% slower per layer
+// on B200 (the down projection's epilogue re-reads both rows of a token and
+// competes with the GEMM; the separate kernel streams them at HBM rate).
 bool layer_fuses_combine(const moe_config& c) { return c.combine == MOE_COMBINE_FUSED && combine_fusable(c); }
 
 // AUTO copies: gathering costs one four-row TMA gather per 512 bytes of A
@@ -167,6 +168,28 @@ bool layer_fuses_combine(const moe_config& c) { return c.combine == MOE_COMBINE_
 // 2.2-2.4x slower per layer on B200 than the row copy plus tiled loads.
 bool layer_gathers(const moe_config& c) {
   return c.dispatch == MOE_DISPATCH_GATHER && gather_supported(c);
+}
+
+// Tile shape of the bf16 grouped GEMMs. The two shapes give the same bits
+// (each output sums its K range in the same order), so this is a speed
+// choice only. AUTO takes CTA-pair tiles where they measured faster on B200,
+// in 10-step and in 250-2000-step loops under the 1 kW cap: experts of at
+// least 1024 rows on average, so that 256-row tiles pad little, with weights
+// of at most 64 MB an expert (3 d F bf16). Pair tiles measured 4-8% faster on
+// the skewed 64-expert layer (d 2048, F 1408) and the scaled Mixtral layer (d
+// 1024, F 3584), even on the skewed layer with capacity 1920, 2% slower with
+// 512-row experts (128 experts, k 8) and 5-8% slower on the Mixtral 8x7B
+// layer (352 MB an expert). Options that need single tiles keep them.
+bool use_pair_tiles(const moe_config& c) {
+  if (c.gemm_tiles == MOE_GEMM_TILES_PAIR) return true;
+  if (c.gemm_tiles != MOE_GEMM_TILES_AUTO) return false;
+  if (c.dtype != MOE_DTYPE_BF16 || c.expert_kind != MOE_EXPERT_SWIGLU || is_mx(c) ||
+      c.dispatch == MOE_DISPATCH_GATHER || c.combine == MOE_COMBINE_FUSED || c.preact == MOE_PREACT_SAVE)
+    return false;
+  long long rows = static_cast<long long>(c.T) * c.k / c.E;
+  if (c.capacity >= 0) rows = c.layout == MOE_LAYOUT_PADDED ? c.capacity : std::min<long long>(rows, c.capacity);
+  const long long expert_weight_bytes = 3LL * c.d * c.d_ff * 2;
+  return rows >= 1024 && expert_weight_bytes <= (64LL << 20);
 }
 
 int check_cfg(const moe_config* c) {
@@ -463,7 +486,7 @@ int ffn_impl(const moe_config& c, const void* x_perm, const int32_t* offsets, co
   const int F = c.d_ff, d = c.d, E = c.E;
   // Tile shape: single-CTA 128x256 tiles unless the caller asks for CTA pairs
   // (256x256, each CTA of the pair stages half of the B tile).
-  const bool pair = c.gemm_tiles == MOE_GEMM_TILES_PAIR;
+  const bool pair = use_pair_tiles(c);
   CUtensorMap a1, b1, a2, b2, d1, d2;
   const bool gather = gather_rows != nullptr && !pair;
   int rc = gather ? make_map(&a1, gather_src, c.T, d, 1) : make_map(&a1, x_perm, rows_max, d, kTileM);
@@ -474,7 +497,7 @@ int ffn_impl(const moe_config& c, const void* x_perm, const int32_t* offsets, co
   if (rc == MOE_OK) rc = make_map_store(&d2, y_perm, rows_max, d);
   if (rc != MOE_OK) return rc;
   cudaError_t e =
-      pair ? launch_grouped_gemm_pair(a1, b1, true, offsets, E, d, 2 * F, F / 128, F, F, h_mid, status, pdl, s)
+      pair ? launch_grouped_gemm_pair(a1, b1, true, offsets, E, d, 2 * F, F / 128, F, F, h_mid, status, pdl, s, &d1)
            : launch_grouped_gemm_tc(a1, b1, true, offsets, E, d, 2 * F, F / 128, F, F, h_mid,
                                     gather ? gather_rows : nullptr, status, pdl, s, preact, &d1);
   if (e != cudaSuccess) return MOE_ERR_CUDA;
@@ -483,7 +506,7 @@ int ffn_impl(const moe_config& c, const void* x_perm, const int32_t* offsets, co
     e = launch_grouped_gemm_combine(a2, b2, offsets, E, F, d, y_perm, fc->perm_src, fc->dest_row, fc->gate,
                                     fc->pair_cnt, fc->y, c.k, status, true, s);
   else
-    e = pair ? launch_grouped_gemm_pair(a2, b2, false, offsets, E, F, d, n2, d, d, y_perm, status, true, s)
+    e = pair ? launch_grouped_gemm_pair(a2, b2, false, offsets, E, F, d, n2, d, d, y_perm, status, true, s, &d2)
              : launch_grouped_gemm_tc(a2, b2, false, offsets, E, F, d, n2, d, d, y_perm, nullptr, status, true, s,
                                       nullptr, &d2);
   return cuda_rc(e);
@@ -496,7 +519,12 @@ using namespace moe;
 
 extern "C" {
 
-int32_t moe_version(void) { return (1 << 16) | 1; }
+int32_t moe_version(void) { return (1 << 16) | 2; }
+
+int32_t moe_gemm_tiles_used(const moe_config* cfg) {
+  if (check_cfg(cfg) != MOE_OK) return MOE_ERR_INVALID_ARG;
+  return use_pair_tiles(*cfg) ? MOE_GEMM_TILES_PAIR : MOE_GEMM_TILES_SINGLE;
+}
 
 const char* moe_status_string(int32_t code) {
   switch (code) {

@@ -49,7 +49,7 @@ constexpr int kStages = 4;
 // tile's columns (the SwiGLU epilogue is as long as a short-K main loop)
 constexpr int kGemmThreads = 320;
 constexpr int kEpiWarps = 8;
-constexpr int kPairThreads = 192;
+constexpr int kPairThreads = 320;  // the same warp roles as the single-CTA kernel
 constexpr uint32_t kABytes = kBM * kBK * 2;
 constexpr uint32_t kBBytes = kBN * kBK * 2;
 constexpr uint32_t kStageBytes = kABytes + kBBytes;
@@ -730,11 +730,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 //   barriers: full[s] lives in the leader and counts both CTAs' bytes; each
 //   CTA's empty[s] and tfull[a] are signalled by the leader's commit to both
 //   CTAs; tempty[a] lives in the leader and takes one arrival per epilogue
-//   warp of both CTAs (8).
+//   warp of both CTAs (16).
+// The epilogue is the single-CTA kernel's: eight warps, two per TMEM lane
+// quadrant, storing whole 32-row blocks through shared memory with TMA stores.
 constexpr int kPairStages = 6;
 constexpr int kPairBM = 256;
 constexpr uint32_t kPairHalfBytes = 128 * kBK * 2;                 // one CTA's A or B slice
-constexpr uint32_t kPairPad = 16384;                               // keeps any operand over-read in bounds
+constexpr uint32_t kPairPad = kEpiWarps * kStgBytes;               // store staging; keeps any operand over-read in bounds
+static_assert(kPairPad >= 16384, "the region after the operand ring must stay at least 16 KB");
 
 constexpr size_t pair_smem_bytes() {
   return 1024 + 2 * kPairStages * static_cast<size_t>(kPairHalfBytes) + kPairPad + (2 * kPairStages + 5) * 8 + 16 +
@@ -744,11 +747,12 @@ constexpr size_t pair_smem_bytes() {
 template <bool kSwiGLU>
 __global__ void __launch_bounds__(kPairThreads, 1)
     grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
-                             const GemmArgs a) {
+                             const __grid_constant__ CUtensorMap tm_d, const GemmArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align_1024(smem_raw);
   uint8_t* sB = smem;                                           // kPairStages x 16 KB
   uint8_t* sA = smem + kPairStages * kPairHalfBytes;             // kPairStages x 16 KB
+  uint8_t* stg_all = smem + 2 * kPairStages * kPairHalfBytes;    // kEpiWarps x kStgBytes, 1024-aligned
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + 2 * kPairStages * kPairHalfBytes + kPairPad);
   uint64_t* empty = full + kPairStages;
   uint64_t* tfull = empty + kPairStages;
@@ -778,7 +782,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&tfull[i], 1);
-      mbar_init(&tempty[i], 8);
+      mbar_init(&tempty[i], 2 * kEpiWarps);
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -786,6 +790,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
     fence_mbar_init();
     tma_prefetch_desc(&tm_a);
     tma_prefetch_desc(&tm_b);
+    if (a.tma_store) tma_prefetch_desc(&tm_d);
   }
   pdl_wait();  // offsets and the A rows come from the kernels before this one
   for (int e = threadIdx.x; e <= E; e += blockDim.x) s_off[e] = a.offsets[e];
@@ -863,6 +868,10 @@ __global__ void __launch_bounds__(kPairThreads, 1)
       uint32_t phase = 0;
       int consumed = 0, local = 0;
       bool stop = false;
+      if (a.stall && !mbar_wait(drain, 0, abort_flag)) {  // nothing arrives on `drain` before the end
+        raise_abort();
+        stop = true;
+      }
       for (long long tile = pair_id; tile < total && !stop; tile += n_pairs, ++local) {
         const int acc = local & 1;
         const uint32_t acc_phase = (local >> 1) & 1;
@@ -901,8 +910,10 @@ __global__ void __launch_bounds__(kPairThreads, 1)
   } else {
     // ---------------------------------------------------------------- epilogue (both CTAs)
     const uint32_t tempty_leader = mapa_shared(smem_addr(&tempty[0]), 0);
-    const int q = warp & 3;
+    const int q = warp & 3;            // TMEM lane quadrant this warp may read
+    const int half = (warp - 2) >> 2;  // which half of the tile's columns it drains
     const int row = q * 32 + lane;
+    uint8_t* stg = stg_all + (warp - 2) * kStgBytes;
     int local = 0;
     for (long long tile = pair_id; tile < total; tile += n_pairs, ++local) {
       int e, m, n;
@@ -919,10 +930,14 @@ __global__ void __launch_bounds__(kPairThreads, 1)
       const bool valid = row < rows_valid;
       const size_t grow = static_cast<size_t>(s_off[e] + row0 + row);
       const uint32_t tbase = tmem + acc * kBN + (static_cast<uint32_t>(q * 32) << 16);
+      // this warp's 32 rows all belong to the expert: stage and TMA-store them
+      const bool staged = a.tma_store != 0 && q * 32 + 32 <= rows_valid;
+      const int srow = s_off[e] + row0 + q * 32;
       if constexpr (kSwiGLU) {
+        // columns [0,128) of the tile are gate, [128,256) the matching up
         __nv_bfloat16* out = a.D + grow * a.ldd + n * (kBN / 2);
 #pragma unroll 1
-        for (int c = 0; c < kBN / 2; c += 32) {
+        for (int c = half * (kBN / 4); c < (half + 1) * (kBN / 4); c += 32) {
           uint32_t g[32], u[32];
           tmem_ld32(tbase + c, g);
           tmem_ld32(tbase + kBN / 2 + c, u);
@@ -935,15 +950,19 @@ __global__ void __launch_bounds__(kPairThreads, 1)
               const float h1 = silu_fast(__uint_as_float(g[2 * i + 1])) * __uint_as_float(u[2 * i + 1]);
               p[i] = pack_bf16x2(h0, h1);
             }
-            uint4* dst = reinterpret_cast<uint4*>(out + c);
+            if (staged) {
+              stage_store(stg, p, lane, &tm_d, n * (kBN / 2) + c, srow);
+            } else {
+              uint4* dst = reinterpret_cast<uint4*>(out + c);
 #pragma unroll
-            for (int i = 0; i < 4; ++i) dst[i] = make_uint4(p[4 * i], p[4 * i + 1], p[4 * i + 2], p[4 * i + 3]);
+              for (int i = 0; i < 4; ++i) dst[i] = make_uint4(p[4 * i], p[4 * i + 1], p[4 * i + 2], p[4 * i + 3]);
+            }
           }
         }
       } else {
         __nv_bfloat16* out = a.D + grow * a.ldd + n * kBN;
 #pragma unroll 1
-        for (int c = 0; c < kBN; c += 32) {
+        for (int c = half * (kBN / 2); c < (half + 1) * (kBN / 2); c += 32) {
           if (n * kBN + c >= a.out_cols) break;
           uint32_t v[32];
           tmem_ld32(tbase + c, v);
@@ -952,9 +971,13 @@ __global__ void __launch_bounds__(kPairThreads, 1)
             uint32_t p[16];
 #pragma unroll
             for (int i = 0; i < 16; ++i) p[i] = pack_bf16x2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
-            uint4* dst = reinterpret_cast<uint4*>(out + c);
+            if (staged) {
+              stage_store(stg, p, lane, &tm_d, n * kBN + c, srow);
+            } else {
+              uint4* dst = reinterpret_cast<uint4*>(out + c);
 #pragma unroll
-            for (int i = 0; i < 4; ++i) dst[i] = make_uint4(p[4 * i], p[4 * i + 1], p[4 * i + 2], p[4 * i + 3]);
+              for (int i = 0; i < 4; ++i) dst[i] = make_uint4(p[4 * i], p[4 * i + 1], p[4 * i + 2], p[4 * i + 3]);
+            }
           }
         }
       }
@@ -964,6 +987,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
     }
   }
   __syncwarp();
+  if (warp >= 2 && lane == 0) bulk_wait_all();  // the epilogue's staged stores have completed
 
   tc_fence_before();
   __syncthreads();
@@ -1113,14 +1137,19 @@ namespace {
 
 std::atomic<int> g_stall_gemms{0};
 
+// 1 when this launch takes one of the stalls moe_debug_stall_next_gemms asked for.
+int take_stall() {
+  int left = g_stall_gemms.load();
+  while (left > 0 && !g_stall_gemms.compare_exchange_weak(left, left - 1)) {
+  }
+  return left > 0 ? 1 : 0;
+}
+
 template <int kEpi, int kMode>
 cudaError_t launch_gemm_inst(const CUtensorMap& tm_a, const CUtensorMap& tm_b, GemmArgs a, bool pdl,
                              cudaStream_t s, const CUtensorMap* tm_d = nullptr) {
   a.tma_store = tm_d != nullptr ? 1 : 0;
-  int left = g_stall_gemms.load();
-  while (left > 0 && !g_stall_gemms.compare_exchange_weak(left, left - 1)) {
-  }
-  a.stall = left > 0 ? 1 : 0;
+  a.stall = take_stall();
   const size_t smem = gemm_smem_bytes();
   cudaError_t err = cudaFuncSetAttribute(grouped_gemm_kernel<kEpi, kMode>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
@@ -1193,9 +1222,13 @@ cudaError_t launch_grouped_gemm_wgrad(const CUtensorMap& tm_a, const CUtensorMap
 
 cudaError_t launch_grouped_gemm_pair(const CUtensorMap& tm_a, const CUtensorMap& tm_b, bool swiglu,
                                      const int32_t* offsets, int E, int K, int n_per_expert, int n_tiles, int out_cols,
-                                     int ldd, void* D, int32_t* status, bool pdl, cudaStream_t s) {
+                                     int ldd, void* D, int32_t* status, bool pdl, cudaStream_t s,
+                                     const CUtensorMap* tm_d) {
   GemmArgs a{offsets, E, K, n_per_expert, n_tiles, out_cols, ldd, static_cast<__nv_bfloat16*>(D), status,
              band_rows(2 * kBM, K, 4, 16), nullptr, nullptr, 0, nullptr, 0, nullptr, nullptr, 0};
+  a.tma_store = tm_d != nullptr ? 1 : 0;
+  a.stall = take_stall();
+  const CUtensorMap& map_d = tm_d != nullptr ? *tm_d : tm_a;
   const size_t smem = pair_smem_bytes();
   const int grid = (device_sm_count() / 2) * 2;
   cudaError_t err;
@@ -1204,13 +1237,13 @@ cudaError_t launch_grouped_gemm_pair(const CUtensorMap& tm_a, const CUtensorMap&
                                static_cast<int>(smem));
     if (err != cudaSuccess) return err;
     err = launch_kernel(grouped_gemm_pair_kernel<true>, dim3(grid), dim3(kPairThreads), smem, s, pdl, 2, tm_a, tm_b,
-                        a);
+                        map_d, a);
   } else {
     err = cudaFuncSetAttribute(grouped_gemm_pair_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                static_cast<int>(smem));
     if (err != cudaSuccess) return err;
     err = launch_kernel(grouped_gemm_pair_kernel<false>, dim3(grid), dim3(kPairThreads), smem, s, pdl, 2, tm_a, tm_b,
-                        a);
+                        map_d, a);
   }
   if (err != cudaSuccess) return err;
   return cudaGetLastError();

@@ -103,7 +103,8 @@ cudaError_t launch_grouped_gemm_wgrad(const CUtensorMap& tm_a, const CUtensorMap
                                       int E, int M, int N, float* D32, int32_t* status, bool pdl, cudaStream_t s);
 cudaError_t launch_grouped_gemm_pair(const CUtensorMap& tm_a, const CUtensorMap& tm_b, bool swiglu,
                                      const int32_t* offsets, int E, int K, int n_per_expert, int n_tiles, int out_cols,
-                                     int ldd, void* D, int32_t* status, bool pdl, cudaStream_t s);
+                                     int ldd, void* D, int32_t* status, bool pdl, cudaStream_t s,
+                                     const CUtensorMap* tm_d = nullptr);
 cudaError_t launch_ffn_f32(const float* x_perm, const int32_t* offsets, const float* w13, const float* wd,
                            float* h_mid, float* y_perm, int rows_max, int d, int F, int E, cudaStream_t s);
 cudaError_t launch_scale_rows(int dtype, int kind, const void* x_perm, const int32_t* offsets, void* y_perm,

@@ -83,9 +83,15 @@ extern "C" {
 
 /* Grouped-GEMM tiles (bf16 path). SINGLE: 128x256 tiles, one SM each. PAIR:
  * 256x256 tiles shared by two SMs of a cluster (tcgen05 cta_group::2), which
- * halves the operand bytes each SM stages but moves operands between the
- * two SMs; under the 1 kW power cap it measured about 5% slower per layer on
- * B200, so AUTO picks SINGLE. */
+ * halves the operand bytes each SM stages. Both give the same bits. AUTO
+ * picks PAIR where it measured faster on B200: bf16 SwiGLU experts of at
+ * least 1024 rows on average (T*k/E, or the capacity if smaller; the
+ * capacity in the padded layout) with at most 64 MB of weights each
+ * (3*d*d_ff bf16), and none of the options that need single tiles (MXFP8,
+ * gather dispatch, fused combine, kept pre-activations). Larger experts (the
+ * Mixtral 8x7B shape, 352 MB each) measured about 5% slower on pair tiles
+ * under the 1 kW power cap, smaller ones pad more. moe_gemm_tiles_used
+ * reports the choice. */
 #define MOE_GEMM_TILES_AUTO   0
 #define MOE_GEMM_TILES_SINGLE 1
 #define MOE_GEMM_TILES_PAIR   2
@@ -204,6 +210,12 @@ MOE_API const char* moe_status_string(int32_t code);
 
 /* ABI version, (major << 16) | minor. */
 MOE_API int32_t moe_version(void);
+
+/* The tile shape (MOE_GEMM_TILES_SINGLE or MOE_GEMM_TILES_PAIR) the bf16
+ * grouped GEMMs of moe_grouped_ffn and moe_layer_forward take for cfg, with
+ * AUTO resolved; MOE_ERR_INVALID_ARG for an invalid cfg. Host only: no GPU
+ * work, no CUDA call. */
+MOE_API int32_t moe_gemm_tiles_used(const moe_config* cfg);
 
 /* moe_pack_weights -- lay out the gate and up projections for the grouped FFN.
  * w_gate, w_up: [E, F, d]. w13_packed: [E, 2F, d], written. For each expert,
@@ -373,8 +385,8 @@ MOE_API int32_t moe_pack_weights_mxfp8(const moe_config* cfg, const void* w13_pa
 
 /* moe_debug_stall_next_gemms -- testing hook for the timeout path. The pages
  * have no counterpart. The next n launches (process-wide, any stream) of the
- * bf16 grouped GEMM kernel make their MMA-issuing thread first wait on a
- * barrier that nothing signals. That wait gives up after the library's
+ * bf16 grouped GEMM kernels (single-CTA or CTA-pair tiles) make their
+ * MMA-issuing thread first wait on a barrier that nothing signals. That wait gives up after the library's
  * on-chip limit (2 s), the kernel unwinds as after any timeout (no MMA was
  * issued; the operand loads already issued are waited for and TMEM is freed)
  * and MOE_STATUS_TIMEOUT is OR-ed into the status word; that call's outputs

@@ -99,6 +99,38 @@ def test_gemm_tiles_value_checked(L):
         assert M.moe_workspace_size(M.config(64, 128, 8, 2, 256, gemm_tiles=tiles), M.MOE_OP_LAYER) > 0
 
 
+def test_gemm_tiles_auto_rule(L):
+    """AUTO resolves to CTA-pair tiles only for bf16 SwiGLU experts of at
+    least 1024 rows on average (T*k/E, capped by a compact capacity; the
+    capacity itself in the padded layout) and at most 64 MB of weights each,
+    and never when an option that needs single tiles is set. Host only."""
+    used = M.moe_gemm_tiles_used
+    S, P = M.MOE_GEMM_TILES_SINGLE, M.MOE_GEMM_TILES_PAIR
+    # the layers this rule was measured on
+    assert used(M.config(4096, 1024, 8, 2, 3584)) == P                      # 1024 rows, 22 MB
+    assert used(M.config(16384, 2048, 64, 6, 1408)) == P                    # 1536 rows, 17 MB
+    assert used(M.config(16384, 2048, 64, 6, 1408, capacity=1920)) == P
+    assert used(M.config(16384, 2048, 64, 6, 1408, capacity=1920, layout="padded")) == P
+    assert used(M.config(32768, 4096, 8, 2, 14336)) == S                    # 352 MB an expert
+    assert used(M.config(8192, 2048, 128, 8, 768)) == S                     # 512 rows
+    # the edges of the rule
+    assert used(M.config(4095, 1024, 8, 2, 3584)) == S                      # 1023 rows
+    assert used(M.config(16384, 2048, 64, 6, 1408, capacity=1000)) == S     # capped below 1024
+    assert used(M.config(1024, 2048, 64, 6, 1408, capacity=1024, layout="padded")) == P
+    assert used(M.config(8192, 4096, 8, 1, 2688)) == P                      # 3 d F 2 = 63 MB
+    assert used(M.config(8192, 4096, 8, 1, 2816)) == S                      # 66 MB
+    # options that need single tiles, other dtypes and expert kinds
+    for kw in (dict(dispatch="gather"), dict(combine="fused"), dict(preact="save"), dict(precision="mxfp8"),
+               dict(dtype="f32"), dict(expert_kind="identity"), dict(gemm_tiles="single")):
+        assert used(M.config(4096, 1024, 8, 2, 3584, **kw)) == S, kw
+    # an explicit request is kept
+    assert used(M.config(64, 128, 8, 2, 256, gemm_tiles="pair")) == P
+    assert used(M.config(64, 128, 8, 2, 256)) == S
+    bad = M.config(64, 128, 8, 2, 256)
+    bad.gemm_tiles = 7
+    assert L.moe_gemm_tiles_used(ctypes.byref(bad)) == M.MOE_ERR_INVALID_ARG
+
+
 def test_null_pointers_rejected(L):
     cfg = M.config(64, 128, 8, 2, 256)
     assert L.moe_route(ctypes.byref(cfg), None, None, None, None, None, None, None, 0, None, None) \

@@ -279,6 +279,24 @@ def test_layer_gather_dispatch_equals_copy(name):
     assert torch.equal(ys["copy"].view(torch.int16), ys["gather"].view(torch.int16))
 
 
+@pytest.mark.parametrize("name", ["small_pair", "small_pair_wide", "small_skewed_pair"])
+def test_layer_pair_tiles_equal_single(name):
+    """256-row CTA-pair tiles accumulate every output over K in the same order
+    as the single-CTA 128-row tiles, so y is the same bit for bit; the cases
+    have ragged last pair tiles in which one CTA of the pair has no rows and
+    32-row blocks cut by an expert's end."""
+    dc = dev_case(name)
+    wl = dc.wl
+    base = dict(T=wl.T, d=wl.d, E=wl.E, k=wl.k, d_ff=wl.F, dtype=wl.dtype, expert_kind=wl.expert_kind,
+                capacity=wl.capacity)
+    ys = {}
+    for tiles in ("single", "pair"):
+        cfg = M.config(**base, gemm_tiles=tiles)
+        ys[tiles] = M.moe_layer_forward(cfg, dc.h, dc.w_router, dc.bias, dc.w13, dc.w_down)
+    torch.cuda.synchronize()
+    assert torch.equal(ys["single"].view(torch.int16), ys["pair"].view(torch.int16))
+
+
 def test_config_layout_checks():
     with pytest.raises(M.MoeError):
         M.moe_layer_forward(M.config(64, 128, 4, 2, 128, layout="padded"),  # padded needs a capacity

@@ -17,9 +17,12 @@ from gpu_cases import DeviceCase, parity_case
 pytestmark = pytest.mark.gpu
 
 
-def test_gemm_wait_timeout_is_reported_and_the_context_stays_usable():
+@pytest.mark.parametrize("name", ["small_ragged", "small_pair"])
+def test_gemm_wait_timeout_is_reported_and_the_context_stays_usable(name):
+    """small_ragged runs single-CTA tiles, small_pair CTA-pair tiles, whose
+    timeout also stops the partner CTA through its shared-memory flag."""
     torch.cuda.set_device(0)
-    dc = DeviceCase(parity_case("small_ragged")[0])
+    dc = DeviceCase(parity_case(name)[0])
     y_ref = dc.layer()["y"].clone()
     torch.cuda.synchronize()
     assert int(dc.status.item()) == 0
