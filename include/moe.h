@@ -115,7 +115,8 @@ extern "C" {
  * permutation (TMA tile::gather4, four rows per load), the fused dispatch of
  * "Dropless MoE Is a Runtime Problem as Much as a Model Design" (fusing
  * dispatch to cut intermediate writes). GATHER needs bf16, SwiGLU experts, the
- * COMPACT layout and single-CTA tiles. The result is the same bit for bit.
+ * COMPACT layout and single-CTA tiles (gemm_tiles SINGLE, or AUTO, which then
+ * keeps them). The result is the same bit for bit.
  * AUTO is COPY: a tile reloads its A rows once per column tile, so the
  * gather repeats for every column tile, and GATHER measured 2.2-2.4x slower
  * per layer on B200. The stage entry points (moe_permute, moe_grouped_ffn)
@@ -153,7 +154,8 @@ extern "C" {
  * two rows of a column tile (a per-token counter decides) reads both back
  * from y_perm and writes y in slot order. y is bit-identical either way, and
  * y_perm is still written (the backward reads it). Needs bf16 SwiGLU
- * experts, single-CTA tiles and bf16 precision. AUTO is SEPARATE: on B200
+ * experts, single-CTA tiles (gemm_tiles SINGLE, or AUTO, which then keeps
+ * them) and bf16 precision. AUTO is SEPARATE: on B200
  * the fused form measured 1-3% slower per layer (its epilogue re-reads both
  * rows of a token while the GEMM runs), so it is opt-in. */
 #define MOE_COMBINE_AUTO     0
@@ -168,8 +170,8 @@ extern "C" {
  * column order), and the backward applies the SwiGLU backward in the epilogue
  * of its dh_mid GEMM from them, with no recompute. The forward then writes
  * 4 P F more bytes; the backward's gradients use the bf16-rounded a and u.
- * SAVE needs bf16 SwiGLU experts, single-CTA tiles, bf16 precision and the
- * COPY dispatch. */
+ * SAVE needs bf16 SwiGLU experts, single-CTA tiles (gemm_tiles SINGLE, or
+ * AUTO, which then keeps them), bf16 precision and the COPY dispatch. */
 #define MOE_PREACT_RECOMPUTE 0
 #define MOE_PREACT_SAVE      1
 
