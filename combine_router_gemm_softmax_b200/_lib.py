@@ -71,7 +71,7 @@ _SIGS = {
     "moe_workspace_size": (SZ, [CFG, I32]),
     "moe_status_string": (ctypes.c_char_p, [I32]),
     "moe_version": (I32, []),
-    "moe_gemm_tiles_used": (I32, [CFG]),
+    "moe_gemm_tiles_used": (I32, [CFG, P]),
     "moe_pack_weights": (I32, [CFG, P, P, P, P]),
     "moe_route": (I32, [CFG, P, P, P, P, P, P, P, SZ, P, P]),
     "moe_permute": (I32, [CFG, P, P, P, P, P, P, P, P, P, SZ, P, P]),
@@ -179,10 +179,9 @@ def moe_workspace_size(cfg: MoeConfig, op: int) -> int:
 def moe_gemm_tiles_used(cfg: MoeConfig) -> int:
     """MOE_GEMM_TILES_SINGLE or MOE_GEMM_TILES_PAIR: the grouped GEMMs' tile
     shape for cfg with AUTO resolved (host only)."""
-    r = int(lib().moe_gemm_tiles_used(ctypes.byref(cfg)))
-    if r < 0:
-        _rc("moe_gemm_tiles_used", r)
-    return r
+    tiles = ctypes.c_int32(-1)
+    _rc("moe_gemm_tiles_used", lib().moe_gemm_tiles_used(ctypes.byref(cfg), ctypes.byref(tiles)))
+    return tiles.value
 
 
 def workspace(cfg: MoeConfig, op: int, device) -> torch.Tensor:

@@ -173,13 +173,15 @@ bool layer_gathers(const moe_config& c) {
 // Tile shape of the bf16 grouped GEMMs. The two shapes give the same bits
 // (each output sums its K range in the same order), so this is a speed
 // choice only. AUTO takes CTA-pair tiles where they measured faster on B200,
-// in 10-step and in 250-2000-step loops under the 1 kW cap: experts of at
+// in 10-step and in 100-2000-step loops under the 1 kW cap: experts of at
 // least 1024 rows on average, so that 256-row tiles pad little, with weights
-// of at most 64 MB an expert (3 d F bf16). Pair tiles measured 4-8% faster on
-// the skewed 64-expert layer (d 2048, F 1408) and the scaled Mixtral layer (d
-// 1024, F 3584), even on the skewed layer with capacity 1920, 2% slower with
-// 512-row experts (128 experts, k 8) and 5-8% slower on the Mixtral 8x7B
-// layer (352 MB an expert). Options that need single tiles keep them.
+// of at most 128 MiB an expert (3 d F bf16; about the L2 size). Pair tiles
+// measured 4-8% faster on the skewed 64-expert layer (d 2048, F 1408) and the
+// scaled Mixtral layer (d 1024, F 3584), 2-3% faster with 63 and 88 MB
+// experts, even with 132 MB ones, even on the skewed layer with capacity
+// 1920, 2% slower with 512-row experts (128 experts, k 8) and 5-8% slower on
+// the Mixtral 8x7B layer (352 MB an expert). Options that need single tiles
+// keep them.
 bool use_pair_tiles(const moe_config& c) {
   if (c.gemm_tiles == MOE_GEMM_TILES_PAIR) return true;
   if (c.gemm_tiles != MOE_GEMM_TILES_AUTO) return false;
@@ -189,7 +191,7 @@ bool use_pair_tiles(const moe_config& c) {
   long long rows = static_cast<long long>(c.T) * c.k / c.E;
   if (c.capacity >= 0) rows = c.layout == MOE_LAYOUT_PADDED ? c.capacity : std::min<long long>(rows, c.capacity);
   const long long expert_weight_bytes = 3LL * c.d * c.d_ff * 2;
-  return rows >= 1024 && expert_weight_bytes <= (64LL << 20);
+  return rows >= 1024 && expert_weight_bytes <= (128LL << 20);
 }
 
 int check_cfg(const moe_config* c) {
@@ -521,9 +523,12 @@ extern "C" {
 
 int32_t moe_version(void) { return (1 << 16) | 2; }
 
-int32_t moe_gemm_tiles_used(const moe_config* cfg) {
-  if (check_cfg(cfg) != MOE_OK) return MOE_ERR_INVALID_ARG;
-  return use_pair_tiles(*cfg) ? MOE_GEMM_TILES_PAIR : MOE_GEMM_TILES_SINGLE;
+int32_t moe_gemm_tiles_used(const moe_config* cfg, int32_t* tiles) {
+  if (tiles == nullptr) return MOE_ERR_INVALID_ARG;
+  const int rc = check_cfg(cfg);
+  if (rc != MOE_OK) return rc;
+  *tiles = use_pair_tiles(*cfg) ? MOE_GEMM_TILES_PAIR : MOE_GEMM_TILES_SINGLE;
+  return MOE_OK;
 }
 
 const char* moe_status_string(int32_t code) {

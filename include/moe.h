@@ -86,7 +86,7 @@ extern "C" {
  * halves the operand bytes each SM stages. Both give the same bits. AUTO
  * picks PAIR where it measured faster on B200: bf16 SwiGLU experts of at
  * least 1024 rows on average (T*k/E, or the capacity if smaller; the
- * capacity in the padded layout) with at most 64 MB of weights each
+ * capacity in the padded layout) with at most 128 MiB of weights each
  * (3*d*d_ff bf16), and none of the options that need single tiles (MXFP8,
  * gather dispatch, fused combine, kept pre-activations). Larger experts (the
  * Mixtral 8x7B shape, 352 MB each) measured about 5% slower on pair tiles
@@ -213,11 +213,13 @@ MOE_API const char* moe_status_string(int32_t code);
 /* ABI version, (major << 16) | minor. */
 MOE_API int32_t moe_version(void);
 
-/* The tile shape (MOE_GEMM_TILES_SINGLE or MOE_GEMM_TILES_PAIR) the bf16
- * grouped GEMMs of moe_grouped_ffn and moe_layer_forward take for cfg, with
- * AUTO resolved; MOE_ERR_INVALID_ARG for an invalid cfg. Host only: no GPU
- * work, no CUDA call. */
-MOE_API int32_t moe_gemm_tiles_used(const moe_config* cfg);
+/* moe_gemm_tiles_used -- writes to *tiles the tile shape
+ * (MOE_GEMM_TILES_SINGLE or MOE_GEMM_TILES_PAIR) that the bf16 grouped GEMMs
+ * of moe_grouped_ffn and moe_layer_forward take for cfg, with AUTO resolved.
+ * Returns MOE_OK, MOE_ERR_INVALID_ARG (NULL tiles, invalid cfg) or
+ * MOE_ERR_UNSUPPORTED (a cfg the library rejects); *tiles is then untouched.
+ * Host only: no GPU work, no CUDA call. */
+MOE_API int32_t moe_gemm_tiles_used(const moe_config* cfg, int32_t* tiles);
 
 /* moe_pack_weights -- lay out the gate and up projections for the grouped FFN.
  * w_gate, w_up: [E, F, d]. w13_packed: [E, 2F, d], written. For each expert,

@@ -102,7 +102,7 @@ def test_gemm_tiles_value_checked(L):
 def test_gemm_tiles_auto_rule(L):
     """AUTO resolves to CTA-pair tiles only for bf16 SwiGLU experts of at
     least 1024 rows on average (T*k/E, capped by a compact capacity; the
-    capacity itself in the padded layout) and at most 64 MB of weights each,
+    capacity itself in the padded layout) and at most 128 MiB of weights each,
     and never when an option that needs single tiles is set. Host only."""
     used = M.moe_gemm_tiles_used
     S, P = M.MOE_GEMM_TILES_SINGLE, M.MOE_GEMM_TILES_PAIR
@@ -117,8 +117,9 @@ def test_gemm_tiles_auto_rule(L):
     assert used(M.config(4095, 1024, 8, 2, 3584)) == S                      # 1023 rows
     assert used(M.config(16384, 2048, 64, 6, 1408, capacity=1000)) == S     # capped below 1024
     assert used(M.config(1024, 2048, 64, 6, 1408, capacity=1024, layout="padded")) == P
-    assert used(M.config(8192, 4096, 8, 1, 2688)) == P                      # 3 d F 2 = 63 MB
-    assert used(M.config(8192, 4096, 8, 1, 2816)) == S                      # 66 MB
+    assert used(M.config(16384, 2048, 8, 2, 7168)) == P                     # 88 MB, measured faster
+    assert used(M.config(8192, 4096, 8, 1, 5376)) == P                      # 3 d F 2 = 132 MB <= 128 MiB
+    assert used(M.config(8192, 4096, 8, 1, 5504)) == S                      # 135 MB > 128 MiB
     # options that need single tiles, other dtypes and expert kinds
     for kw in (dict(dispatch="gather"), dict(combine="fused"), dict(preact="save"), dict(precision="mxfp8"),
                dict(dtype="f32"), dict(expert_kind="identity"), dict(gemm_tiles="single")):
@@ -126,9 +127,17 @@ def test_gemm_tiles_auto_rule(L):
     # an explicit request is kept
     assert used(M.config(64, 128, 8, 2, 256, gemm_tiles="pair")) == P
     assert used(M.config(64, 128, 8, 2, 256)) == S
+    # errors come back as the return code and leave the output alone
+    out = ctypes.c_int32(-1)
     bad = M.config(64, 128, 8, 2, 256)
     bad.gemm_tiles = 7
-    assert L.moe_gemm_tiles_used(ctypes.byref(bad)) == M.MOE_ERR_INVALID_ARG
+    assert L.moe_gemm_tiles_used(ctypes.byref(bad), ctypes.byref(out)) == M.MOE_ERR_INVALID_ARG
+    odd = M.config(64, 128, 8, 2, 200)                                      # d_ff not a multiple of 128
+    assert L.moe_gemm_tiles_used(ctypes.byref(odd), ctypes.byref(out)) == M.MOE_ERR_UNSUPPORTED
+    assert L.moe_gemm_tiles_used(ctypes.byref(M.config(64, 128, 8, 2, 256)), None) == M.MOE_ERR_INVALID_ARG
+    assert out.value == -1
+    with pytest.raises(M.MoeError):
+        used(odd)
 
 
 def test_null_pointers_rejected(L):
