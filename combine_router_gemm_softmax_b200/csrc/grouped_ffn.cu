@@ -743,6 +743,7 @@ constexpr size_t pair_smem_bytes() {
   return 1024 + 2 * kPairStages * static_cast<size_t>(kPairHalfBytes) + kPairPad + (2 * kPairStages + 5) * 8 + 16 +
          2 * (kMaxE + 1) * 4;
 }
+static_assert(pair_smem_bytes() <= 227 * 1024, "shared memory");
 
 template <bool kSwiGLU>
 __global__ void __launch_bounds__(kPairThreads, 1)
