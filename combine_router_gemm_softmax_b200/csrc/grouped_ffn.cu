@@ -15,13 +15,22 @@
 // projection with K = 14336), so the band stays in L2 while the weights stream
 // through it once. grid = number of SMs; CTA c takes tiles c, c + grid, ...
 //
-// Inside a CTA (192 threads): warp 0 issues TMA loads into a 4-stage ring of
+// Inside a CTA (320 threads): warp 0 issues TMA loads into a 4-stage ring of
 // shared-memory buffers, warp 1 allocates TMEM and one of its threads issues
-// tcgen05.mma into one of two 256-column fp32 accumulators, warps 2..5 drain
-// the other accumulator (tcgen05.ld, 32x32b: one thread per output row) and
-// store it, so the epilogue of tile i overlaps the main loop of tile i+1.
-// Rows past the end of an expert's group are computed on whatever the buffer
-// holds there and never stored.
+// tcgen05.mma into one of two 256-column fp32 accumulators, warps 2..9 (two
+// per TMEM lane quadrant, each taking half of the columns) drain the other
+// accumulator (tcgen05.ld, 32x32b: one thread per output row), so the
+// epilogue of tile i overlaps the main loop of tile i+1. A warp whose 32 rows
+// all belong to the expert writes each 32-column block into its own staging
+// buffer in shared memory and stores it with one TMA store; the others store
+// row by row. Rows past the end of an expert's group are computed on whatever
+// the buffer holds there and never stored.
+//
+// CTA-pair variant (grouped_gemm_pair_kernel): 256 x 256 tiles on a cluster
+// of two SMs with tcgen05.mma.cta_group::2, each CTA staging its own 128 A
+// rows and half of B, so each SM stages a third fewer operand bytes per
+// flop; same epilogue, same bits. The layer takes it for mid-sized experts
+// (the rule is use_pair_tiles in api.cu).
 //
 // The same kernel, by template arguments, also serves the layer's backward:
 // a plain bf16 store (the down projection and both dgrad GEMMs), the gate/up
