@@ -55,6 +55,9 @@ def test_launch_count_per_step():
     import bench
     import combine_router_gemm_softmax_b200 as M
     assert bench.launches(M.config(64, 128, 8, 2, 128)) == 6
+    # CTA-pair GEMM tiles (AUTO's choice here) are one launch per GEMM too
+    cfg = M.config(4096, 1024, 8, 2, 3584)
+    assert M.moe_gemm_tiles_used(cfg) == M.MOE_GEMM_TILES_PAIR and bench.launches(cfg) == 6
     # combine fused into the down projection (opt-in): no combine kernel
     assert bench.launches(M.config(64, 128, 8, 2, 128, combine="fused")) == 5
     # MXFP8: the row copy is replaced by the dispatch that quantises the rows
